@@ -1,0 +1,434 @@
+"""Pins of the CPU oracle to facts fixed outside itself (CPU only).
+
+Each test checks the oracle against a closed form, an invariant the pages state,
+brute force on tiny inputs, an independent library routine, or a figure the
+pages print (tests/golden/).  A plausible slip in the oracle (a dropped term, a
+swapped operand, a wrong index, a missed rounding point) fails one of them.
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from routing_dispatch_grouped_top_b200 import inputs
+from routing_dispatch_grouped_top_b200.config import DEEPSEEK_R1_DECODE, TINY
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def bf(vals):
+    return oracle.f64_to_bf16_bits(np.asarray(vals, dtype=np.float64))
+
+
+def val(bits):
+    return oracle.bf16_bits_to_f64(bits)
+
+
+# ---------------------------------------------------------------------------
+# bf16 rounding
+# ---------------------------------------------------------------------------
+
+def test_bf16_rounding_hand_values():
+    # 1 + 2^-8 is the midpoint of 1.0 and 1.0078125: ties go to the even pattern 0x3F80.
+    assert bf([1.0 + 2 ** -8])[0] == 0x3F80
+    assert bf([1.0 + 3 * 2 ** -8])[0] == 0x3F82       # midpoint of 0x3F81/0x3F82 -> even
+    assert bf([1.0 + 1.5 * 2 ** -8])[0] == 0x3F81
+    assert bf([-2.0])[0] == 0xC000
+    assert bf([65504.0])[0] == 0x4780                  # rounds up to 65536
+    assert bf([3 * 2.0 ** -133])[0] == 0x0003          # subnormal spacing 2^-133
+    assert bf([np.inf])[0] == 0x7F80 and bf([-np.inf])[0] == 0xFF80
+
+
+def test_bf16_rounding_matches_torch_on_float32_values():
+    # Every float32 value is exact in float64, so direct f64->bf16 rounding must
+    # agree with torch's float32->bf16 conversion (an independent implementation).
+    g = torch.Generator().manual_seed(0)
+    f = torch.cat([torch.randn(200000, generator=g) * 10.0 ** torch.randint(-30, 30, (200000,), generator=g),
+                   torch.tensor([0.0, -0.0, 1e-40, -3e-39, 3.3e38])]).to(torch.float32)
+    ref = f.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = bf(f.numpy().astype(np.float64))
+    assert np.array_equal(got, ref)
+
+
+# ---------------------------------------------------------------------------
+# S0 gating logits
+# ---------------------------------------------------------------------------
+
+def test_logits_one_hot_rows_select_router_rows():
+    H, E = 16, 5
+    w_g = np.random.default_rng(1).standard_normal((H, E)).astype(np.float32)
+    x = np.zeros((H, H)); x[np.arange(H), np.arange(H)] = 1.0
+    l = oracle.gating_logits(bf(x), w_g)
+    assert np.array_equal(l, w_g)                      # row h of W_g, not a column
+    bias = np.arange(E, dtype=np.float32) * 0.25
+    lb = oracle.gating_logits(bf(x), w_g, bias)
+    assert np.array_equal(lb, (w_g + bias).astype(np.float32))
+
+
+def test_logits_exact_small_integer_sum():
+    x = bf([[1.0, 2.0, -3.0]])
+    w_g = np.array([[1.0, 0.5], [2.0, 0.25], [1.0, -1.0]], np.float32)
+    assert np.array_equal(oracle.gating_logits(x, w_g), np.array([[2.0, 4.0]], np.float32))
+
+
+# ---------------------------------------------------------------------------
+# S1 top-k selection (brute force over all subsets) and weights (closed forms)
+# ---------------------------------------------------------------------------
+
+def _beats(va, a, vb, b):
+    """a ranks above b: larger value; equal values -> lower id; NaN below all."""
+    na, nb = math.isnan(va), math.isnan(vb)
+    if na or nb:
+        if na and nb:
+            return a < b
+        return nb
+    if va != vb:
+        return va > vb
+    return a < b
+
+
+def _brute_topk(row, K):
+    E = len(row)
+    winners = []
+    for S in itertools.combinations(range(E), K):
+        rest = [j for j in range(E) if j not in S]
+        if all(_beats(row[i], i, row[j], j) for i in S for j in rest):
+            winners.append(S)
+    assert len(winners) == 1
+    S = list(winners[0])
+    # order inside the set: best first (insertion sort with the same relation)
+    out = []
+    for i in S:
+        pos = 0
+        while pos < len(out) and _beats(row[out[pos]], out[pos], row[i], i):
+            pos += 1
+        out.insert(pos, i)
+    return out
+
+
+@pytest.mark.parametrize("gen", ["random", "quantized", "special"])
+@pytest.mark.parametrize("E,K", [(5, 2), (7, 3), (8, 8), (8, 1), (6, 4)])
+def test_topk_matches_brute_force(gen, E, K):
+    T = 40
+    if gen == "random":
+        l = inputs.random_logits(T, E, seed=E * 10 + K)
+    elif gen == "quantized":
+        l = inputs.quantized_logits(T, E, levels=3, seed=E * 10 + K)
+    else:
+        l = inputs.special_logits(T, E, seed=E * 10 + K)
+    l = l.numpy()
+    ids, _ = oracle.route(l, K)
+    for t in range(T):
+        assert list(ids[t]) == _brute_topk([float(v) for v in l[t]], K), (t, l[t])
+
+
+def test_topk_all_equal_logits_gives_lowest_ids():
+    ids, w = oracle.route(np.full((3, 9), 0.5, np.float32), 4)
+    assert (ids == np.arange(4)).all()
+    assert np.allclose(w, 0.25, atol=0)
+
+
+def test_topk_signed_zero_is_a_tie():
+    l = np.array([[-0.0, 0.0, -1.0]], np.float32)
+    ids, _ = oracle.route(l, 1)
+    assert ids[0, 0] == 0                              # -0.0 == +0.0 -> lower id
+
+
+def test_weights_closed_form_renormalised():
+    # logits ln1, ln2, ln3 (+ a loser): renormalised top-3 weights are 3/6, 2/6, 1/6.
+    l = np.array([[0.0, math.log(2.0), math.log(3.0), -50.0]], np.float32)
+    ids, w = oracle.route(l, 3, renormalize=True)
+    assert list(ids[0]) == [2, 1, 0]
+    e = np.exp(l[0, [2, 1, 0]].astype(np.float64))
+    assert np.allclose(w[0], [0.5, 1 / 3, 1 / 6], atol=2e-7)
+    assert abs(float(w.sum()) - 1.0) < 1e-6
+    assert e[0] > e[1] > e[2]
+
+
+def test_weights_closed_form_plain_softmax():
+    # logits ln1..ln4, K = 2 without renormalising: weights 4/10 and 3/10.
+    l = np.log(np.array([[1.0, 2.0, 3.0, 4.0]])).astype(np.float32)
+    ids, w = oracle.route(l, 2, renormalize=False)
+    assert list(ids[0]) == [3, 2]
+    assert np.allclose(w[0], [0.4, 0.3], atol=2e-7)
+
+
+def test_weights_sum_to_one_and_K_equal_E_is_full_softmax_order():
+    l = inputs.random_logits(64, 12, seed=3).numpy()
+    ids, w = oracle.route(l, 12)
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-6)
+    for t in range(64):
+        assert sorted(ids[t]) == list(range(12))       # K = E selects every expert
+        assert np.all(np.diff(w[t]) <= 0)              # weights follow the slot order
+    # K = E with renormalisation equals the plain softmax over E (same weights).
+    _, w2 = oracle.route(l, 12, renormalize=False)
+    assert np.allclose(w, w2, atol=1e-7)
+
+
+# ---------------------------------------------------------------------------
+# S2 counting / scan / permutation
+# ---------------------------------------------------------------------------
+
+def _count_definition(ids_flat, E):
+    """Row of each assignment straight from the counting definition, in loops."""
+    counts = [0] * E
+    for e in ids_flat:
+        counts[e] += 1
+    off = [0]
+    for c in counts:
+        off.append(off[-1] + c)
+    seen = [0] * E
+    rows = []
+    for e in ids_flat:
+        rows.append(off[e] + seen[e])
+        seen[e] += 1
+    return counts, off, rows
+
+
+@pytest.mark.parametrize("T,E,K,P,zipf", [(37, 8, 2, 2, None), (64, 16, 4, 4, 1.1), (5, 32, 3, 8, None),
+                                          (1, 4, 4, 1, None), (100, 6, 1, 3, 2.0)])
+def test_count_scan_matches_counting_definition(T, E, K, P, zipf):
+    ids = inputs.random_topk_ids(T, E, K, seed=T + E, zipf_s=zipf).numpy()
+    cs = oracle.count_scan(ids, E, P)
+    counts, off, rows = _count_definition(list(ids.reshape(-1)), E)
+    assert list(cs["counts"]) == counts
+    assert list(cs["offsets"]) == off
+    assert list(cs["row_of_assign"]) == rows
+    # invariants: counts sum to T*K (every token contributes K rows)
+    assert cs["counts"].sum() == T * K and cs["offsets"][-1] == T * K
+    # bijection
+    roa, aor = cs["row_of_assign"], cs["assign_of_row"]
+    assert np.array_equal(aor[roa], np.arange(T * K)) and np.array_equal(roa[aor], np.arange(T * K))
+    # partitions: part_offsets[p] = offsets[p*E/P]; rows of partition p hold its experts
+    epp = E // P
+    assert np.array_equal(cs["part_offsets"], cs["offsets"][::epp])
+    flat = ids.reshape(-1)
+    for p in range(P):
+        lo, hi = cs["part_offsets"][p], cs["part_offsets"][p + 1]
+        assert cs["part_counts"][p] == hi - lo
+        e_rows = flat[aor[lo:hi]]
+        assert np.all((e_rows >= p * epp) & (e_rows < (p + 1) * epp))
+
+
+def test_rows_per_token_figure():
+    fig = json.load(open(os.path.join(GOLDEN, "sizing_figures.json")))["rows_per_token"]
+    ids = inputs.random_topk_ids(50, 8, fig["K"], seed=5).numpy()
+    cs = oracle.count_scan(ids, 8)
+    assert cs["counts"].sum() == 50 * fig["rows_per_token"]
+
+
+# ---------------------------------------------------------------------------
+# S3 permute
+# ---------------------------------------------------------------------------
+
+def test_permute_roundtrip_bytes_and_metadata():
+    T, H, E, K, P = 29, 24, 8, 3, 4
+    x = inputs.to_bits(inputs.random_bf16((T, H), seed=1))
+    ids = inputs.random_topk_ids(T, E, K, seed=2).numpy()
+    w = inputs.random_weights(T, K, seed=3).numpy()
+    cs = oracle.count_scan(ids, E, P)
+    xp, meta = oracle.permute(x, cs["row_of_assign"], ids, w, E, P)
+    # dispatch bytes = T x K x H x b, no padding
+    assert xp.nbytes == oracle.dispatch_bytes(T, K, H, 2) == T * K * H * 2
+    # unpermute(permute(x)) = x for every slot
+    roa = cs["row_of_assign"].reshape(T, K)
+    for k in range(K):
+        assert np.array_equal(xp[roa[:, k]], x)
+    # metadata reproduces the route
+    assert np.array_equal(xp, x[meta["token"]])
+    assert np.array_equal(ids[meta["token"], meta["slot"]] % (E // P), meta["local_expert"])
+    assert np.array_equal(w[meta["token"], meta["slot"]], meta["w"])
+    # rows are expert-contiguous: expert of row r is non-decreasing
+    e_of_row = ids[meta["token"], meta["slot"]]
+    assert np.all(np.diff(e_of_row) >= 0)
+
+
+# ---------------------------------------------------------------------------
+# S4/S5 SwiGLU expert FFN (closed forms on structured weights)
+# ---------------------------------------------------------------------------
+
+def _sel(rows, cols, pairs, scale=1.0):
+    w = np.zeros((rows, cols))
+    for r, c in pairs:
+        w[r, c] = scale
+    return bf(w)
+
+
+def test_ffn_silu_known_value_and_rounding_points():
+    # x = [1, 1]; gate selects x0, up selects x1 -> a = silu(1) * 1 = sigma(1).
+    # sigma(1) = 0.7310585786300049 (logistic at 1); bf16 -> 0.73046875.
+    x = bf([[1.0, 1.0]])
+    wg = _sel(1, 2, [(0, 0)])
+    wu = _sel(1, 2, [(0, 1)])
+    wd = bf([[1.0078125], [1.0]])                    # W_down [H=2][F=1]
+    h, y = oracle.ffn_rows(x, wg, wu, wd)
+    assert val(h)[0, 0] == 0.73046875
+    # y rounds h to bf16 first: 0.73046875 * 1.0078125 = 0.7361755... -> 0.734375.
+    # (Rounding only once, sigma(1) * 1.0078125 = 0.73677... would give 0.73828125.)
+    assert val(y)[0, 0] == 0.734375 and val(y)[0, 1] == 0.73046875
+
+
+def test_ffn_silu_odd_part_identity_and_gate_up_order():
+    # silu(v) - silu(-v) = v exactly in real arithmetic; with u = 1 the rows for x and -x
+    # give h(v) - h(-v) = v up to two bf16 roundings.  With gate <-> up swapped the
+    # second row below would be silu(1)*4 instead of silu(4)*1.
+    v = np.array([0.5, 1.5, 3.0, 6.0, 0.0])
+    x = bf(np.stack([np.concatenate([v, [1.0]]), np.concatenate([-v, [1.0]])]))
+    H = 6
+    wg = _sel(5, H, [(i, i) for i in range(5)])
+    wu = _sel(5, H, [(i, 5) for i in range(5)])
+    wd = _sel(H, 5, [(i, i) for i in range(5)])
+    h, _ = oracle.ffn_rows(x, wg, wu, wd)
+    hv = val(h)
+    assert np.all(np.abs((hv[0] - hv[1]) - v) <= 2 ** -7 * np.maximum(np.abs(v), 1))
+    assert hv[0, 4] == 0.0
+    # order check: gate = 4, up = 1 vs gate = 1, up = 4
+    x2 = bf([[4.0, 1.0]])
+    h2, _ = oracle.ffn_rows(x2, _sel(1, 2, [(0, 0)]), _sel(1, 2, [(0, 1)]), _sel(2, 1, [(0, 0)]))
+    # silu(4) = 4 * sigma(4) with sigma(4) in (0.98, 0.99); silu(1)*4 would be ~2.92
+    assert 3.9 < val(h2)[0, 0] < 3.96
+
+
+def test_ffn_transposition_non_square():
+    # H = 3, F = 2: gate row f reads x[(f+1) % 3], up row f reads x[f]; down maps h_f -> y_{2-f}.
+    x = bf([[2.0, -1.0, 0.5]])
+    wg = _sel(2, 3, [(0, 1), (1, 2)], scale=0.0)        # gate = 0 -> silu(0) = 0 everywhere
+    wu = _sel(2, 3, [(0, 0), (1, 1)])
+    wd = _sel(3, 2, [(2, 0), (1, 1)])
+    h, y = oracle.ffn_rows(x, wg, wu, wd)
+    assert np.all(val(h) == 0.0) and np.all(val(y) == 0.0)
+    big = 16.0                                          # silu(16) = 16 * (1 - 1.1e-7) -> bf16 16
+    x = bf([[big, big, big]])
+    wu = _sel(2, 3, [(0, 0), (1, 1)], scale=0.5)        # u = 8 for both features
+    wg = _sel(2, 3, [(0, 1), (1, 2)])                  # g = 16
+    wd = _sel(3, 2, [(2, 0), (1, 1)], scale=0.25)
+    h, y = oracle.ffn_rows(x, wg, wu, wd)
+    assert np.array_equal(val(h), [[128.0, 128.0]])
+    assert np.array_equal(val(y), [[0.0, 32.0, 32.0]])  # output 0 gets nothing: Wd[0,:] = 0
+
+
+def test_grouped_ffn_uses_each_experts_weights_on_its_rows():
+    E, H, F = 4, 2, 1
+    counts = [3, 0, 2, 1]
+    off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    xp = bf(np.full((6, H), 16.0))
+    wg = np.stack([_sel(F, H, [(0, 0)]) for _ in range(E)])
+    wu = np.stack([_sel(F, H, [(0, 1)], scale=e + 1.0) for e in range(E)])
+    wd = np.stack([_sel(H, F, [(0, 0)]) for _ in range(E)])
+    h, y = oracle.grouped_ffn(xp, off, wg, wu, wd)
+    expect = [16.0 * 16 * 1] * 3 + [16.0 * 16 * 3] * 2 + [16.0 * 16 * 4]
+    assert np.array_equal(val(h)[:, 0], expect)
+    assert np.array_equal(val(y)[:, 0], expect) and np.all(val(y)[:, 1] == 0)
+
+
+# ---------------------------------------------------------------------------
+# S6 combine
+# ---------------------------------------------------------------------------
+
+def test_combine_identity_experts_returns_x():
+    # Identity experts (y = xp): combine gives (sum_k w) * x = x when renormalised.
+    T, H, E, K = 33, 40, 8, 4
+    x = inputs.to_bits(inputs.random_bf16((T, H), seed=11))
+    l = inputs.random_logits(T, E, seed=12).numpy()
+    ids, w = oracle.route(l, K, renormalize=True)
+    cs = oracle.count_scan(ids, E)
+    xp, _ = oracle.permute(x, cs["row_of_assign"], ids, w, E)
+    out = oracle.combine(xp, cs["row_of_assign"], w)
+    assert np.array_equal(out, x)
+    # without renormalisation: out = bf16(sum_k w * x)
+    ids2, w2 = oracle.route(l, K, renormalize=False)
+    cs2 = oracle.count_scan(ids2, E)
+    xp2, _ = oracle.permute(x, cs2["row_of_assign"], ids2, w2, E)
+    out2 = val(oracle.combine(xp2, cs2["row_of_assign"], w2))
+    s = w2.astype(np.float64).sum(axis=1, keepdims=True)
+    assert np.allclose(out2, val(x) * s, rtol=2 ** -8, atol=0)
+
+
+def test_combine_weighted_slots_closed_form():
+    y = bf([[1.0, 2.0], [4.0, 8.0], [16.0, 32.0]])
+    roa = np.array([2, 0, 1, 2], np.int32)           # token 0 -> rows 2,0; token 1 -> rows 1,2
+    w = np.array([[0.25, 0.75], [0.5, 0.125]], np.float32)
+    out = val(oracle.combine(y, roa, w))
+    assert np.array_equal(out, [[0.25 * 16 + 0.75 * 1, 0.25 * 32 + 0.75 * 2],
+                                [0.5 * 4 + 0.125 * 16, 0.5 * 8 + 0.125 * 32]])
+
+
+# ---------------------------------------------------------------------------
+# S7 skew statistics
+# ---------------------------------------------------------------------------
+
+def test_skew_ratio_and_p95():
+    assert oracle.skew_ratio([4, 4, 4, 4]) == 1.0
+    assert oracle.skew_ratio([16, 0, 0, 0]) == 4.0
+    assert oracle.skew_ratio([3, 1, 0, 0]) == 3.0
+    assert oracle.skew_ratio([0, 0]) == 0.0
+    assert oracle.p95_nearest_rank(np.arange(1, 101)) == 95.0
+    assert oracle.p95_nearest_rank(np.arange(20, 0, -1)) == 19.0
+    assert oracle.p95_nearest_rank([7.0]) == 7.0
+
+
+def test_zipf_decode_workload_reaches_p95_skew_4():
+    # The skewed decode router is calibrated to a p95 max/mean load near 4.
+    cfg = DEEPSEEK_R1_DECODE
+    w_g, bias = inputs.make_router(cfg)
+    ratios = []
+    for s in range(64):
+        l = oracle.gating_logits(inputs.to_bits(inputs.make_tokens(cfg, "cpu", s)), w_g.numpy(), bias.numpy())
+        ids, _ = oracle.route(l, cfg.K)
+        ratios.append(oracle.skew_ratio(oracle.count_scan(ids, cfg.E)["counts"]))
+    assert 3.75 <= oracle.p95_nearest_rank(ratios) <= 4.25
+
+
+# ---------------------------------------------------------------------------
+# S8 latent projections
+# ---------------------------------------------------------------------------
+
+def test_dense_projection_layout():
+    x = bf([[1.0, 2.0, 3.0, 4.0]])
+    w = _sel(2, 4, [(0, 3), (1, 0)], scale=0.5)       # [D_out=2][D_in=4]
+    assert np.array_equal(val(oracle.dense_bf16(x, w)), [[2.0, 0.5]])
+
+
+def test_layer_forward_tiny_is_consistent():
+    cfg = TINY
+    d = inputs.make_layer(cfg)
+    r = oracle.layer_forward(inputs.to_bits(d["x"]), d["w_g"].numpy(), inputs.to_bits(d["w_gate"]),
+                             inputs.to_bits(d["w_up"]), inputs.to_bits(d["w_down"]), cfg.K, cfg.P)
+    assert r["counts"].sum() == cfg.TK
+    assert r["xp"].shape == (cfg.TK, cfg.H) and r["out"].shape == (cfg.T, cfg.H)
+    # row-by-row evaluation of one token equals the grouped evaluation
+    t = 5
+    acc = np.zeros(cfg.H)
+    for k in range(cfg.K):
+        e = r["topk_ids"][t, k]
+        _, yk = oracle.ffn_rows(inputs.to_bits(d["x"])[t:t + 1], inputs.to_bits(d["w_gate"][e]),
+                                inputs.to_bits(d["w_up"][e]), inputs.to_bits(d["w_down"][e]))
+        acc += float(r["topk_w"][t, k]) * val(yk)[0]
+    assert np.array_equal(oracle.f64_to_bf16_bits(acc), r["out"][t])
+
+
+# ---------------------------------------------------------------------------
+# Figures the pages print
+# ---------------------------------------------------------------------------
+
+def test_sizing_figures_from_pages():
+    g = json.load(open(os.path.join(GOLDEN, "sizing_figures.json")))
+    c = g["checkpoint"]
+    nbytes = oracle.checkpoint_bytes(c["params"], c["bytes_per_param"])
+    assert nbytes / 1e9 == pytest.approx(c["bytes_decimal_GB"])
+    assert round(nbytes / 2 ** 30, 1) == c["GiB"]
+    for row in g["experts_per_partition"]:
+        assert oracle.experts_per_partition(row["E"], row["P"]) == row["per_partition"]
+    a = g["activated_share"]
+    assert round(100.0 * a["K"] / a["E"], 1) == a["percent"]
+    u = g["unselected_experts"]
+    assert u["E"] - u["K"] == u["unselected"]
+    cs = g["cold_share_ep8"]
+    assert 100.0 * (cs["local_experts"] - cs["K"]) / cs["local_experts"] == cs["cold_percent"]
+    th = g["topk_halving"]
+    assert oracle.dispatch_bytes(4096, th["K_to"], 2048, 2) / oracle.dispatch_bytes(4096, th["K_from"], 2048, 2) == th["ratio"]
