@@ -1,0 +1,305 @@
+/*
+ * moe.h - C ABI of the B200 (sm_100a) routed Mixture-of-Experts layer.
+ *
+ * One routed MoE layer on one GPU, in the order the "WideEP: Wide Expert
+ * Parallelism and Kimi K3" essay gives in its section "The router writes a
+ * network schedule": gating scores and top-k expert ids; count destinations
+ * and allocate slots; permute token activations into destination-contiguous
+ * buffers and attach routing metadata; run the experts' matrix multiplies per
+ * local expert; combine reverses the route, unpermutes and applies the routing
+ * weights.  The same essay's table of communication regimes (row "Same GPU":
+ * no fabric hop, still a permute and HBM traffic; fused layouts, grouped GEMM)
+ * is the regime of this library: logical expert-parallel partitions are only a
+ * buffer layout, nothing is transferred between GPUs.
+ *
+ * Notation (the pages' statement of the problem): T tokens, E experts, top-K,
+ * H dispatch width, F expert FFN width, b = 2 bytes per bf16 activation,
+ * P logical partitions, TK = T*K assignments.  Assignment a = t*K + k is slot k
+ * of token t.
+ *
+ * Conventions for every call:
+ *  - Pointers are DEVICE pointers unless the name ends in _host.  bf16 data is
+ *    passed as raw IEEE bfloat16 (void*), row-major, densely packed.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
+ *    enqueues work and returns; none synchronizes with the host except
+ *    moe_read_device_status.
+ *  - The caller owns every buffer, including the workspace.  The library never
+ *    allocates device memory and keeps no per-call state; it caches only device
+ *    properties and the driver's tensor-map encoder.
+ *  - Output shapes are static (TK rows, no capacity factor, no dropped tokens).
+ *  - Argument and shape errors are returned synchronously and enqueue nothing.
+ *    Launch failures return MOE_ERR_CUDA.  Conditions detected on the device
+ *    (an expert id outside [0, E), a wait that exceeded its time limit) are
+ *    OR-ed into the status word inside the workspace and read back with
+ *    moe_read_device_status; no kernel traps or asserts.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Layer shape.  d_model = 0 except for the latent layer, whose tokens arrive at
+ * width d_model and are projected down to H before routing ("Latent MoE" page,
+ * sections "Definition" and "Current Synthesis"). */
+typedef struct moe_dims {
+  int64_t T;
+  int32_t H;
+  int32_t E;
+  int32_t K;
+  int32_t F;
+  int32_t P;            /* logical partitions, E % P == 0 (1 = no partitioning) */
+  int32_t renormalize;  /* 1: weights = softmax over the K selected logits;
+                           0: weights = softmax over all E at the selected ids */
+  int32_t d_model;      /* 0, or the model width of a latent layer */
+} moe_dims;
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,        /* null pointer, T < 0, K > E, E % P != 0, ... */
+  MOE_ERR_UNSUPPORTED_SHAPE = 2,  /* valid but outside this build's limits    */
+  MOE_ERR_WORKSPACE = 3,          /* workspace missing or too small           */
+  MOE_ERR_CUDA = 4,               /* a CUDA runtime / driver call failed      */
+  MOE_ERR_DEVICE_TIMEOUT = 5,     /* a device-side wait ran out of time       */
+  MOE_ERR_DEVICE_BAD_INDEX = 6,   /* an expert id or row index out of range   */
+  MOE_ERR_NO_DEVICE = 7           /* no sm_100 device current                 */
+} moe_status;
+
+/* Device status bits OR-ed into the workspace status word. */
+#define MOE_DEV_BAD_INDEX 0x1
+#define MOE_DEV_TIMEOUT   0x2
+
+/* Limits of this build (checked; larger shapes return MOE_ERR_UNSUPPORTED_SHAPE). */
+#define MOE_MAX_E 1024
+#define MOE_MAX_K 32
+
+/* ------------------------------------------------------------------------- */
+/* Workspace                                                                 */
+/* ------------------------------------------------------------------------- */
+
+/* Bytes of workspace the calls that take `ws` need for `d` (a multiple of 256).
+ * One workspace may serve every call of one layer shape, on one stream at a
+ * time.  Returns 0 for an invalid shape. */
+size_t moe_workspace_bytes(const moe_dims* d);
+
+/* Clears the workspace's status word and the count/scan kernel's grid-barrier
+ * counters (an async memset on `stream`).  Call once after allocating the
+ * workspace, and again after a device-side error has been reported. */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronizes `stream`, then copies the workspace status word to *status
+ * (0 = no device-side error; otherwise MOE_DEV_* bits).  Off the hot path. */
+moe_status moe_read_device_status(const void* ws, int32_t* status, void* stream);
+
+const char* moe_status_str(moe_status s);
+
+/* ------------------------------------------------------------------------- */
+/* S0  Gating logits                                                         */
+/* "The source rank computes the gating scores" (WideEP essay, "The router   */
+/* writes a network schedule"); the gating network is replicated non-expert  */
+/* work (InferenceX v2 review claim IX2-0406).                               */
+/* ------------------------------------------------------------------------- */
+
+/* One-time weight preparation: splits the fp32 router W_g [H][E] into three
+ * bf16 planes hi, mid, lo with W_g = hi + mid + lo to float32 accuracy and
+ * stores them transposed as w_g_split [3][E][H] (bf16, 6*E*H bytes, caller
+ * allocated).  Not part of the per-token path. */
+moe_status moe_pack_router(const float* w_g, const moe_dims* d, void* w_g_split, void* stream);
+
+/* logits[t][e] = sum_h x[t][h] * W_g[h][e] (+ bias[e]), fp32 out [T][E].
+ * x: [T][H] bf16.  w_g_split: from moe_pack_router.  bias: [E] fp32 or NULL.
+ * Tensor-core products of the exact bf16 x with the three bf16 planes,
+ * accumulated in fp32. */
+moe_status moe_gating(const void* x, const void* w_g_split, const float* bias,
+                      const moe_dims* d, float* logits, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* S1  Router top-K + routing weights                                        */
+/* "computes the gating scores and top-k expert IDs" (WideEP essay, "The     */
+/* router writes a network schedule").                                       */
+/* ------------------------------------------------------------------------- */
+
+/* logits: [T][E] fp32.  Out: topk_ids [T][K] int32 and topk_w [T][K] fp32, slot
+ * 0 the best.  Order: larger logit first; equal logits (-0.0 == +0.0) go to the
+ * lower expert id; NaN ranks below every number.  Weights: exp(l_k - l_max)
+ * normalised over the K selected (renormalize = 1) or over all E. */
+moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids,
+                     float* topk_w, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* S2  Count destinations, allocate slots                                    */
+/* "A dispatcher counts destinations, allocates or selects communication     */
+/* slots" (WideEP essay); per-expert assignment counts, "assignments, not    */
+/* unique tokens" ("Three Parameter Counts...", "What the utilization        */
+/* dashboard smooths away").                                                 */
+/* ------------------------------------------------------------------------- */
+
+/* topk_ids: [T][K] int32.  Out (all int32):
+ *   counts[E], offsets[E+1] (exclusive scan, offsets[E] = TK),
+ *   part_counts[P], part_offsets[P+1] (partition p owns experts
+ *     [p*E/P, (p+1)*E/P); part_offsets[p] = offsets[p*E/P]),
+ *   row_of_assign[TK]: row of assignment a in the expert-major buffer, a stable
+ *     counting sort (rows of one expert keep increasing a),
+ *   assign_of_row[TK]: its inverse.
+ * An id outside [0, E) sets MOE_DEV_BAD_INDEX; such assignments are given no row
+ * and the outputs are then unspecified.  Uses the workspace (grid barrier and
+ * per-block histograms). */
+moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* counts,
+                          int32_t* offsets, int32_t* part_counts, int32_t* part_offsets,
+                          int32_t* row_of_assign, int32_t* assign_of_row,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* S3  Permute into destination-contiguous rows + routing metadata           */
+/* "permutes token activations into destination-contiguous buffers, attaches */
+/* routing metadata" (WideEP essay); payload T x K x H x b ("Top-k           */
+/* multiplies traffic"; "Three Parameter Counts...", "Halving top-k is a     */
+/* network change first").                                                  */
+/* ------------------------------------------------------------------------- */
+
+/* xp[row_of_assign[t*K+k]][:] = x[t][:] for every (t, k); x [T][H] bf16,
+ * xp [TK][H] bf16 (exactly T*K*H*2 bytes, no padding).  Metadata per row r
+ * (each pointer may be NULL to skip it): meta_token[r] = t, meta_slot[r] = k,
+ * meta_w[r] = topk_w[t][k], meta_local_expert[r] = e - p*E/P for the row's
+ * expert e in partition p.  topk_ids is read only for meta_local_expert,
+ * topk_w only for meta_w (either may be NULL when its output is NULL).
+ * H must be a multiple of 8 (16-byte rows). */
+moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_t* topk_ids,
+                       const float* topk_w, const moe_dims* d, void* xp,
+                       int32_t* meta_token, int32_t* meta_slot, float* meta_w,
+                       int32_t* meta_local_expert, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* S4 + S5  Expert SwiGLU FFN as grouped GEMMs over variable row counts      */
+/* "The receiver groups tokens by local expert and launches expert matrix    */
+/* multiplies" (WideEP essay); grouped GEMM runs several expert matrices in  */
+/* one launch despite differing row counts ("Three Parameter Counts...",     */
+/* "Which optimizations need a task-level gate").                            */
+/* ------------------------------------------------------------------------- */
+
+/* For every expert e and row r in [offsets[e], offsets[e+1]):
+ *   h[r][f] = bf16( silu(sum_k xp[r][k] w_gate[e][f][k]) * (sum_k xp[r][k] w_up[e][f][k]) )
+ *   y[r][j] = bf16( sum_f h[r][f] w_down[e][j][f] )
+ * xp [TK][H], w_gate/w_up [E][F][H], w_down [E][H][F] (nn.Linear layout),
+ * h [TK][F], y [TK][H]; all bf16.  offsets: device [E+1] from moe_count_scan;
+ * it is read on the device, so launch shapes never depend on the counts.
+ * Experts with no rows cost nothing.  H and F must be multiples of 8.  Offsets
+ * that decrease or leave [0, TK] set MOE_DEV_BAD_INDEX and the call computes
+ * nothing.  The GEMM calls use only the workspace's status word; any workspace
+ * of moe_workspace_bytes(d) bytes serves (moe_dense needs 256 bytes). */
+moe_status moe_grouped_ffn(const void* xp, const int32_t* offsets, const void* w_gate,
+                           const void* w_up, const void* w_down, const moe_dims* d,
+                           void* h, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* The two halves of moe_grouped_ffn as separate launches (S4 and S5). */
+moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const void* w_gate,
+                               const void* w_up, const moe_dims* d, void* h, void* ws,
+                               size_t ws_bytes, void* stream);
+moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w_down,
+                            const moe_dims* d, void* y, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* S6  Combine: unpermute + weighted sum                                     */
+/* "A combine phase reverses the route, after which the source rank          */
+/* unpermutes and applies routing weights" (WideEP essay).                   */
+/* ------------------------------------------------------------------------- */
+
+/* out[t][:] = bf16( sum_{k<K} topk_w[t][k] * y[row_of_assign[t*K+k]][:] ),
+ * accumulated in fp32 in slot order.  y [TK][H] bf16, out [T][H] bf16. */
+moe_status moe_combine(const void* y, const int32_t* row_of_assign, const float* topk_w,
+                       const moe_dims* d, void* out, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* S7  Skew statistics                                                       */
+/* "Skew ratio at p95: max expert load divided by mean expert load"          */
+/* ("Three Parameter Counts...", "What the utilization dashboard smooths     */
+/* away").                                                                   */
+/* ------------------------------------------------------------------------- */
+
+/* *d_ratio (device fp32) = max_e counts[e] / (sum_e counts[e] / E); 0 if no rows. */
+moe_status moe_skew_stats(const int32_t* counts, const moe_dims* d, float* d_ratio, void* stream);
+
+/* Host helper: 95th percentile of n per-step ratios by nearest rank (the
+ * ceil(0.95 n)-th smallest).  Returns NaN for n <= 0. */
+double moe_p95(const float* ratios, int n);
+
+/* ------------------------------------------------------------------------- */
+/* S8  Latent projections ("Latent MoE" page: dispatch on a reduced width)   */
+/* ------------------------------------------------------------------------- */
+
+/* out[m][n] = bf16( sum_k a[m][k] * w[n][k] ): a [M][Kd] bf16, w [N][Kd] bf16
+ * (nn.Linear layout), out [M][N] bf16.  Used for z = x W_dp^T (d_model -> H)
+ * before routing and final = out W_up^T (H -> d_model) after combine.
+ * Kd and N must be multiples of 8. */
+moe_status moe_dense(const void* a, const void* w, int64_t M, int32_t N, int32_t Kd,
+                     void* out, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Whole layer                                                               */
+/* ------------------------------------------------------------------------- */
+
+typedef struct moe_layer_weights {
+  const void*  w_g_split;   /* [3][E][H] bf16 from moe_pack_router          */
+  const float* bias;        /* [E] fp32 router bias, or NULL                 */
+  const void*  w_gate;      /* [E][F][H] bf16                                */
+  const void*  w_up;        /* [E][F][H] bf16                                */
+  const void*  w_down;      /* [E][H][F] bf16                                */
+  const void*  w_dp;        /* latent only: [H][d_model] bf16, else NULL     */
+  const void*  w_upp;       /* latent only: [d_model][H] bf16, else NULL     */
+} moe_layer_weights;
+
+typedef struct moe_layer_buffers {
+  void*    z;               /* latent only: [T][H] bf16 (routed activations) */
+  float*   logits;          /* [T][E] fp32                                   */
+  int32_t* topk_ids;        /* [T][K]                                        */
+  float*   topk_w;          /* [T][K]                                        */
+  int32_t* counts;          /* [E]                                           */
+  int32_t* offsets;         /* [E+1]                                         */
+  int32_t* part_counts;     /* [P]                                           */
+  int32_t* part_offsets;    /* [P+1]                                         */
+  int32_t* row_of_assign;   /* [TK]                                          */
+  int32_t* assign_of_row;   /* [TK]                                          */
+  void*    xp;              /* [TK][H] bf16                                  */
+  int32_t* meta_token;      /* [TK] or NULL                                  */
+  int32_t* meta_slot;       /* [TK] or NULL                                  */
+  float*   meta_w;          /* [TK] or NULL                                  */
+  int32_t* meta_local_expert; /* [TK] or NULL                                */
+  void*    h;               /* [TK][F] bf16                                  */
+  void*    y;               /* [TK][H] bf16                                  */
+  void*    out;             /* [T][H] bf16 (combine output)                  */
+  void*    final_out;       /* latent only: [T][d_model] bf16                */
+  float*   skew;            /* [1] fp32 max/mean expert load                 */
+} moe_layer_buffers;
+
+/* Number of stage boundaries recorded when stage events are given. */
+#define MOE_NUM_STAGE_EVENTS 10
+
+/* Runs every step on `stream` in pipeline order: [latent down-projection] ->
+ * gating -> route -> count/scan -> permute -> gate/up+SwiGLU -> down -> combine
+ * -> [latent up-projection] -> skew statistics.  x: [T][d_in] bf16 with
+ * d_in = d_model for a latent layer, else H.  stage_events: NULL, or an array of
+ * MOE_NUM_STAGE_EVENTS cudaEvent_t (created by the caller) recorded at: start,
+ * after latent-down, gating, route, count/scan, permute, gate/up, down,
+ * combine, latent-up/skew (end).  Events of absent stages are still recorded. */
+moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const moe_dims* d,
+                             const moe_layer_buffers* b, void* ws, size_t ws_bytes,
+                             void* const* stage_events, void* stream);
+
+/* The same layer with HOST activations: copies x_host (pinned, [T][d_in] bf16)
+ * into x_dev, runs moe_layer_forward, and copies the final output ([T][d_out]
+ * bf16, d_out = d_model for a latent layer, else H) back to out_host, all
+ * enqueued on `stream` (the host data must stay valid until the stream reaches
+ * the copies). */
+moe_status moe_layer_forward_host(const void* x_host, void* x_dev, const moe_layer_weights* w,
+                                  const moe_dims* d, const moe_layer_buffers* b, void* ws,
+                                  size_t ws_bytes, void* out_host, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

@@ -1,0 +1,317 @@
+// api.cu - the C ABI of libmoe_b200 (declared in include/moe.h): argument
+// checks, workspace layout and the order of the layer's launches.
+#include <algorithm>
+#include <cmath>
+#include <mutex>
+#include <vector>
+
+#include "device.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+// Workspace: [0] status word, [64] grid-barrier count, [128] grid-barrier
+// generation, [256 ...) per-block expert histograms of the count/scan kernel.
+constexpr size_t kWsHeader = 256;
+
+bool device_ok() {
+  static int cache[64] = {0};  // 0 unknown, 1 ok, -1 not sm_100
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (cache[dev] == 0) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cache[dev] = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return cache[dev] == 1;
+}
+
+moe_status check_dims(const moe_dims* d) {
+  if (!d) return MOE_ERR_INVALID_ARG;
+  if (d->T < 0 || d->E < 1 || d->K < 1 || d->K > d->E || d->P < 1 || d->E % d->P != 0 || d->H < 8 ||
+      d->F < 8 || d->d_model < 0)
+    return MOE_ERR_INVALID_ARG;
+  if (d->H % 8 != 0 || d->F % 8 != 0 || d->d_model % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (d->E > MOE_MAX_E || d->K > MOE_MAX_K) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (d->T * static_cast<long long>(d->K) > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED_SHAPE;
+  return MOE_OK;
+}
+
+size_t ws_bytes_for(const moe_dims* d) {
+  const long long TK = d->T * static_cast<long long>(d->K);
+  const size_t hist = static_cast<size_t>(scan_max_blocks(TK)) * d->E * sizeof(int);
+  return kWsHeader + (hist + 255) / 256 * 256;
+}
+
+int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
+
+ScanWorkspace scan_ws(void* ws, const moe_dims* d) {
+  uint8_t* p = reinterpret_cast<uint8_t*>(ws);
+  ScanWorkspace s;
+  s.status = reinterpret_cast<int*>(p);
+  s.bar_count = reinterpret_cast<unsigned int*>(p + 64);
+  s.bar_gen = reinterpret_cast<unsigned int*>(p + 128);
+  s.block_counts = reinterpret_cast<int*>(p + kWsHeader);
+  s.max_blocks = scan_max_blocks(d->T * static_cast<long long>(d->K));
+  return s;
+}
+
+moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
+
+#define MOE_TRY(expr)                      \
+  do {                                     \
+    const moe_status _s = (expr);          \
+    if (_s != MOE_OK) return _s;           \
+  } while (0)
+
+#define MOE_CUDA(expr)                                        \
+  do {                                                        \
+    if ((expr) != cudaSuccess) return MOE_ERR_CUDA;           \
+  } while (0)
+
+moe_status common_checks(const moe_dims* d) {
+  MOE_TRY(check_dims(d));
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  return MOE_OK;
+}
+
+moe_status check_ws(const void* ws, size_t ws_bytes, const moe_dims* d) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < ws_bytes_for(d)) return MOE_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+size_t moe_workspace_bytes(const moe_dims* d) {
+  if (check_dims(d) != MOE_OK) return 0;
+  return ws_bytes_for(d);
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < kWsHeader) return MOE_ERR_WORKSPACE;
+  MOE_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, as_stream(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_read_device_status(const void* ws, int32_t* status, void* stream) {
+  if (!ws || !status) return MOE_ERR_INVALID_ARG;
+  MOE_CUDA(cudaStreamSynchronize(as_stream(stream)));
+  MOE_CUDA(cudaMemcpy(status, ws, sizeof(int32_t), cudaMemcpyDeviceToHost));
+  return MOE_OK;
+}
+
+const char* moe_status_str(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case MOE_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case MOE_ERR_CUDA: return "CUDA call failed";
+    case MOE_ERR_DEVICE_TIMEOUT: return "device-side wait timed out";
+    case MOE_ERR_DEVICE_BAD_INDEX: return "device-side index out of range";
+    case MOE_ERR_NO_DEVICE: return "no sm_100 device is current";
+  }
+  return "unknown status";
+}
+
+moe_status moe_pack_router(const float* w_g, const moe_dims* d, void* w_g_split, void* stream) {
+  MOE_TRY(common_checks(d));
+  if (!w_g || !w_g_split) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_pack_router(w_g, d->H, d->E, w_g_split, as_stream(stream)));
+}
+
+moe_status moe_gating(const void* x, const void* w_g_split, const float* bias, const moe_dims* d, float* logits,
+                      void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(common_checks(d));
+  MOE_TRY(check_ws(ws, ws_bytes, d));
+  if (d->T == 0) return MOE_OK;
+  if (!x || !w_g_split || !logits) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_g_split)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(gemm_gating(x, w_g_split, bias, d->T, d->H, d->E, logits, ws_status(ws), as_stream(stream)));
+}
+
+moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids, float* topk_w, void* stream) {
+  MOE_TRY(common_checks(d));
+  if (d->T == 0) return MOE_OK;
+  if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_route(logits, d->T, d->E, d->K, d->renormalize, topk_ids, topk_w, as_stream(stream)));
+}
+
+moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* counts, int32_t* offsets,
+                          int32_t* part_counts, int32_t* part_offsets, int32_t* row_of_assign,
+                          int32_t* assign_of_row, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(common_checks(d));
+  MOE_TRY(check_ws(ws, ws_bytes, d));
+  if (!counts || !offsets || !part_counts || !part_offsets || (d->T > 0 && (!topk_ids || !row_of_assign ||
+                                                                           !assign_of_row)))
+    return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_count_scan(topk_ids, d->T * static_cast<long long>(d->K), d->E, d->P, counts, offsets,
+                                       part_counts, part_offsets, row_of_assign, assign_of_row, nullptr,
+                                       scan_ws(ws, d), as_stream(stream)));
+}
+
+moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_t* topk_ids, const float* topk_w,
+                       const moe_dims* d, void* xp, int32_t* meta_token, int32_t* meta_slot, float* meta_w,
+                       int32_t* meta_local_expert, void* stream) {
+  MOE_TRY(common_checks(d));
+  if (d->T == 0) return MOE_OK;
+  if (!x || !row_of_assign || !xp || (meta_w && !topk_w) || (meta_local_expert && !topk_ids))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_permute(x, row_of_assign, topk_ids, topk_w, d->T, d->H, d->E, d->K, d->P, xp,
+                                    meta_token, meta_slot, meta_w, meta_local_expert, as_stream(stream)));
+}
+
+moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up,
+                               const moe_dims* d, void* h, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(common_checks(d));
+  MOE_TRY(check_ws(ws, ws_bytes, d));
+  if (d->T == 0) return MOE_OK;
+  if (!xp || !offsets || !w_gate || !w_up || !h) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xp) || !aligned16(w_gate) || !aligned16(w_up)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(gemm_gate_up(xp, offsets, w_gate, w_up, d->E, d->T * static_cast<long long>(d->K), d->H,
+                                  d->F, h, ws_status(ws), as_stream(stream)));
+}
+
+moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w_down, const moe_dims* d, void* y,
+                            void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(common_checks(d));
+  MOE_TRY(check_ws(ws, ws_bytes, d));
+  if (d->T == 0) return MOE_OK;
+  if (!h || !offsets || !w_down || !y) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_down)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(gemm_down(h, offsets, w_down, d->E, d->T * static_cast<long long>(d->K), d->H, d->F, y,
+                               ws_status(ws), as_stream(stream)));
+}
+
+moe_status moe_grouped_ffn(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up,
+                           const void* w_down, const moe_dims* d, void* h, void* y, void* ws, size_t ws_bytes,
+                           void* stream) {
+  MOE_TRY(moe_grouped_gate_up(xp, offsets, w_gate, w_up, d, h, ws, ws_bytes, stream));
+  return moe_grouped_down(h, offsets, w_down, d, y, ws, ws_bytes, stream);
+}
+
+moe_status moe_combine(const void* y, const int32_t* row_of_assign, const float* topk_w, const moe_dims* d,
+                       void* out, void* stream) {
+  MOE_TRY(common_checks(d));
+  if (d->T == 0) return MOE_OK;
+  if (!y || !row_of_assign || !topk_w || !out) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_combine(y, row_of_assign, topk_w, d->T, d->H, d->K, out, as_stream(stream)));
+}
+
+moe_status moe_skew_stats(const int32_t* counts, const moe_dims* d, float* d_ratio, void* stream) {
+  MOE_TRY(common_checks(d));
+  if (!counts || !d_ratio) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_skew(counts, d->E, d_ratio, as_stream(stream)));
+}
+
+double moe_p95(const float* ratios, int n) {
+  if (!ratios || n <= 0) return NAN;
+  std::vector<float> v(ratios, ratios + n);
+  std::sort(v.begin(), v.end());
+  const int r = std::max(1, static_cast<int>(std::ceil(0.95 * n - 1e-9)));
+  return static_cast<double>(v[r - 1]);
+}
+
+moe_status moe_dense(const void* a, const void* w, int64_t M, int32_t N, int32_t Kd, void* out, void* ws,
+                     size_t ws_bytes, void* stream) {
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  if (!a || !w || !out || !ws || M < 0 || N < 8 || Kd < 8) return MOE_ERR_INVALID_ARG;
+  if (N % 8 != 0 || Kd % 8 != 0 || M > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (ws_bytes < kWsHeader || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_WORKSPACE;
+  if (!aligned16(a) || !aligned16(w)) return MOE_ERR_INVALID_ARG;
+  if (M == 0) return MOE_OK;
+  return cuda_status(gemm_dense(a, w, M, N, Kd, out, ws_status(ws), as_stream(stream)));
+}
+
+moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const moe_dims* d,
+                             const moe_layer_buffers* b, void* ws, size_t ws_bytes, void* const* stage_events,
+                             void* stream) {
+  MOE_TRY(common_checks(d));
+  MOE_TRY(check_ws(ws, ws_bytes, d));
+  if (!x || !w || !b) return MOE_ERR_INVALID_ARG;
+  const bool latent = d->d_model > 0;
+  if (!w->w_g_split || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if (latent && (!w->w_dp || !w->w_upp || !b->z || !b->final_out)) return MOE_ERR_INVALID_ARG;
+  if (!b->logits || !b->topk_ids || !b->topk_w || !b->counts || !b->offsets || !b->part_counts ||
+      !b->part_offsets || !b->row_of_assign || !b->assign_of_row || !b->xp || !b->h || !b->y || !b->out)
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  auto mark = [&](int i) -> moe_status {
+    if (stage_events && stage_events[i])
+      return cuda_status(cudaEventRecord(reinterpret_cast<cudaEvent_t>(stage_events[i]), s));
+    return MOE_OK;
+  };
+  int* status = ws_status(ws);
+  const long long T = d->T, TK = d->T * static_cast<long long>(d->K);
+  MOE_TRY(mark(0));
+  const void* routed = x;
+  if (latent) {
+    if (T > 0) MOE_CUDA(gemm_dense(x, w->w_dp, T, d->H, d->d_model, b->z, status, s));
+    routed = b->z;
+  }
+  MOE_TRY(mark(1));
+  if (T > 0) MOE_CUDA(gemm_gating(routed, w->w_g_split, w->bias, T, d->H, d->E, b->logits, status, s));
+  MOE_TRY(mark(2));
+  MOE_CUDA(launch_route(b->logits, T, d->E, d->K, d->renormalize, b->topk_ids, b->topk_w, s));
+  MOE_TRY(mark(3));
+  MOE_CUDA(launch_count_scan(b->topk_ids, TK, d->E, d->P, b->counts, b->offsets, b->part_counts, b->part_offsets,
+                             b->row_of_assign, b->assign_of_row, b->skew, scan_ws(ws, d), s));
+  MOE_TRY(mark(4));
+  MOE_CUDA(launch_permute(routed, b->row_of_assign, b->topk_ids, b->topk_w, T, d->H, d->E, d->K, d->P, b->xp,
+                          b->meta_token, b->meta_slot, b->meta_w, b->meta_local_expert, s));
+  MOE_TRY(mark(5));
+  if (T > 0) MOE_CUDA(gemm_gate_up(b->xp, b->offsets, w->w_gate, w->w_up, d->E, TK, d->H, d->F, b->h, status, s));
+  MOE_TRY(mark(6));
+  if (T > 0) MOE_CUDA(gemm_down(b->h, b->offsets, w->w_down, d->E, TK, d->H, d->F, b->y, status, s));
+  MOE_TRY(mark(7));
+  MOE_CUDA(launch_combine(b->y, b->row_of_assign, b->topk_w, T, d->H, d->K, b->out, s));
+  MOE_TRY(mark(8));
+  if (latent && T > 0) MOE_CUDA(gemm_dense(b->out, w->w_upp, T, d->d_model, d->H, b->final_out, status, s));
+  MOE_TRY(mark(9));
+  return MOE_OK;
+}
+
+moe_status moe_layer_forward_host(const void* x_host, void* x_dev, const moe_layer_weights* w, const moe_dims* d,
+                                  const moe_layer_buffers* b, void* ws, size_t ws_bytes, void* out_host,
+                                  void* stream) {
+  MOE_TRY(common_checks(d));
+  if (!x_host || !x_dev || !out_host || !b) return MOE_ERR_INVALID_ARG;
+  const bool latent = d->d_model > 0;
+  const size_t d_in = latent ? d->d_model : d->H;
+  cudaStream_t s = as_stream(stream);
+  MOE_CUDA(cudaMemcpyAsync(x_dev, x_host, static_cast<size_t>(d->T) * d_in * 2, cudaMemcpyHostToDevice, s));
+  MOE_TRY(moe_layer_forward(x_dev, w, d, b, ws, ws_bytes, nullptr, stream));
+  const void* res = latent ? b->final_out : b->out;
+  MOE_CUDA(cudaMemcpyAsync(out_host, res, static_cast<size_t>(d->T) * d_in * 2, cudaMemcpyDeviceToHost, s));
+  return MOE_OK;
+}
+
+}  // extern "C"

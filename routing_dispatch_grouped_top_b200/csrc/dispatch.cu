@@ -1,0 +1,199 @@
+// dispatch.cu - permute (dispatch into expert-contiguous rows + routing
+// metadata), combine (unpermute + weighted sum) and the one-time router split.
+//
+// "permutes token activations into destination-contiguous buffers, attaches
+// routing metadata ... A combine phase reverses the route, after which the
+// source rank unpermutes and applies routing weights" (WideEP essay, "The
+// router writes a network schedule").  On one GPU this is the "Same GPU" row of
+// the essay's regime table: no fabric hop, but a permute and its HBM traffic,
+// T x K x H x b bytes out and a similar volume back ("Top-k multiplies
+// traffic").
+//
+// Both copy kernels are HBM-bound.  They work on 16-byte vectors (8 bf16): the
+// item space is (token, vector) flattened, so consecutive threads touch
+// consecutive 16-byte pieces of one row (coalesced on both sides), and each
+// thread keeps several independent items in flight.
+#include <algorithm>
+
+#include "device.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kCopyThreads = 256;
+constexpr int kUnroll = 4;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__global__ void __launch_bounds__(kCopyThreads) permute_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ roa, const int32_t* __restrict__ ids,
+    const float* __restrict__ w, long long T, int vpr, int E, int K, int P, uint4* __restrict__ xp,
+    int32_t* __restrict__ meta_token, int32_t* __restrict__ meta_slot, float* __restrict__ meta_w,
+    int32_t* __restrict__ meta_local) {
+  const long long n_items = T * vpr;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (long long base = tid; base < n_items; base += stride * kUnroll) {
+    uint4 v[kUnroll];
+    long long tok[kUnroll];
+    int vec[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long it = base + u * stride;
+      tok[u] = it / vpr;
+      vec[u] = static_cast<int>(it - tok[u] * vpr);
+      if (it < n_items) v[u] = ld_stream(x + it);
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const long long it = base + u * stride;
+      if (it < n_items) {
+        const int32_t* r = roa + tok[u] * K;
+        for (int k = 0; k < K; ++k) {
+          const int row = __ldg(r + k);
+          if (static_cast<unsigned long long>(row) < static_cast<unsigned long long>(T * K))
+            xp[static_cast<long long>(row) * vpr + vec[u]] = v[u];
+        }
+      }
+    }
+  }
+  // routing metadata of every row
+  const long long TK = T * K;
+  const int epp = E / P;
+  for (long long a = tid; a < TK; a += stride) {
+    const int r = __ldg(roa + a);
+    if (static_cast<unsigned long long>(r) >= static_cast<unsigned long long>(TK)) continue;
+    const int t = static_cast<int>(a / K);
+    if (meta_token) meta_token[r] = t;
+    if (meta_slot) meta_slot[r] = static_cast<int>(a - static_cast<long long>(t) * K);
+    if (meta_w) meta_w[r] = __ldg(w + a);
+    if (meta_local) meta_local[r] = __ldg(ids + a) % epp;
+  }
+}
+
+template <int KC>
+__global__ void __launch_bounds__(kCopyThreads) combine_kernel(const uint4* __restrict__ y,
+                                                               const int32_t* __restrict__ roa,
+                                                               const float* __restrict__ w, long long T, int vpr,
+                                                               int K, uint4* __restrict__ out) {
+  const long long n_items = T * vpr;
+  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
+  for (long long it = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; it < n_items; it += stride) {
+    const long long t = it / vpr;
+    const int vec = static_cast<int>(it - t * vpr);
+    const int32_t* r = roa + t * K;
+    const float* wt = w + t * K;
+    float acc[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+    // slots in order; KC rows fetched before they are summed
+    for (int k0 = 0; k0 < K; k0 += KC) {
+      uint4 yv[KC];
+      float wk[KC];
+#pragma unroll
+      for (int u = 0; u < KC; ++u) {
+        yv[u] = make_uint4(0u, 0u, 0u, 0u);
+        wk[u] = 0.0f;
+        if (k0 + u < K) {
+          const int row = __ldg(r + k0 + u);
+          if (static_cast<unsigned long long>(row) < static_cast<unsigned long long>(T * K)) {
+            yv[u] = ld_stream(y + static_cast<long long>(row) * vpr + vec);
+            wk[u] = __ldg(wt + k0 + u);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < KC; ++u) {
+        if (k0 + u < K) {
+          const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&yv[u]);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float2 f = __bfloat1622float2(p[j]);
+            acc[2 * j] = fmaf(wk[u], f.x, acc[2 * j]);
+            acc[2 * j + 1] = fmaf(wk[u], f.y, acc[2 * j + 1]);
+          }
+        }
+      }
+    }
+    uint4 o;
+    __nv_bfloat162* po = reinterpret_cast<__nv_bfloat162*>(&o);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) po[j] = __floats2bfloat162_rn(acc[2 * j], acc[2 * j + 1]);
+    out[it] = o;
+  }
+}
+
+// W_g [H][E] fp32 -> [3][E][H] bf16 planes hi, mid, lo (hi = rn(w), mid = rn(w - hi),
+// lo = rn(w - hi - mid); both differences are exact in fp32).
+__global__ void pack_router_kernel(const float* __restrict__ w_g, int H, int E, __nv_bfloat16* __restrict__ out) {
+  __shared__ float tile[32][33];
+  const int h0 = blockIdx.y * 32, e0 = blockIdx.x * 32;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int h = h0 + i, e = e0 + threadIdx.x;
+    tile[i][threadIdx.x] = (h < H && e < E) ? w_g[static_cast<long long>(h) * E + e] : 0.0f;
+  }
+  __syncthreads();
+  const long long plane = static_cast<long long>(E) * H;
+  for (int i = threadIdx.y; i < 32; i += blockDim.y) {
+    const int e = e0 + i, h = h0 + threadIdx.x;
+    if (e < E && h < H) {
+      const float v = tile[threadIdx.x][i];
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      const float r1 = v - __bfloat162float(hi);
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const float r2 = r1 - __bfloat162float(mid);
+      const long long o = static_cast<long long>(e) * H + h;
+      out[o] = hi;
+      out[plane + o] = mid;
+      out[2 * plane + o] = __float2bfloat16_rn(r2);
+    }
+  }
+}
+
+int copy_blocks(long long items) {
+  const long long want = (items + kCopyThreads - 1) / kCopyThreads;
+  return static_cast<int>(std::max<long long>(1, std::min<long long>(want, 8LL * num_sms())));
+}
+
+}  // namespace
+
+cudaError_t launch_permute(const void* x, const int32_t* roa, const int32_t* ids, const float* w, long long T,
+                           int H, int E, int K, int P, void* xp, int32_t* meta_token, int32_t* meta_slot,
+                           float* meta_w, int32_t* meta_local, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int vpr = H / 8;
+  permute_kernel<<<copy_blocks(T * vpr / 2), kCopyThreads, 0, s>>>(
+      reinterpret_cast<const uint4*>(x), roa, ids, w, T, vpr, E, K, P, reinterpret_cast<uint4*>(xp), meta_token,
+      meta_slot, meta_w, meta_local);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const void* y, const int32_t* roa, const float* w, long long T, int H, int K, void* out,
+                           cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int vpr = H / 8;
+  const int blocks = copy_blocks(T * vpr);
+  if (K <= 2)
+    combine_kernel<2><<<blocks, kCopyThreads, 0, s>>>(reinterpret_cast<const uint4*>(y), roa, w, T, vpr, K,
+                                                     reinterpret_cast<uint4*>(out));
+  else
+    combine_kernel<4><<<blocks, kCopyThreads, 0, s>>>(reinterpret_cast<const uint4*>(y), roa, w, T, vpr, K,
+                                                     reinterpret_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack_router(const float* w_g, int H, int E, void* w_split, cudaStream_t s) {
+  dim3 grid((E + 31) / 32, (H + 31) / 32), block(32, 8);
+  pack_router_kernel<<<grid, block, 0, s>>>(w_g, H, E, reinterpret_cast<__nv_bfloat16*>(w_split));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,59 @@
+// kernels.h - launchers of libmoe_b200's kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace moe {
+
+enum Epi : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2 };
+
+struct GemmArgs {
+  const int32_t* offsets;  // [G + 1] device row offsets of the groups, or nullptr: one group of M rows
+  int G;
+  int M;
+  int N;                   // output features
+  int Kd;                  // reduction length
+  void* out;
+  long long ldo;           // output row stride in elements
+  const float* bias;       // kEpiF32 only: [N] or nullptr
+  int* status;             // device status word (MOE_DEV_* bits)
+};
+
+int num_sms();             // SM count of the current device (cached per device)
+int gemm_smem_bytes(int epi);
+
+cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
+                         long long rows, int H, int F, void* h, int* status, cudaStream_t stream);
+cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down, int E, long long rows, int H,
+                      int F, void* y, int* status, cudaStream_t stream);
+cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd, void* out, int* status,
+                       cudaStream_t stream);
+cudaError_t gemm_gating(const void* x, const void* w_split, const float* bias, long long T, int H, int E,
+                        float* logits, int* status, cudaStream_t stream);
+
+cudaError_t launch_route(const float* logits, long long T, int E, int K, int renormalize, int32_t* ids, float* w,
+                         cudaStream_t stream);
+
+// Count/scan workspace: status word, grid-barrier words, per-block histograms.
+struct ScanWorkspace {
+  int* status;
+  unsigned int* bar_count;
+  unsigned int* bar_gen;
+  int* block_counts;   // [max_blocks][E]
+  int max_blocks;
+};
+int scan_max_blocks(long long TK);
+cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, int32_t* counts, int32_t* offsets,
+                              int32_t* part_counts, int32_t* part_offsets, int32_t* row_of_assign,
+                              int32_t* assign_of_row, float* skew, const ScanWorkspace& ws, cudaStream_t stream);
+cudaError_t launch_skew(const int32_t* counts, int E, float* ratio, cudaStream_t stream);
+
+cudaError_t launch_permute(const void* x, const int32_t* row_of_assign, const int32_t* ids, const float* w,
+                           long long T, int H, int E, int K, int P, void* xp, int32_t* meta_token,
+                           int32_t* meta_slot, float* meta_w, int32_t* meta_local, cudaStream_t stream);
+cudaError_t launch_combine(const void* y, const int32_t* row_of_assign, const float* w, long long T, int H, int K,
+                           void* out, cudaStream_t stream);
+cudaError_t launch_pack_router(const float* w_g, int H, int E, void* w_split, cudaStream_t stream);
+
+}  // namespace moe

@@ -1,0 +1,356 @@
+// routing.cu - router top-K, per-expert count + stable scan, skew statistics.
+//
+// "The source rank computes the gating scores and top-k expert IDs.  A
+// dispatcher counts destinations, allocates or selects communication slots"
+// (WideEP essay, "The router writes a network schedule").  Counts are of
+// assignments, not unique tokens, and the skew ratio is max expert load over
+// mean expert load ("Three Parameter Counts...", "What the utilization
+// dashboard smooths away").
+#include <cuda/atomic>
+
+#include <algorithm>
+#include <mutex>
+
+#include "device.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+// ---------------------------------------------------------------------------
+// Top-K: one warp per token.  Each lane holds logits e = lane + 32 i.  A logit
+// becomes a 64-bit key: high word = order-preserving image of the float (NaN ->
+// 0, the lowest; -0.0 folded into +0.0), low word = ~e so that equal values
+// prefer the lower expert id.  K rounds of (lane-local max, warp max by
+// butterfly shuffles, the winner's slot is cleared).
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t order_key(float v) {
+  if (v != v) return 0u;   // NaN ranks below every number
+  if (v == 0.0f) v = 0.0f;  // -0.0 == +0.0
+  const uint32_t u = __float_as_uint(v);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float key_value(uint32_t k) {
+  if (k == 0u) return __uint_as_float(0x7fc00000u);
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, long long T, int E, int K,
+                                                    int renormalize, int32_t* __restrict__ ids,
+                                                    float* __restrict__ w) {
+  const int lane = threadIdx.x & 31;
+  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
+  for (long long t = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
+       t += warps) {
+    const float* row = logits + t * E;
+    unsigned long long key[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      const int e = lane + 32 * i;
+      key[i] = 0ull;
+      if (e < E) {
+        const float v = __ldg(row + e);
+        key[i] = (static_cast<unsigned long long>(order_key(v)) << 32) | static_cast<uint32_t>(~e);
+      }
+    }
+    // Every real candidate has key > 0 (low word ~e != 0), padding has key 0.
+    int my_id = 0;
+    float my_val = 0.0f;
+    for (int k = 0; k < K; ++k) {
+      unsigned long long best = 0ull;
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) best = key[i] > best ? key[i] : best;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+        best = other > best ? other : best;
+      }
+      const int e = static_cast<int>(~static_cast<uint32_t>(best));
+      // Keys are unique (the low word is the id): the owner of the winner retires it.
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) key[i] = (key[i] == best) ? 0ull : key[i];
+      if (lane == k) {
+        my_id = e;
+        my_val = key_value(static_cast<uint32_t>(best >> 32));
+      }
+    }
+    // Weights: exp(l_k - l_top) / (sum over the K selected, or over all E).
+    const float top = __shfl_sync(0xffffffffu, my_val, 0);
+    const float num = (lane < K) ? expf(my_val - top) : 0.0f;
+    float den = 0.0f;
+    if (renormalize) {
+      den = num;
+    } else {
+      const float* r = row;
+      for (int e = lane; e < E; e += 32) den += expf(__ldg(r + e) - top);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    if (lane < K) {
+      ids[t * K + lane] = my_id;
+      w[t * K + lane] = num / den;
+    }
+  }
+}
+
+template <int VPL>
+cudaError_t launch_route_vpl(const float* logits, long long T, int E, int K, int renorm, int32_t* ids, float* w,
+                             cudaStream_t s) {
+  const long long blocks = std::min<long long>((T + 7) / 8, 64LL * num_sms());
+  route_kernel<VPL><<<static_cast<int>(std::max<long long>(blocks, 1)), 256, 0, s>>>(logits, T, E, K, renorm,
+                                                                                       ids, w);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Count + scan + stable rank, one cooperative launch.
+//  phase 1: block b histograms its contiguous slice of assignments -> block_counts[b][e]
+//  grid barrier (bounded wait; all blocks are co-resident by the cooperative launch)
+//  phase 2: offsets[e] = sum of all counts of experts < e; base[b][e] = offsets[e] +
+//           counts of expert e in blocks < b.  Block 0 writes counts, offsets,
+//           partition counts/offsets and the skew ratio.
+//  phase 3: block b walks its slice in order, 256 assignments at a time; the rank of
+//           an assignment among equal ids = earlier warps' counts (shared) + its rank
+//           inside the warp (__match_any_sync); row = base + rank.
+// ---------------------------------------------------------------------------
+
+constexpr int kScanThreads = 256;
+constexpr int kScanWarps = kScanThreads / 32;
+constexpr int kScanMinChunk = 1024;
+
+__device__ bool grid_barrier(unsigned int* count, unsigned int* gen, unsigned int nblocks, int* status,
+                             int* s_ok) {
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    cuda::atomic_ref<unsigned int, cuda::thread_scope_device> c(*count), g(*gen);
+    const unsigned int my_gen = g.load(cuda::memory_order_acquire);
+    const unsigned int arrived = c.fetch_add(1u, cuda::memory_order_acq_rel);
+    int ok = 1;
+    if (arrived == nblocks - 1) {
+      c.store(0u, cuda::memory_order_relaxed);
+      g.fetch_add(1u, cuda::memory_order_release);
+    } else {
+      const uint64_t t0 = global_timer_ns();
+      unsigned int i = 0;
+      while (g.load(cuda::memory_order_acquire) == my_gen) {
+        if ((++i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+          report(status, MOE_DEV_TIMEOUT);
+          ok = 0;
+          break;
+        }
+      }
+    }
+    *s_ok = ok;
+  }
+  __syncthreads();
+  return *s_ok != 0;
+}
+
+__global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
+    const int32_t* __restrict__ ids, int TK, int E, int P, int chunk, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ part_counts, int32_t* __restrict__ part_offsets,
+    int32_t* __restrict__ row_of_assign, int32_t* __restrict__ assign_of_row, float* __restrict__ skew,
+    int* block_counts, unsigned int* bar_count, unsigned int* bar_gen, int* status) {
+  extern __shared__ int sm[];
+  int* s_hist = sm;                    // [E]   this block's histogram, then its running base
+  int* s_off = s_hist + E;             // [E+1] global exclusive offsets
+  int* s_wcnt = s_off + E + 1;         // [kScanWarps][E] per-warp counts of one 256-slice
+  __shared__ int s_ok, s_bad, s_red[kScanWarps], s_max[kScanWarps];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int b = blockIdx.x;
+  const int lo = min(TK, b * chunk), hi = min(TK, lo + chunk);
+
+  for (int e = tid; e < E; e += kScanThreads) s_hist[e] = 0;
+  for (int i = tid; i < kScanWarps * E; i += kScanThreads) s_wcnt[i] = 0;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+
+  // phase 1
+  for (int a = lo + tid; a < hi; a += kScanThreads) {
+    const int e = __ldg(ids + a);
+    if (e >= 0 && e < E) atomicAdd(&s_hist[e], 1);
+    else s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad && tid == 0) report(status, MOE_DEV_BAD_INDEX);
+  for (int e = tid; e < E; e += kScanThreads) block_counts[static_cast<long long>(b) * E + e] = s_hist[e];
+
+  if (!grid_barrier(bar_count, bar_gen, gridDim.x, status, &s_ok)) return;
+
+  // phase 2: column sums over blocks
+  int my_max = 0;
+  for (int e = tid; e < E; e += kScanThreads) {
+    int before = 0, total = 0;
+    for (int bb = 0; bb < static_cast<int>(gridDim.x); ++bb) {
+      const int c = __ldcg(block_counts + static_cast<long long>(bb) * E + e);
+      before += (bb < b) ? c : 0;
+      total += c;
+    }
+    s_hist[e] = before;
+    s_off[e] = total;
+    my_max = max(my_max, total);
+  }
+  __syncthreads();
+  // exclusive scan of s_off[0..E) in place (E <= 1024: 4 per thread)
+  {
+    const int per = (E + kScanThreads - 1) / kScanThreads;
+    const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
+    int local = 0;
+    for (int e = e0; e < e1; ++e) local += s_off[e];
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    if (lane == 31) s_red[warp] = incl;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, o));
+    if (lane == 0) s_max[warp] = my_max;
+    __syncthreads();
+    int wbase = 0, total = 0, mx = 0;
+    for (int w = 0; w < kScanWarps; ++w) {
+      if (w < warp) wbase += s_red[w];
+      total += s_red[w];
+      mx = max(mx, s_max[w]);
+    }
+    int run = wbase + incl - local;
+    __syncthreads();
+    for (int e = e0; e < e1; ++e) {
+      const int c = s_off[e];
+      s_off[e] = run;
+      run += c;
+    }
+    if (tid == 0) s_off[E] = total;
+    __syncthreads();
+    if (b == 0) {
+      for (int e = tid; e <= E; e += kScanThreads) {
+        offsets[e] = s_off[e];
+        if (e < E) counts[e] = s_off[e + 1] - s_off[e];
+      }
+      const int epp = E / P;
+      for (int p = tid; p <= P; p += kScanThreads) {
+        part_offsets[p] = s_off[p * epp];
+        if (p < P) part_counts[p] = s_off[(p + 1) * epp] - s_off[p * epp];
+      }
+      if (tid == 0 && skew) skew[0] = total > 0 ? static_cast<float>(mx) * static_cast<float>(E) / total : 0.0f;
+    }
+  }
+  for (int e = tid; e < E; e += kScanThreads) s_hist[e] += s_off[e];
+  __syncthreads();
+
+  // phase 3
+  const unsigned lt_mask = (1u << lane) - 1u;
+  for (int base = lo; base < hi; base += kScanThreads) {
+    const int a = base + tid;
+    int e = -1;
+    if (a < hi) {
+      e = __ldg(ids + a);
+      if (e < 0 || e >= E) e = -1;
+    }
+    const unsigned same = __match_any_sync(0xffffffffu, e);
+    const int leader = __ffs(same) - 1;
+    const int rank_in_warp = __popc(same & lt_mask);
+    if (e >= 0 && lane == leader) s_wcnt[warp * E + e] = __popc(same);
+    __syncthreads();
+    if (a < hi && e < 0) row_of_assign[a] = -1;  // an invalid id gets no row
+    if (e >= 0) {
+      int r = s_hist[e] + rank_in_warp;
+      for (int w = 0; w < warp; ++w) r += s_wcnt[w * E + e];
+      row_of_assign[a] = r;
+      assign_of_row[r] = a;
+    }
+    __syncthreads();
+    if (e >= 0 && lane == leader) {
+      atomicAdd(&s_hist[e], __popc(same));
+      s_wcnt[warp * E + e] = 0;
+    }
+    __syncthreads();
+  }
+}
+
+__global__ void skew_kernel(const int32_t* __restrict__ counts, int E, float* ratio) {
+  __shared__ int s_max[32], s_sum[32];
+  int mx = 0, sum = 0;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const int c = counts[e];
+    mx = max(mx, c);
+    sum += c;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    mx = max(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    sum += __shfl_xor_sync(0xffffffffu, sum, o);
+  }
+  if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = mx, s_sum[threadIdx.x >> 5] = sum;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mx = 0, sum = 0;
+    for (int w = 0; w < static_cast<int>(blockDim.x >> 5); ++w) mx = max(mx, s_max[w]), sum += s_sum[w];
+    ratio[0] = sum > 0 ? static_cast<float>(mx) * static_cast<float>(E) / sum : 0.0f;
+  }
+}
+
+size_t scan_smem_bytes(int E) { return static_cast<size_t>(E * 2 + 1 + kScanWarps * E) * sizeof(int); }
+
+}  // namespace
+
+cudaError_t launch_route(const float* logits, long long T, int E, int K, int renorm, int32_t* ids, float* w,
+                         cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int vpl = (E + 31) / 32;
+  if (vpl <= 1) return launch_route_vpl<1>(logits, T, E, K, renorm, ids, w, s);
+  if (vpl <= 2) return launch_route_vpl<2>(logits, T, E, K, renorm, ids, w, s);
+  if (vpl <= 4) return launch_route_vpl<4>(logits, T, E, K, renorm, ids, w, s);
+  if (vpl <= 8) return launch_route_vpl<8>(logits, T, E, K, renorm, ids, w, s);
+  if (vpl <= 16) return launch_route_vpl<16>(logits, T, E, K, renorm, ids, w, s);
+  return launch_route_vpl<32>(logits, T, E, K, renorm, ids, w, s);
+}
+
+int scan_max_blocks(long long TK) {
+  const long long b = (TK + kScanMinChunk - 1) / kScanMinChunk;
+  return static_cast<int>(std::max<long long>(1, std::min<long long>(b, 1024)));
+}
+
+cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, int32_t* counts, int32_t* offsets,
+                              int32_t* part_counts, int32_t* part_offsets, int32_t* row_of_assign,
+                              int32_t* assign_of_row, float* skew, const ScanWorkspace& ws, cudaStream_t s) {
+  const size_t smem = scan_smem_bytes(E);
+  static std::once_flag once;
+  static cudaError_t attr = cudaSuccess;
+  std::call_once(once, [] {
+    attr = cudaFuncSetAttribute(count_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(scan_smem_bytes(MOE_MAX_E)));
+  });
+  if (attr != cudaSuccess) return attr;
+  int occ = 0;
+  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, count_scan_kernel, kScanThreads, smem);
+  if (err != cudaSuccess) return err;
+  const long long resident = static_cast<long long>(std::max(occ, 1)) * num_sms();
+  int blocks = static_cast<int>(std::min<long long>({static_cast<long long>(ws.max_blocks), resident,
+                                                     std::max<long long>(1, (TK + kScanMinChunk - 1) / kScanMinChunk)}));
+  blocks = std::max(blocks, 1);
+  long long chunk = (TK + blocks - 1) / blocks;
+  chunk = (chunk + kScanThreads - 1) / kScanThreads * kScanThreads;
+  int TKi = static_cast<int>(TK), chunki = static_cast<int>(std::max<long long>(chunk, kScanThreads));
+  int* block_counts = ws.block_counts;
+  unsigned int* bc = ws.bar_count;
+  unsigned int* bg = ws.bar_gen;
+  int* status = ws.status;
+  void* args[] = {&ids, &TKi, &E, &P, &chunki, &counts, &offsets, &part_counts, &part_offsets,
+                  &row_of_assign, &assign_of_row, &skew, &block_counts, &bc, &bg, &status};
+  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(count_scan_kernel), dim3(blocks), dim3(kScanThreads),
+                                     args, smem, s);
+}
+
+cudaError_t launch_skew(const int32_t* counts, int E, float* ratio, cudaStream_t s) {
+  skew_kernel<<<1, 256, 0, s>>>(counts, E, ratio);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,275 @@
+"""End-to-end parity of moe_layer_forward (C ABI) with the CPU oracle.
+
+Small layers are compared output by output against the whole oracle.  The full
+workloads (the sizes bench.py times, same launch path) are checked on sampled
+tokens that the oracle evaluates one by one, and on properties that hold at any
+size (counting sort = bijection, expert-sorted and stable; xp rows are copies of
+x rows; partition ranges).
+
+Routing is compared token by token: a token whose K-th and (K+1)-th oracle
+logits are closer than the observed GPU-vs-oracle logit error has two correct
+answers, so it is only checked for validity; every other token must get exactly
+the oracle's ids.  When every token is unambiguous, all integer outputs are
+compared bit for bit.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from routing_dispatch_grouped_top_b200 import binding as B
+from routing_dispatch_grouped_top_b200 import build, inputs
+from routing_dispatch_grouped_top_b200.config import (DEEPSEEK_R1_DECODE, DEEPSEEK_R1_PREFILL, LATENT_896E,
+                                                      QWEN3_30B_A3B_PREFILL, TINY)
+from parity import BF16_MAX_RMS, BF16_REL_FROB, check_bf16, check_logits, rel_frob, topk_margin
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_ok):
+    build.build()
+    B.lib()
+
+
+def bits(t):
+    return inputs.to_bits(t)
+
+
+def cpu(t):
+    return t.detach().cpu().numpy()
+
+
+def run_gpu_layer(cfg, inp):
+    d = B.dims_of(cfg)
+    w = B.pack_layer_weights(d, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"], inp["w_dp"],
+                             inp["w_upp"])
+    bufs = B.alloc_layer_buffers(d)
+    ws = B.make_workspace(d)
+    B.moe_layer_forward(inp["x"], w, d, bufs, ws)
+    assert B.read_device_status(ws) == 0
+    return bufs
+
+
+def routing_split(ref_logits, got_logits, K):
+    """Boolean mask of tokens whose top-K set is unambiguous given the logit error."""
+    err = float(np.abs(np.asarray(got_logits, np.float64) - ref_logits).max()) if ref_logits.size else 0.0
+    return topk_margin(ref_logits, K) > 4.0 * err + 1e-7, err
+
+
+def check_routing(got_ids, ref_ids, ref_logits, safe, err, K):
+    assert np.array_equal(got_ids[safe], ref_ids[safe])
+    for t in np.nonzero(~safe)[0]:   # ambiguous tokens: the GPU's choice must be a valid top-K
+        kth = np.sort(ref_logits[t])[::-1][K - 1]
+        assert len(set(got_ids[t].tolist())) == K
+        assert np.all(ref_logits[t][got_ids[t]] >= kth - 2.0 * err - 1e-7)
+
+
+def check_count_scan_properties(ids, E, P, res):
+    """Properties that fix the stable counting sort at any size (checked with torch on the GPU)."""
+    ids = ids.reshape(-1).long()
+    TK = ids.numel()
+    counts = torch.bincount(ids, minlength=E)
+    assert torch.equal(res["counts"].long(), counts)
+    off = torch.zeros(E + 1, dtype=torch.long, device=ids.device)
+    off[1:] = torch.cumsum(counts, 0)
+    assert torch.equal(res["offsets"].long(), off)
+    roa, aor = res["row_of_assign"].long(), res["assign_of_row"].long()
+    ar = torch.arange(TK, device=ids.device)
+    assert torch.equal(aor[roa], ar) and torch.equal(roa[aor], ar)       # bijection
+    e_of_row = ids[aor]
+    assert bool((e_of_row[1:] >= e_of_row[:-1]).all())                     # expert-major
+    same = e_of_row[1:] == e_of_row[:-1]
+    assert bool((aor[1:][same] > aor[:-1][same]).all())                    # stable inside an expert
+    epp = E // P
+    assert torch.equal(res["part_offsets"].long(), off[::epp])
+    assert torch.equal(res["part_counts"].long(), off[epp::epp] - off[:-1:epp])
+
+
+# ---------------------------------------------------------------------------
+# Small layers against the whole oracle
+# ---------------------------------------------------------------------------
+
+SMALL = [
+    TINY,
+    TINY.with_(name="tiny_T100_P2_plain_softmax", T=100, P=2, renormalize=False),
+    QWEN3_30B_A3B_PREFILL.with_(name="qwen3_shape_T256_H512_F384", T=256, H=512, F=384),
+    DEEPSEEK_R1_PREFILL.with_(name="r1_shape_T64_H1024_F256_E64_P8", T=64, H=1024, F=256, E=64),
+    DEEPSEEK_R1_DECODE.with_(name="r1_decode_shape_T32_H1024_F512", T=32, H=1024, F=512),
+    LATENT_896E.with_(name="latent_shape_T48_D1024_H256_E112_P8", T=48, d_model=1024, H=256, E=112, F=128, P=8),
+    TINY.with_(name="one_token", T=1),
+]
+
+
+@pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
+def test_layer_matches_oracle(cfg):
+    inp = inputs.make_layer(cfg, DEV)
+    g = run_gpu_layer(cfg, inp)
+    torch.cuda.synchronize()
+    cpu_in = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
+    r = oracle.layer_forward(bits(cpu_in["x"]), cpu_in["w_g"].numpy(), bits(cpu_in["w_gate"]),
+                             bits(cpu_in["w_up"]), bits(cpu_in["w_down"]), cfg.K, cfg.P, cfg.renormalize,
+                             bias=None if cpu_in["bias"] is None else cpu_in["bias"].numpy(),
+                             w_dp_bits=None if cpu_in["w_dp"] is None else bits(cpu_in["w_dp"]),
+                             w_upp_bits=None if cpu_in["w_upp"] is None else bits(cpu_in["w_upp"]))
+    latent = bool(cfg.d_model)
+    if latent:
+        check_bf16("z", bits(g["z"]), r["z"])
+        # logits of a latent layer inherit z's bf16 rounding flips: bf16-in / fp32-out tolerance
+        gl = cpu(g["logits"])
+        assert rel_frob(gl, r["logits"]) <= BF16_REL_FROB
+        assert np.abs(gl - r["logits"]).max() <= BF16_MAX_RMS * np.sqrt(np.mean(r["logits"].astype(np.float64) ** 2))
+    else:
+        check_logits("logits", cpu(g["logits"]), r["logits"])
+    safe, err = routing_split(r["logits"], cpu(g["logits"]), cfg.K)
+    gid = cpu(g["topk_ids"])
+    check_routing(gid, r["topk_ids"], r["logits"], safe, err, cfg.K)
+    check_count_scan_properties(g["topk_ids"], cfg.E, cfg.P, g)
+    if safe.all():
+        for k in ("counts", "offsets", "part_counts", "part_offsets", "row_of_assign", "assign_of_row"):
+            assert np.array_equal(cpu(g[k]), r[k]), k
+        if not latent:
+            assert np.array_equal(bits(g["xp"]), r["xp"])
+        for key, mk in (("meta_token", "token"), ("meta_slot", "slot"), ("meta_local_expert", "local_expert")):
+            assert np.array_equal(cpu(g[key]), r["meta"][mk]), key
+        np.testing.assert_allclose(cpu(g["meta_w"]), r["meta"]["w"], atol=2e-6, rtol=0)
+        if not latent:
+            check_bf16("h", bits(g["h"]), r["h"])
+            check_bf16("y", bits(g["y"]), r["y"])
+    # per assignment of unambiguous tokens: h, y at each side's own row
+    T, K = cfg.T, cfg.K
+    ga, ra = cpu(g["row_of_assign"]).reshape(T, K), r["row_of_assign"].reshape(T, K)
+    st = np.nonzero(safe)[0]
+    if not latent and st.size:
+        check_bf16("h(assign)", bits(g["h"])[ga[st].reshape(-1)], r["h"][ra[st].reshape(-1)])
+        check_bf16("y(assign)", bits(g["y"])[ga[st].reshape(-1)], r["y"][ra[st].reshape(-1)])
+        check_bf16("out", bits(g["out"])[st], r["out"][st])
+    if latent:
+        # z flips move h, y and out by more than their rounding: the latent layer's
+        # outputs are compared at the whole-layer tolerance on unambiguous tokens.
+        for name, gv, rv in (("out", bits(g["out"])[st], r["out"][st]),
+                             ("final", bits(g["final_out"])[st], r["final"][st])):
+            assert rel_frob(oracle.bf16_bits_to_f64(gv), oracle.bf16_bits_to_f64(rv)) <= BF16_REL_FROB, name
+    assert float(g["skew"].item()) == pytest.approx(oracle.skew_ratio(cpu(g["counts"])), rel=1e-6)
+
+
+def test_layer_forward_host_io_matches_device_call():
+    cfg = TINY.with_(T=200, name="tiny_T200")
+    inp = inputs.make_layer(cfg, DEV)
+    g = run_gpu_layer(cfg, inp)
+    d = B.dims_of(cfg)
+    w = B.pack_layer_weights(d, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"])
+    bufs = B.alloc_layer_buffers(d)
+    ws = B.make_workspace(d)
+    xh = inp["x"].cpu().pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    xd = torch.empty_like(inp["x"])
+    B.moe_layer_forward_host(xh, xd, w, d, bufs, ws, oh)
+    torch.cuda.synchronize()
+    assert torch.equal(oh.view(torch.int16), g["out"].cpu().view(torch.int16))
+
+
+def test_layer_stage_events_are_recorded():
+    cfg = TINY
+    inp = inputs.make_layer(cfg, DEV)
+    d = B.dims_of(cfg)
+    w = B.pack_layer_weights(d, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"])
+    bufs = B.alloc_layer_buffers(d)
+    ws = B.make_workspace(d)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(B.MOE_NUM_STAGE_EVENTS)]
+    B.moe_layer_forward(inp["x"], w, d, bufs, ws, stage_events=ev)
+    torch.cuda.synchronize()
+    times = [ev[i].elapsed_time(ev[i + 1]) for i in range(len(ev) - 1)]
+    assert all(t >= 0 for t in times) and sum(times) > 0
+
+
+# ---------------------------------------------------------------------------
+# Full workloads: sampled tokens + size-independent properties
+# ---------------------------------------------------------------------------
+
+FULL = [QWEN3_30B_A3B_PREFILL, DEEPSEEK_R1_PREFILL, DEEPSEEK_R1_DECODE, LATENT_896E]
+HOST_EXPERT_BUDGET = 2.5e9   # bytes of expert weights copied to the host for the oracle
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("cfg", FULL, ids=lambda c: c.name)
+def test_full_size_sampled(cfg):
+    torch.cuda.empty_cache()
+    inp = inputs.make_layer(cfg, DEV)
+    g = run_gpu_layer(cfg, inp)
+    T, K, E, H, F = cfg.T, cfg.K, cfg.E, cfg.H, cfg.F
+    latent = bool(cfg.d_model)
+    # properties at full size
+    check_count_scan_properties(g["topk_ids"], E, cfg.P, g)
+    routed = g["z"] if latent else inp["x"]
+    roa = g["row_of_assign"].long()
+    tok = torch.arange(T * K, device=DEV) // K
+    assert torch.equal(g["xp"][roa].view(torch.int16), routed[tok].view(torch.int16))
+    assert torch.equal(g["meta_token"][roa].long(), tok)
+    assert g["xp"].numel() * 2 == oracle.dispatch_bytes(T, K, H, 2)
+    # sampled tokens through the oracle
+    rng = np.random.default_rng(cfg.T + cfg.E)
+    cand = rng.permutation(T)[:256]
+    x_rows = bits(inp["x"][torch.from_numpy(cand).to(DEV)])
+    w_g = inp["w_g"].cpu().numpy()
+    bias = None if inp["bias"] is None else inp["bias"].cpu().numpy()
+    if latent:
+        z_rows = oracle.dense_bf16(x_rows, bits(inp["w_dp"]))
+        check_bf16("z(sampled)", bits(g["z"])[cand], z_rows)
+    else:
+        z_rows = x_rows
+    lref = oracle.gating_logits(z_rows, w_g, bias)
+    lgot = cpu(g["logits"])[cand]
+    if latent:
+        assert rel_frob(lgot, lref) <= BF16_REL_FROB
+    else:
+        check_logits("logits(sampled)", lgot, lref)
+    ids_ref, w_ref = oracle.route(lref, K, cfg.renormalize)
+    safe, err = routing_split(lref, lgot, K)
+    check_routing(cpu(g["topk_ids"])[cand], ids_ref, lref, safe, err, K)
+    # FFN + combine for unambiguous sampled tokens, within a host-memory budget
+    per_expert = 3 * H * F * 2
+    max_experts = max(K, int(HOST_EXPERT_BUDGET // per_expert))
+    chosen, experts = [], set()
+    for i in np.nonzero(safe)[0]:
+        need = experts | set(ids_ref[i].tolist())
+        if len(need) > max_experts and chosen:
+            break
+        chosen.append(i)
+        experts = need
+        if len(chosen) >= 64:
+            break
+    assert chosen, "no unambiguous sampled token"
+    wcache = {e: (bits(inp["w_gate"][e]), bits(inp["w_up"][e]), bits(inp["w_down"][e])) for e in sorted(experts)}
+    ga = cpu(g["row_of_assign"]).reshape(T, K)
+    gh, gy, gout = [], [], []
+    rh, ry, rout = [], [], []
+    for i in chosen:
+        t = cand[i]
+        acc = np.zeros(H)
+        for k in range(K):
+            e = int(ids_ref[i, k])
+            h_, y_ = oracle.ffn_rows(z_rows[i:i + 1], *wcache[e])
+            rh.append(h_[0])
+            ry.append(y_[0])
+            acc += float(w_ref[i, k]) * oracle.bf16_bits_to_f64(y_)[0]
+            row = ga[t, k]
+            gh.append(bits(g["h"][row]))
+            gy.append(bits(g["y"][row]))
+        rout.append(oracle.f64_to_bf16_bits(acc))
+        gout.append(bits(g["out"][t]))
+    if latent:
+        # the GPU's h/y/out rows descend from its own z (rounding flips of z move them a little)
+        for name, a, b in (("h", gh, rh), ("y", gy, ry), ("out", gout, rout)):
+            assert rel_frob(oracle.bf16_bits_to_f64(np.stack(a)), oracle.bf16_bits_to_f64(np.stack(b))) <= BF16_REL_FROB, name
+        fin = oracle.dense_bf16(np.stack(rout), bits(inp["w_upp"]))
+        got_fin = bits(g["final_out"])[cand[chosen]]
+        assert rel_frob(oracle.bf16_bits_to_f64(got_fin), oracle.bf16_bits_to_f64(fin)) <= BF16_REL_FROB
+    else:
+        check_bf16("h(sampled)", np.stack(gh), np.stack(rh))
+        check_bf16("y(sampled)", np.stack(gy), np.stack(ry))
+        check_bf16("out(sampled)", np.stack(gout), np.stack(rout))
+    assert float(g["skew"].item()) == pytest.approx(oracle.skew_ratio(cpu(g["counts"])), rel=1e-6)
+    del g, inp
+    torch.cuda.empty_cache()

@@ -1,0 +1,325 @@
+"""GPU parity of each step, called through the C ABI, against the CPU oracle.
+
+Both sides get the same seeded inputs from routing_dispatch_grouped_top_b200.inputs;
+nothing the GPU computes is fed to the oracle.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from routing_dispatch_grouped_top_b200 import binding as B
+from routing_dispatch_grouped_top_b200 import build, inputs
+from parity import WEIGHT_ABS, check_bf16, check_logits
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(cuda_ok):
+    build.build()
+    B.lib()
+
+
+def bits(t):
+    return inputs.to_bits(t)
+
+
+def cpu(t):
+    return t.detach().cpu().numpy()
+
+
+# ---------------------------------------------------------------------------
+# S1 route
+# ---------------------------------------------------------------------------
+
+ROUTE_CASES = [  # T, E, K, renormalize, generator
+    (300, 8, 2, True, "random"), (257, 128, 8, True, "random"), (100, 256, 8, False, "random"),
+    (77, 896, 16, True, "random"), (64, 33, 5, True, "quantized"), (50, 1024, 32, True, "random"),
+    (129, 64, 6, True, "special"), (40, 1000, 7, False, "quantized"), (1, 5, 5, True, "random"),
+    (0, 16, 4, True, "random"), (4096, 128, 8, True, "random"),
+]
+
+
+@pytest.mark.parametrize("T,E,K,renorm,gen", ROUTE_CASES)
+def test_route_matches_oracle(T, E, K, renorm, gen):
+    seed = T * 7 + E
+    if gen == "random":
+        l = inputs.random_logits(T, E, seed=seed, scale=2.0)
+    elif gen == "quantized":
+        l = inputs.quantized_logits(T, E, levels=5, seed=seed)
+    else:
+        l = inputs.special_logits(T, E, seed=seed)
+    d = B.dims(T=T, H=8, E=E, K=K, F=8, renormalize=renorm)
+    ids = torch.full((T, K), -7, dtype=torch.int32, device=DEV)
+    w = torch.empty((T, K), dtype=torch.float32, device=DEV)
+    B.moe_route(l.to(DEV), d, ids, w)
+    torch.cuda.synchronize()
+    if T == 0:
+        return
+    rid, rw = oracle.route(l.numpy(), K, renorm)
+    assert np.array_equal(cpu(ids), rid)
+    if gen == "special":
+        sel = np.take_along_axis(l.numpy(), rid, axis=1)
+        ok_rows = np.all(np.isfinite(sel), axis=1) & np.all(np.isfinite(l.numpy()) | renorm, axis=1)
+        np.testing.assert_allclose(cpu(w)[ok_rows], rw[ok_rows], atol=WEIGHT_ABS, rtol=0)
+    else:
+        np.testing.assert_allclose(cpu(w), rw, atol=WEIGHT_ABS, rtol=0)
+        if renorm:
+            assert np.allclose(cpu(w).sum(axis=1), 1.0, atol=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# S2 count + scan
+# ---------------------------------------------------------------------------
+
+SCAN_CASES = [  # T, E, K, P, zipf
+    (64, 8, 2, 1, None), (300, 16, 4, 4, None), (1, 4, 4, 2, None), (0, 8, 2, 1, None),
+    (128, 256, 8, 8, 1.1), (4096, 128, 8, 1, None), (8192, 256, 8, 8, None), (4096, 896, 16, 64, None),
+    (3000, 1024, 3, 16, 2.0), (5000, 7, 7, 7, None), (20000, 64, 6, 4, 1.1),
+]
+
+
+def run_count_scan(ids, E, P):
+    T, K = ids.shape
+    d = B.dims(T=T, H=8, E=E, K=K, F=8, P=P)
+    ws = B.make_workspace(d)
+    TK = T * K
+    mk = lambda n: torch.full((n,), -3, dtype=torch.int32, device=DEV)  # noqa: E731
+    out = dict(counts=mk(E), offsets=mk(E + 1), part_counts=mk(P), part_offsets=mk(P + 1),
+               row_of_assign=mk(max(TK, 1)), assign_of_row=mk(max(TK, 1)))
+    B.moe_count_scan(ids.to(DEV).contiguous(), d, out["counts"], out["offsets"], out["part_counts"],
+                     out["part_offsets"], out["row_of_assign"], out["assign_of_row"], ws)
+    status = B.read_device_status(ws)
+    res = {k: cpu(v) for k, v in out.items()}
+    res["row_of_assign"] = res["row_of_assign"][:TK]
+    res["assign_of_row"] = res["assign_of_row"][:TK]
+    return res, status
+
+
+@pytest.mark.parametrize("T,E,K,P,zipf", SCAN_CASES)
+def test_count_scan_matches_oracle(T, E, K, P, zipf):
+    ids = inputs.random_topk_ids(T, E, K, seed=T + E + K, zipf_s=zipf) if T else torch.zeros((0, K), dtype=torch.int32)
+    got, status = run_count_scan(ids, E, P)
+    assert status == 0
+    ref = oracle.count_scan(ids.numpy(), E, P)
+    for k in ("counts", "offsets", "part_counts", "part_offsets", "row_of_assign", "assign_of_row"):
+        assert np.array_equal(got[k], ref[k]), k
+
+
+def test_count_scan_repeated_calls_reuse_workspace():
+    ids = inputs.random_topk_ids(2000, 64, 4, seed=3)
+    d = B.dims(T=2000, H=8, E=64, K=4, F=8, P=4)
+    ws = B.make_workspace(d)
+    ref = oracle.count_scan(ids.numpy(), 64, 4)
+    idd = ids.to(DEV)
+    bufs = [torch.empty(n, dtype=torch.int32, device=DEV) for n in (64, 65, 4, 5, 8000, 8000)]
+    for _ in range(5):
+        B.moe_count_scan(idd, d, *bufs, ws)
+    assert B.read_device_status(ws) == 0
+    assert np.array_equal(cpu(bufs[4]), ref["row_of_assign"])
+
+
+def test_count_scan_flags_out_of_range_ids():
+    ids = inputs.random_topk_ids(100, 16, 2, seed=1)
+    ids[17, 1] = 16
+    ids[50, 0] = -2
+    got, status = run_count_scan(ids, 16, 1)
+    assert status & B.DEV_BAD_INDEX
+    flat = ids.numpy().reshape(-1)
+    assert got["counts"].sum() == int(((flat >= 0) & (flat < 16)).sum())
+    assert got["row_of_assign"][17 * 2 + 1] == -1 and got["row_of_assign"][100] == -1
+
+
+def test_count_scan_barrier_wait_times_out_and_reports():
+    # A grid-barrier counter that can never reach its target (set on the host):
+    # every block's bounded wait must give up, report MOE_DEV_TIMEOUT and return.
+    ids = inputs.random_topk_ids(4000, 32, 4, seed=9)
+    d = B.dims(T=4000, H=8, E=32, K=4, F=8)
+    ws = B.make_workspace(d)
+    ws[64:68] = torch.tensor([0xF0, 0xFF, 0xFF, 0x7F], dtype=torch.uint8, device=DEV)
+    bufs = [torch.empty(n, dtype=torch.int32, device=DEV) for n in (32, 33, 1, 2, 16000, 16000)]
+    B.moe_count_scan(ids.to(DEV), d, *bufs, ws)
+    assert B.read_device_status(ws) & B.DEV_TIMEOUT
+    B.workspace_init(ws)   # the context stays usable: the next call works
+    B.moe_count_scan(ids.to(DEV), d, *bufs, ws)
+    assert B.read_device_status(ws) == 0
+    assert np.array_equal(cpu(bufs[4]), oracle.count_scan(ids.numpy(), 32)["row_of_assign"])
+
+
+# ---------------------------------------------------------------------------
+# S3 permute
+# ---------------------------------------------------------------------------
+
+PERMUTE_CASES = [(300, 256, 16, 4, 4), (1, 8, 4, 1, 1), (64, 7168, 256, 8, 8), (1000, 2048, 128, 8, 1),
+                 (33, 72, 6, 6, 3), (0, 64, 8, 2, 1)]
+
+
+@pytest.mark.parametrize("T,H,E,K,P", PERMUTE_CASES)
+def test_permute_matches_oracle(T, H, E, K, P):
+    x = inputs.random_bf16((T, H), seed=T + H)
+    ids = inputs.random_topk_ids(T, E, K, seed=T + E) if T else torch.zeros((0, K), dtype=torch.int32)
+    w = inputs.random_weights(T, K, seed=5)
+    cs = oracle.count_scan(ids.numpy(), E, P)
+    roa = torch.from_numpy(cs["row_of_assign"])
+    d = B.dims(T=T, H=H, E=E, K=K, F=8, P=P)
+    TK = T * K
+    xp = torch.zeros((TK, H), dtype=torch.bfloat16, device=DEV)
+    meta = [torch.full((TK,), -1, dtype=dt, device=DEV) for dt in (torch.int32, torch.int32, torch.float32, torch.int32)]
+    B.moe_permute(x.to(DEV), roa.to(DEV), ids.to(DEV), w.to(DEV), d, xp, *meta)
+    torch.cuda.synchronize()
+    rxp, rmeta = oracle.permute(bits(x), cs["row_of_assign"], ids.numpy(), w.numpy(), E, P)
+    assert np.array_equal(bits(xp), rxp)
+    assert xp.numel() * xp.element_size() == oracle.dispatch_bytes(T, K, H, 2)
+    for got, key in zip(meta, ("token", "slot", "w", "local_expert")):
+        assert np.array_equal(cpu(got), rmeta[key]), key
+
+
+def test_permute_then_combine_of_identity_experts_returns_x():
+    # Identity experts (y = xp): combine(permute(x)) = (sum of weights) * x = x.
+    T, H, E, K = 500, 1024, 32, 8
+    x = inputs.random_bf16((T, H), seed=1).to(DEV)
+    l = inputs.random_logits(T, E, seed=2).to(DEV)
+    d = B.dims(T=T, H=H, E=E, K=K, F=8)
+    ws = B.make_workspace(d)
+    b = B.alloc_layer_buffers(d)
+    B.moe_route(l, d, b["topk_ids"], b["topk_w"])
+    B.moe_count_scan(b["topk_ids"], d, b["counts"], b["offsets"], b["part_counts"], b["part_offsets"],
+                     b["row_of_assign"], b["assign_of_row"], ws)
+    B.moe_permute(x, b["row_of_assign"], b["topk_ids"], b["topk_w"], d, b["xp"])
+    B.moe_combine(b["xp"], b["row_of_assign"], b["topk_w"], d, b["out"])
+    torch.cuda.synchronize()
+    assert torch.equal(b["out"].view(torch.int16), x.view(torch.int16))
+
+
+# ---------------------------------------------------------------------------
+# S4/S5 grouped SwiGLU FFN
+# ---------------------------------------------------------------------------
+
+FFN_CASES = [  # E, H, F, rows, zipf, zero_frac
+    (8, 256, 512, 300, None, 0.25), (4, 200, 200, 260, None, 0.0), (16, 2048, 768, 2000, 1.1, 0.2),
+    (3, 64, 136, 1, None, 0.0), (32, 512, 256, 700, 2.0, 0.3), (1, 1024, 384, 513, None, 0.0),
+    (64, 128, 128, 64, None, 0.5),
+]
+
+
+def ffn_inputs(E, H, F, rows, zipf, zero_frac, seed=0):
+    counts = inputs.random_counts(E, rows, seed=seed + E + rows, zipf_s=zipf, zero_frac=zero_frac)
+    off = np.zeros(E + 1, np.int32)
+    off[1:] = np.cumsum(counts.numpy())
+    xp = inputs.random_bf16((rows, H), seed=seed + 1)
+    wg = inputs.random_bf16((E, F, H), seed=seed + 2, std=H ** -0.5)
+    wu = inputs.random_bf16((E, F, H), seed=seed + 3, std=H ** -0.5)
+    wd = inputs.random_bf16((E, H, F), seed=seed + 4, std=F ** -0.5)
+    return off, xp, wg, wu, wd
+
+
+@pytest.mark.parametrize("E,H,F,rows,zipf,zf", FFN_CASES)
+def test_grouped_ffn_matches_oracle(E, H, F, rows, zipf, zf):
+    off, xp, wg, wu, wd = ffn_inputs(E, H, F, rows, zipf, zf)
+    d = B.dims(T=rows, H=H, E=E, K=1, F=F)
+    ws = B.make_workspace(d)
+    h = torch.zeros((rows, F), dtype=torch.bfloat16, device=DEV)
+    y = torch.zeros((rows, H), dtype=torch.bfloat16, device=DEV)
+    B.moe_grouped_ffn(xp.to(DEV), torch.from_numpy(off).to(DEV), wg.to(DEV), wu.to(DEV), wd.to(DEV), d, h, y, ws)
+    assert B.read_device_status(ws) == 0
+    rh, ry = oracle.grouped_ffn(bits(xp), off, bits(wg), bits(wu), bits(wd))
+    check_bf16("h", bits(h), rh)
+    check_bf16("y", bits(y), ry)
+
+
+def test_grouped_down_alone_matches_oracle():
+    E, H, F, rows = 12, 1024, 512, 900
+    counts = inputs.random_counts(E, rows, seed=4, zero_frac=0.2)
+    off = np.concatenate([[0], np.cumsum(counts.numpy())]).astype(np.int32)
+    hin = inputs.random_bf16((rows, F), seed=5, std=0.5)
+    wd = inputs.random_bf16((E, H, F), seed=6, std=F ** -0.5)
+    d = B.dims(T=rows, H=H, E=E, K=1, F=F)
+    ws = B.make_workspace(d)
+    y = torch.zeros((rows, H), dtype=torch.bfloat16, device=DEV)
+    B.moe_grouped_down(hin.to(DEV), torch.from_numpy(off).to(DEV), wd.to(DEV), d, y, ws)
+    assert B.read_device_status(ws) == 0
+    ry = np.zeros((rows, H), np.uint16)
+    for e in range(E):
+        lo, hi = off[e], off[e + 1]
+        if hi > lo:
+            ry[lo:hi] = oracle.f64_to_bf16_bits(oracle.bf16_bits_to_f64(bits(hin)[lo:hi]) @
+                                                oracle.bf16_bits_to_f64(bits(wd)[e]).T)
+    check_bf16("y", bits(y), ry)
+
+
+def test_grouped_gemm_rejects_bad_offsets_without_touching_memory():
+    E, H, F, rows = 4, 128, 128, 64
+    off, xp, wg, wu, wd = ffn_inputs(E, H, F, rows, None, 0.0)
+    off_bad = off.copy()
+    off_bad[2] = rows + 5000                          # beyond the buffer
+    d = B.dims(T=rows, H=H, E=E, K=1, F=F)
+    ws = B.make_workspace(d)
+    h = torch.zeros((rows, F), dtype=torch.bfloat16, device=DEV)
+    B.moe_grouped_gate_up(xp.to(DEV), torch.from_numpy(off_bad).to(DEV), wg.to(DEV), wu.to(DEV), d, h, ws)
+    assert B.read_device_status(ws) & B.DEV_BAD_INDEX
+    assert int(h.view(torch.int16).abs().sum()) == 0
+
+
+# ---------------------------------------------------------------------------
+# S6 combine
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,H,K", [(300, 256, 2), (77, 7168, 8), (1000, 2048, 16), (5, 8, 1), (64, 512, 32)])
+def test_combine_matches_oracle(T, H, K):
+    y = inputs.random_bf16((T * K, H), seed=T + H)
+    roa = inputs.random_bijection(T * K, seed=K)
+    w = inputs.random_weights(T, K, seed=T)
+    d = B.dims(T=T, H=H, E=max(K, 2), K=K, F=8)
+    out = torch.zeros((T, H), dtype=torch.bfloat16, device=DEV)
+    B.moe_combine(y.to(DEV), roa.to(DEV), w.to(DEV), d, out)
+    torch.cuda.synchronize()
+    ref = oracle.combine(bits(y), roa.numpy(), w.numpy())
+    check_bf16("out", bits(out), ref)
+
+
+# ---------------------------------------------------------------------------
+# S7 skew
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("E,total,zipf", [(8, 128, None), (256, 1024, 1.1), (896, 65536, None), (4, 0, None)])
+def test_skew_matches_oracle(E, total, zipf):
+    c = inputs.random_counts(E, total, seed=E, zipf_s=zipf)
+    d = B.dims(T=max(total, 1), H=8, E=E, K=1, F=8)
+    r = torch.zeros(1, dtype=torch.float32, device=DEV)
+    B.moe_skew_stats(c.to(DEV), d, r)
+    torch.cuda.synchronize()
+    assert float(r.item()) == pytest.approx(oracle.skew_ratio(c.numpy()), rel=1e-6)
+
+
+# ---------------------------------------------------------------------------
+# S0 gating and S8 dense projections
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,H,E,bias", [(300, 256, 8, False), (200, 2048, 128, False), (130, 7168, 256, True),
+                                        (97, 2048, 896, False), (5, 64, 1000, True)])
+def test_gating_matches_oracle(T, H, E, bias):
+    x = inputs.random_bf16((T, H), seed=T)
+    w_g = (torch.randn((H, E), generator=torch.Generator().manual_seed(H + E)) * H ** -0.5).float()
+    b = (torch.randn(E, generator=torch.Generator().manual_seed(E)) * 0.5).float() if bias else None
+    d = B.dims(T=T, H=H, E=E, K=1, F=8)
+    ws = B.make_workspace(d)
+    split = torch.empty((3, E, H), dtype=torch.bfloat16, device=DEV)
+    B.moe_pack_router(w_g.to(DEV), d, split)
+    logits = torch.empty((T, E), dtype=torch.float32, device=DEV)
+    B.moe_gating(x.to(DEV), split, b.to(DEV) if bias else None, d, logits, ws)
+    assert B.read_device_status(ws) == 0
+    ref = oracle.gating_logits(bits(x), w_g.numpy(), b.numpy() if bias else None)
+    check_logits("logits", cpu(logits), ref)
+
+
+@pytest.mark.parametrize("M,Kd,N", [(300, 1024, 256), (64, 7168, 2048), (257, 2048, 7168), (3, 72, 40)])
+def test_dense_projection_matches_oracle(M, Kd, N):
+    a = inputs.random_bf16((M, Kd), seed=M)
+    w = inputs.random_bf16((N, Kd), seed=N, std=Kd ** -0.5)
+    out = torch.zeros((M, N), dtype=torch.bfloat16, device=DEV)
+    ws = torch.zeros(256, dtype=torch.uint8, device=DEV)
+    B.moe_dense(a.to(DEV), w.to(DEV), out, ws)
+    assert B.read_device_status(ws) == 0
+    check_bf16("dense", bits(out), oracle.dense_bf16(bits(a), bits(w)))
