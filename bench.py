@@ -39,8 +39,8 @@ FLUSH_BYTES = 256 << 20
 def parse():
     p = argparse.ArgumentParser()
     p.add_argument("--gpus", type=int, default=1)
-    p.add_argument("--steps", type=int, default=50)
-    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--config", default=DEFAULT_CONFIG)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -55,6 +55,15 @@ def dist_env():
     return ws, rank, local
 
 
+def reduce_max(x: float, dist=None, device="cpu") -> float:
+    """Largest value over all ranks (the slowest rank's time); identity without a process group."""
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -66,59 +75,93 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+    """Samples the SM clock and clock-event (throttle) reasons through NVML (read-only
+    queries, the interface nvidia-smi reads) in a thread while the timed region runs."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    def __init__(self, device: int):
+        self.device = device
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+        self._nvml = None
+
+    def _handle(self, nv):
+        try:
+            props = torch.cuda.get_device_properties(self.device)
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return nv.nvmlDeviceGetHandleByPciBusId(bus.encode())
+        except Exception:
+            return nv.nvmlDeviceGetHandleByIndex(self.device)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
-                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            self._nvml = nv
+            self._h = self._handle(nv)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        except Exception:
+            self._nvml = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self._nvml
+        while not self._stop.is_set():
+            try:
+                sm = nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM)
+                rs = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                self.samples.append((sm, rs))
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
+        self._stop.set()
+        if self._t:
+            self._t.join(timeout=2)
+        if self._nvml:
             try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+                self._nvml.nvmlShutdown()
+            except Exception:
+                pass
 
     def summary(self):
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0, "source": "nvml"}
+        nv = self._nvml
+        reasons = set()
+        for _, rs in self.samples:
+            for name, const in self.REASONS:
+                if nv is not None and rs & getattr(nv, const, 0):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s for s, _ in self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
+
+
+def kernel_traffic(workload: str, stage: str):
+    """DRAM bytes per launch of one kernel from a committed ncu summary, or None when the
+    kernel source changed since the counters were taken (the summary records its hash)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
+    if not os.path.exists(path):
+        return None
+    for ln in open(path):
+        f = ln.split("#")[0].split()
+        if len(f) >= 4 and f[0] == workload and f[1] == stage:
+            src = os.path.join(ROOT, "routing_dispatch_grouped_top_b200", "csrc", f[3].split(":")[0])
+            if not os.path.exists(src):
+                return None
+            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
+            return float(f[2]) if h == f[3].split(":")[1] else None
+    return None
 
 
 def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 16):
@@ -185,6 +228,12 @@ def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 16):
                        f"(numpy float64, {el:.1f} s of oracle compute; weights prepared outside the clock)")
 
 
+def config_dict(cfg, world: int) -> dict:
+    return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K, "F": cfg.F, "P": cfg.P,
+            "d_model": cfg.d_model, "parallelism": f"replicas{world}",
+            "l2": "flushed (256 MiB write) before every timed step, outside its events"}
+
+
 def run_reference(args, cfg):
     ws, rank, _ = dist_env()
     if rank != 0:
@@ -199,8 +248,7 @@ def run_reference(args, cfg):
     line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1000.0 * 16 / val, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference", "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K,
-                                            "F": cfg.F, "P": cfg.P, "d_model": cfg.d_model},
+            "impl": "reference", "config": config_dict(cfg, ws),
             "cpu_baseline": cb, "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
                                         "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -261,11 +309,7 @@ def main():
         raise RuntimeError("device status set during the timed steps")
     step_ms = [ev[0].elapsed_time(ev[-1]) for ev in events]
     stage_ms = [[ev[j].elapsed_time(ev[j + 1]) for ev in events] for j in range(n_ev - 1)]
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = reduce_max(sum(step_ms), dist, dev)
     ms_per_step = total_ms / args.steps
     value = world * cfg.T / (ms_per_step / 1e3)
 
@@ -284,11 +328,7 @@ def main():
         B.moe_layer_forward_host(xh, xd, w, d, bufs, ws, oh)
         b.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = reduce_max(sum(a.elapsed_time(b) for a, b in e2e_ev), dist, dev)
     e2e_value = world * cfg.T / (e2e_ms / args.steps / 1e3)
 
     if rank == 0:
@@ -298,33 +338,60 @@ def main():
         stage_mean = {n: statistics.mean(v) for n, v in zip(names, stage_ms)}
         long_run = total_ms > 1000.0
         bf16_peak = peaks["bf16_sustained"] if long_run else peaks["bf16"]
-        gate_up_tflops = cfg.gate_up_flops() / (stage_mean["gate_up"] / 1e3) / 1e12
-        down_tflops = cfg.down_flops() / (stage_mean["down"] / 1e3) / 1e12
+        n_touched = int((bufs["counts"] > 0).sum().item())
+        T, H, F, TK = cfg.T, cfg.H, cfg.F, cfg.TK
+        # algorithmic work per launch: (flops, HBM bytes)
+        work = {
+            "gate_up": (4 * H * F * TK, 2 * H * F * 2 * n_touched + TK * H * 2 + TK * F * 2),
+            "down": (2 * H * F * TK, H * F * 2 * n_touched + TK * F * 2 + TK * H * 2),
+            "permute": (0, T * H * 2 + TK * H * 2 + TK * (4 + 8 + 16)),
+            "combine": (0, TK * H * 2 + T * H * 2 + TK * 8),
+            "gating": (2 * T * H * cfg.E * 3, T * H * 2 + 3 * cfg.E * H * 2 + T * cfg.E * 4),
+            "route": (0, T * cfg.E * 4 + TK * 8),
+        }
+        dominant = max(work, key=lambda n: stage_mean[n])
+        fl, by = work[dominant]
+        t_s = stage_mean[dominant] / 1e3
+        hbm_time, tc_time = by / (peaks["hbm"] * 1e9), fl / (bf16_peak * 1e12)
+        if hbm_time >= tc_time:
+            roof = {"bound": "hbm", "achieved": by / t_s / 1e9, "peak": peaks["hbm"], "unit": "GB/s"}
+        else:
+            roof = {"bound": "tensor", "achieved": fl / t_s / 1e12, "peak": bf16_peak, "unit": "TFLOP/s"}
+        roof["frac"] = roof["achieved"] / roof["peak"]
+        roof["traffic"] = kernel_traffic(cfg.name, dominant)
+        roof["kernel"] = dominant
+        roof["algorithmic_bytes"] = by
+        roof["algorithmic_flops"] = fl
+        roof["peak_source"] = (f"{peaks['source']} " + ("HBM copy" if roof["bound"] == "hbm" else
+                                                         f"bf16 {'sustained' if long_run else 'burst'}"))
         ffn_ms = stage_mean["gate_up"] + stage_mean["down"]
         ffn_tflops = cfg.expert_flops() / (ffn_ms / 1e3) / 1e12
-        perm_bytes = cfg.T * cfg.H * 2 + cfg.TK * cfg.H * 2
-        perm_gbs = perm_bytes / (stage_mean["permute"] / 1e3) / 1e9
-        comb_gbs = perm_bytes / (stage_mean["combine"] / 1e3) / 1e9
-        dominant = max(("gate_up", "down"), key=lambda n: stage_mean[n])
-        dom_tf = gate_up_tflops if dominant == "gate_up" else down_tflops
+        ffn_bytes = work["gate_up"][1] + work["down"][1]
+        frac = {n: {"ms": stage_mean[n],
+                    "tflops": (work[n][0] / (stage_mean[n] / 1e3) / 1e12) if work[n][0] else None,
+                    "gbs": work[n][1] / (stage_mean[n] / 1e3) / 1e9} for n in work}
+        for n in frac:
+            frac[n]["frac_hbm"] = frac[n]["gbs"] / peaks["hbm"]
+            if frac[n]["tflops"]:
+                frac[n]["frac_bf16"] = frac[n]["tflops"] / bf16_peak
+        frac["grouped_ffn"] = {"ms": ffn_ms, "tflops": ffn_tflops, "frac_bf16": ffn_tflops / bf16_peak,
+                               "gbs": ffn_bytes / (ffn_ms / 1e3) / 1e9,
+                               "frac_hbm": ffn_bytes / (ffn_ms / 1e3) / 1e9 / peaks["hbm"],
+                               "roofline_ms": 1e3 * max(ffn_bytes / (peaks["hbm"] * 1e9),
+                                                        cfg.expert_flops() / (bf16_peak * 1e12))}
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K, "F": cfg.F,
-                       "P": cfg.P, "d_model": cfg.d_model, "parallelism": f"replicas{world}",
-                       "l2": "flushed (256 MiB write) before every timed step, outside its events"},
-            "roofline": {"bound": "tensor", "kernel": f"grouped_gemm<{dominant}>", "achieved": dom_tf,
-                         "peak": bf16_peak, "unit": "TFLOP/s", "frac": dom_tf / bf16_peak, "traffic": None,
-                         "peak_source": f"{peaks['source']} bf16 {'sustained' if long_run else 'burst'}"},
+            "config": config_dict(cfg, world),
+            "roofline": roof,
             "stages_ms": stage_mean,
-            "fractions": {"grouped_gemm_tflops": ffn_tflops, "grouped_gemm_frac_bf16": ffn_tflops / bf16_peak,
-                          "permute_gbs": perm_gbs, "permute_frac_hbm": perm_gbs / peaks["hbm"],
-                          "combine_gbs": comb_gbs, "combine_frac_hbm": comb_gbs / peaks["hbm"]},
+            "fractions": frac,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": cfg.T * d_in * 2,
                     "d2h_bytes_per_step": cfg.T * d_in * 2},
             "gpu_launches": (7 + (2 if cfg.d_model else 0)) * args.steps,
             "clocks": clk.summary(),
+            "skew_max_over_mean": float(bufs["skew"].item()),
         }
         if not args.no_cpu_baseline and world == 1:
             line["cpu_baseline"] = cpu_oracle_rate(cfg, args.cpu_seconds)

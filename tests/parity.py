@@ -77,8 +77,12 @@ def check_logits(name, got, ref):
 
 
 def topk_margin(logits, K):
-    """Per token: gap between the K-th and (K+1)-th largest logit (inf when K == E)."""
+    """Per token: (gap between the K-th and (K+1)-th largest logit, smallest gap
+    between neighbours among the K+1 largest).  The first decides the selected
+    set, the second also the slot order.  inf where there is no such pair."""
     l = np.sort(np.asarray(logits, np.float64), axis=1)[:, ::-1]
-    if K >= l.shape[1]:
-        return np.full(l.shape[0], np.inf)
-    return l[:, K - 1] - l[:, K]
+    n = l.shape[0]
+    boundary = l[:, K - 1] - l[:, K] if K < l.shape[1] else np.full(n, np.inf)
+    top = l[:, :min(K + 1, l.shape[1])]
+    order = np.min(top[:, :-1] - top[:, 1:], axis=1) if top.shape[1] > 1 else np.full(n, np.inf)
+    return boundary, order
