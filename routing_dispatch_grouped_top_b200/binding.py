@@ -14,7 +14,8 @@ from typing import Optional, Sequence
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
+# MOE_B200_LIB may name another build of the same library (e.g. a tuning variant).
+LIB_PATH = os.environ.get("MOE_B200_LIB") or os.path.join(_HERE, "libmoe_b200.so")
 
 MOE_NUM_STAGE_EVENTS = 10
 STAGE_NAMES = ["latent_down", "gating", "route", "count_scan", "permute", "gate_up", "down", "combine",

@@ -18,7 +18,7 @@
 // tile at run time.
 //
 // Roles (192 threads, one CTA per SM, persistent over a static tile order):
-//   warp 0      TMA producer: weight tile(s) 128 x 64 and token boxes 32 x 64,
+//   warp 0      TMA producer: weight tile(s) 128 x 64 and token boxes (16..256) x 64,
 //               128-byte swizzle, into a STAGES-deep ring of shared memory;
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer;
 //   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp reads
@@ -40,7 +40,12 @@ namespace {
 constexpr int kBM = 128;                  // output features per tile (MMA M)
 constexpr int kBK = 64;                   // K per stage: one 128-byte swizzle atom of bf16
 constexpr int kABytes = kBM * kBK * 2;    // 16 KB per weight tile
-constexpr int kBoxB = 32;                 // token rows per TMA box of the B operand
+// The token operand of a tile (nround rows, a multiple of 16) is fetched with one TMA box
+// per set bit of nround / 16: boxes of 256, 128, 64, 32 and 16 rows, at most 4 per stage.
+constexpr int kNumBoxes = 5;
+struct BoxMaps {
+  CUtensorMap box[kNumBoxes];  // box[i] is (256 >> i) rows x 64 columns
+};
 constexpr int kThreads = 192;
 constexpr int kEpiThreads = 128;
 constexpr int kMaxGroups = MOE_MAX_E;
@@ -48,15 +53,23 @@ constexpr int kMaxGroups = MOE_MAX_E;
 template <int EPI>
 struct Cfg;
 // SwiGLU: gate and up tiles share one token tile; two accumulators per tile.
+#ifndef MOE_SWIGLU_NT
+#define MOE_SWIGLU_NT 128
+#define MOE_SWIGLU_STAGES 4
+#endif
+#ifndef MOE_BF16_NT
+#define MOE_BF16_NT 256
+#define MOE_BF16_STAGES 4
+#endif
 template <>
 struct Cfg<kEpiSwiGLU> {
-  static constexpr int NA = 2, NT = 128, STAGES = 4;
+  static constexpr int NA = 2, NT = MOE_SWIGLU_NT, STAGES = MOE_SWIGLU_STAGES;
   static constexpr bool SEP = true;
 };
 // Plain bf16 output (down projection, latent projections).
 template <>
 struct Cfg<kEpiBF16> {
-  static constexpr int NA = 1, NT = 256, STAGES = 4;
+  static constexpr int NA = 1, NT = MOE_BF16_NT, STAGES = MOE_BF16_STAGES;
   static constexpr bool SEP = false;
 };
 // fp32 output: three bf16 weight planes accumulated into one fp32 accumulator.
@@ -76,7 +89,7 @@ struct Layout {
   static constexpr int kBarBytes = 8 * (2 * C::STAGES + 5) + 16;
   static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
   static constexpr int kSmemBytes = 1024 + C::STAGES * kStageBytes + kBarBytes + kTableBytes;
-  static_assert(kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
+  static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
 
@@ -84,8 +97,11 @@ struct Tile {
   int g, n0, row0, nvalid, nround;
 };
 
-// Tile t -> (group, weight tile, token chunk).  s_pre[g] = first tile of group g.
-__device__ __forceinline__ Tile decode_tile(int t, const int* s_pre, const int* s_off, int G, int NT) {
+// Tile t -> (group, weight tile, token chunk).  s_pre[g] = first tile of group g.  A group of
+// cnt rows is cut into ceil(cnt / NT) balanced chunks of a multiple of ROUND rows; a weight
+// tile covers FEAT output features.
+template <int NT, int ROUND, int FEAT>
+__device__ __forceinline__ Tile decode_tile(int t, const int* s_pre, const int* s_off, int G) {
   int lo = 0, hi = G;  // s_pre[lo] <= t < s_pre[hi]
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -97,13 +113,13 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* s_pre, const int* 
   const int nch = (cnt + NT - 1) / NT;
   const int ft = local / nch;
   const int c = local - ft * nch;
-  const int sz = (((cnt + nch - 1) / nch) + 15) & ~15;
+  const int sz = (((cnt + nch - 1) / nch) + ROUND - 1) & ~(ROUND - 1);
   Tile r;
   r.g = lo;
-  r.n0 = ft * kBM;
+  r.n0 = ft * FEAT;
   r.row0 = s_off[lo] + c * sz;
   r.nvalid = min(sz, cnt - c * sz);
-  r.nround = (r.nvalid + 15) & ~15;
+  r.nround = (r.nvalid + ROUND - 1) & ~(ROUND - 1);
   return r;
 }
 
@@ -143,7 +159,7 @@ __device__ void build_tile_table(int* s_pre, const int* s_off, int G, int NT, in
 template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                        const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ BoxMaps tmB,
                         const GemmArgs args) {
   using C = Cfg<EPI>;
   using L = Layout<EPI>;
@@ -199,7 +215,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmA0);
-    tma_prefetch_map(&tmB);
+    for (int i = 0; i < kNumBoxes; ++i) tma_prefetch_map(&tmB.box[i]);
   }
   if (warp == 1) {
     tmem_alloc(tmem_slot, L::kTmemCols);
@@ -222,9 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < STAGES; ++s) pend[s] = false, pend_phase[s] = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
-        const Tile tl = decode_tile(t, s_pre, s_off, G, NT);
-        const int nbox = (tl.nround + kBoxB - 1) / kBoxB;
-        const uint32_t bytes = NA * kABytes + nbox * kBoxB * 128;
+        const Tile tl = decode_tile<NT, 16, kBM>(t, s_pre, s_off, G);
+        const uint32_t bytes = NA * kABytes + tl.nround * 128;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
             ok = false;
@@ -239,8 +254,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int z = (EPI == kEpiF32) ? i : tl.g;
             tma_load_3d(st + i * kABytes, m, &full[stage], kx, tl.n0, z);
           }
-          for (int b = 0; b < nbox; ++b)
-            tma_load_2d(st + NA * kABytes + b * kBoxB * 128, &tmB, &full[stage], kx, tl.row0 + b * kBoxB);
+          int r = 0;
+#pragma unroll
+          for (int i = 0; i < kNumBoxes; ++i) {
+            const int rows = 256 >> i;
+            if (tl.nround & rows) {
+              tma_load_2d(st + NA * kABytes + r * 128, &tmB.box[i], &full[stage], kx, tl.row0 + r);
+              r += rows;
+            }
+          }
           pend[stage] = true;
           pend_phase[stage] = phase;
           if (++stage == STAGES) {
@@ -261,7 +283,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
-        const Tile tl = decode_tile(t, s_pre, s_off, G, NT);
+        const Tile tl = decode_tile<NT, 16, kBM>(t, s_pre, s_off, G);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) {
           ok = false;
           break;
@@ -309,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lanes [32q, 32q + 32) are visible to this warp
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = decode_tile(t, s_pre, s_off, G, NT);
+      const Tile tl = decode_tile<NT, 16, kBM>(t, s_pre, s_off, G);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
       const int f = tl.n0 + q * 32 + lane;
@@ -371,6 +393,291 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
+// CTA-pair kernel (cta_group::2): one M = 256 x N (<= 256) MMA per K-step spans the
+// two SMs of a cluster.  Each CTA stages its own 128 weight rows and N/2 token rows
+// (32 KB per stage, 6 stages), so shared-memory traffic per MMA cycle is two thirds of
+// the single-CTA tiles'; the token tile crosses L2 once per pair.  The leader CTA
+// (rank 0) issues the MMAs; both CTAs' TMA loads complete on the leader's "full"
+// barrier, the leader's commits release both CTAs' "empty" and "tmem full" barriers,
+// and both CTAs' epilogues release the leader's "tmem empty" barrier.
+//   SwiGLU: CTA r holds gate rows [f0 + 64 r, +64) over up rows of the same features,
+//           so TMEM lanes 0-63 are gate and 64-127 up; the epilogue warps swap halves of
+//           each 32-token chunk through shared memory (warp q and q + 2 own the gate and
+//           up of the same features).  128 output features per pair tile.
+//   bf16:   CTA r holds weight rows [n0 + 128 r, +128).  256 output features per pair tile.
+// ---------------------------------------------------------------------------
+
+template <int EPI>
+struct PairLayout {
+  static constexpr int NT = 256;                      // token columns per tile (MMA N)
+  static constexpr int STAGES = 6;
+  static constexpr int kFeat = (EPI == kEpiSwiGLU) ? 128 : 256;
+  static constexpr int kABytes = 128 * kBK * 2;       // this CTA's 128 weight rows
+  static constexpr int kBBytes = (NT / 2) * 128;      // this CTA's token rows
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr uint32_t kAccCols = NT;
+  static constexpr uint32_t kTmemCols = 2 * kAccCols;
+  static constexpr int kExchFloats = 2 * 16 * 64;     // one chunk: 16 tokens x 64 features, each direction
+  static constexpr int kExchBytes = (EPI == kEpiSwiGLU) ? 2 * kExchFloats * 4 : 0;  // double-buffered
+  static constexpr int kBarBytes = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
+  static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kExchBytes + kBarBytes + kTableBytes;
+  static_assert(kSmemBytes <= 232448, "shared memory budget");
+};
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
+                     const __grid_constant__ BoxMaps tmB, const GemmArgs args) {
+  using L = PairLayout<EPI>;
+  constexpr int NT = L::NT, STAGES = L::STAGES;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* ring = smem;
+  float* exch = reinterpret_cast<float*>(smem + STAGES * L::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::kStageBytes + L::kExchBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_off = reinterpret_cast<int*>(smem + STAGES * L::kStageBytes + L::kExchBytes + L::kBarBytes);
+  int* s_pre = s_off + (kMaxGroups + 1);
+  __shared__ int s_warp_sums[kThreads / 32];
+  __shared__ int s_bad;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int G = args.offsets ? args.G : 1;
+  const int NFT = (args.N + L::kFeat - 1) / L::kFeat;
+  const int KB = (args.Kd + kBK - 1) / kBK;
+
+  if (threadIdx.x == 0) s_bad = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i <= G; i += kThreads)
+    s_off[i] = args.offsets ? __ldg(args.offsets + i) : (i == 0 ? 0 : args.M);
+  __syncthreads();
+  for (int i = threadIdx.x; i <= G; i += kThreads) {
+    const bool bad = s_off[i] < 0 || s_off[i] > args.M || (i > 0 && s_off[i] < s_off[i - 1]);
+    if (bad) s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (threadIdx.x == 0 && rank == 0) report(args.status, MOE_DEV_BAD_INDEX);
+    for (int i = threadIdx.x; i <= G; i += kThreads) s_off[i] = 0;
+  }
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * (kEpiThreads / 32));  // one arrival per epilogue warp of each CTA
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    mbar_init_fence();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_map(&tmA0);
+    tma_prefetch_map(&tmA1);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, L::kTmemCols);
+    tmem_relinquish_pair();
+    tc_fence_before();
+  }
+  __syncthreads();
+  build_tile_table(s_pre, s_off, G, NT, NFT, s_warp_sums);  // ends with __syncthreads
+  cluster_sync();  // both CTAs' barriers exist before any remote arrival
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_pre[G];
+  const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      uint32_t pend_phase[STAGES];
+      bool pend[STAGES];
+#pragma unroll
+      for (int s = 0; s < STAGES; ++s) pend[s] = false, pend_phase[s] = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < total; t += npairs) {
+        const Tile tl = decode_tile<NT, 32, L::kFeat>(t, s_pre, s_off, G);
+        const int half = tl.nround >> 1;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = ring + stage * L::kStageBytes;
+          const uint32_t bar = full_leader + stage * 8;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kABytes + half * 128));
+          const int kx = kb * kBK;
+          if constexpr (EPI == kEpiSwiGLU) {
+            const int fr = tl.n0 + 64 * static_cast<int>(rank);
+            tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);             // gate rows -> lanes 0..63
+            tma_load_3d_pair(st + L::kABytes / 2, &tmA1, bar, kx, fr, tl.g);  // up rows -> lanes 64..127
+          } else {
+            tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
+          }
+          const int rbase = tl.row0 + static_cast<int>(rank) * half;
+          int r = 0;
+#pragma unroll
+          for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
+            const int rows = 256 >> i;
+            if (half & rows) {
+              tma_load_2d_pair(st + L::kABytes + r * 128, &tmB.box[i], bar, kx, rbase + r);
+              r += rows;
+            }
+          }
+          pend[stage] = true;
+          pend_phase[stage] = phase;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        if (rank == 0) {
+#pragma unroll
+          for (int s = 0; s < STAGES; ++s)
+            if (pend[s]) mbar_drain(&full[s], pend_phase[s], 200000000ull);
+        } else {  // the peer's copies complete on the leader's barrier: give them time to land
+          const uint64_t t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 2000000ull) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader only)
+    if (lane == 0 && rank == 0) {
+      const uint32_t empty_peer = mapa_shared(smem_u32(empty), 1);
+      const uint32_t tfull_peer = mapa_shared(smem_u32(tfull), 1);
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = pair; ok && t < total; t += npairs) {
+        const Tile tl = decode_tile<NT, 32, L::kFeat>(t, s_pre, s_off, G);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t idesc = idesc_bf16_f32(256, tl.nround);
+        const uint32_t d = tmem_base + acc * L::kAccCols;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(ring + stage * L::kStageBytes);
+          const uint32_t sb = sa + L::kABytes;
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16_pair(d, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), idesc,
+                           (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_pair(smem_u32(&empty[stage]));  // both CTAs' stage buffers are free again
+          umma_commit_pair(empty_peer + stage * 8);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit_pair(smem_u32(&tfull[acc]));
+        umma_commit_pair(tfull_peer + acc * 8);
+        acc ^= 1u;
+        if (acc == 0) acc_phase ^= 1u;
+      }
+      if (!ok) {
+        umma_commit_pair(smem_u32(drain));
+        mbar_drain(drain, 0, 200000000ull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    const int q = warp & 3;  // TMEM lanes [32q, 32q + 32)
+    const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
+    uint32_t acc = 0, acc_phase = 0, chunk = 0;
+    for (int t = pair; t < total; t += npairs) {
+      const Tile tl = decode_tile<NT, 32, L::kFeat>(t, s_pre, s_off, G);
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
+      tc_fence_after();
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
+      for (int j0 = 0; j0 < tl.nvalid; j0 += 32, ++chunk) {
+        uint32_t r[32];
+        tmem_ld_32cols(tbase + j0, r);
+        tmem_wait_ld();
+        if constexpr (EPI == kEpiSwiGLU) {
+          // warps q < 2 own gate of features fi, warps q >= 2 own up of the same fi
+          const int fi = 32 * (q & 1) + lane;
+          const bool is_gate = q < 2;
+          float* xb = exch + (chunk & 1) * L::kExchFloats;
+          float* to_up = xb;                 // gate of tokens 16..31, read by the up owner
+          float* to_gate = xb + 16 * 64;     // up of tokens 0..15, read by the gate owner
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            if (is_gate) to_up[j * 64 + fi] = __uint_as_float(r[16 + j]);
+            else to_gate[j * 64 + fi] = __uint_as_float(r[j]);
+          }
+          named_bar_sync(1, kEpiThreads);
+          const int f = tl.n0 + 64 * static_cast<int>(rank) + fi;
+          const int jbase = is_gate ? 0 : 16;
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.out);
+          if (f < args.N) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int tok = j0 + jbase + j;
+              if (tok < tl.nvalid) {
+                const float g = is_gate ? __uint_as_float(r[j]) : to_up[j * 64 + fi];
+                const float u = is_gate ? to_gate[j * 64 + fi] : __uint_as_float(r[16 + j]);
+                const float h = g / (1.0f + __expf(-g)) * u;
+                out[static_cast<long long>(tl.row0 + tok) * args.ldo + f] = __float2bfloat16_rn(h);
+              }
+            }
+          }
+        } else {
+          const int f = tl.n0 + 128 * static_cast<int>(rank) + q * 32 + lane;
+          const int jn = min(32, tl.nvalid - j0);
+          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.out);
+          if (f < args.N) {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+              if (j < jn)
+                out[static_cast<long long>(tl.row0 + j0 + j) * args.ldo + f] = __float2bfloat16_rn(__uint_as_float(r[j]));
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_cluster(tempty_leader + acc * 8);
+      }
+      acc ^= 1u;
+      if (acc == 0) acc_phase ^= 1u;
+    }
+  }
+
+  __syncthreads();
+  cluster_sync();  // no CTA leaves while its peer may still touch its barriers or smem
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, L::kTmemCols);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------
 
@@ -416,8 +723,14 @@ bool map_bf16_2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uin
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+bool map_token_boxes(BoxMaps* m, const void* base, uint64_t d0, uint64_t rows) {
+  for (int i = 0; i < kNumBoxes; ++i)
+    if (!map_bf16_2d(&m->box[i], base, d0, rows, 256u >> i)) return false;
+  return true;
+}
+
 template <int EPI>
-cudaError_t launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const CUtensorMap& b,
+cudaError_t launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const BoxMaps& b,
                    const GemmArgs& args, long long tile_bound, cudaStream_t stream) {
   using L = Layout<EPI>;
   static std::once_flag once;
@@ -433,8 +746,25 @@ cudaError_t launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   return cudaGetLastError();
 }
 
-long long tile_bound(long long rows, int groups, int NT, int N) {
-  const long long nft = (N + kBM - 1) / kBM;
+template <int EPI>
+cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const BoxMaps& b, const GemmArgs& args,
+                        long long tile_bound, cudaStream_t stream) {
+  using L = PairLayout<EPI>;
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(pair_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    L::kSmemBytes);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  if (tile_bound <= 0) return cudaSuccess;
+  const int pairs = static_cast<int>(std::min<long long>(num_sms() / 2, tile_bound));
+  pair_gemm_kernel<EPI><<<2 * pairs, kThreads, L::kSmemBytes, stream>>>(a0, a1, b, args);
+  return cudaGetLastError();
+}
+
+long long tile_bound(long long rows, int groups, int NT, int N, int feat) {
+  const long long nft = (N + feat - 1) / feat;
   return ((rows + NT - 1) / NT + (groups > 1 ? groups : 0)) * nft;
 }
 
@@ -448,43 +778,60 @@ int gemm_smem_bytes(int epi) {
   }
 }
 
+// The CTA-pair kernel is correct (it passes the same parity tests when built with
+// MOE_GEMM_PAIR=1) and faster on long-K dense shapes, but slower than the single-CTA
+// kernel on the layer workloads measured so far, so the single-CTA kernel is the default.
+#ifndef MOE_GEMM_PAIR
+#define MOE_GEMM_PAIR 0
+#endif
+
 // h = silu(xp Wg^T) * (xp Wu^T) per expert group.
 cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
                          long long rows, int H, int F, void* h, int* status, cudaStream_t stream) {
-  CUtensorMap a0, a1, b;
-  if (!map_bf16_3d(&a0, w_gate, H, F, E, kBM) || !map_bf16_3d(&a1, w_up, H, F, E, kBM) ||
-      !map_bf16_2d(&b, xp, H, rows, kBoxB))
-    return cudaErrorInvalidValue;
   GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status};
-  return launch<kEpiSwiGLU>(a0, a1, a1, b, args, tile_bound(rows, E, Cfg<kEpiSwiGLU>::NT, F), stream);
+  CUtensorMap a0, a1;
+  BoxMaps b;
+  if (!map_token_boxes(&b, xp, H, rows)) return cudaErrorInvalidValue;
+  if (MOE_GEMM_PAIR) {
+    if (!map_bf16_3d(&a0, w_gate, H, F, E, 64) || !map_bf16_3d(&a1, w_up, H, F, E, 64)) return cudaErrorInvalidValue;
+    return launch_pair<kEpiSwiGLU>(a0, a1, b, args, tile_bound(rows, E, PairLayout<kEpiSwiGLU>::NT, F, 128), stream);
+  }
+  if (!map_bf16_3d(&a0, w_gate, H, F, E, kBM) || !map_bf16_3d(&a1, w_up, H, F, E, kBM)) return cudaErrorInvalidValue;
+  return launch<kEpiSwiGLU>(a0, a1, a1, b, args, tile_bound(rows, E, Cfg<kEpiSwiGLU>::NT, F, kBM), stream);
 }
 
 // y = h Wd^T per expert group.
 cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down, int E, long long rows, int H,
                       int F, void* y, int* status, cudaStream_t stream) {
-  CUtensorMap a0, b;
-  if (!map_bf16_3d(&a0, w_down, F, H, E, kBM) || !map_bf16_2d(&b, h, F, rows, kBoxB))
-    return cudaErrorInvalidValue;
   GemmArgs args{offsets, E, static_cast<int>(rows), H, F, y, H, nullptr, status};
-  return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(rows, E, Cfg<kEpiBF16>::NT, H), stream);
+  CUtensorMap a0;
+  BoxMaps b;
+  if (!map_bf16_3d(&a0, w_down, F, H, E, kBM) || !map_token_boxes(&b, h, F, rows)) return cudaErrorInvalidValue;
+  if (MOE_GEMM_PAIR)
+    return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(rows, E, PairLayout<kEpiBF16>::NT, H, 256), stream);
+  return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(rows, E, Cfg<kEpiBF16>::NT, H, kBM), stream);
 }
 
 // out[M][N] = a[M][Kd] w[N][Kd]^T, bf16 out.
 cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd, void* out, int* status,
                        cudaStream_t stream) {
-  CUtensorMap a0, b;
-  if (!map_bf16_3d(&a0, w, Kd, N, 1, kBM) || !map_bf16_2d(&b, a, Kd, M, kBoxB)) return cudaErrorInvalidValue;
+  CUtensorMap a0;
+  BoxMaps b;
+  if (!map_bf16_3d(&a0, w, Kd, N, 1, kBM) || !map_token_boxes(&b, a, Kd, M)) return cudaErrorInvalidValue;
   GemmArgs args{nullptr, 1, static_cast<int>(M), N, Kd, out, N, nullptr, status};
-  return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(M, 1, Cfg<kEpiBF16>::NT, N), stream);
+  if (MOE_GEMM_PAIR)
+    return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(M, 1, PairLayout<kEpiBF16>::NT, N, 256), stream);
+  return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(M, 1, Cfg<kEpiBF16>::NT, N, kBM), stream);
 }
 
 // logits[T][E] = x[T][H] (hi + mid + lo)^T (+ bias), fp32 out; w_split is [3][E][H] bf16.
 cudaError_t gemm_gating(const void* x, const void* w_split, const float* bias, long long T, int H, int E,
                         float* logits, int* status, cudaStream_t stream) {
-  CUtensorMap a0, b;
-  if (!map_bf16_3d(&a0, w_split, H, E, 3, kBM) || !map_bf16_2d(&b, x, H, T, kBoxB)) return cudaErrorInvalidValue;
+  CUtensorMap a0;
+  BoxMaps b;
+  if (!map_bf16_3d(&a0, w_split, H, E, 3, kBM) || !map_token_boxes(&b, x, H, T)) return cudaErrorInvalidValue;
   GemmArgs args{nullptr, 1, static_cast<int>(T), E, H, logits, E, bias, status};
-  return launch<kEpiF32>(a0, a0, a0, b, args, tile_bound(T, 1, Cfg<kEpiF32>::NT, E), stream);
+  return launch<kEpiF32>(a0, a0, a0, b, args, tile_bound(T, 1, Cfg<kEpiF32>::NT, E, kBM), stream);
 }
 
 }  // namespace moe
