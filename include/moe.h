@@ -153,6 +153,31 @@ moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* c
                           int32_t* row_of_assign, int32_t* assign_of_row,
                           void* ws, size_t ws_bytes, void* stream);
 
+/* Bytes of device memory that moe_count_scan_noalloc keeps as its scratch.  Every GPU
+ * that loads this library holds them until the process exits. */
+#define MOE_NOALLOC_SCRATCH_BYTES (1u << 20)
+
+/* moe_count_scan without a caller workspace (the source pages have no counterpart for
+ * this call; it exists for callers that cannot allocate device memory: a plugin inside
+ * a host framework that owns every device allocation, or a real-time loop that may not
+ * call cudaMalloc/cudaFree, which can also synchronize the device, once it runs).
+ * Same arguments and results as moe_count_scan minus the workspace.  The scratch is a
+ * fixed device array inside the library: 256 bytes of status and grid-barrier words
+ * plus one E-entry int32 histogram per block (ceil(T*K / 1024) blocks, at most 1024),
+ * at most MOE_NOALLOC_SCRATCH_BYTES in all; larger shapes return
+ * MOE_ERR_UNSUPPORTED_SHAPE (with E = 1024 up to T*K = 261 120 assignments).
+ * The call allocates nothing: it clears the scratch's status and barrier words with
+ * an async memset on `stream`, then launches the count/scan kernel.  The first call on
+ * a device looks up the scratch's device address once (with that device current);
+ * make that first call before any stream capture.  All calls share the one scratch
+ * and it keeps the last call's contents, so calls that overlap on the GPU (other
+ * streams, other host threads) race: serialize them.  Device-side conditions are not
+ * reported back (no workspace to read): an id outside [0, E) shows up as row -1 in
+ * row_of_assign. */
+moe_status moe_count_scan_noalloc(const int32_t* topk_ids, const moe_dims* d, int32_t* counts,
+                                  int32_t* offsets, int32_t* part_counts, int32_t* part_offsets,
+                                  int32_t* row_of_assign, int32_t* assign_of_row, void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* S3  Permute into destination-contiguous rows + routing metadata           */
 /* "permutes token activations into destination-contiguous buffers, attaches */

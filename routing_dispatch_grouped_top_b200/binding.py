@@ -59,6 +59,7 @@ _SIGS = {
     "moe_gating": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
     "moe_route": (C.c_int, [_VP, _DP, _VP, _VP, _VP]),
     "moe_count_scan": (C.c_int, [_VP, _DP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
+    "moe_count_scan_noalloc": (C.c_int, [_VP, _DP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_permute": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_grouped_ffn": (C.c_int, [_VP, _VP, _VP, _VP, _VP, _DP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_gate_up": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
@@ -189,6 +190,19 @@ def moe_count_scan(topk_ids, d: moe_dims, counts, offsets, part_counts, part_off
         _ptr(row_of_assign, torch.int32, "row_of_assign", TK),
         _ptr(assign_of_row, torch.int32, "assign_of_row", TK), _ptr(ws, torch.uint8, "ws"), ws.numel(),
         _stream(stream)))
+
+
+def moe_count_scan_noalloc(topk_ids, d: moe_dims, counts, offsets, part_counts, part_offsets, row_of_assign,
+                           assign_of_row, stream=None):
+    """moe_count_scan for callers that cannot allocate: the library's own fixed scratch
+    replaces the workspace (see include/moe.h for its limit and sharing rules)."""
+    TK = d.T * d.K
+    _check("moe_count_scan_noalloc", lib().moe_count_scan_noalloc(
+        _ptr(topk_ids, torch.int32, "topk_ids", TK), C.byref(d), _ptr(counts, torch.int32, "counts", d.E),
+        _ptr(offsets, torch.int32, "offsets", d.E + 1), _ptr(part_counts, torch.int32, "part_counts", d.P),
+        _ptr(part_offsets, torch.int32, "part_offsets", d.P + 1),
+        _ptr(row_of_assign, torch.int32, "row_of_assign", TK),
+        _ptr(assign_of_row, torch.int32, "assign_of_row", TK), _stream(stream)))
 
 
 def moe_permute(x, row_of_assign, topk_ids, topk_w, d: moe_dims, xp, meta_token=None, meta_slot=None,
