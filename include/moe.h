@@ -1,16 +1,18 @@
 /*
  * moe.h - C ABI of the B200 (sm_100a) routed Mixture-of-Experts layer.
  *
- * One routed MoE layer on one GPU, in the order the "WideEP: Wide Expert
- * Parallelism and Kimi K3" essay gives in its section "The router writes a
- * network schedule": gating scores and top-k expert ids; count destinations
- * and allocate slots; permute token activations into destination-contiguous
- * buffers and attach routing metadata; run the experts' matrix multiplies per
- * local expert; combine reverses the route, unpermutes and applies the routing
- * weights.  The same essay's table of communication regimes (row "Same GPU":
- * no fabric hop, still a permute and HBM traffic; fused layouts, grouped GEMM)
- * is the regime of this library: logical expert-parallel partitions are only a
- * buffer layout, nothing is transferred between GPUs.
+ * One routed MoE layer on one GPU, following the pipeline of the "WideEP: Wide
+ * Expert Parallelism and Kimi K3" essay, section "The router writes a network
+ * schedule": the router scores every expert and keeps the top K per token; the
+ * dispatcher counts the assignments bound for each destination, reserves their
+ * rows and gathers the activations into one contiguous block per destination,
+ * with routing metadata per row; each expert multiplies its block; the combine
+ * step brings every output back to its token and sums the K of them with the
+ * routing weights.  The essay's table of communication regimes says that local
+ * (same-GPU) assignments avoid the fabric but still pay the permute's HBM
+ * traffic, and points to fused layouts and grouped GEMM: that is the regime of
+ * this library.  Logical expert-parallel partitions are only a buffer layout;
+ * nothing is transferred between GPUs.
  *
  * Notation (the pages' statement of the problem): T tokens, E experts, top-K,
  * H dispatch width, F expert FFN width, b = 2 bytes per bf16 activation,
@@ -99,9 +101,9 @@ const char* moe_status_str(moe_status s);
 
 /* ------------------------------------------------------------------------- */
 /* S0  Gating logits                                                         */
-/* "The source rank computes the gating scores" (WideEP essay, "The router   */
-/* writes a network schedule"); the gating network is replicated non-expert  */
-/* work (InferenceX v2 review claim IX2-0406).                               */
+/* The sending rank scores each token against every expert (WideEP essay,   */
+/* "The router writes a network schedule"); the gating network is non-expert */
+/* work every rank replicates (InferenceX v2 review, claim IX2-0406).        */
 /* ------------------------------------------------------------------------- */
 
 /* One-time weight preparation: splits the fp32 router W_g [H][E] into three
@@ -119,7 +121,7 @@ moe_status moe_gating(const void* x, const void* w_g_split, const float* bias,
 
 /* ------------------------------------------------------------------------- */
 /* S1  Router top-K + routing weights                                        */
-/* "computes the gating scores and top-k expert IDs" (WideEP essay, "The     */
+/* Per-token choice of the K best-scoring experts (WideEP essay, "The       */
 /* router writes a network schedule").                                       */
 /* ------------------------------------------------------------------------- */
 
@@ -132,10 +134,10 @@ moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids,
 
 /* ------------------------------------------------------------------------- */
 /* S2  Count destinations, allocate slots                                    */
-/* "A dispatcher counts destinations, allocates or selects communication     */
-/* slots" (WideEP essay); per-expert assignment counts, "assignments, not    */
-/* unique tokens" ("Three Parameter Counts...", "What the utilization        */
-/* dashboard smooths away").                                                 */
+/* Counting what each expert receives and reserving its rows (WideEP essay, */
+/* "The router writes a network schedule"); counts are of token-expert       */
+/* assignments, so a token routed to K experts counts K times ("Three        */
+/* Parameter Counts...", "What the utilization dashboard smooths away").     */
 /* ------------------------------------------------------------------------- */
 
 /* topk_ids: [T][K] int32.  Out (all int32):
@@ -180,9 +182,10 @@ moe_status moe_count_scan_noalloc(const int32_t* topk_ids, const moe_dims* d, in
 
 /* ------------------------------------------------------------------------- */
 /* S3  Permute into destination-contiguous rows + routing metadata           */
-/* "permutes token activations into destination-contiguous buffers, attaches */
-/* routing metadata" (WideEP essay); payload T x K x H x b ("Top-k           */
-/* multiplies traffic"; "Three Parameter Counts...", "Halving top-k is a     */
+/* Gathering each destination's activations into one contiguous block with */
+/* per-row routing metadata (WideEP essay, "The router writes a network     */
+/* schedule"); the block holds T x K x H x b bytes (same essay, "Top-k      */
+/* multiplies traffic"; "Three Parameter Counts...", "Halving top-k is a    */
 /* network change first").                                                  */
 /* ------------------------------------------------------------------------- */
 
@@ -200,10 +203,10 @@ moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_
 
 /* ------------------------------------------------------------------------- */
 /* S4 + S5  Expert SwiGLU FFN as grouped GEMMs over variable row counts      */
-/* "The receiver groups tokens by local expert and launches expert matrix    */
-/* multiplies" (WideEP essay); grouped GEMM runs several expert matrices in  */
-/* one launch despite differing row counts ("Three Parameter Counts...",     */
-/* "Which optimizations need a task-level gate").                            */
+/* Each expert multiplies the rows routed to it (WideEP essay, "The router  */
+/* writes a network schedule"); one grouped launch serves every expert,      */
+/* whatever its row count ("Three Parameter Counts...", "Which               */
+/* optimizations need a task-level gate").                                   */
 /* ------------------------------------------------------------------------- */
 
 /* For every expert e and row r in [offsets[e], offsets[e+1]):
@@ -229,8 +232,9 @@ moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w
 
 /* ------------------------------------------------------------------------- */
 /* S6  Combine: unpermute + weighted sum                                     */
-/* "A combine phase reverses the route, after which the source rank          */
-/* unpermutes and applies routing weights" (WideEP essay).                   */
+/* Every expert output goes back to its token and the K outputs are summed */
+/* with the routing weights (WideEP essay, "The router writes a network     */
+/* schedule").                                                               */
 /* ------------------------------------------------------------------------- */
 
 /* out[t][:] = bf16( sum_{k<K} topk_w[t][k] * y[row_of_assign[t*K+k]][:] ),
@@ -240,9 +244,9 @@ moe_status moe_combine(const void* y, const int32_t* row_of_assign, const float*
 
 /* ------------------------------------------------------------------------- */
 /* S7  Skew statistics                                                       */
-/* "Skew ratio at p95: max expert load divided by mean expert load"          */
-/* ("Three Parameter Counts...", "What the utilization dashboard smooths     */
-/* away").                                                                   */
+/* Load skew = the busiest expert's load over the mean load, followed at    */
+/* its 95th percentile over steps ("Three Parameter Counts...", "What the   */
+/* utilization dashboard smooths away").                                     */
 /* ------------------------------------------------------------------------- */
 
 /* *d_ratio (device fp32) = max_e counts[e] / (sum_e counts[e] / E); 0 if no rows. */

@@ -12,31 +12,33 @@ and section:
 
 * [WideEP/router]  "WideEP: Wide Expert Parallelism and Kimi K3" essay
   (manishklach.github.io/writings/wideep-kimi-expert-parallelism), section
-  "The router writes a network schedule": gating scores and top-k expert ids;
-  count destinations; allocate slots; permute activations into
-  destination-contiguous buffers with routing metadata; group by local expert;
-  expert matrix multiplies; combine reverses the route; unpermute and apply
-  routing weights.
+  "The router writes a network schedule": the pipeline of a routed layer
+  (score experts and keep the top k; count each destination's assignments and
+  reserve their slots; gather activations per destination with routing
+  metadata; run each expert on its rows; send outputs back, undo the
+  permutation and weight them).
 * [WideEP/bytes]  same essay, section "Top-k multiplies traffic. Locality
-  subtracts it.": dispatch moves about T x k x H x B bytes, combine a similar
-  volume.
-* [WideEP/regimes]  same essay, table of communication regimes, row "Same GPU":
-  no fabric hop, still a permute and HBM traffic; fused layouts, grouped GEMM.
-* [WideEP/placement]  same essay, section "896 experts across 64 ranks":
-  experts evenly placed over the EP ranks (896 / 64 = 14 per rank).
+  subtracts it.": one dispatch carries about T x k x H x B activation bytes
+  and the combine about as many.
+* [WideEP/regimes]  same essay, table of communication regimes: assignments
+  that stay on the same GPU cross no fabric but still cost a permute in HBM.
+* [WideEP/placement]  same essay, section "896 experts across 64 ranks": an
+  even split of the experts over the ranks (896 / 64 = 14 per rank).
 * [ParamCounts/network]  "Three Parameter Counts, and Only One Tells You Whether
   the Model Fits" (clarity-us-archive, 2026-09-24 science edition), section
-  "Halving top-k is a network change first": payload bound T x K x H x b.
+  "Halving top-k is a network change first": the dispatch payload is bounded by
+  T x K x H x b.
 * [ParamCounts/dashboard]  same article, section "What the utilization
-  dashboard smooths away": per-expert assignment counts (assignments, not unique
-  tokens), skew ratio at p95 = max expert load / mean expert load.
+  dashboard smooths away": count per expert every token-expert assignment, and
+  watch the busiest expert's load over the mean load at its 95th percentile.
 * [ParamCounts/gate]  same article, section "Which optimizations need a
-  task-level gate": grouped GEMM runs several expert matrices in one launch
-  despite different row counts and must preserve expert selection.
+  task-level gate": a grouped GEMM serves experts with different row counts in
+  one launch and leaves the expert selection unchanged.
 * [LatentMoE]  "Latent MoE" concept page (podcastatlas.ai wiki), sections
-  "Definition" and "Current Synthesis": dispatch on a reduced latent width.
+  "Definition" and "Current Synthesis": experts receive a narrower, projected
+  hidden state.
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
 
 * Top-k order: a beats b iff value(a) > value(b), or the values compare equal
   and id(a) < id(b).  -0.0 equals +0.0; NaN ranks below every number (also

@@ -1,13 +1,13 @@
 // dispatch.cu - permute (dispatch into expert-contiguous rows + routing
 // metadata), combine (unpermute + weighted sum) and the one-time router split.
 //
-// "permutes token activations into destination-contiguous buffers, attaches
-// routing metadata ... A combine phase reverses the route, after which the
-// source rank unpermutes and applies routing weights" (WideEP essay, "The
-// router writes a network schedule").  On one GPU this is the "Same GPU" row of
-// the essay's regime table: no fabric hop, but a permute and its HBM traffic,
-// T x K x H x b bytes out and a similar volume back ("Top-k multiplies
-// traffic").
+// The dispatcher gathers each destination's activations into one contiguous
+// block with routing metadata per row, and the combine step returns every
+// expert output to its token and sums them with the routing weights (WideEP
+// essay, "The router writes a network schedule").  On one GPU no fabric is
+// crossed, but the permute still moves T x K x H x b bytes through HBM and the
+// combine about as many back (same essay: its regime table and "Top-k
+// multiplies traffic").
 //
 // Both copy kernels are HBM-bound.  They work on 16-byte vectors (8 bf16): the
 // item space is (token, vector) flattened, so consecutive threads touch

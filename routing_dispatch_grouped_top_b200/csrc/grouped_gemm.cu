@@ -3,11 +3,10 @@
 // routed MoE layer), plus its dense single-group uses (gating, latent
 // projections).
 //
-// "The receiver groups tokens by local expert and launches expert matrix
-// multiplies" (WideEP essay, "The router writes a network schedule"); "Grouped
-// GEMM ... runs several expert matrices in one launch and cuts launch overhead
-// even when row counts differ" ("Three Parameter Counts...", "Which
-// optimizations need a task-level gate").
+// Each expert multiplies the rows routed to it (WideEP essay, "The router
+// writes a network schedule"); a grouped GEMM serves all experts in a single
+// launch whatever their row counts, without changing those counts ("Three
+// Parameter Counts...", "Which optimizations need a task-level gate").
 //
 // Orientation: the weight rows (output features) are the MMA's M side (128 per
 // tile) and an expert's tokens are its N side (a multiple of 16, at most NT per

@@ -1,11 +1,10 @@
 // routing.cu - router top-K, per-expert count + stable scan, skew statistics.
 //
-// "The source rank computes the gating scores and top-k expert IDs.  A
-// dispatcher counts destinations, allocates or selects communication slots"
-// (WideEP essay, "The router writes a network schedule").  Counts are of
-// assignments, not unique tokens, and the skew ratio is max expert load over
-// mean expert load ("Three Parameter Counts...", "What the utilization
-// dashboard smooths away").
+// The router keeps the K best-scoring experts of each token, and the dispatcher
+// counts what every expert receives and reserves its rows (WideEP essay, "The
+// router writes a network schedule").  Counts are per token-expert assignment
+// and the skew statistic is the busiest expert's load over the mean load
+// ("Three Parameter Counts...", "What the utilization dashboard smooths away").
 #include <cuda/atomic>
 
 #include <algorithm>
