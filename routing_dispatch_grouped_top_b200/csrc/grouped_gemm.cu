@@ -52,29 +52,33 @@ constexpr int kMaxGroups = MOE_MAX_E;
 template <int EPI>
 struct Cfg;
 // SwiGLU: gate and up tiles share one token tile; two accumulators per tile.
-#ifndef MOE_SWIGLU_NT
-#define MOE_SWIGLU_NT 128
-#define MOE_SWIGLU_STAGES 4
-#endif
-#ifndef MOE_BF16_NT
-#define MOE_BF16_NT 256
-#define MOE_BF16_STAGES 4
-#endif
+// NA weight tiles of 128 rows per stage share one token tile of NT rows.  SEP: each
+// weight tile has its own accumulator (SwiGLU: gate and up; wide bf16 tiles: rows
+// 0-127 and 128-255 of the output features); otherwise all accumulate into one.
+// FEAT output features per tile.  Accumulators are double-buffered in TMEM when two fit
+// in its 512 columns (the epilogue of one tile then overlaps the next tile's main loop).
+//
+// Measured on B200: the per-SM rate at which TMA can fill shared memory, not the MMA,
+// bounds these kernels; a 128 x 256 tile needs 48 KB per 542 MMA cycles.  The bf16
+// kernel therefore uses 256 x 256 tiles (two 128-row weight tiles, 42 B per MMA cycle),
+// single-buffered, which measured 15-30 % faster than 128 x 256 on every workload.  For
+// SwiGLU the same widening was slower (its epilogue is heavier and no longer overlapped),
+// so it keeps 128 x (128 gate + 128 up) tiles with double-buffered accumulators.
 template <>
 struct Cfg<kEpiSwiGLU> {
-  static constexpr int NA = 2, NT = MOE_SWIGLU_NT, STAGES = MOE_SWIGLU_STAGES;
+  static constexpr int NA = 2, NT = 128, STAGES = 4, FEAT = 128;
   static constexpr bool SEP = true;
 };
 // Plain bf16 output (down projection, latent projections).
 template <>
 struct Cfg<kEpiBF16> {
-  static constexpr int NA = 1, NT = MOE_BF16_NT, STAGES = MOE_BF16_STAGES;
-  static constexpr bool SEP = false;
+  static constexpr int NA = 2, NT = 256, STAGES = 3, FEAT = 256;
+  static constexpr bool SEP = true;
 };
 // fp32 output: three bf16 weight planes accumulated into one fp32 accumulator.
 template <>
 struct Cfg<kEpiF32> {
-  static constexpr int NA = 3, NT = 128, STAGES = 3;
+  static constexpr int NA = 3, NT = 128, STAGES = 3, FEAT = 128;
   static constexpr bool SEP = false;
 };
 
@@ -84,7 +88,8 @@ struct Layout {
   static constexpr int kBBytes = C::NT * 128;
   static constexpr int kStageBytes = C::NA * kABytes + kBBytes;
   static constexpr int kAccCols = C::SEP ? C::NA * C::NT : C::NT;
-  static constexpr uint32_t kTmemCols = 2 * kAccCols;
+  static constexpr int kNumAcc = (2 * kAccCols <= 512) ? 2 : 1;
+  static constexpr uint32_t kTmemCols = kNumAcc * kAccCols;
   static constexpr int kBarBytes = 8 * (2 * C::STAGES + 5) + 16;
   static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
   static constexpr int kSmemBytes = 1024 + C::STAGES * kStageBytes + kBarBytes + kTableBytes;
@@ -180,7 +185,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.offsets ? args.G : 1;
-  const int NFT = (args.N + kBM - 1) / kBM;
+  const int NFT = (args.N + C::FEAT - 1) / C::FEAT;
   const int KB = (args.Kd + kBK - 1) / kBK;
 
   __shared__ int s_bad;
@@ -237,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int s = 0; s < STAGES; ++s) pend[s] = false, pend_phase[s] = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
-        const Tile tl = decode_tile<NT, 16, kBM>(t, s_pre, s_off, G);
+        const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
         const uint32_t bytes = NA * kABytes + tl.nround * 128;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
@@ -251,7 +256,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int i = 0; i < NA; ++i) {
             const CUtensorMap* m = (i == 0) ? &tmA0 : ((i == 1) ? &tmA1 : &tmA2);
             const int z = (EPI == kEpiF32) ? i : tl.g;
-            tma_load_3d(st + i * kABytes, m, &full[stage], kx, tl.n0, z);
+            const int row = (EPI == kEpiBF16) ? tl.n0 + i * kBM : tl.n0;  // wide bf16: rows n0 + 128 i
+            tma_load_3d(st + i * kABytes, m, &full[stage], kx, row, z);
           }
           int r = 0;
 #pragma unroll
@@ -282,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
       bool ok = true;
       for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
-        const Tile tl = decode_tile<NT, 16, kBM>(t, s_pre, s_off, G);
+        const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) {
           ok = false;
           break;
@@ -317,8 +323,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         umma_commit(&tfull[acc]);
-        acc ^= 1u;
-        if (acc == 0) acc_phase ^= 1u;
+        if (++acc == L::kNumAcc) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       if (!ok) {  // wait for the MMAs already issued before TMEM is released
         umma_commit(drain);
@@ -330,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;  // TMEM lanes [32q, 32q + 32) are visible to this warp
     uint32_t acc = 0, acc_phase = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = decode_tile<NT, 16, kBM>(t, s_pre, s_off, G);
+      const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
       const int f = tl.n0 + q * 32 + lane;
@@ -365,6 +373,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; ++j)
               if (j < jn) out[(row0 + j) * args.ldo + f] = __float2bfloat16_rn(__uint_as_float(r0[j]));
           }
+          if constexpr (C::SEP) {  // wide tile: second accumulator = features n0 + 128 ..
+            uint32_t r1[32];
+            tmem_ld_32cols(tbase + NT + j0, r1);
+            tmem_wait_ld();
+            const int f1 = f + kBM;
+            if (f1 < args.N) {
+#pragma unroll
+              for (int j = 0; j < 32; ++j)
+                if (j < jn) out[(row0 + j) * args.ldo + f1] = __float2bfloat16_rn(__uint_as_float(r1[j]));
+            }
+          }
         } else {
           tmem_wait_ld();
           float* out = reinterpret_cast<float*>(args.out);
@@ -378,8 +397,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       mbar_arrive(&tempty[acc]);
-      acc ^= 1u;
-      if (acc == 0) acc_phase ^= 1u;
+      if (++acc == L::kNumAcc) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
 
@@ -796,7 +817,7 @@ cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_g
     return launch_pair<kEpiSwiGLU>(a0, a1, b, args, tile_bound(rows, E, PairLayout<kEpiSwiGLU>::NT, F, 128), stream);
   }
   if (!map_bf16_3d(&a0, w_gate, H, F, E, kBM) || !map_bf16_3d(&a1, w_up, H, F, E, kBM)) return cudaErrorInvalidValue;
-  return launch<kEpiSwiGLU>(a0, a1, a1, b, args, tile_bound(rows, E, Cfg<kEpiSwiGLU>::NT, F, kBM), stream);
+  return launch<kEpiSwiGLU>(a0, a1, a1, b, args, tile_bound(rows, E, Cfg<kEpiSwiGLU>::NT, F, Cfg<kEpiSwiGLU>::FEAT), stream);
 }
 
 // y = h Wd^T per expert group.
@@ -808,7 +829,7 @@ cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down,
   if (!map_bf16_3d(&a0, w_down, F, H, E, kBM) || !map_token_boxes(&b, h, F, rows)) return cudaErrorInvalidValue;
   if (MOE_GEMM_PAIR)
     return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(rows, E, PairLayout<kEpiBF16>::NT, H, 256), stream);
-  return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(rows, E, Cfg<kEpiBF16>::NT, H, kBM), stream);
+  return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(rows, E, Cfg<kEpiBF16>::NT, H, Cfg<kEpiBF16>::FEAT), stream);
 }
 
 // out[M][N] = a[M][Kd] w[N][Kd]^T, bf16 out.
@@ -820,7 +841,7 @@ cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd,
   GemmArgs args{nullptr, 1, static_cast<int>(M), N, Kd, out, N, nullptr, status};
   if (MOE_GEMM_PAIR)
     return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(M, 1, PairLayout<kEpiBF16>::NT, N, 256), stream);
-  return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(M, 1, Cfg<kEpiBF16>::NT, N, kBM), stream);
+  return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(M, 1, Cfg<kEpiBF16>::NT, N, Cfg<kEpiBF16>::FEAT), stream);
 }
 
 // logits[T][E] = x[T][H] (hi + mid + lo)^T (+ bias), fp32 out; w_split is [3][E][H] bf16.
