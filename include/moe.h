@@ -223,6 +223,21 @@ moe_status moe_grouped_ffn(const void* xp, const int32_t* offsets, const void* w
                            const void* w_up, const void* w_down, const moe_dims* d,
                            void* h, void* y, void* ws, size_t ws_bytes, void* stream);
 
+/* One-time weight preparation for the gate/up GEMM: interleaves w_gate and w_up
+ * ([E][F][H] each) in blocks of 64 rows into w_gu [E][2 Fp][H] bf16, Fp = F rounded up
+ * to a multiple of 64 (rows [128 j, 128 j + 64) = gate rows [64 j, 64 j + 64), the next 64
+ * = the up rows of the same features, rows of features >= F zero).  Then one TMA box
+ * carries gate and up of 128 features and the GEMM runs N = 256 MMAs.  Size in bytes:
+ * moe_packed_gate_up_bytes(d).  Not part of the per-token path. */
+size_t moe_packed_gate_up_bytes(const moe_dims* d);
+moe_status moe_pack_gate_up(const void* w_gate, const void* w_up, const moe_dims* d, void* w_gu,
+                            void* stream);
+
+/* moe_grouped_gate_up on packed weights: identical h. */
+moe_status moe_grouped_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu,
+                                      const moe_dims* d, void* h, void* ws, size_t ws_bytes,
+                                      void* stream);
+
 /* The two halves of moe_grouped_ffn as separate launches (S4 and S5). */
 moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const void* w_gate,
                                const void* w_up, const moe_dims* d, void* h, void* ws,
@@ -279,6 +294,8 @@ typedef struct moe_layer_weights {
   const void*  w_down;      /* [E][H][F] bf16                                */
   const void*  w_dp;        /* latent only: [H][d_model] bf16, else NULL     */
   const void*  w_upp;       /* latent only: [d_model][H] bf16, else NULL     */
+  const void*  w_gate_up;   /* optional: w_gate/w_up packed by moe_pack_gate_up;
+                               when set the layer uses it (w_gate/w_up may be NULL) */
 } moe_layer_weights;
 
 typedef struct moe_layer_buffers {

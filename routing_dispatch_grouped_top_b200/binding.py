@@ -35,8 +35,11 @@ class moe_dims(C.Structure):
                 ("P", C.c_int32), ("renormalize", C.c_int32), ("d_model", C.c_int32)]
 
 
+_W_FIELDS = ("w_g_split", "bias", "w_gate", "w_up", "w_down", "w_dp", "w_upp", "w_gate_up")
+
+
 class moe_layer_weights(C.Structure):
-    _fields_ = [(n, C.c_void_p) for n in ("w_g_split", "bias", "w_gate", "w_up", "w_down", "w_dp", "w_upp")]
+    _fields_ = [(n, C.c_void_p) for n in _W_FIELDS]
 
 
 _BUF_FIELDS = ("z", "logits", "topk_ids", "topk_w", "counts", "offsets", "part_counts", "part_offsets",
@@ -64,6 +67,9 @@ _SIGS = {
     "moe_grouped_ffn": (C.c_int, [_VP, _VP, _VP, _VP, _VP, _DP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_gate_up": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_down": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
+    "moe_packed_gate_up_bytes": (_SZ, [_DP]),
+    "moe_pack_gate_up": (C.c_int, [_VP, _VP, _DP, _VP, _VP]),
+    "moe_grouped_gate_up_packed": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
     "moe_combine": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP]),
     "moe_skew_stats": (C.c_int, [_VP, _DP, _VP, _VP]),
     "moe_p95": (C.c_double, [C.POINTER(C.c_float), C.c_int]),
@@ -234,6 +240,31 @@ def moe_grouped_gate_up(xp, offsets, w_gate, w_up, d: moe_dims, h, ws, stream=No
         _stream(stream)))
 
 
+def packed_gate_up_bytes(d: moe_dims) -> int:
+    return int(lib().moe_packed_gate_up_bytes(C.byref(d)))
+
+
+def moe_pack_gate_up(w_gate, w_up, d: moe_dims, w_gu, stream=None):
+    n = d.E * d.F * d.H
+    _check("moe_pack_gate_up", lib().moe_pack_gate_up(
+        _ptr(w_gate, torch.bfloat16, "w_gate", n), _ptr(w_up, torch.bfloat16, "w_up", n), C.byref(d),
+        _ptr(w_gu, torch.bfloat16, "w_gu", packed_gate_up_bytes(d) // 2), _stream(stream)))
+
+
+def pack_gate_up(w_gate, w_up, d: moe_dims, stream=None) -> torch.Tensor:
+    w_gu = torch.empty(packed_gate_up_bytes(d) // 2, dtype=torch.bfloat16, device=w_gate.device)
+    moe_pack_gate_up(w_gate, w_up, d, w_gu, stream)
+    return w_gu
+
+
+def moe_grouped_gate_up_packed(xp, offsets, w_gu, d: moe_dims, h, ws, stream=None):
+    TK = d.T * d.K
+    _check("moe_grouped_gate_up_packed", lib().moe_grouped_gate_up_packed(
+        _ptr(xp, torch.bfloat16, "xp", TK * d.H), _ptr(offsets, torch.int32, "offsets", d.E + 1),
+        _ptr(w_gu, torch.bfloat16, "w_gu", packed_gate_up_bytes(d) // 2), C.byref(d),
+        _ptr(h, torch.bfloat16, "h", TK * d.F), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
 def moe_grouped_down(h, offsets, w_down, d: moe_dims, y, ws, stream=None):
     TK = d.T * d.K
     _check("moe_grouped_down", lib().moe_grouped_down(
@@ -294,12 +325,22 @@ def _buffers_struct(b: dict) -> moe_layer_buffers:
 
 
 def _weights_struct(w: dict) -> moe_layer_weights:
-    names = ("w_g_split", "bias", "w_gate", "w_up", "w_down", "w_dp", "w_upp")
-    return moe_layer_weights(*[(w[n].data_ptr() if w.get(n) is not None else None) for n in names])
+    return moe_layer_weights(*[(w[n].data_ptr() if w.get(n) is not None else None) for n in _W_FIELDS])
 
 
-def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, w_upp=None, stream=None) -> dict:
-    """One-time weight preparation (router split into three bf16 planes)."""
+# Packed gate/up weights (256 x 256 tiles, single-buffered accumulators) measured faster
+# than the separate-weight kernel only when the reduction is long (H = 7168) and slower at
+# H = 2048, where the unoverlapped epilogue weighs more: pack from this width up.
+PACK_GATE_UP_MIN_H = 4096
+
+
+def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, w_upp=None, stream=None,
+                       pack_gate_up_weights=None) -> dict:
+    """One-time weight preparation: router split into three bf16 planes and, when
+    ``pack_gate_up_weights`` (default: H >= PACK_GATE_UP_MIN_H), gate/up interleaved for the
+    packed gate/up GEMM."""
+    if pack_gate_up_weights is None:
+        pack_gate_up_weights = d.H >= PACK_GATE_UP_MIN_H
     split = torch.empty((3, d.E, d.H), dtype=torch.bfloat16, device=w_g.device)
     moe_pack_router(w_g.contiguous(), d, split, stream)
     for name, t, n in (("w_gate", w_gate, d.E * d.F * d.H), ("w_up", w_up, d.E * d.F * d.H),
@@ -310,7 +351,9 @@ def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, 
         _ptr(w_upp, torch.bfloat16, "w_upp", d.H * d.d_model)
     if bias is not None:
         _ptr(bias, torch.float32, "bias", d.E)
-    return dict(w_g_split=split, bias=bias, w_gate=w_gate, w_up=w_up, w_down=w_down, w_dp=w_dp, w_upp=w_upp)
+    w_gu = pack_gate_up(w_gate, w_up, d, stream) if pack_gate_up_weights else None
+    return dict(w_g_split=split, bias=bias, w_gate=w_gate, w_up=w_up, w_down=w_down, w_dp=w_dp, w_upp=w_upp,
+                w_gate_up=w_gu)
 
 
 def moe_layer_forward(x, weights: dict, d: moe_dims, buffers: dict, ws, stage_events=None, stream=None):

@@ -199,6 +199,29 @@ moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const voi
                                   d->F, h, ws_status(ws), as_stream(stream)));
 }
 
+size_t moe_packed_gate_up_bytes(const moe_dims* d) {
+  if (check_dims(d) != MOE_OK) return 0;
+  return static_cast<size_t>(d->E) * static_cast<size_t>(packed_gate_up_rows(d->F)) * d->H * 2;
+}
+
+moe_status moe_pack_gate_up(const void* w_gate, const void* w_up, const moe_dims* d, void* w_gu, void* stream) {
+  MOE_TRY(common_checks(d));
+  if (!w_gate || !w_up || !w_gu) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_gu)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_pack_gate_up(w_gate, w_up, d->E, d->H, d->F, w_gu, as_stream(stream)));
+}
+
+moe_status moe_grouped_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, const moe_dims* d,
+                                      void* h, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(common_checks(d));
+  MOE_TRY(check_ws(ws, ws_bytes, d));
+  if (d->T == 0) return MOE_OK;
+  if (!xp || !offsets || !w_gu || !h) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xp) || !aligned16(w_gu)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(gemm_gate_up_packed(xp, offsets, w_gu, d->E, d->T * static_cast<long long>(d->K), d->H, d->F,
+                                         h, ws_status(ws), as_stream(stream)));
+}
+
 moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w_down, const moe_dims* d, void* y,
                             void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(common_checks(d));
@@ -258,7 +281,7 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   MOE_TRY(check_ws(ws, ws_bytes, d));
   if (!x || !w || !b) return MOE_ERR_INVALID_ARG;
   const bool latent = d->d_model > 0;
-  if (!w->w_g_split || !w->w_gate || !w->w_up || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if (!w->w_g_split || !w->w_down || (!w->w_gate_up && (!w->w_gate || !w->w_up))) return MOE_ERR_INVALID_ARG;
   if (latent && (!w->w_dp || !w->w_upp || !b->z || !b->final_out)) return MOE_ERR_INVALID_ARG;
   if (!b->logits || !b->topk_ids || !b->topk_w || !b->counts || !b->offsets || !b->part_counts ||
       !b->part_offsets || !b->row_of_assign || !b->assign_of_row || !b->xp || !b->h || !b->y || !b->out)
@@ -288,7 +311,12 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   MOE_CUDA(launch_permute(routed, b->row_of_assign, b->topk_ids, b->topk_w, T, d->H, d->E, d->K, d->P, b->xp,
                           b->meta_token, b->meta_slot, b->meta_w, b->meta_local_expert, s));
   MOE_TRY(mark(5));
-  if (T > 0) MOE_CUDA(gemm_gate_up(b->xp, b->offsets, w->w_gate, w->w_up, d->E, TK, d->H, d->F, b->h, status, s));
+  if (T > 0) {
+    if (w->w_gate_up)
+      MOE_CUDA(gemm_gate_up_packed(b->xp, b->offsets, w->w_gate_up, d->E, TK, d->H, d->F, b->h, status, s));
+    else
+      MOE_CUDA(gemm_gate_up(b->xp, b->offsets, w->w_gate, w->w_up, d->E, TK, d->H, d->F, b->h, status, s));
+  }
   MOE_TRY(mark(6));
   if (T > 0) MOE_CUDA(gemm_down(b->h, b->offsets, w->w_down, d->E, TK, d->H, d->F, b->y, status, s));
   MOE_TRY(mark(7));

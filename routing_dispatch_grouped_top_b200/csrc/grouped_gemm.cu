@@ -69,6 +69,14 @@ struct Cfg<kEpiSwiGLU> {
   static constexpr int NA = 2, NT = 128, STAGES = 4, FEAT = 128;
   static constexpr bool SEP = true;
 };
+// SwiGLU on packed weights: one 256-row box holds two 128-row weight tiles, each
+// [64 gate rows; the 64 up rows of the same features]; two N = 256 accumulators, so gate
+// (lanes 0-63) and up (lanes 64-127) meet through a shared-memory swap in the epilogue.
+template <>
+struct Cfg<kEpiSwiGLUPacked> {
+  static constexpr int NA = 2, NT = 256, STAGES = 3, FEAT = 128;
+  static constexpr bool SEP = true;
+};
 // Plain bf16 output (down projection, latent projections).
 template <>
 struct Cfg<kEpiBF16> {
@@ -90,9 +98,11 @@ struct Layout {
   static constexpr int kAccCols = C::SEP ? C::NA * C::NT : C::NT;
   static constexpr int kNumAcc = (2 * kAccCols <= 512) ? 2 : 1;
   static constexpr uint32_t kTmemCols = kNumAcc * kAccCols;
+  static constexpr int kExchFloats = 2 * 16 * 64;  // SwiGLU swap of one 32-token chunk, both directions
+  static constexpr int kExchBytes = (EPI == kEpiSwiGLUPacked) ? 2 * kExchFloats * 4 : 0;  // double-buffered
   static constexpr int kBarBytes = 8 * (2 * C::STAGES + 5) + 16;
   static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
-  static constexpr int kSmemBytes = 1024 + C::STAGES * kStageBytes + kBarBytes + kTableBytes;
+  static constexpr int kSmemBytes = 1024 + C::STAGES * kStageBytes + kExchBytes + kBarBytes + kTableBytes;
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
   static_assert(kSmemBytes <= 232448, "shared memory budget");
 };
@@ -100,6 +110,10 @@ struct Layout {
 struct Tile {
   int g, n0, row0, nvalid, nround;
 };
+
+// silu(g) * u = g u / (1 + e^-g) with the fast exponential and divide (2 MUFU ops):
+// for g -> -inf the denominator overflows and the result is 0, for g -> +inf it is g u.
+__device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g * u, 1.0f + __expf(-g)); }
 
 // Tile t -> (group, weight tile, token chunk).  s_pre[g] = first tile of group g.  A group of
 // cnt rows is cut into ceil(cnt / NT) balanced chunks of a multiple of ROUND rows; a weight
@@ -172,16 +186,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::kStageBytes);
+  float* exch = reinterpret_cast<float*>(smem + STAGES * L::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::kStageBytes + L::kExchBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_off = reinterpret_cast<int*>(smem + STAGES * L::kStageBytes + L::kBarBytes);
+  int* s_off = reinterpret_cast<int*>(smem + STAGES * L::kStageBytes + L::kExchBytes + L::kBarBytes);
   int* s_pre = s_off + (kMaxGroups + 1);
   __shared__ int s_warp_sums[kThreads / 32];
+  (void)exch;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.offsets ? args.G : 1;
@@ -252,12 +268,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = ring + stage * L::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
           const int kx = kb * kBK;
+          if constexpr (EPI == kEpiBF16 || EPI == kEpiSwiGLUPacked) {
+            // both 128-row weight tiles in one 256-row box (packed rows are 2 per feature)
+            tma_load_3d(st, &tmA0, &full[stage], kx, (EPI == kEpiSwiGLUPacked) ? 2 * tl.n0 : tl.n0, tl.g);
+          } else {
 #pragma unroll
-          for (int i = 0; i < NA; ++i) {
-            const CUtensorMap* m = (i == 0) ? &tmA0 : ((i == 1) ? &tmA1 : &tmA2);
-            const int z = (EPI == kEpiF32) ? i : tl.g;
-            const int row = (EPI == kEpiBF16) ? tl.n0 + i * kBM : tl.n0;  // wide bf16: rows n0 + 128 i
-            tma_load_3d(st + i * kABytes, m, &full[stage], kx, row, z);
+            for (int i = 0; i < NA; ++i) {
+              const CUtensorMap* m = (i == 0) ? &tmA0 : ((i == 1) ? &tmA1 : &tmA2);
+              tma_load_3d(st + i * kABytes, m, &full[stage], kx, tl.n0, (EPI == kEpiF32) ? i : tl.g);
+            }
           }
           int r = 0;
 #pragma unroll
@@ -336,11 +355,57 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lanes [32q, 32q + 32) are visible to this warp
-    uint32_t acc = 0, acc_phase = 0;
+    uint32_t acc = 0, acc_phase = 0, chunk = 0;
     for (int t = blockIdx.x; t < total; t += gridDim.x) {
       const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
+      if constexpr (EPI == kEpiSwiGLUPacked) {
+        // Accumulator i covers features n0 + 64 i + fi: gate in warps q < 2, up in warps q >= 2.
+        // The gate owner keeps tokens 0..15 of each 32-token chunk and hands 16..31 to the up
+        // owner, who hands back the up of tokens 0..15; each then finishes 16 tokens of h.
+        const int fi = 32 * (q & 1) + lane;
+        const bool is_gate = q < 2;
+        const int jbase = is_gate ? 0 : 16;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.out);
+        const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
+#pragma unroll 1
+        for (int i = 0; i < NA; ++i) {
+          const int f = tl.n0 + 64 * i + fi;
+          for (int j0 = 0; j0 < tl.nvalid; j0 += 32, ++chunk) {
+            uint32_t r[32];
+            tmem_ld_32cols(tb + i * NT + j0, r);
+            tmem_wait_ld();
+            float* xb = exch + (chunk & 1) * L::kExchFloats;
+            float* to_up = xb;              // gate of tokens 16..31
+            float* to_gate = xb + 16 * 64;  // up of tokens 0..15
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              if (is_gate) to_up[j * 64 + fi] = __uint_as_float(r[16 + j]);
+              else to_gate[j * 64 + fi] = __uint_as_float(r[j]);
+            }
+            named_bar_sync(1, kEpiThreads);
+            if (f < args.N) {
+              const long long row0 = static_cast<long long>(tl.row0) + j0 + jbase;
+#pragma unroll
+              for (int j = 0; j < 16; ++j) {
+                if (j0 + jbase + j < tl.nvalid) {
+                  const float g = is_gate ? __uint_as_float(r[j]) : to_up[j * 64 + fi];
+                  const float u = is_gate ? to_gate[j * 64 + fi] : __uint_as_float(r[16 + j]);
+                  out[(row0 + j) * args.ldo + f] = __float2bfloat16_rn(silu_mul(g, u));
+                }
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        if (++acc == L::kNumAcc) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+        continue;
+      }
       const int f = tl.n0 + q * 32 + lane;
       const bool f_ok = f < args.N;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
@@ -358,10 +423,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               if (j < jn) {
-                const float g = __uint_as_float(r0[j]);
-                const float u = __uint_as_float(r1[j]);
-                const float h = g / (1.0f + __expf(-g)) * u;
-                out[(row0 + j) * args.ldo + f] = __float2bfloat16_rn(h);
+                out[(row0 + j) * args.ldo + f] =
+                    __float2bfloat16_rn(silu_mul(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
               }
             }
           }
@@ -660,8 +723,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               if (tok < tl.nvalid) {
                 const float g = is_gate ? __uint_as_float(r[j]) : to_up[j * 64 + fi];
                 const float u = is_gate ? to_gate[j * 64 + fi] : __uint_as_float(r[16 + j]);
-                const float h = g / (1.0f + __expf(-g)) * u;
-                out[static_cast<long long>(tl.row0 + tok) * args.ldo + f] = __float2bfloat16_rn(h);
+                out[static_cast<long long>(tl.row0 + tok) * args.ldo + f] = __float2bfloat16_rn(silu_mul(g, u));
               }
             }
           }
@@ -793,6 +855,7 @@ long long tile_bound(long long rows, int groups, int NT, int N, int feat) {
 int gemm_smem_bytes(int epi) {
   switch (epi) {
     case kEpiSwiGLU: return Layout<kEpiSwiGLU>::kSmemBytes;
+    case kEpiSwiGLUPacked: return Layout<kEpiSwiGLUPacked>::kSmemBytes;
     case kEpiBF16: return Layout<kEpiBF16>::kSmemBytes;
     default: return Layout<kEpiF32>::kSmemBytes;
   }
@@ -820,13 +883,30 @@ cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_g
   return launch<kEpiSwiGLU>(a0, a1, a1, b, args, tile_bound(rows, E, Cfg<kEpiSwiGLU>::NT, F, Cfg<kEpiSwiGLU>::FEAT), stream);
 }
 
+long long packed_gate_up_rows(int F) { return 2LL * ((F + 63) / 64 * 64); }
+
+// Same result as gemm_gate_up, from weights packed by launch_pack_gate_up.
+cudaError_t gemm_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, int E, long long rows,
+                                int H, int F, void* h, int* status, cudaStream_t stream) {
+  GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status};
+  CUtensorMap a0;
+  BoxMaps b;
+  if (!map_bf16_3d(&a0, w_gu, H, static_cast<uint64_t>(packed_gate_up_rows(F)), E, 256) ||
+      !map_token_boxes(&b, xp, H, rows))
+    return cudaErrorInvalidValue;
+  return launch<kEpiSwiGLUPacked>(a0, a0, a0, b, args,
+                                  tile_bound(rows, E, Cfg<kEpiSwiGLUPacked>::NT, F, Cfg<kEpiSwiGLUPacked>::FEAT),
+                                  stream);
+}
+
 // y = h Wd^T per expert group.
 cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down, int E, long long rows, int H,
                       int F, void* y, int* status, cudaStream_t stream) {
   GemmArgs args{offsets, E, static_cast<int>(rows), H, F, y, H, nullptr, status};
   CUtensorMap a0;
   BoxMaps b;
-  if (!map_bf16_3d(&a0, w_down, F, H, E, kBM) || !map_token_boxes(&b, h, F, rows)) return cudaErrorInvalidValue;
+  if (!map_bf16_3d(&a0, w_down, F, H, E, MOE_GEMM_PAIR ? kBM : 256) || !map_token_boxes(&b, h, F, rows))
+    return cudaErrorInvalidValue;
   if (MOE_GEMM_PAIR)
     return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(rows, E, PairLayout<kEpiBF16>::NT, H, 256), stream);
   return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(rows, E, Cfg<kEpiBF16>::NT, H, Cfg<kEpiBF16>::FEAT), stream);
@@ -837,7 +917,8 @@ cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd,
                        cudaStream_t stream) {
   CUtensorMap a0;
   BoxMaps b;
-  if (!map_bf16_3d(&a0, w, Kd, N, 1, kBM) || !map_token_boxes(&b, a, Kd, M)) return cudaErrorInvalidValue;
+  if (!map_bf16_3d(&a0, w, Kd, N, 1, MOE_GEMM_PAIR ? kBM : 256) || !map_token_boxes(&b, a, Kd, M))
+    return cudaErrorInvalidValue;
   GemmArgs args{nullptr, 1, static_cast<int>(M), N, Kd, out, N, nullptr, status};
   if (MOE_GEMM_PAIR)
     return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(M, 1, PairLayout<kEpiBF16>::NT, N, 256), stream);

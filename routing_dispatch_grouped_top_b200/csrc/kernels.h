@@ -6,7 +6,7 @@
 
 namespace moe {
 
-enum Epi : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2 };
+enum Epi : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2, kEpiSwiGLUPacked = 3 };
 
 struct GemmArgs {
   const int32_t* offsets;  // [G + 1] device row offsets of the groups, or nullptr: one group of M rows
@@ -25,6 +25,12 @@ int gemm_smem_bytes(int epi);
 
 cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
                          long long rows, int H, int F, void* h, int* status, cudaStream_t stream);
+// Gate and up weights interleaved in 64-row blocks ([E][2 Fp][H], Fp = F rounded up to 64).
+long long packed_gate_up_rows(int F);
+cudaError_t launch_pack_gate_up(const void* w_gate, const void* w_up, int E, int H, int F, void* w_gu,
+                                cudaStream_t stream);
+cudaError_t gemm_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, int E, long long rows,
+                                int H, int F, void* h, int* status, cudaStream_t stream);
 cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down, int E, long long rows, int H,
                       int F, void* y, int* status, cudaStream_t stream);
 cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd, void* out, int* status,

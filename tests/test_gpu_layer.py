@@ -42,10 +42,10 @@ def cpu(t):
     return t.detach().cpu().numpy()
 
 
-def run_gpu_layer(cfg, inp):
+def run_gpu_layer(cfg, inp, packed=True):
     d = B.dims_of(cfg)
     w = B.pack_layer_weights(d, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"], inp["w_dp"],
-                             inp["w_upp"])
+                             inp["w_upp"], pack_gate_up_weights=packed)
     bufs = B.alloc_layer_buffers(d)
     ws = B.make_workspace(d)
     B.moe_layer_forward(inp["x"], w, d, bufs, ws)
@@ -117,7 +117,8 @@ SMALL = [
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
 def test_layer_matches_oracle(cfg):
     inp = inputs.make_layer(cfg, DEV)
-    g = run_gpu_layer(cfg, inp)
+    # both gate/up paths: separate weights for two layers, packed weights for the others
+    g = run_gpu_layer(cfg, inp, packed=cfg.name not in ("tiny_T100_P2_plain_softmax", "one_token"))
     torch.cuda.synchronize()
     cpu_in = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
     r = oracle.layer_forward(bits(cpu_in["x"]), cpu_in["w_g"].numpy(), bits(cpu_in["w_gate"]),

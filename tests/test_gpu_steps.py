@@ -215,18 +215,42 @@ def ffn_inputs(E, H, F, rows, zipf, zero_frac, seed=0):
     return off, xp, wg, wu, wd
 
 
+@pytest.mark.parametrize("packed", [False, True], ids=["separate", "packed"])
 @pytest.mark.parametrize("E,H,F,rows,zipf,zf", FFN_CASES)
-def test_grouped_ffn_matches_oracle(E, H, F, rows, zipf, zf):
+def test_grouped_ffn_matches_oracle(E, H, F, rows, zipf, zf, packed):
     off, xp, wg, wu, wd = ffn_inputs(E, H, F, rows, zipf, zf)
     d = B.dims(T=rows, H=H, E=E, K=1, F=F)
     ws = B.make_workspace(d)
     h = torch.zeros((rows, F), dtype=torch.bfloat16, device=DEV)
     y = torch.zeros((rows, H), dtype=torch.bfloat16, device=DEV)
-    B.moe_grouped_ffn(xp.to(DEV), torch.from_numpy(off).to(DEV), wg.to(DEV), wu.to(DEV), wd.to(DEV), d, h, y, ws)
+    offd = torch.from_numpy(off).to(DEV)
+    if packed:
+        w_gu = B.pack_gate_up(wg.to(DEV), wu.to(DEV), d)
+        B.moe_grouped_gate_up_packed(xp.to(DEV), offd, w_gu, d, h, ws)
+        B.moe_grouped_down(h, offd, wd.to(DEV), d, y, ws)
+    else:
+        B.moe_grouped_ffn(xp.to(DEV), offd, wg.to(DEV), wu.to(DEV), wd.to(DEV), d, h, y, ws)
     assert B.read_device_status(ws) == 0
     rh, ry = oracle.grouped_ffn(bits(xp), off, bits(wg), bits(wu), bits(wd))
     check_bf16("h", bits(h), rh)
     check_bf16("y", bits(y), ry)
+
+
+def test_pack_gate_up_layout():
+    # packed rows [128 j, 128 j + 64) = gate rows [64 j, +64), next 64 = up rows; padding rows zero
+    E, H, F = 3, 16, 136
+    wg = inputs.random_bf16((E, F, H), seed=1)
+    wu = inputs.random_bf16((E, F, H), seed=2)
+    d = B.dims(T=1, H=H, E=E, K=1, F=F)
+    w_gu = B.pack_gate_up(wg.to(DEV), wu.to(DEV), d).view(E, -1, H).cpu()
+    Fp = 192
+    assert w_gu.shape[1] == 2 * Fp
+    for j in range(Fp // 64):
+        for half, src in ((0, wg), (1, wu)):
+            rows = w_gu[:, 128 * j + 64 * half: 128 * j + 64 * half + 64]
+            n = max(0, min(64, F - 64 * j))
+            assert torch.equal(rows[:, :n].view(torch.int16), src[:, 64 * j: 64 * j + n].view(torch.int16))
+            assert int(rows[:, n:].view(torch.int16).abs().sum()) == 0
 
 
 def test_grouped_down_alone_matches_oracle():
