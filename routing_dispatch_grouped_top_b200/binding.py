@@ -329,9 +329,11 @@ def _weights_struct(w: dict) -> moe_layer_weights:
 
 
 # Packed gate/up weights (256 x 256 tiles, single-buffered accumulators) measured faster
-# than the separate-weight kernel only when the reduction is long (H = 7168) and slower at
-# H = 2048, where the unoverlapped epilogue weighs more: pack from this width up.
+# than the separate-weight kernel in the layer only with a long reduction and prefill-sized
+# expert batches (H = 7168, 256 rows per expert: 5.0 vs 5.3 ms); slower at H = 2048 and for
+# decode (few rows per expert).  Pack when both hold.
 PACK_GATE_UP_MIN_H = 4096
+PACK_GATE_UP_MIN_ROWS_PER_EXPERT = 64
 
 
 def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, w_upp=None, stream=None,
@@ -340,7 +342,8 @@ def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, 
     ``pack_gate_up_weights`` (default: H >= PACK_GATE_UP_MIN_H), gate/up interleaved for the
     packed gate/up GEMM."""
     if pack_gate_up_weights is None:
-        pack_gate_up_weights = d.H >= PACK_GATE_UP_MIN_H
+        pack_gate_up_weights = (d.H >= PACK_GATE_UP_MIN_H and
+                                d.T * d.K >= PACK_GATE_UP_MIN_ROWS_PER_EXPERT * d.E)
     split = torch.empty((3, d.E, d.H), dtype=torch.bfloat16, device=w_g.device)
     moe_pack_router(w_g.contiguous(), d, split, stream)
     for name, t, n in (("w_gate", w_gate, d.E * d.F * d.H), ("w_up", w_up, d.E * d.F * d.H),
