@@ -366,9 +366,10 @@ def moe_layer_forward(x, weights: dict, d: moe_dims, buffers: dict, ws, stage_ev
         if len(stage_events) != MOE_NUM_STAGE_EVENTS:
             raise ValueError(f"need {MOE_NUM_STAGE_EVENTS} events")
         for e in stage_events:          # torch creates the CUDA event on its first record
-            if not e.cuda_event:
+            if e is not None and not e.cuda_event:
                 e.record(torch.cuda.current_stream() if stream is None else stream)
-        ev = (C.c_void_p * MOE_NUM_STAGE_EVENTS)(*[e.cuda_event for e in stage_events])
+        ev = (C.c_void_p * MOE_NUM_STAGE_EVENTS)(*[(e.cuda_event if e is not None else None)
+                                                   for e in stage_events])
     wst, bst = _weights_struct(weights), _buffers_struct(buffers)
     _check("moe_layer_forward", lib().moe_layer_forward(
         _ptr(x, torch.bfloat16, "x", d.T * d_in), C.byref(wst), C.byref(d), C.byref(bst),

@@ -38,6 +38,8 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
     const float* __restrict__ w, long long T, int vpr, int E, int K, int P, uint4* __restrict__ xp,
     int32_t* __restrict__ meta_token, int32_t* __restrict__ meta_slot, float* __restrict__ meta_w,
     int32_t* __restrict__ meta_local) {
+  pdl_wait();  // row_of_assign comes from the count/scan kernel
+  pdl_launch_dependents();
   const long long n_items = T * vpr;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
@@ -84,6 +86,8 @@ __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const uint4* __re
                                                                const int32_t* __restrict__ roa,
                                                                const float* __restrict__ w, long long T, int vpr,
                                                                int K, uint4* __restrict__ out) {
+  pdl_wait();  // y comes from the down-projection GEMM
+  pdl_launch_dependents();
   const long long n_items = T * vpr;
   const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
   for (long long it = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; it < n_items; it += stride) {
@@ -193,10 +197,9 @@ cudaError_t launch_permute(const void* x, const int32_t* roa, const int32_t* ids
                            float* meta_w, int32_t* meta_local, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int vpr = H / 8;
-  permute_kernel<<<copy_blocks(T * vpr / 2), kCopyThreads, 0, s>>>(
-      reinterpret_cast<const uint4*>(x), roa, ids, w, T, vpr, E, K, P, reinterpret_cast<uint4*>(xp), meta_token,
-      meta_slot, meta_w, meta_local);
-  return cudaGetLastError();
+  return launch_pdl(permute_kernel, dim3(copy_blocks(T * vpr / 2)), dim3(kCopyThreads), 0, s,
+                    reinterpret_cast<const uint4*>(x), roa, ids, w, T, vpr, E, K, P, reinterpret_cast<uint4*>(xp),
+                    meta_token, meta_slot, meta_w, meta_local);
 }
 
 cudaError_t launch_combine(const void* y, const int32_t* roa, const float* w, long long T, int H, int K, void* out,
@@ -205,12 +208,10 @@ cudaError_t launch_combine(const void* y, const int32_t* roa, const float* w, lo
   const int vpr = H / 8;
   const int blocks = copy_blocks(T * vpr);
   if (K <= 2)
-    combine_kernel<2><<<blocks, kCopyThreads, 0, s>>>(reinterpret_cast<const uint4*>(y), roa, w, T, vpr, K,
-                                                     reinterpret_cast<uint4*>(out));
-  else
-    combine_kernel<4><<<blocks, kCopyThreads, 0, s>>>(reinterpret_cast<const uint4*>(y), roa, w, T, vpr, K,
-                                                     reinterpret_cast<uint4*>(out));
-  return cudaGetLastError();
+    return launch_pdl(combine_kernel<2>, dim3(blocks), dim3(kCopyThreads), 0, s, reinterpret_cast<const uint4*>(y),
+                      roa, w, T, vpr, K, reinterpret_cast<uint4*>(out));
+  return launch_pdl(combine_kernel<4>, dim3(blocks), dim3(kCopyThreads), 0, s, reinterpret_cast<const uint4*>(y),
+                    roa, w, T, vpr, K, reinterpret_cast<uint4*>(out));
 }
 
 cudaError_t launch_pack_gate_up(const void* w_gate, const void* w_up, int E, int H, int F, void* w_gu,

@@ -204,23 +204,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int NFT = (args.N + C::FEAT - 1) / C::FEAT;
   const int KB = (args.Kd + kBK - 1) / kBK;
 
+  // Set-up that reads no global input runs before the wait on the previous kernel.
   __shared__ int s_bad;
-  if (threadIdx.x == 0) s_bad = 0;
-  __syncthreads();
-  for (int i = threadIdx.x; i <= G; i += kThreads)
-    s_off[i] = args.offsets ? __ldg(args.offsets + i) : (i == 0 ? 0 : args.M);
-  __syncthreads();
-  // Offsets must be non-decreasing inside [0, M]; otherwise no tile runs.
-  for (int i = threadIdx.x; i <= G; i += kThreads) {
-    const bool bad = s_off[i] < 0 || s_off[i] > args.M || (i > 0 && s_off[i] < s_off[i - 1]);
-    if (bad) s_bad = 1;
-  }
-  __syncthreads();
-  if (s_bad) {
-    if (threadIdx.x == 0) report(args.status, MOE_DEV_BAD_INDEX);
-    for (int i = threadIdx.x; i <= G; i += kThreads) s_off[i] = 0;
-  }
   if (threadIdx.x == 0) {
+    s_bad = 0;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
@@ -241,6 +228,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_alloc(tmem_slot, L::kTmemCols);
     tmem_relinquish();
     tc_fence_before();
+  }
+  pdl_wait();  // offsets and the token operand come from earlier kernels
+  pdl_launch_dependents();
+  __syncthreads();
+  for (int i = threadIdx.x; i <= G; i += kThreads)
+    s_off[i] = args.offsets ? __ldg(args.offsets + i) : (i == 0 ? 0 : args.M);
+  __syncthreads();
+  // Offsets must be non-decreasing inside [0, M]; otherwise no tile runs.
+  for (int i = threadIdx.x; i <= G; i += kThreads) {
+    const bool bad = s_off[i] < 0 || s_off[i] > args.M || (i > 0 && s_off[i] < s_off[i - 1]);
+    if (bad) s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (threadIdx.x == 0) report(args.status, MOE_DEV_BAD_INDEX);
+    for (int i = threadIdx.x; i <= G; i += kThreads) s_off[i] = 0;
   }
   __syncthreads();
   build_tile_table(s_pre, s_off, G, NT, NFT, s_warp_sums);  // ends with __syncthreads
@@ -539,6 +542,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const int KB = (args.Kd + kBK - 1) / kBK;
 
   if (threadIdx.x == 0) s_bad = 0;
+  pdl_wait();
   __syncthreads();
   for (int i = threadIdx.x; i <= G; i += kThreads)
     s_off[i] = args.offsets ? __ldg(args.offsets + i) : (i == 0 ? 0 : args.M);
@@ -824,8 +828,7 @@ cudaError_t launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   if (attr_err != cudaSuccess) return attr_err;
   if (tile_bound <= 0) return cudaSuccess;
   const int grid = static_cast<int>(std::min<long long>(num_sms(), tile_bound));
-  grouped_gemm_kernel<EPI><<<grid, kThreads, L::kSmemBytes, stream>>>(a0, a1, a2, b, args);
-  return cudaGetLastError();
+  return launch_pdl(grouped_gemm_kernel<EPI>, dim3(grid), dim3(kThreads), L::kSmemBytes, stream, a0, a1, a2, b, args);
 }
 
 template <int EPI>

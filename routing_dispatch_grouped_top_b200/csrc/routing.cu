@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
                                                     int renormalize, int32_t* __restrict__ ids,
                                                     float* __restrict__ w) {
   const int lane = threadIdx.x & 31;
+  pdl_wait();  // logits come from the previous kernel
+  pdl_launch_dependents();
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
   for (long long t = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
        t += warps) {
@@ -100,9 +102,8 @@ template <int VPL>
 cudaError_t launch_route_vpl(const float* logits, long long T, int E, int K, int renorm, int32_t* ids, float* w,
                              cudaStream_t s) {
   const long long blocks = std::min<long long>((T + 7) / 8, 64LL * num_sms());
-  route_kernel<VPL><<<static_cast<int>(std::max<long long>(blocks, 1)), 256, 0, s>>>(logits, T, E, K, renorm,
-                                                                                       ids, w);
-  return cudaGetLastError();
+  return launch_pdl(route_kernel<VPL>, dim3(static_cast<unsigned>(std::max<long long>(blocks, 1))), dim3(256), 0, s,
+                    logits, T, E, K, renorm, ids, w);
 }
 
 // ---------------------------------------------------------------------------
