@@ -45,6 +45,8 @@ def parse():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--group-limit", type=int, default=0,
+                   help="node-limited routing: experts from the M best partitions (0 = off)")
     return p.parse_args()
 
 
@@ -258,6 +260,8 @@ def run_reference(args, cfg):
 def main():
     args = parse()
     cfg = CFG.get(args.config)
+    if args.group_limit:
+        cfg = cfg.with_(group_limit=args.group_limit, name=f"{cfg.name}_node_limited_M{args.group_limit}")
     if args.impl == "reference":
         return run_reference(args, cfg)
 

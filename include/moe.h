@@ -58,6 +58,9 @@ typedef struct moe_dims {
   int32_t renormalize;  /* 1: weights = softmax over the K selected logits;
                            0: weights = softmax over all E at the selected ids */
   int32_t d_model;      /* 0, or the model width of a latent layer */
+  int32_t group_limit;  /* 0, or M: node-limited routing, each token takes its K experts from
+                           its M best partitions (a partition ranks by its best expert);
+                           needs P <= MOE_MAX_LIMITED_GROUPS and K <= M * E / P */
 } moe_dims;
 
 typedef enum moe_status {
@@ -78,6 +81,7 @@ typedef enum moe_status {
 /* Limits of this build (checked; larger shapes return MOE_ERR_UNSUPPORTED_SHAPE). */
 #define MOE_MAX_E 1024
 #define MOE_MAX_K 32
+#define MOE_MAX_LIMITED_GROUPS 256
 
 /* ------------------------------------------------------------------------- */
 /* Workspace                                                                 */
@@ -128,7 +132,11 @@ moe_status moe_gating(const void* x, const void* w_g_split, const float* bias,
 /* logits: [T][E] fp32.  Out: topk_ids [T][K] int32 and topk_w [T][K] fp32, slot
  * 0 the best.  Order: larger logit first; equal logits (-0.0 == +0.0) go to the
  * lower expert id; NaN ranks below every number.  Weights: exp(l_k - l_max)
- * normalised over the K selected (renormalize = 1) or over all E. */
+ * normalised over the K selected (renormalize = 1) or over all E.
+ * With d->group_limit = M > 0 (node-limited routing, DeepSeek-V3's bound on how many
+ * nodes a token's experts span: "Three Parameter Counts...", "Halving top-k is a
+ * network change first"), the K experts are the best among the experts of the token's
+ * M best partitions, a partition ranking by its best expert under the same order. */
 moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids,
                      float* topk_w, void* stream);
 

@@ -37,6 +37,9 @@ and section:
 * [LatentMoE]  "Latent MoE" concept page (podcastatlas.ai wiki), sections
   "Definition" and "Current Synthesis": experts receive a narrower, projected
   hidden state.
+* [ParamCounts/layout]  "Three Parameter Counts...", section "Halving top-k is
+  a network change first": DeepSeek-V3's node-limited routing bounds how many
+  nodes (expert groups) one token's experts may span.
 
 Readings where the pages are silent:
 
@@ -47,6 +50,9 @@ Readings where the pages are silent:
   E followed by renormalising the top-K); with ``renormalize=False`` the weight
   is the plain softmax over all E at the selected experts.
 * Order of rows inside one expert: stable (assignment a = t*K + k ascending).
+* Node-limited routing: the groups are the P partitions; a group ranks by its best
+  expert under the top-k order; each token keeps its M best groups and takes its K
+  experts from those groups only.
 * Partition p owns experts [p*E/P, (p+1)*E/P); metadata per row is
   (token, slot, weight, expert - p*E/P).
 * Expert FFN: SwiGLU, h = silu(x Wg^T) * (x Wu^T), y = h Wd^T with nn.Linear
@@ -65,7 +71,7 @@ import numpy as np
 __all__ = [
     "bf16_bits_to_f64", "f64_to_bf16_bits", "gating_logits", "route",
     "count_scan", "permute", "grouped_ffn", "ffn_rows", "combine",
-    "skew_ratio", "p95_nearest_rank", "dense_bf16", "layer_forward",
+    "skew_ratio", "p95_nearest_rank", "dense_bf16", "layer_forward", "route_limited",
     "dispatch_bytes", "expert_weight_bytes", "experts_per_partition",
     "checkpoint_bytes",
 ]
@@ -158,6 +164,54 @@ def route(logits, K: int, renormalize: bool = True):
             mall = np.max(np.where(is_nan, -np.inf, v), axis=1, keepdims=True)
             num = np.exp(sel - mall)
             w = num / np.exp(v - mall).sum(axis=1, keepdims=True)
+    return ids, w.astype(np.float32)
+
+
+def _expert_order(v64):
+    """Per token, expert ids best first (larger value; ties -> lower id; NaN last)."""
+    T, E = v64.shape
+    is_nan = np.isnan(v64)
+    key_val = np.where(is_nan, 0.0, -v64)
+    ids_e = np.broadcast_to(np.arange(E), (T, E))
+    return np.lexsort((ids_e, key_val, is_nan.astype(np.int8)), axis=1)
+
+
+def route_limited(logits, K: int, P: int, M: int, renormalize: bool = True):
+    """Node-limited top-K: the K experts come from the token's M best groups.
+
+    Group p holds experts [p*E/P, (p+1)*E/P).  A group ranks by its best expert under
+    the top-k order of ``route``; the M groups whose best experts come first are kept
+    and the K best experts among their experts are selected.  Weights as in ``route``
+    (over the K selected, or over all E when not renormalising).  [ParamCounts/layout]
+    """
+    l = np.asarray(logits, dtype=np.float32)
+    T, E = l.shape
+    if E % P or not (1 <= M <= P) or K > M * (E // P):
+        raise ValueError("need E % P == 0, 1 <= M <= P and K <= M * E / P")
+    epp = E // P
+    v = l.astype(np.float64) + 0.0
+    order = _expert_order(v)                      # [T, E] expert ids, best first
+    group_of = order // epp
+    ids = np.empty((T, K), np.int64)
+    for t in range(T):
+        kept, seen = [], set()
+        for g in group_of[t]:                     # groups in the order of their best expert
+            if g not in seen:
+                seen.add(g)
+                kept.append(g)
+                if len(kept) == M:
+                    break
+        allowed = np.isin(group_of[t], kept)
+        ids[t] = order[t][allowed][:K]
+    ids = ids.astype(np.int32)
+    sel = np.take_along_axis(v, ids, axis=1)
+    with np.errstate(invalid="ignore", over="ignore"):
+        if renormalize:
+            num = np.exp(sel - sel[:, :1])
+            w = num / num.sum(axis=1, keepdims=True)
+        else:
+            mall = np.max(np.where(np.isnan(v), -np.inf, v), axis=1, keepdims=True)
+            w = np.exp(sel - mall) / np.exp(v - mall).sum(axis=1, keepdims=True)
     return ids, w.astype(np.float32)
 
 
@@ -321,7 +375,7 @@ def dense_bf16(x_bits, w_bits):
 
 def layer_forward(x_bits, w_g, w_gate_bits, w_up_bits, w_down_bits, K: int, P: int = 1,
                   renormalize: bool = True, bias=None, w_dp_bits=None, w_upp_bits=None,
-                  logits=None):
+                  logits=None, group_limit: int = 0):
     """All steps in pipeline order.  Returns a dict with every intermediate.
 
     If ``logits`` is given it replaces the oracle's own gating output (used by
@@ -335,7 +389,10 @@ def layer_forward(x_bits, w_g, w_gate_bits, w_up_bits, w_down_bits, K: int, P: i
     l = gating_logits(z, w_g, bias) if logits is None else np.asarray(logits, np.float32)
     res["logits"] = l
     E = l.shape[1]
-    ids, w = route(l, K, renormalize)
+    if group_limit:
+        ids, w = route_limited(l, K, P, group_limit, renormalize)
+    else:
+        ids, w = route(l, K, renormalize)
     res["topk_ids"], res["topk_w"] = ids, w
     cs = count_scan(ids, E, P)
     res.update(cs)

@@ -32,7 +32,7 @@ class MoEError(RuntimeError):
 
 class moe_dims(C.Structure):
     _fields_ = [("T", C.c_int64), ("H", C.c_int32), ("E", C.c_int32), ("K", C.c_int32), ("F", C.c_int32),
-                ("P", C.c_int32), ("renormalize", C.c_int32), ("d_model", C.c_int32)]
+                ("P", C.c_int32), ("renormalize", C.c_int32), ("d_model", C.c_int32), ("group_limit", C.c_int32)]
 
 
 _W_FIELDS = ("w_g_split", "bias", "w_gate", "w_up", "w_down", "w_dp", "w_upp", "w_gate_up")
@@ -105,12 +105,14 @@ def _check(fn: str, status: int):
         raise MoEError(fn, status, lib().moe_status_str(status).decode())
 
 
-def dims(T, H, E, K, F, P=1, renormalize=True, d_model=0) -> moe_dims:
-    return moe_dims(int(T), int(H), int(E), int(K), int(F), int(P), int(bool(renormalize)), int(d_model or 0))
+def dims(T, H, E, K, F, P=1, renormalize=True, d_model=0, group_limit=0) -> moe_dims:
+    return moe_dims(int(T), int(H), int(E), int(K), int(F), int(P), int(bool(renormalize)), int(d_model or 0),
+                    int(group_limit or 0))
 
 
 def dims_of(cfg, T=None) -> moe_dims:
-    return dims(cfg.T if T is None else T, cfg.H, cfg.E, cfg.K, cfg.F, cfg.P, cfg.renormalize, cfg.d_model or 0)
+    return dims(cfg.T if T is None else T, cfg.H, cfg.E, cfg.K, cfg.F, cfg.P, cfg.renormalize, cfg.d_model or 0,
+                cfg.group_limit or 0)
 
 
 def _stream(stream) -> int:

@@ -24,6 +24,7 @@ class MoEConfig:
     renormalize: bool = True
     zipf_s: Optional[float] = None      # per-expert logit bias drawn from rank-Zipf popularity
     d_model: Optional[int] = None       # latent layer: model width before the down-projection
+    group_limit: int = 0                # node-limited routing: experts from the M best partitions
     seed: int = 0
 
     @property

@@ -48,6 +48,10 @@ moe_status check_dims(const moe_dims* d) {
     return MOE_ERR_INVALID_ARG;
   if (d->H % 8 != 0 || d->F % 8 != 0 || d->d_model % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (d->E > MOE_MAX_E || d->K > MOE_MAX_K) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (d->group_limit < 0 || d->group_limit > d->P ||
+      (d->group_limit > 0 && d->K > static_cast<long long>(d->group_limit) * (d->E / d->P)))
+    return MOE_ERR_INVALID_ARG;
+  if (d->group_limit > 0 && d->P > MOE_MAX_LIMITED_GROUPS) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (d->T * static_cast<long long>(d->K) > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
@@ -160,7 +164,8 @@ moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids, 
   MOE_TRY(common_checks(d));
   if (d->T == 0) return MOE_OK;
   if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_route(logits, d->T, d->E, d->K, d->renormalize, topk_ids, topk_w, as_stream(stream)));
+  return cuda_status(launch_route(logits, d->T, d->E, d->K, d->renormalize, d->P, d->group_limit, topk_ids, topk_w,
+                                  as_stream(stream)));
 }
 
 moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* counts, int32_t* offsets,
@@ -303,7 +308,7 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   MOE_TRY(mark(1));
   if (T > 0) MOE_CUDA(gemm_gating(routed, w->w_g_split, w->bias, T, d->H, d->E, b->logits, status, s));
   MOE_TRY(mark(2));
-  MOE_CUDA(launch_route(b->logits, T, d->E, d->K, d->renormalize, b->topk_ids, b->topk_w, s));
+  MOE_CUDA(launch_route(b->logits, T, d->E, d->K, d->renormalize, d->P, d->group_limit, b->topk_ids, b->topk_w, s));
   MOE_TRY(mark(3));
   MOE_CUDA(launch_count_scan(b->topk_ids, TK, d->E, d->P, b->counts, b->offsets, b->part_counts, b->part_offsets,
                              b->row_of_assign, b->assign_of_row, b->skew, scan_ws(ws, d), s));

@@ -56,8 +56,8 @@ cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd,
 cudaError_t gemm_gating(const void* x, const void* w_split, const float* bias, long long T, int H, int E,
                         float* logits, int* status, cudaStream_t stream);
 
-cudaError_t launch_route(const float* logits, long long T, int E, int K, int renormalize, int32_t* ids, float* w,
-                         cudaStream_t stream);
+cudaError_t launch_route(const float* logits, long long T, int E, int K, int renormalize, int P, int group_limit,
+                         int32_t* ids, float* w, cudaStream_t stream);
 
 // Count/scan workspace: status word, grid-barrier words, per-block histograms.
 struct ScanWorkspace {

@@ -37,11 +37,19 @@ __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
+constexpr int kRouteWarps = 8;
+
 template <int VPL>
 __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, long long T, int E, int K,
-                                                    int renormalize, int32_t* __restrict__ ids,
+                                                    int renormalize, int P, int M, int32_t* __restrict__ ids,
                                                     float* __restrict__ w) {
+  // node-limited routing: best expert key of each group, then the kept groups (per warp)
+  __shared__ unsigned long long s_gkey[kRouteWarps][MOE_MAX_LIMITED_GROUPS];
+  __shared__ unsigned char s_kept[kRouteWarps][MOE_MAX_LIMITED_GROUPS];
   const int lane = threadIdx.x & 31;
+  const int wib = threadIdx.x >> 5;
+  const bool limited = M > 0 && M < P;
+  const int epp = E / P;
   pdl_wait();  // logits come from the previous kernel
   pdl_launch_dependents();
   const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
@@ -59,6 +67,49 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
       }
     }
     // Every real candidate has key > 0 (low word ~e != 0), padding has key 0.
+    if (limited) {
+      for (int g = lane; g < P; g += 32) s_gkey[wib][g] = 0ull;
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) atomicMax(&s_gkey[wib][e / epp], key[i]);
+      }
+      __syncwarp();
+      // M rounds of warp arg-max over the group keys; lane owns groups lane + 32 j
+      constexpr int GPL = MOE_MAX_LIMITED_GROUPS / 32;
+      unsigned long long gk[GPL];
+#pragma unroll
+      for (int j = 0; j < GPL; ++j) {
+        const int g = lane + 32 * j;
+        gk[j] = g < P ? s_gkey[wib][g] : 0ull;
+        if (g < P) s_kept[wib][g] = 0;
+      }
+      for (int m = 0; m < M; ++m) {
+        unsigned long long best = 0ull;
+#pragma unroll
+        for (int j = 0; j < GPL; ++j) best = gk[j] > best ? gk[j] : best;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+          best = other > best ? other : best;
+        }
+#pragma unroll
+        for (int j = 0; j < GPL; ++j) {
+          if (gk[j] == best && best != 0ull) {  // keys are unique: the owner marks its group kept
+            s_kept[wib][lane + 32 * j] = 1;
+            gk[j] = 0ull;
+          }
+        }
+      }
+      __syncwarp();
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E && !s_kept[wib][e / epp]) key[i] = 0ull;  // experts of dropped groups leave the race
+      }
+      __syncwarp();
+    }
     int my_id = 0;
     float my_val = 0.0f;
     for (int k = 0; k < K; ++k) {
@@ -99,11 +150,11 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 }
 
 template <int VPL>
-cudaError_t launch_route_vpl(const float* logits, long long T, int E, int K, int renorm, int32_t* ids, float* w,
-                             cudaStream_t s) {
-  const long long blocks = std::min<long long>((T + 7) / 8, 64LL * num_sms());
-  return launch_pdl(route_kernel<VPL>, dim3(static_cast<unsigned>(std::max<long long>(blocks, 1))), dim3(256), 0, s,
-                    logits, T, E, K, renorm, ids, w);
+cudaError_t launch_route_vpl(const float* logits, long long T, int E, int K, int renorm, int P, int M, int32_t* ids,
+                             float* w, cudaStream_t s) {
+  const long long blocks = std::min<long long>((T + kRouteWarps - 1) / kRouteWarps, 64LL * num_sms());
+  return launch_pdl(route_kernel<VPL>, dim3(static_cast<unsigned>(std::max<long long>(blocks, 1))),
+                    dim3(32 * kRouteWarps), 0, s, logits, T, E, K, renorm, P, M, ids, w);
 }
 
 // ---------------------------------------------------------------------------
@@ -300,16 +351,16 @@ size_t scan_smem_bytes(int E) { return static_cast<size_t>(E * 2 + 1 + kScanWarp
 
 }  // namespace
 
-cudaError_t launch_route(const float* logits, long long T, int E, int K, int renorm, int32_t* ids, float* w,
-                         cudaStream_t s) {
+cudaError_t launch_route(const float* logits, long long T, int E, int K, int renorm, int P, int M, int32_t* ids,
+                         float* w, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int vpl = (E + 31) / 32;
-  if (vpl <= 1) return launch_route_vpl<1>(logits, T, E, K, renorm, ids, w, s);
-  if (vpl <= 2) return launch_route_vpl<2>(logits, T, E, K, renorm, ids, w, s);
-  if (vpl <= 4) return launch_route_vpl<4>(logits, T, E, K, renorm, ids, w, s);
-  if (vpl <= 8) return launch_route_vpl<8>(logits, T, E, K, renorm, ids, w, s);
-  if (vpl <= 16) return launch_route_vpl<16>(logits, T, E, K, renorm, ids, w, s);
-  return launch_route_vpl<32>(logits, T, E, K, renorm, ids, w, s);
+  if (vpl <= 1) return launch_route_vpl<1>(logits, T, E, K, renorm, P, M, ids, w, s);
+  if (vpl <= 2) return launch_route_vpl<2>(logits, T, E, K, renorm, P, M, ids, w, s);
+  if (vpl <= 4) return launch_route_vpl<4>(logits, T, E, K, renorm, P, M, ids, w, s);
+  if (vpl <= 8) return launch_route_vpl<8>(logits, T, E, K, renorm, P, M, ids, w, s);
+  if (vpl <= 16) return launch_route_vpl<16>(logits, T, E, K, renorm, P, M, ids, w, s);
+  return launch_route_vpl<32>(logits, T, E, K, renorm, P, M, ids, w, s);
 }
 
 int scan_max_blocks(long long TK) {

@@ -70,6 +70,36 @@ def test_route_matches_oracle(T, E, K, renorm, gen):
             assert np.allclose(cpu(w).sum(axis=1), 1.0, atol=1e-6)
 
 
+LIMITED_CASES = [  # T, E, K, P, M, renormalize, generator
+    (300, 256, 8, 8, 4, True, "random"), (200, 896, 16, 64, 8, True, "random"), (100, 16, 3, 4, 2, True, "quantized"),
+    (129, 64, 6, 16, 3, False, "special"), (77, 1024, 8, 256, 4, True, "random"), (50, 32, 4, 32, 4, True, "random"),
+    (64, 48, 5, 6, 1, True, "quantized"),
+]
+
+
+@pytest.mark.parametrize("T,E,K,P,M,renorm,gen", LIMITED_CASES)
+def test_route_limited_matches_oracle(T, E, K, P, M, renorm, gen):
+    seed = T + E + M
+    l = {"random": lambda: inputs.random_logits(T, E, seed=seed, scale=2.0),
+         "quantized": lambda: inputs.quantized_logits(T, E, levels=4, seed=seed),
+         "special": lambda: inputs.special_logits(T, E, seed=seed)}[gen]()
+    d = B.dims(T=T, H=8, E=E, K=K, F=8, P=P, renormalize=renorm, group_limit=M)
+    ids = torch.full((T, K), -7, dtype=torch.int32, device=DEV)
+    w = torch.empty((T, K), dtype=torch.float32, device=DEV)
+    B.moe_route(l.to(DEV), d, ids, w)
+    torch.cuda.synchronize()
+    rid, rw = oracle.route_limited(l.numpy(), K, P, M, renorm)
+    assert np.array_equal(cpu(ids), rid)
+    if gen != "special":
+        np.testing.assert_allclose(cpu(w), rw, atol=WEIGHT_ABS, rtol=0)
+
+
+def test_route_limited_argument_checks():
+    with pytest.raises(B.MoEError):
+        B.moe_route(torch.zeros((4, 16), device=DEV), B.dims(T=4, H=8, E=16, K=5, F=8, P=4, group_limit=1),
+                    torch.empty((4, 5), dtype=torch.int32, device=DEV), torch.empty((4, 5), device=DEV))
+
+
 # ---------------------------------------------------------------------------
 # S2 count + scan
 # ---------------------------------------------------------------------------

@@ -432,3 +432,70 @@ def test_sizing_figures_from_pages():
     assert 100.0 * (cs["local_experts"] - cs["K"]) / cs["local_experts"] == cs["cold_percent"]
     th = g["topk_halving"]
     assert oracle.dispatch_bytes(4096, th["K_to"], 2048, 2) / oracle.dispatch_bytes(4096, th["K_from"], 2048, 2) == th["ratio"]
+
+
+# ---------------------------------------------------------------------------
+# Node-limited routing (a variant of S1)
+# ---------------------------------------------------------------------------
+
+def _brute_limited(row, K, P, M):
+    """Every choice of M groups, every K-subset of their experts: the selection is the
+    unique K-set that beats every other expert of the kept groups, where the kept groups
+    are the M whose best experts beat the best experts of the others."""
+    E = len(row)
+    epp = E // P
+
+    def best(g):
+        b = g * epp
+        for j in range(g * epp, (g + 1) * epp):
+            if _beats(row[j], j, row[b], b):
+                b = j
+        return b
+
+    bests = [best(g) for g in range(P)]
+    kept = None
+    for G in itertools.combinations(range(P), M):
+        rest = [g for g in range(P) if g not in G]
+        if all(_beats(row[bests[a]], bests[a], row[bests[b]], bests[b]) for a in G for b in rest):
+            assert kept is None
+            kept = G
+    allowed = [j for j in range(E) if j // epp in kept]
+    return sorted_topk(row, allowed, K)
+
+
+def sorted_topk(row, allowed, K):
+    out = []
+    for i in allowed:
+        pos = 0
+        while pos < len(out) and _beats(row[out[pos]], out[pos], row[i], i):
+            pos += 1
+        out.insert(pos, i)
+    return out[:K]
+
+
+@pytest.mark.parametrize("gen", ["random", "quantized", "special"])
+@pytest.mark.parametrize("E,P,M,K", [(8, 4, 2, 3), (12, 6, 1, 2), (9, 3, 2, 4), (8, 8, 3, 3), (6, 2, 2, 5)])
+def test_route_limited_matches_brute_force(gen, E, P, M, K):
+    T = 30
+    l = {"random": inputs.random_logits, "quantized": lambda T, E, seed: inputs.quantized_logits(T, E, 3, seed),
+         "special": inputs.special_logits}[gen](T, E, seed=E * P + M).numpy()
+    ids, _ = oracle.route_limited(l, K, P, M)
+    for t in range(T):
+        assert list(ids[t]) == _brute_limited([float(v) for v in l[t]], K, P, M), (t, l[t])
+
+
+def test_route_limited_special_cases():
+    l = inputs.random_logits(50, 16, seed=4).numpy()
+    # all groups kept -> plain top-K
+    assert np.array_equal(oracle.route_limited(l, 5, 4, 4)[0], oracle.route(l, 5)[0])
+    # one expert per group and M >= K -> plain top-K
+    assert np.array_equal(oracle.route_limited(l, 3, 16, 5)[0], oracle.route(l, 3)[0])
+    # M = 1: all K experts in one group (the group of the best expert)
+    ids, w = oracle.route_limited(l, 3, 4, 1)
+    best = oracle.route(l, 1)[0][:, 0]
+    assert np.all(ids // 4 == (best // 4)[:, None])
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-6)
+    # hand example: groups {0,1} {2,3} {4,5}; best group is {4,5} (logit 9); then {0,1} (5)
+    row = np.array([[5.0, 1.0, 4.0, 4.5, 9.0, 0.0]], np.float32)
+    ids, _ = oracle.route_limited(row, 3, 3, 2)
+    assert list(ids[0]) == [4, 0, 1]          # 3 and 2 are excluded although 4.5 > 1.0
