@@ -47,6 +47,8 @@ def parse():
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     p.add_argument("--group-limit", type=int, default=0,
                    help="node-limited routing: experts from the M best partitions (0 = off)")
+    p.add_argument("--shared-expert", type=int, default=0, metavar="F_SHARED",
+                   help="add a shared expert of this width, run on a second stream beside the routed path")
     return p.parse_args()
 
 
@@ -194,13 +196,18 @@ def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 16):
     bias_np = None if bias is None else bias.numpy()
     w_dp_b = None if w_dp is None else inputs.to_bits(w_dp)
     w_upp_b = None if w_upp is None else inputs.to_bits(w_upp)
+    sh = inputs.make_shared_expert(cfg, "cpu")
+    sh_b = None if sh is None else tuple(inputs.to_bits(t) for t in sh)
     while True:
         idx = torch.randperm(cfg.T, generator=g)[:seed_tokens]
         xs = inputs.to_bits(x_all[idx])
         t0 = time.perf_counter()
         z = oracle.dense_bf16(xs, w_dp_b) if w_dp_b is not None else xs
         logits = oracle.gating_logits(z, w_g_np, bias_np)
-        ids, w = oracle.route(logits, cfg.K, cfg.renormalize)
+        if cfg.group_limit:
+            ids, w = oracle.route_limited(logits, cfg.K, cfg.P, cfg.group_limit, cfg.renormalize)
+        else:
+            ids, w = oracle.route(logits, cfg.K, cfg.renormalize)
         cs = oracle.count_scan(ids, cfg.E, cfg.P)
         xp, _ = oracle.permute(z, cs["row_of_assign"], ids, w, cfg.E, cfg.P)
         busy += time.perf_counter() - t0
@@ -213,7 +220,8 @@ def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 16):
         for e in np.nonzero(cs["counts"])[0]:
             lo, hi = off[e], off[e + 1]
             h[lo:hi], y[lo:hi] = oracle.ffn_rows(xp[lo:hi], *expert(int(e)))
-        out = oracle.combine(y, cs["row_of_assign"], w)
+        y_sh = None if sh_b is None else oracle.ffn_rows(z, *sh_b)[1]
+        out = oracle.combine(y, cs["row_of_assign"], w, y_sh)
         if w_upp_b is not None:
             oracle.dense_bf16(out, w_upp_b)
         busy += time.perf_counter() - t0
@@ -228,6 +236,41 @@ def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 16):
     return dict(value=n_tok / el, unit=UNIT, cores=int(threads), kind="oracle",
                 sample=f"{runs} runs x {seed_tokens} random tokens of {cfg.name} through the whole layer "
                        f"(numpy float64, {el:.1f} s of oracle compute; weights prepared outside the clock)")
+
+
+def shared_expert_overlap(cfg, inp, w, bufs, ws, flush, stream, n, dev) -> dict:
+    """How much of the shared expert the auxiliary stream hides behind the routed path: the
+    routed-only layer, the shared expert alone (one-group FFN over all T rows) and the whole
+    layer, each timed on its own (mean of n L2-flushed runs; not part of the timed value)."""
+    from routing_dispatch_grouped_top_b200 import binding as B
+    d, d0 = B.dims_of(cfg), B.dims_of(cfg.with_(F_shared=0))
+    ds = B.dims(T=cfg.T, H=cfg.H, E=1, K=1, F=cfg.F_shared)
+    w0 = dict(w, w_shared_gate=None, w_shared_up=None, w_shared_down=None)
+    off = torch.tensor([0, cfg.T], dtype=torch.int32, device=dev)
+    rows = bufs["z"] if cfg.d_model else inp["x"]
+    sg, su, sd = w["w_shared_gate"], w["w_shared_up"], w["w_shared_down"]
+    runs = {
+        "layer": lambda: B.moe_layer_forward(inp["x"], w, d, bufs, ws),
+        "routed_only": lambda: B.moe_layer_forward(inp["x"], w0, d0, bufs, ws),
+        "shared_alone": lambda: B.moe_grouped_ffn(rows, off, sg, su, sd, ds, bufs["h_shared"], bufs["y_shared"], ws),
+    }
+    ms = {}
+    for name, fn in runs.items():
+        fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+        for a, b in ev:
+            flush.fill_(1)
+            a.record(stream)
+            fn()
+            b.record(stream)
+        torch.cuda.synchronize()
+        ms[name] = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    if B.read_device_status(ws) != 0:
+        raise RuntimeError("device status set during the shared-expert pass")
+    hidden = (ms["routed_only"] + ms["shared_alone"] - ms["layer"]) / ms["shared_alone"]
+    return {"F_shared": cfg.F_shared, "layer_ms": ms["layer"], "routed_only_ms": ms["routed_only"],
+            "shared_alone_ms": ms["shared_alone"], "hidden_frac": hidden,
+            "stream": "shared expert on an auxiliary stream, forked after the latent down-projection"}
 
 
 def config_dict(cfg, world: int) -> dict:
@@ -262,6 +305,8 @@ def main():
     cfg = CFG.get(args.config)
     if args.group_limit:
         cfg = cfg.with_(group_limit=args.group_limit, name=f"{cfg.name}_node_limited_M{args.group_limit}")
+    if args.shared_expert:
+        cfg = cfg.with_(F_shared=args.shared_expert, name=f"{cfg.name}_shared_expert_Fs{args.shared_expert}")
     if args.impl == "reference":
         return run_reference(args, cfg)
 
@@ -281,8 +326,10 @@ def main():
     d = B.dims_of(cfg)
     inp = inputs.make_layer(cfg, dev)
     w = B.pack_layer_weights(d, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"], inp["w_dp"],
-                             inp["w_upp"])
+                             inp["w_upp"], shared=inp["shared"])
     bufs = B.alloc_layer_buffers(d, dev)
+    if cfg.F_shared:
+        B.attach_aux_stream(bufs, torch.cuda.Stream(dev))
     ws = B.make_workspace(d, dev)
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
@@ -333,6 +380,7 @@ def main():
         step(events[i])
     torch.cuda.synchronize()
     stage_ms = [[ev[j].elapsed_time(ev[j + 1]) for ev in events] for j in range(n_ev - 1)]
+    shared_diag = shared_expert_overlap(cfg, inp, w, bufs, ws, flush, stream, n_diag, dev) if cfg.F_shared else None
 
     # End to end through the host-buffer entry point: every step copies its x from pinned host
     # memory and its output back, inside the timed region.  Steps alternate between two streams,
@@ -341,7 +389,10 @@ def main():
     d_in = cfg.d_model or cfg.H
     lanes = []
     for i in range(2):
-        lanes.append(dict(stream=torch.cuda.Stream(dev), bufs=bufs if i == 0 else B.alloc_layer_buffers(d, dev),
+        lb = bufs if i == 0 else B.alloc_layer_buffers(d, dev)
+        if cfg.F_shared and i > 0:
+            B.attach_aux_stream(lb, torch.cuda.Stream(dev))
+        lanes.append(dict(stream=torch.cuda.Stream(dev), bufs=lb,
                           ws=ws if i == 0 else B.make_workspace(d, dev), xd=torch.empty_like(inp["x"]),
                           oh=torch.empty((cfg.T, d_in), dtype=torch.bfloat16).pin_memory()))
     xh = inp["x"].cpu().pin_memory()
@@ -432,10 +483,11 @@ def main():
             "config": config_dict(cfg, world),
             "roofline": roof,
             "stages_ms": stage_mean,
+            **({"shared_expert": shared_diag} if shared_diag else {}),
             "fractions": frac,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": cfg.T * d_in * 2,
                     "d2h_bytes_per_step": cfg.T * d_in * 2},
-            "gpu_launches": (7 + (2 if cfg.d_model else 0)) * args.steps,
+            "gpu_launches": (7 + (2 if cfg.d_model else 0) + (2 if cfg.F_shared else 0)) * args.steps,
             "clocks": clk.summary(),
             "skew_max_over_mean": float(bufs["skew"].item()),
         }

@@ -61,6 +61,8 @@ typedef struct moe_dims {
   int32_t group_limit;  /* 0, or M: node-limited routing, each token takes its K experts from
                            its M best partitions (a partition ranks by its best expert);
                            needs P <= MOE_MAX_LIMITED_GROUPS and K <= M * E / P */
+  int32_t F_shared;     /* 0, or the width of a shared expert that every token passes through
+                           (a multiple of 8) */
 } moe_dims;
 
 typedef enum moe_status {
@@ -260,10 +262,13 @@ moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w
 /* schedule").                                                               */
 /* ------------------------------------------------------------------------- */
 
-/* out[t][:] = bf16( sum_{k<K} topk_w[t][k] * y[row_of_assign[t*K+k]][:] ),
- * accumulated in fp32 in slot order.  y [TK][H] bf16, out [T][H] bf16. */
+/* out[t][:] = bf16( sum_{k<K} topk_w[t][k] * y[row_of_assign[t*K+k]][:] + shared[t][:] ),
+ * accumulated in fp32 in slot order.  y [TK][H] bf16, out [T][H] bf16; shared: [T][H] bf16
+ * output of a shared expert (added with weight 1: shared experts run on every token
+ * regardless of the router, "Three Parameter Counts...", "What the utilization dashboard
+ * smooths away"), or NULL. */
 moe_status moe_combine(const void* y, const int32_t* row_of_assign, const float* topk_w,
-                       const moe_dims* d, void* out, void* stream);
+                       const void* shared, const moe_dims* d, void* out, void* stream);
 
 /* ------------------------------------------------------------------------- */
 /* S7  Skew statistics                                                       */
@@ -304,6 +309,9 @@ typedef struct moe_layer_weights {
   const void*  w_upp;       /* latent only: [d_model][H] bf16, else NULL     */
   const void*  w_gate_up;   /* optional: w_gate/w_up packed by moe_pack_gate_up;
                                when set the layer uses it (w_gate/w_up may be NULL) */
+  const void*  w_shared_gate; /* shared expert (F_shared > 0): [F_shared][H] bf16    */
+  const void*  w_shared_up;   /* [F_shared][H] bf16                                  */
+  const void*  w_shared_down; /* [H][F_shared] bf16                                  */
 } moe_layer_weights;
 
 typedef struct moe_layer_buffers {
@@ -327,6 +335,12 @@ typedef struct moe_layer_buffers {
   void*    out;             /* [T][H] bf16 (combine output)                  */
   void*    final_out;       /* latent only: [T][d_model] bf16                */
   float*   skew;            /* [1] fp32 max/mean expert load                 */
+  void*    h_shared;        /* shared expert: [T][F_shared] bf16             */
+  void*    y_shared;        /* shared expert output: [T][H] bf16             */
+  void*    aux_stream;      /* NULL, or a cudaStream_t on which the shared expert
+                               runs alongside the routed path                */
+  void*    fork_event;      /* with aux_stream: two cudaEvent_t created by the */
+  void*    join_event;      /* caller (timing disabled is fine)              */
 } moe_layer_buffers;
 
 /* Number of stage boundaries recorded when stage events are given. */
@@ -334,7 +348,10 @@ typedef struct moe_layer_buffers {
 
 /* Runs every step on `stream` in pipeline order: [latent down-projection] ->
  * gating -> route -> count/scan -> permute -> gate/up+SwiGLU -> down -> combine
- * -> [latent up-projection] -> skew statistics.  x: [T][d_in] bf16 with
+ * -> [latent up-projection] -> skew statistics.  With d->F_shared > 0 the shared
+ * expert (gate/up+SwiGLU and down over all T tokens of the routed activations) runs
+ * on b->aux_stream, forked after the routed activations are ready and joined before
+ * the combine, or on `stream` when aux_stream is NULL.  x: [T][d_in] bf16 with
  * d_in = d_model for a latent layer, else H.  stage_events: NULL, or an array of
  * MOE_NUM_STAGE_EVENTS cudaEvent_t (created by the caller) recorded at: start,
  * after latent-down, gating, route, count/scan, permute, gate/up, down,

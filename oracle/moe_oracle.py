@@ -50,6 +50,11 @@ Readings where the pages are silent:
   E followed by renormalising the top-K); with ``renormalize=False`` the weight
   is the plain softmax over all E at the selected experts.
 * Order of rows inside one expert: stable (assignment a = t*K + k ascending).
+* Shared expert [ParamCounts/dashboard: DeepSeekMoE-style shared experts run on every
+  token whatever the router says; InferenceX review claim IX2-0406 lists the shared
+  expert among the replicated non-expert weights]: a SwiGLU FFN of its own width on
+  every token, rounded like a routed expert, added with weight 1 in the combine:
+  out[t] = bf16( sum_k w[t,k] y[row(t,k)] + s[t] ).
 * Node-limited routing: the groups are the P partitions; a group ranks by its best
   expert under the top-k order; each token keeps its M best groups and takes its K
   experts from those groups only.
@@ -326,13 +331,16 @@ def grouped_ffn(xp_bits, offsets, w_gate_bits, w_up_bits, w_down_bits):
 # Step S6: combine = unpermute + weighted sum   [WideEP/router], [WideEP/bytes]
 # ----------------------------------------------------------------------------
 
-def combine(y_bits, row_of_assign, topk_w):
-    """out[t] = bf16( sum_{k<K} w[t,k] * y[row_of_assign[t*K+k]] ), summed in slot order."""
+def combine(y_bits, row_of_assign, topk_w, shared_bits=None):
+    """out[t] = bf16( sum_{k<K} w[t,k] * y[row_of_assign[t*K+k]] (+ s[t]) ), summed in slot order;
+    s is the shared expert's output when given."""
     w = np.asarray(topk_w, dtype=np.float32).astype(np.float64)
     T, K = w.shape
     y = bf16_bits_to_f64(y_bits)
     roa = np.asarray(row_of_assign, dtype=np.int64).reshape(T, K)
     acc = np.zeros((T, y.shape[1]), dtype=np.float64)
+    if shared_bits is not None:
+        acc = acc + bf16_bits_to_f64(shared_bits)
     for k in range(K):
         acc = acc + w[:, k:k + 1] * y[roa[:, k]]
     return f64_to_bf16_bits(acc)
@@ -375,8 +383,11 @@ def dense_bf16(x_bits, w_bits):
 
 def layer_forward(x_bits, w_g, w_gate_bits, w_up_bits, w_down_bits, K: int, P: int = 1,
                   renormalize: bool = True, bias=None, w_dp_bits=None, w_upp_bits=None,
-                  logits=None, group_limit: int = 0):
+                  logits=None, group_limit: int = 0, shared=None):
     """All steps in pipeline order.  Returns a dict with every intermediate.
+
+    ``shared`` = (W_gate_s [Fs][d], W_up_s [Fs][d], W_down_s [d][Fs]) bf16 bits adds a shared
+    expert on the routed activations (x, or z for a latent layer).
 
     If ``logits`` is given it replaces the oracle's own gating output (used by
     the routing tests, which hand both sides the same float32 logits).
@@ -401,7 +412,11 @@ def layer_forward(x_bits, w_g, w_gate_bits, w_up_bits, w_down_bits, K: int, P: i
     res["meta"] = meta
     h, y = grouped_ffn(xp, cs["offsets"], w_gate_bits, w_up_bits, w_down_bits)
     res["h"], res["y"] = h, y
-    out = combine(y, cs["row_of_assign"], w)
+    s_bits = None
+    if shared is not None:
+        res["h_shared"], s_bits = ffn_rows(z, *shared)
+        res["y_shared"] = s_bits
+    out = combine(y, cs["row_of_assign"], w, s_bits)
     res["out"] = out
     if w_upp_bits is not None:
         res["final"] = dense_bf16(out, w_upp_bits)

@@ -32,10 +32,12 @@ class MoEError(RuntimeError):
 
 class moe_dims(C.Structure):
     _fields_ = [("T", C.c_int64), ("H", C.c_int32), ("E", C.c_int32), ("K", C.c_int32), ("F", C.c_int32),
-                ("P", C.c_int32), ("renormalize", C.c_int32), ("d_model", C.c_int32), ("group_limit", C.c_int32)]
+                ("P", C.c_int32), ("renormalize", C.c_int32), ("d_model", C.c_int32), ("group_limit", C.c_int32),
+                ("F_shared", C.c_int32)]
 
 
-_W_FIELDS = ("w_g_split", "bias", "w_gate", "w_up", "w_down", "w_dp", "w_upp", "w_gate_up")
+_W_FIELDS = ("w_g_split", "bias", "w_gate", "w_up", "w_down", "w_dp", "w_upp", "w_gate_up", "w_shared_gate",
+             "w_shared_up", "w_shared_down")
 
 
 class moe_layer_weights(C.Structure):
@@ -44,7 +46,7 @@ class moe_layer_weights(C.Structure):
 
 _BUF_FIELDS = ("z", "logits", "topk_ids", "topk_w", "counts", "offsets", "part_counts", "part_offsets",
                "row_of_assign", "assign_of_row", "xp", "meta_token", "meta_slot", "meta_w", "meta_local_expert",
-               "h", "y", "out", "final_out", "skew")
+               "h", "y", "out", "final_out", "skew", "h_shared", "y_shared", "aux_stream", "fork_event", "join_event")
 
 
 class moe_layer_buffers(C.Structure):
@@ -70,7 +72,7 @@ _SIGS = {
     "moe_packed_gate_up_bytes": (_SZ, [_DP]),
     "moe_pack_gate_up": (C.c_int, [_VP, _VP, _DP, _VP, _VP]),
     "moe_grouped_gate_up_packed": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
-    "moe_combine": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP]),
+    "moe_combine": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP]),
     "moe_skew_stats": (C.c_int, [_VP, _DP, _VP, _VP]),
     "moe_p95": (C.c_double, [C.POINTER(C.c_float), C.c_int]),
     "moe_dense": (C.c_int, [_VP, _VP, _I64, _I32, _I32, _VP, _VP, _SZ, _VP]),
@@ -105,14 +107,14 @@ def _check(fn: str, status: int):
         raise MoEError(fn, status, lib().moe_status_str(status).decode())
 
 
-def dims(T, H, E, K, F, P=1, renormalize=True, d_model=0, group_limit=0) -> moe_dims:
+def dims(T, H, E, K, F, P=1, renormalize=True, d_model=0, group_limit=0, F_shared=0) -> moe_dims:
     return moe_dims(int(T), int(H), int(E), int(K), int(F), int(P), int(bool(renormalize)), int(d_model or 0),
-                    int(group_limit or 0))
+                    int(group_limit or 0), int(F_shared or 0))
 
 
 def dims_of(cfg, T=None) -> moe_dims:
     return dims(cfg.T if T is None else T, cfg.H, cfg.E, cfg.K, cfg.F, cfg.P, cfg.renormalize, cfg.d_model or 0,
-                cfg.group_limit or 0)
+                cfg.group_limit or 0, cfg.F_shared or 0)
 
 
 def _stream(stream) -> int:
@@ -275,12 +277,12 @@ def moe_grouped_down(h, offsets, w_down, d: moe_dims, y, ws, stream=None):
         _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
 
 
-def moe_combine(y, row_of_assign, topk_w, d: moe_dims, out, stream=None):
+def moe_combine(y, row_of_assign, topk_w, d: moe_dims, out, shared=None, stream=None):
     TK = d.T * d.K
     _check("moe_combine", lib().moe_combine(
         _ptr(y, torch.bfloat16, "y", TK * d.H), _ptr(row_of_assign, torch.int32, "row_of_assign", TK),
-        _ptr(topk_w, torch.float32, "topk_w", TK), C.byref(d), _ptr(out, torch.bfloat16, "out", d.T * d.H),
-        _stream(stream)))
+        _ptr(topk_w, torch.float32, "topk_w", TK), _ptr(shared, torch.bfloat16, "shared", d.T * d.H), C.byref(d),
+        _ptr(out, torch.bfloat16, "out", d.T * d.H), _stream(stream)))
 
 
 def moe_skew_stats(counts, d: moe_dims, d_ratio, stream=None):
@@ -318,12 +320,36 @@ def alloc_layer_buffers(d: moe_dims, device="cuda", meta=True) -> dict:
              xp=e((TK, d.H), bf), meta_token=e((TK,), i32) if meta else None,
              meta_slot=e((TK,), i32) if meta else None, meta_w=e((TK,), f32) if meta else None,
              meta_local_expert=e((TK,), i32) if meta else None, h=e((TK, d.F), bf), y=e((TK, d.H), bf),
-             out=e((T, d.H), bf), final_out=e((T, d.d_model), bf) if d.d_model else None, skew=e((1,), f32))
+             out=e((T, d.H), bf), final_out=e((T, d.d_model), bf) if d.d_model else None, skew=e((1,), f32),
+             h_shared=e((T, d.F_shared), bf) if d.F_shared else None,
+             y_shared=e((T, d.H), bf) if d.F_shared else None)
     return b
 
 
+def attach_aux_stream(buffers: dict, stream: torch.cuda.Stream) -> dict:
+    """Lets the shared expert run on ``stream`` beside the routed path (events created here)."""
+    buffers["aux_stream"] = stream
+    buffers["fork_event"] = torch.cuda.Event()
+    buffers["join_event"] = torch.cuda.Event()
+    for ev in (buffers["fork_event"], buffers["join_event"]):
+        ev.record(stream)               # torch creates the CUDA event on its first record
+    return buffers
+
+
+def _handle(v):
+    if v is None:
+        return None
+    if isinstance(v, torch.Tensor):
+        return v.data_ptr()
+    if isinstance(v, torch.cuda.Stream):
+        return v.cuda_stream
+    if isinstance(v, torch.cuda.Event):
+        return v.cuda_event
+    raise TypeError(type(v))
+
+
 def _buffers_struct(b: dict) -> moe_layer_buffers:
-    return moe_layer_buffers(*[(b[n].data_ptr() if b.get(n) is not None else None) for n in _BUF_FIELDS])
+    return moe_layer_buffers(*[_handle(b.get(n)) for n in _BUF_FIELDS])
 
 
 def _weights_struct(w: dict) -> moe_layer_weights:
@@ -339,7 +365,7 @@ PACK_GATE_UP_MIN_ROWS_PER_EXPERT = 64
 
 
 def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, w_upp=None, stream=None,
-                       pack_gate_up_weights=None) -> dict:
+                       pack_gate_up_weights=None, shared=None) -> dict:
     """One-time weight preparation: router split into three bf16 planes and, when
     ``pack_gate_up_weights`` (default: H >= PACK_GATE_UP_MIN_H), gate/up interleaved for the
     packed gate/up GEMM."""
@@ -357,8 +383,12 @@ def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, 
     if bias is not None:
         _ptr(bias, torch.float32, "bias", d.E)
     w_gu = pack_gate_up(w_gate, w_up, d, stream) if pack_gate_up_weights else None
+    sg, su, sd = shared if shared is not None else (None, None, None)
+    if d.F_shared:
+        for name, t in (("w_shared_gate", sg), ("w_shared_up", su), ("w_shared_down", sd)):
+            _ptr(t, torch.bfloat16, name, d.F_shared * d.H)
     return dict(w_g_split=split, bias=bias, w_gate=w_gate, w_up=w_up, w_down=w_down, w_dp=w_dp, w_upp=w_upp,
-                w_gate_up=w_gu)
+                w_gate_up=w_gu, w_shared_gate=sg, w_shared_up=su, w_shared_down=sd)
 
 
 def moe_layer_forward(x, weights: dict, d: moe_dims, buffers: dict, ws, stage_events=None, stream=None):

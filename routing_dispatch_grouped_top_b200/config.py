@@ -25,6 +25,7 @@ class MoEConfig:
     zipf_s: Optional[float] = None      # per-expert logit bias drawn from rank-Zipf popularity
     d_model: Optional[int] = None       # latent layer: model width before the down-projection
     group_limit: int = 0                # node-limited routing: experts from the M best partitions
+    F_shared: int = 0                   # width of a shared expert every token passes through (0: none)
     seed: int = 0
 
     @property

@@ -52,6 +52,8 @@ moe_status check_dims(const moe_dims* d) {
       (d->group_limit > 0 && d->K > static_cast<long long>(d->group_limit) * (d->E / d->P)))
     return MOE_ERR_INVALID_ARG;
   if (d->group_limit > 0 && d->P > MOE_MAX_LIMITED_GROUPS) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (d->F_shared < 0) return MOE_ERR_INVALID_ARG;
+  if (d->F_shared % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (d->T * static_cast<long long>(d->K) > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
@@ -245,13 +247,13 @@ moe_status moe_grouped_ffn(const void* xp, const int32_t* offsets, const void* w
   return moe_grouped_down(h, offsets, w_down, d, y, ws, ws_bytes, stream);
 }
 
-moe_status moe_combine(const void* y, const int32_t* row_of_assign, const float* topk_w, const moe_dims* d,
-                       void* out, void* stream) {
+moe_status moe_combine(const void* y, const int32_t* row_of_assign, const float* topk_w, const void* shared,
+                       const moe_dims* d, void* out, void* stream) {
   MOE_TRY(common_checks(d));
   if (d->T == 0) return MOE_OK;
   if (!y || !row_of_assign || !topk_w || !out) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(y) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_combine(y, row_of_assign, topk_w, d->T, d->H, d->K, out, as_stream(stream)));
+  if (!aligned16(y) || !aligned16(out) || !aligned16(shared)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_combine(y, row_of_assign, topk_w, shared, d->T, d->H, d->K, out, as_stream(stream)));
 }
 
 moe_status moe_skew_stats(const int32_t* counts, const moe_dims* d, float* d_ratio, void* stream) {
@@ -288,6 +290,10 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   const bool latent = d->d_model > 0;
   if (!w->w_g_split || !w->w_down || (!w->w_gate_up && (!w->w_gate || !w->w_up))) return MOE_ERR_INVALID_ARG;
   if (latent && (!w->w_dp || !w->w_upp || !b->z || !b->final_out)) return MOE_ERR_INVALID_ARG;
+  const bool shared = d->F_shared > 0;
+  if (shared && (!w->w_shared_gate || !w->w_shared_up || !w->w_shared_down || !b->h_shared || !b->y_shared))
+    return MOE_ERR_INVALID_ARG;
+  if (shared && b->aux_stream && (!b->fork_event || !b->join_event)) return MOE_ERR_INVALID_ARG;
   if (!b->logits || !b->topk_ids || !b->topk_w || !b->counts || !b->offsets || !b->part_counts ||
       !b->part_offsets || !b->row_of_assign || !b->assign_of_row || !b->xp || !b->h || !b->y || !b->out)
     return MOE_ERR_INVALID_ARG;
@@ -306,6 +312,19 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
     routed = b->z;
   }
   MOE_TRY(mark(1));
+  // Shared expert: a dense SwiGLU over every token, beside the routed path.
+  cudaStream_t sh = s;
+  if (shared && T > 0) {
+    if (b->aux_stream) {
+      sh = as_stream(b->aux_stream);
+      MOE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(b->fork_event), s));
+      MOE_CUDA(cudaStreamWaitEvent(sh, reinterpret_cast<cudaEvent_t>(b->fork_event), 0));
+    }
+    MOE_CUDA(gemm_gate_up(routed, nullptr, w->w_shared_gate, w->w_shared_up, 1, T, d->H, d->F_shared, b->h_shared,
+                          status, sh));
+    MOE_CUDA(gemm_down(b->h_shared, nullptr, w->w_shared_down, 1, T, d->H, d->F_shared, b->y_shared, status, sh));
+    if (b->aux_stream) MOE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(b->join_event), sh));
+  }
   if (T > 0) MOE_CUDA(gemm_gating(routed, w->w_g_split, w->bias, T, d->H, d->E, b->logits, status, s));
   MOE_TRY(mark(2));
   MOE_CUDA(launch_route(b->logits, T, d->E, d->K, d->renormalize, d->P, d->group_limit, b->topk_ids, b->topk_w, s));
@@ -325,7 +344,10 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   MOE_TRY(mark(6));
   if (T > 0) MOE_CUDA(gemm_down(b->h, b->offsets, w->w_down, d->E, TK, d->H, d->F, b->y, status, s));
   MOE_TRY(mark(7));
-  MOE_CUDA(launch_combine(b->y, b->row_of_assign, b->topk_w, T, d->H, d->K, b->out, s));
+  if (shared && T > 0 && b->aux_stream)
+    MOE_CUDA(cudaStreamWaitEvent(s, reinterpret_cast<cudaEvent_t>(b->join_event), 0));
+  MOE_CUDA(launch_combine(b->y, b->row_of_assign, b->topk_w, shared ? b->y_shared : nullptr, T, d->H, d->K,
+                          b->out, s));
   MOE_TRY(mark(8));
   if (latent && T > 0) MOE_CUDA(gemm_dense(b->out, w->w_upp, T, d->d_model, d->H, b->final_out, status, s));
   MOE_TRY(mark(9));

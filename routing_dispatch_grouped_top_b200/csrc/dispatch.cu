@@ -84,8 +84,9 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
 template <int KC>
 __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const uint4* __restrict__ y,
                                                                const int32_t* __restrict__ roa,
-                                                               const float* __restrict__ w, long long T, int vpr,
-                                                               int K, uint4* __restrict__ out) {
+                                                               const float* __restrict__ w,
+                                                               const uint4* __restrict__ shared, long long T,
+                                                               int vpr, int K, uint4* __restrict__ out) {
   pdl_wait();  // y comes from the down-projection GEMM
   pdl_launch_dependents();
   const long long n_items = T * vpr;
@@ -98,6 +99,16 @@ __global__ void __launch_bounds__(kCopyThreads) combine_kernel(const uint4* __re
     float acc[8];
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[j] = 0.0f;
+    if (shared) {  // shared expert output, weight 1
+      const uint4 sv = ld_stream(shared + it);
+      const __nv_bfloat162* ps = reinterpret_cast<const __nv_bfloat162*>(&sv);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float2 f = __bfloat1622float2(ps[j]);
+        acc[2 * j] = f.x;
+        acc[2 * j + 1] = f.y;
+      }
+    }
     // slots in order; KC rows fetched before they are summed
     for (int k0 = 0; k0 < K; k0 += KC) {
       uint4 yv[KC];
@@ -202,16 +213,16 @@ cudaError_t launch_permute(const void* x, const int32_t* roa, const int32_t* ids
                     meta_token, meta_slot, meta_w, meta_local);
 }
 
-cudaError_t launch_combine(const void* y, const int32_t* roa, const float* w, long long T, int H, int K, void* out,
-                           cudaStream_t s) {
+cudaError_t launch_combine(const void* y, const int32_t* roa, const float* w, const void* shared, long long T, int H,
+                           int K, void* out, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int vpr = H / 8;
   const int blocks = copy_blocks(T * vpr);
   if (K <= 2)
     return launch_pdl(combine_kernel<2>, dim3(blocks), dim3(kCopyThreads), 0, s, reinterpret_cast<const uint4*>(y),
-                      roa, w, T, vpr, K, reinterpret_cast<uint4*>(out));
+                      roa, w, reinterpret_cast<const uint4*>(shared), T, vpr, K, reinterpret_cast<uint4*>(out));
   return launch_pdl(combine_kernel<4>, dim3(blocks), dim3(kCopyThreads), 0, s, reinterpret_cast<const uint4*>(y),
-                    roa, w, T, vpr, K, reinterpret_cast<uint4*>(out));
+                    roa, w, reinterpret_cast<const uint4*>(shared), T, vpr, K, reinterpret_cast<uint4*>(out));
 }
 
 cudaError_t launch_pack_gate_up(const void* w_gate, const void* w_up, int E, int H, int F, void* w_gu,

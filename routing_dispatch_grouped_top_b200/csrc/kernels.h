@@ -76,8 +76,8 @@ cudaError_t launch_skew(const int32_t* counts, int E, float* ratio, cudaStream_t
 cudaError_t launch_permute(const void* x, const int32_t* row_of_assign, const int32_t* ids, const float* w,
                            long long T, int H, int E, int K, int P, void* xp, int32_t* meta_token,
                            int32_t* meta_slot, float* meta_w, int32_t* meta_local, cudaStream_t stream);
-cudaError_t launch_combine(const void* y, const int32_t* row_of_assign, const float* w, long long T, int H, int K,
-                           void* out, cudaStream_t stream);
+cudaError_t launch_combine(const void* y, const int32_t* row_of_assign, const float* w, const void* shared,
+                           long long T, int H, int K, void* out, cudaStream_t stream);
 cudaError_t launch_pack_router(const float* w_g, int H, int E, void* w_split, cudaStream_t stream);
 
 }  // namespace moe

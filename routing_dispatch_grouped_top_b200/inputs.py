@@ -11,6 +11,7 @@ Recipe (the pages name no dataset; these stand in for real activations):
   [E][F][H]; W_down ~ N(0, 1/F), [E][H][F].
 * Latent layer: W_dp ~ N(0, 1/d_model), [H][d_model]; W_up_proj ~ N(0, 1/H),
   [d_model][H].
+* Shared expert (optional): like a routed expert of width F_shared.
 * Skewed decode router: popularity p_r proportional to r^(-s) over ranks
   r = 1..E, ranks assigned to experts by a seeded random permutation pi, and a
   logit bias bias_e = beta * ln(p_pi(e) * E).  beta is a fixed constant,
@@ -90,12 +91,22 @@ def make_latent(cfg: MoEConfig, device="cpu"):
     return w_dp, w_upp
 
 
+def make_shared_expert(cfg: MoEConfig, device="cpu"):
+    """(W_gate_s, W_up_s [F_shared][H], W_down_s [H][F_shared]) bf16, or None."""
+    if not cfg.F_shared:
+        return None
+    g = _gen(device, 307 + cfg.seed)
+    Fs, H = cfg.F_shared, cfg.H
+    return (_randn((Fs, H), H ** -0.5, g, device, torch.bfloat16), _randn((Fs, H), H ** -0.5, g, device, torch.bfloat16),
+            _randn((H, Fs), Fs ** -0.5, g, device, torch.bfloat16))
+
+
 def make_layer(cfg: MoEConfig, device="cpu", step: int = 0) -> dict:
     w_g, bias = make_router(cfg, device)
     w_gate, w_up, w_down = make_experts(cfg, device)
     w_dp, w_upp = make_latent(cfg, device)
     return dict(x=make_tokens(cfg, device, step), w_g=w_g, bias=bias, w_gate=w_gate,
-                w_up=w_up, w_down=w_down, w_dp=w_dp, w_upp=w_upp)
+                w_up=w_up, w_down=w_down, w_dp=w_dp, w_upp=w_upp, shared=make_shared_expert(cfg, device))
 
 
 # ---------------------------------------------------------------------------

@@ -42,11 +42,13 @@ def cpu(t):
     return t.detach().cpu().numpy()
 
 
-def run_gpu_layer(cfg, inp, packed=True):
+def run_gpu_layer(cfg, inp, packed=True, aux=False):
     d = B.dims_of(cfg)
     w = B.pack_layer_weights(d, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"], inp["w_dp"],
-                             inp["w_upp"], pack_gate_up_weights=packed)
+                             inp["w_upp"], pack_gate_up_weights=packed, shared=inp["shared"])
     bufs = B.alloc_layer_buffers(d)
+    if aux:
+        B.attach_aux_stream(bufs, torch.cuda.Stream())
     ws = B.make_workspace(d)
     B.moe_layer_forward(inp["x"], w, d, bufs, ws)
     assert B.read_device_status(ws) == 0
@@ -112,23 +114,33 @@ SMALL = [
     LATENT_896E.with_(name="latent_shape_T48_D1024_H256_E112_P8", T=48, d_model=1024, H=256, E=112, F=128, P=8),
     TINY.with_(name="one_token", T=1),
     DEEPSEEK_R1_PREFILL.with_(name="r1_shape_node_limited_T96_H512_F256_M4", T=96, H=512, F=256, group_limit=4),
+    DEEPSEEK_R1_PREFILL.with_(name="r1_shape_shared_expert_T80_H512_F256_E32_Fs384", T=80, H=512, F=256, E=32,
+                              F_shared=384),
+    LATENT_896E.with_(name="latent_shared_expert_T40_D512_H256_E64_Fs128", T=40, d_model=512, H=256, E=64, F=128,
+                      P=8, F_shared=128),
 ]
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
 def test_layer_matches_oracle(cfg):
     inp = inputs.make_layer(cfg, DEV)
-    # both gate/up paths: separate weights for two layers, packed weights for the others
-    g = run_gpu_layer(cfg, inp, packed=cfg.name not in ("tiny_T100_P2_plain_softmax", "one_token"))
+    # both gate/up paths: separate weights for two layers, packed weights for the others;
+    # the shared expert on its own stream in one layer and in line in the other
+    g = run_gpu_layer(cfg, inp, packed=cfg.name not in ("tiny_T100_P2_plain_softmax", "one_token"),
+                      aux=cfg.name.startswith("r1_shape_shared"))
     torch.cuda.synchronize()
-    cpu_in = {k: (v.cpu() if v is not None else None) for k, v in inp.items()}
+    cpu_in = {k: (v.cpu() if isinstance(v, torch.Tensor) else None) for k, v in inp.items()}
+    shared = None if inp["shared"] is None else tuple(bits(t) for t in inp["shared"])
     r = oracle.layer_forward(bits(cpu_in["x"]), cpu_in["w_g"].numpy(), bits(cpu_in["w_gate"]),
                              bits(cpu_in["w_up"]), bits(cpu_in["w_down"]), cfg.K, cfg.P, cfg.renormalize,
                              bias=None if cpu_in["bias"] is None else cpu_in["bias"].numpy(),
                              w_dp_bits=None if cpu_in["w_dp"] is None else bits(cpu_in["w_dp"]),
                              w_upp_bits=None if cpu_in["w_upp"] is None else bits(cpu_in["w_upp"]),
-                             group_limit=cfg.group_limit)
+                             group_limit=cfg.group_limit, shared=shared)
     latent = bool(cfg.d_model)
+    if shared is not None and not latent:
+        check_bf16("h_shared", bits(g["h_shared"]), r["h_shared"])
+        check_bf16("y_shared", bits(g["y_shared"]), r["y_shared"])
     if latent:
         check_bf16("z", bits(g["z"]), r["z"])
         # logits of a latent layer inherit z's bf16 rounding flips: bf16-in / fp32-out tolerance

@@ -320,16 +320,18 @@ def test_grouped_gemm_rejects_bad_offsets_without_touching_memory():
 # S6 combine
 # ---------------------------------------------------------------------------
 
+@pytest.mark.parametrize("with_shared", [False, True], ids=["routed", "plus_shared"])
 @pytest.mark.parametrize("T,H,K", [(300, 256, 2), (77, 7168, 8), (1000, 2048, 16), (5, 8, 1), (64, 512, 32)])
-def test_combine_matches_oracle(T, H, K):
+def test_combine_matches_oracle(T, H, K, with_shared):
     y = inputs.random_bf16((T * K, H), seed=T + H)
     roa = inputs.random_bijection(T * K, seed=K)
     w = inputs.random_weights(T, K, seed=T)
+    s = inputs.random_bf16((T, H), seed=T + 3, std=0.5) if with_shared else None
     d = B.dims(T=T, H=H, E=max(K, 2), K=K, F=8)
     out = torch.zeros((T, H), dtype=torch.bfloat16, device=DEV)
-    B.moe_combine(y.to(DEV), roa.to(DEV), w.to(DEV), d, out)
+    B.moe_combine(y.to(DEV), roa.to(DEV), w.to(DEV), d, out, shared=None if s is None else s.to(DEV))
     torch.cuda.synchronize()
-    ref = oracle.combine(bits(y), roa.numpy(), w.numpy())
+    ref = oracle.combine(bits(y), roa.numpy(), w.numpy(), None if s is None else bits(s))
     check_bf16("out", bits(out), ref)
 
 

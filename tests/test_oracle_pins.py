@@ -499,3 +499,39 @@ def test_route_limited_special_cases():
     row = np.array([[5.0, 1.0, 4.0, 4.5, 9.0, 0.0]], np.float32)
     ids, _ = oracle.route_limited(row, 3, 3, 2)
     assert list(ids[0]) == [4, 0, 1]          # 3 and 2 are excluded although 4.5 > 1.0
+
+
+# ---------------------------------------------------------------------------
+# Shared expert (added in the combine)
+# ---------------------------------------------------------------------------
+
+def test_combine_with_shared_expert_closed_form():
+    y = bf([[1.0, 2.0], [4.0, 8.0]])
+    roa = np.array([1, 0], np.int32)                # token 0 -> rows 1, 0
+    w = np.array([[0.25, 0.75]], np.float32)
+    s = bf([[0.5, -6.0]])
+    out = val(oracle.combine(y, roa, w, s))
+    assert np.array_equal(out, [[0.25 * 4 + 0.75 * 1 + 0.5, 0.25 * 8 + 0.75 * 2 - 6.0]])
+
+
+def test_layer_shared_expert_is_a_dense_swiglu_added_to_every_token():
+    cfg = TINY
+    d = inputs.make_layer(cfg)
+    xs = inputs.to_bits(d["x"])
+    args = (xs, d["w_g"].numpy(), inputs.to_bits(d["w_gate"]), inputs.to_bits(d["w_up"]),
+            inputs.to_bits(d["w_down"]), cfg.K, cfg.P)
+    Fs = 64
+    sh = (inputs.to_bits(inputs.random_bf16((Fs, cfg.H), seed=7, std=cfg.H ** -0.5)),
+          inputs.to_bits(inputs.random_bf16((Fs, cfg.H), seed=8, std=cfg.H ** -0.5)),
+          inputs.to_bits(inputs.random_bf16((cfg.H, Fs), seed=9, std=Fs ** -0.5)))
+    plain = oracle.layer_forward(*args)
+    with_s = oracle.layer_forward(*args, shared=sh)
+    # routing and the routed experts are untouched
+    for k in ("topk_ids", "row_of_assign", "xp", "h", "y"):
+        assert np.array_equal(plain[k], with_s[k])
+    # the shared expert equals a dense SwiGLU of every token
+    _, s_dense = oracle.ffn_rows(xs, *sh)
+    assert np.array_equal(with_s["y_shared"], s_dense)
+    # zero shared weights leave the output unchanged
+    zero = tuple(np.zeros_like(a) for a in sh)
+    assert np.array_equal(oracle.layer_forward(*args, shared=zero)["out"], plain["out"])
