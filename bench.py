@@ -49,6 +49,9 @@ def parse():
                    help="node-limited routing: experts from the M best partitions (0 = off)")
     p.add_argument("--shared-expert", type=int, default=0, metavar="F_SHARED",
                    help="add a shared expert of this width, run on a second stream beside the routed path")
+    p.add_argument("--shape", action="append", default=[], metavar="FIELD=INT",
+                   help="override one integer field of the workload (T, E, H, F, K, P); for reduced-size "
+                        "profiling captures of a workload's kernels, e.g. --shape T=1024 --shape E=32")
     return p.parse_args()
 
 
@@ -275,7 +278,8 @@ def shared_expert_overlap(cfg, inp, w, bufs, ws, flush, stream, n, dev) -> dict:
 
 def config_dict(cfg, world: int) -> dict:
     return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K, "F": cfg.F, "P": cfg.P,
-            "d_model": cfg.d_model, "parallelism": f"replicas{world}",
+            "d_model": cfg.d_model, "group_limit": cfg.group_limit, "F_shared": cfg.F_shared,
+            "parallelism": f"replicas{world}",
             "l2": "flushed (256 MiB write) before every timed step, outside its events"}
 
 
@@ -305,6 +309,13 @@ def main():
     cfg = CFG.get(args.config)
     if args.group_limit:
         cfg = cfg.with_(group_limit=args.group_limit, name=f"{cfg.name}_node_limited_M{args.group_limit}")
+    for kv in args.shape:
+        k, v = kv.split("=")
+        if k not in ("T", "E", "H", "F", "K", "P"):
+            raise SystemExit(f"--shape: unknown field {k}")
+        cfg = cfg.with_(**{k: int(v)})
+    if args.shape:
+        cfg = cfg.with_(name=f"{cfg.name}_reshaped_" + "_".join(args.shape).replace("=", ""))
     if args.shared_expert:
         cfg = cfg.with_(F_shared=args.shared_expert, name=f"{cfg.name}_shared_expert_Fs{args.shared_expert}")
     if args.impl == "reference":
