@@ -66,6 +66,17 @@ Readings where the pages are silent:
 * Combine: out[t] = bf16( sum_k w[t,k] * y[row(t,k)] ), summed in slot order.
 * Latent layer: z = bf16(x Wdp^T) is routed and dispatched; the final output is
   bf16(out Wup^T).
+* FP8 dispatch [WideEP/bytes: low-precision dispatch quantizes the outbound
+  activation, carries its scales, computes in the other format and returns at higher
+  precision; DeepEP's published examples dispatch in FP8 and combine in BF16]: the
+  format is E4M3 (bias 7, 3 mantissa bits, largest finite 448, no infinities, code
+  0x7F/0xFF = NaN) with one fp32 scale per row, s = amax(|row|) / 448 (1 for an
+  all-zero row) and code = round-to-nearest-even(x / s) saturated to +-448, the
+  scale and the quotient both taken in fp32 (the float decides an integer code, so
+  it is decided in the kernel's precision).  Activations are quantized per token (the
+  K dispatched copies share the token's codes and scale), gate and up weights per
+  output feature.  g = s_x s_wg sum_k q_x q_wg (likewise u) from the codes; h, the
+  down projection (bf16 weights) and the combine are as in the bf16 layer.
 """
 from __future__ import annotations
 
@@ -78,6 +89,8 @@ __all__ = [
     "count_scan", "permute", "grouped_ffn", "ffn_rows", "combine",
     "skew_ratio", "p95_nearest_rank", "dense_bf16", "layer_forward", "route_limited",
     "dispatch_bytes", "expert_weight_bytes", "experts_per_partition",
+    "E4M3_MAX", "e4m3_to_f64", "f32_to_e4m3", "quantize_rows_fp8", "dispatch_fp8", "ffn_rows_fp8",
+    "grouped_ffn_fp8", "quantize_experts_fp8", "dispatch_bytes_fp8",
     "checkpoint_bytes",
 ]
 
@@ -328,6 +341,107 @@ def grouped_ffn(xp_bits, offsets, w_gate_bits, w_up_bits, w_down_bits):
 
 
 # ----------------------------------------------------------------------------
+# FP8 dispatch: E4M3 codes with one fp32 scale per row   [WideEP/bytes]
+# ----------------------------------------------------------------------------
+
+E4M3_MAX = 448.0
+
+
+def e4m3_to_f64(codes) -> np.ndarray:
+    """Value of each E4M3 code: sign bit 7, exponent bits 6..3 (bias 7), mantissa bits 2..0;
+    exponent 0 is subnormal (m * 2^-9); exponent 15 with mantissa 7 is NaN."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m * 2.0 ** -9, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7.0))
+    mag = np.where((e == 15) & ((c & 7) == 7), np.nan, mag)
+    return np.where(c & 0x80, -mag, mag)
+
+
+def f32_to_e4m3(v) -> np.ndarray:
+    """Nearest E4M3 code of each fp32 value (ties to an even mantissa), saturating to +-448
+    (infinities included); NaN gives 0x7F."""
+    v32 = np.asarray(v, dtype=np.float32)
+    finite = np.isfinite(v32)
+    a = np.where(finite, np.abs(v32).astype(np.float64), 0.0)
+    frac, ex = np.frexp(a)                       # a = frac * 2^ex, frac in [0.5, 1)
+    unb = ex.astype(np.int64) - 1                # a = (2 frac) * 2^unb
+    q = np.rint((2.0 * frac - 1.0) * 8.0)        # mantissa steps, ties to even
+    carry = q == 8.0
+    unb = np.where(carry, unb + 1, unb)
+    q = np.where(carry, 0.0, q)
+    normal_code = (unb + 7) * 8 + q.astype(np.int64)
+    sub_code = np.rint(np.minimum(a, 2.0 ** -6) / 2.0 ** -9).astype(np.int64)  # 8 steps of 2^-9 = code 8, the smallest normal
+    mag = np.where(a >= 2.0 ** -6, normal_code, sub_code)
+    mag = np.minimum(np.where(finite, mag, 0x7E), 0x7E)   # 0x7E = 448; anything larger saturates
+    mag = np.where(np.isnan(v32), 0x7F, mag)
+    sign = np.where(np.signbit(v32) & ~np.isnan(v32), 0x80, 0)
+    return (mag | sign).astype(np.uint8)
+
+
+def quantize_rows_fp8(x_bits):
+    """Per-row E4M3 quantization of bf16 rows: (codes uint8 [R][C], scales fp32 [R]).
+    s = fp32(amax) / 448 in fp32 (1 for an all-zero row); code = f32_to_e4m3(fp32(x) / s)."""
+    x = bf16_bits_to_f64(x_bits).astype(np.float32)          # exact
+    amax = np.abs(x).max(axis=-1) if x.shape[-1] else np.zeros(x.shape[:-1], np.float32)
+    s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    q = f32_to_e4m3((x / s[..., None]).astype(np.float32))
+    return q, s
+
+
+def dispatch_fp8(z_bits, row_of_assign, K: int):
+    """FP8 dispatch buffer: every token quantized once, its codes and scale placed at the
+    rows of its K assignments (xq[row_of_assign[t*K+k]] = q[t], xs[...] = s[t])."""
+    q, s = quantize_rows_fp8(z_bits)
+    T = q.shape[0]
+    roa = np.asarray(row_of_assign, dtype=np.int64).reshape(-1)
+    t = np.arange(T * K) // K
+    xq = np.empty((T * K, q.shape[1]), dtype=np.uint8)
+    xs = np.empty(T * K, dtype=np.float32)
+    xq[roa] = q[t]
+    xs[roa] = s[t]
+    return xq, xs
+
+
+def quantize_experts_fp8(w_bits):
+    """Gate or up weights [E][F][H] quantized per output feature: codes [E][F][H], scales [E][F]."""
+    w = np.asarray(w_bits, dtype=np.uint16)
+    q, s = quantize_rows_fp8(w.reshape(-1, w.shape[-1]))
+    return q.reshape(w.shape), s.reshape(w.shape[:-1])
+
+
+def ffn_rows_fp8(xq, xs, wg_q, wg_s, wu_q, wu_s, w_down_e_bits):
+    """SwiGLU expert FFN on E4M3 rows: g = s_x s_wg (q_x q_wg^T), u likewise (float64),
+    h = bf16(silu(g) * u), y = bf16(h Wd^T) with bf16 Wd.  Returns (h, y) bits."""
+    x = e4m3_to_f64(xq)
+    sx = np.asarray(xs, dtype=np.float32).astype(np.float64)[:, None]
+    g = (x @ e4m3_to_f64(wg_q).T) * sx * np.asarray(wg_s, np.float32).astype(np.float64)[None, :]
+    u = (x @ e4m3_to_f64(wu_q).T) * sx * np.asarray(wu_s, np.float32).astype(np.float64)[None, :]
+    h_bits = f64_to_bf16_bits(_silu(g) * u)
+    y_bits = f64_to_bf16_bits(bf16_bits_to_f64(h_bits) @ bf16_bits_to_f64(w_down_e_bits).T)
+    return h_bits, y_bits
+
+
+def grouped_ffn_fp8(xq, xs, offsets, wg_q, wg_s, wu_q, wu_s, w_down_bits):
+    """ffn_rows_fp8 of expert e on rows [offsets[e], offsets[e+1]), for every e."""
+    off = np.asarray(offsets, dtype=np.int64)
+    rows, F, H = xq.shape[0], wg_q.shape[1], w_down_bits.shape[1]
+    h = np.zeros((rows, F), dtype=np.uint16)
+    y = np.zeros((rows, H), dtype=np.uint16)
+    for e in range(off.size - 1):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi > lo:
+            h[lo:hi], y[lo:hi] = ffn_rows_fp8(xq[lo:hi], xs[lo:hi], wg_q[e], wg_s[e], wu_q[e], wu_s[e],
+                                              w_down_bits[e])
+    return h, y
+
+
+def dispatch_bytes_fp8(T: int, K: int, H: int) -> int:
+    """FP8 dispatch payload: T K H one-byte codes plus one 4-byte scale per dispatched row."""
+    return T * K * H + 4 * T * K
+
+
+# ----------------------------------------------------------------------------
 # Step S6: combine = unpermute + weighted sum   [WideEP/router], [WideEP/bytes]
 # ----------------------------------------------------------------------------
 
@@ -383,7 +497,7 @@ def dense_bf16(x_bits, w_bits):
 
 def layer_forward(x_bits, w_g, w_gate_bits, w_up_bits, w_down_bits, K: int, P: int = 1,
                   renormalize: bool = True, bias=None, w_dp_bits=None, w_upp_bits=None,
-                  logits=None, group_limit: int = 0, shared=None):
+                  logits=None, group_limit: int = 0, shared=None, fp8: bool = False):
     """All steps in pipeline order.  Returns a dict with every intermediate.
 
     ``shared`` = (W_gate_s [Fs][d], W_up_s [Fs][d], W_down_s [d][Fs]) bf16 bits adds a shared
@@ -391,6 +505,9 @@ def layer_forward(x_bits, w_g, w_gate_bits, w_up_bits, w_down_bits, K: int, P: i
 
     If ``logits`` is given it replaces the oracle's own gating output (used by
     the routing tests, which hand both sides the same float32 logits).
+
+    ``fp8`` dispatches E4M3 codes with per-token scales and runs gate/up on E4M3 weights
+    quantized per output feature (results "xq", "xs", "wg_q", "wg_s", "wu_q", "wu_s").
     """
     res = {}
     z = x_bits
@@ -410,7 +527,14 @@ def layer_forward(x_bits, w_g, w_gate_bits, w_up_bits, w_down_bits, K: int, P: i
     xp, meta = permute(z, cs["row_of_assign"], ids, w, E, P)
     res["xp"] = xp
     res["meta"] = meta
-    h, y = grouped_ffn(xp, cs["offsets"], w_gate_bits, w_up_bits, w_down_bits)
+    if fp8:
+        xq, xs = dispatch_fp8(z, cs["row_of_assign"], K)
+        wg_q, wg_s = quantize_experts_fp8(w_gate_bits)
+        wu_q, wu_s = quantize_experts_fp8(w_up_bits)
+        res.update(xq=xq, xs=xs, wg_q=wg_q, wg_s=wg_s, wu_q=wu_q, wu_s=wu_s)
+        h, y = grouped_ffn_fp8(xq, xs, cs["offsets"], wg_q, wg_s, wu_q, wu_s, w_down_bits)
+    else:
+        h, y = grouped_ffn(xp, cs["offsets"], w_gate_bits, w_up_bits, w_down_bits)
     res["h"], res["y"] = h, y
     s_bits = None
     if shared is not None:

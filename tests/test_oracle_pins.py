@@ -535,3 +535,146 @@ def test_layer_shared_expert_is_a_dense_swiglu_added_to_every_token():
     # zero shared weights leave the output unchanged
     zero = tuple(np.zeros_like(a) for a in sh)
     assert np.array_equal(oracle.layer_forward(*args, shared=zero)["out"], plain["out"])
+
+
+# ---------------------------------------------------------------------------
+# FP8 dispatch (E4M3 codes, one fp32 scale per row)
+# ---------------------------------------------------------------------------
+
+def test_e4m3_decode_matches_torch_and_hand_values():
+    codes = np.arange(256, dtype=np.uint8)
+    v = oracle.e4m3_to_f64(codes)
+    t = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()   # torch's own decoder
+    assert np.array_equal(np.isnan(v), np.isnan(t))
+    assert np.array_equal(v[~np.isnan(v)], t[~np.isnan(t)])
+    hand = {0x00: 0.0, 0x01: 2.0 ** -9, 0x07: 7 * 2.0 ** -9, 0x08: 2.0 ** -6, 0x38: 1.0, 0x39: 1.125,
+            0xB8: -1.0, 0x7E: 448.0, 0xFE: -448.0, 0x77: 240.0, 0x40: 2.0}
+    for c, x in hand.items():
+        assert oracle.e4m3_to_f64(np.array([c], np.uint8))[0] == x, hex(c)
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF]) and np.isnan(v).sum() == 2
+    assert np.signbit(v[0x80]) and v[0x80] == 0.0
+
+
+def test_e4m3_encode_roundtrip_ties_to_even_and_saturation():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    v = oracle.e4m3_to_f64(codes)
+    assert np.array_equal(oracle.f32_to_e4m3(v.astype(np.float32)), codes)
+    # midpoints between neighbouring positive codes go to the code with the even mantissa
+    pos = np.arange(0, 0x7F, dtype=np.uint8)
+    pv = oracle.e4m3_to_f64(pos)
+    mid = ((pv[:-1] + pv[1:]) / 2).astype(np.float32)
+    assert np.array_equal(mid.astype(np.float64), (pv[:-1] + pv[1:]) / 2)   # midpoints are fp32-exact
+    got = oracle.f32_to_e4m3(mid)
+    want = np.where(pos[:-1] % 2 == 0, pos[:-1], pos[1:])
+    assert np.array_equal(got, want)
+    assert np.array_equal(oracle.f32_to_e4m3(-mid), want | 0x80)
+    # just off the midpoints the nearest code wins
+    up = np.nextafter(mid, np.float32(np.inf))
+    dn = np.nextafter(mid, np.float32(0))
+    assert np.array_equal(oracle.f32_to_e4m3(up), pos[1:])
+    assert np.array_equal(oracle.f32_to_e4m3(dn), pos[:-1])
+    # saturation to +-448; NaN stays NaN
+    big = np.array([448.0, 449.0, 463.99, 464.0, 480.0, 1e6, 3.0e38, np.inf], np.float32)
+    assert np.all(oracle.f32_to_e4m3(big) == 0x7E)
+    assert np.all(oracle.f32_to_e4m3(-big) == 0xFE)
+    assert oracle.f32_to_e4m3(np.array([np.nan], np.float32))[0] == 0x7F
+    # below half the smallest subnormal: zero; the sign survives
+    assert oracle.f32_to_e4m3(np.array([2.0 ** -11, -2.0 ** -11], np.float32)).tolist() == [0x00, 0x80]
+
+
+def test_e4m3_encode_matches_torch_on_random_values():
+    rng = np.random.default_rng(11)
+    v = np.concatenate([rng.standard_normal(20000) * s for s in (1e-3, 0.05, 1.0, 30.0, 150.0)])
+    v = np.clip(v, -447.0, 447.0).astype(np.float32)
+    t = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()   # torch's own encoder
+    assert np.array_equal(oracle.f32_to_e4m3(v), t)
+
+
+def test_quantize_rows_fp8_scale_amax_and_error_bound():
+    rng = np.random.default_rng(5)
+    x = bf(rng.standard_normal((40, 96)) * np.exp(rng.uniform(-6, 6, (40, 1))))
+    x[3] = bf(np.zeros(96))
+    q, s = oracle.quantize_rows_fp8(x)
+    xv = val(x)
+    assert s.dtype == np.float32 and q.dtype == np.uint8
+    assert s[3] == 1.0 and np.all(q[3] == 0)
+    amax = np.abs(xv).max(axis=1)
+    nz = amax > 0
+    assert np.array_equal(s[nz], (amax[nz].astype(np.float32) / np.float32(448.0)))
+    # the largest element of each row lands on +-448
+    i = np.abs(xv).argmax(axis=1)
+    assert np.all(oracle.e4m3_to_f64(q[np.arange(40), i])[nz] == np.sign(xv[np.arange(40), i])[nz] * 448.0)
+    # dequantization error: half a step of 3 mantissa bits, or half a subnormal step
+    err = np.abs(xv - oracle.e4m3_to_f64(q) * s[:, None].astype(np.float64))
+    bound = 2.0 ** -4 * np.abs(xv) * (1 + 2.0 ** -20) + 2.0 ** -10 * s[:, None]
+    assert np.all(err <= bound)
+    # scaling a row by a power of two scales s and leaves the codes unchanged
+    q2, s2 = oracle.quantize_rows_fp8(bf(xv * 2.0 ** 7))
+    assert np.array_equal(q2, q) and np.array_equal(s2[nz], s[nz] * np.float32(2 ** 7))
+
+
+def _exact_fp8_rows(rng, R, C):
+    """bf16 rows that per-row E4M3 quantization represents exactly: codes times 2^a_r, with one
+    element per row at +-448 so that the scale comes out as 2^a_r."""
+    codes = rng.integers(0, 0x7E, size=(R, C)).astype(np.uint8) | (rng.integers(0, 2, (R, C)) * 0x80).astype(np.uint8)
+    codes[np.arange(R), rng.integers(0, C, R)] = np.where(rng.integers(0, 2, R) > 0, 0x7E, 0xFE)
+    a = rng.integers(-14, -6, R).astype(np.float64)
+    x = oracle.e4m3_to_f64(codes) * np.exp2(a)[:, None]
+    bits = bf(x)
+    assert np.array_equal(val(bits), x)
+    return bits, codes, np.exp2(a).astype(np.float32)
+
+
+def test_quantize_rows_fp8_recovers_exact_codes_and_scales():
+    rng = np.random.default_rng(8)
+    bits, codes, scale = _exact_fp8_rows(rng, 17, 50)
+    q, s = oracle.quantize_rows_fp8(bits)
+    assert np.array_equal(q, codes) and np.array_equal(s, scale)
+
+
+def test_ffn_rows_fp8_equals_bf16_ffn_on_exactly_representable_inputs():
+    # per-token and per-feature scales differ, T != F: a scale on the wrong axis changes g and u
+    rng = np.random.default_rng(9)
+    T, H, F = 7, 64, 24
+    x, qx, sx = _exact_fp8_rows(rng, T, H)
+    wg, qg, sg = _exact_fp8_rows(rng, F, H)
+    wu, qu, su = _exact_fp8_rows(rng, F, H)
+    wd = bf(rng.standard_normal((H, F)) / np.sqrt(F))
+    h8, y8 = oracle.ffn_rows_fp8(qx, sx, qg, sg, qu, su, wd)
+    h, y = oracle.ffn_rows(x, wg, wu, wd)
+    assert np.array_equal(h8, h) and np.array_equal(y8, y)
+    # a swapped pair of scales is visible
+    h_bad, _ = oracle.ffn_rows_fp8(qx, sx, qg, su, qu, sg, wd)
+    assert not np.array_equal(h_bad, h)
+
+
+def test_dispatch_fp8_rows_and_bytes():
+    rng = np.random.default_rng(2)
+    T, K, E, H = 30, 3, 8, 40
+    z = bf(rng.standard_normal((T, H)))
+    ids = np.stack([rng.permutation(E)[:K] for _ in range(T)])
+    cs = oracle.count_scan(ids, E, 1)
+    xq, xs = oracle.dispatch_fp8(z, cs["row_of_assign"], K)
+    q, s = oracle.quantize_rows_fp8(z)
+    roa = cs["row_of_assign"].reshape(T, K)
+    for t in range(T):
+        for k in range(K):
+            assert np.array_equal(xq[roa[t, k]], q[t]) and xs[roa[t, k]] == s[t]
+    assert xq.nbytes + xs.nbytes == oracle.dispatch_bytes_fp8(T, K, H) == oracle.dispatch_bytes(T, K, H, 1) + 4 * T * K
+    assert 2 * oracle.dispatch_bytes(T, K, H, 1) == oracle.dispatch_bytes(T, K, H, 2)   # FP8 halves the payload
+
+
+def test_layer_fp8_equals_bf16_layer_on_exactly_representable_inputs():
+    rng = np.random.default_rng(4)
+    T, H, F, E, K = 24, 64, 32, 6, 2
+    x, _, _ = _exact_fp8_rows(rng, T, H)
+    wg = np.stack([_exact_fp8_rows(rng, F, H)[0] for _ in range(E)])
+    wu = np.stack([_exact_fp8_rows(rng, F, H)[0] for _ in range(E)])
+    wd = bf(rng.standard_normal((E, H, F)) / np.sqrt(F))
+    w_g = (rng.standard_normal((H, E)) / np.sqrt(H)).astype(np.float32)
+    r16 = oracle.layer_forward(x, w_g, wg, wu, wd, K)
+    r8 = oracle.layer_forward(x, w_g, wg, wu, wd, K, fp8=True)
+    assert np.array_equal(r8["topk_ids"], r16["topk_ids"])
+    for k in ("h", "y", "out"):
+        assert np.array_equal(r8[k], r16[k]), k
+    assert np.array_equal(oracle.e4m3_to_f64(r8["xq"]) * r8["xs"][:, None], val(r16["xp"]))
