@@ -49,6 +49,8 @@ def parse():
                    help="node-limited routing: experts from the M best partitions (0 = off)")
     p.add_argument("--shared-expert", type=int, default=0, metavar="F_SHARED",
                    help="add a shared expert of this width, run on a second stream beside the routed path")
+    p.add_argument("--fp8-dispatch", action="store_true",
+                   help="dispatch E4M3 rows with per-token scales and run gate/up on E4M3 weights")
     p.add_argument("--shape", action="append", default=[], metavar="FIELD=INT",
                    help="override one integer field of the workload (T, E, H, F, K, P); for reduced-size "
                         "profiling captures of a workload's kernels, e.g. --shape T=1024 --shape E=32")
@@ -191,8 +193,12 @@ def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 16):
         if e not in expert_cache:
             ge = torch.Generator().manual_seed(10_000 + e)
             F, H = cfg.F, cfg.H
-            expert_cache[e] = tuple(inputs.to_bits((torch.randn(s, generator=ge) * std).to(torch.bfloat16))
-                                    for s, std in (((F, H), H ** -0.5), ((F, H), H ** -0.5), ((H, F), F ** -0.5)))
+            wts = tuple(inputs.to_bits((torch.randn(s, generator=ge) * std).to(torch.bfloat16))
+                        for s, std in (((F, H), H ** -0.5), ((F, H), H ** -0.5), ((H, F), F ** -0.5)))
+            if cfg.fp8_dispatch:   # one-time weight preparation, like the GPU's
+                (qg, sg), (qu, su) = oracle.quantize_rows_fp8(wts[0]), oracle.quantize_rows_fp8(wts[1])
+                wts = (qg, sg, qu, su, wts[2])
+            expert_cache[e] = wts
         return expert_cache[e]
 
     w_g_np = w_g.numpy()
@@ -220,9 +226,14 @@ def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 16):
         off = cs["offsets"]
         h = np.zeros((xp.shape[0], cfg.F), np.uint16)
         y = np.zeros((xp.shape[0], cfg.H), np.uint16)
+        if cfg.fp8_dispatch:
+            xq, xs = oracle.dispatch_fp8(z, cs["row_of_assign"], cfg.K)
         for e in np.nonzero(cs["counts"])[0]:
             lo, hi = off[e], off[e + 1]
-            h[lo:hi], y[lo:hi] = oracle.ffn_rows(xp[lo:hi], *expert(int(e)))
+            if cfg.fp8_dispatch:
+                h[lo:hi], y[lo:hi] = oracle.ffn_rows_fp8(xq[lo:hi], xs[lo:hi], *expert(int(e)))
+            else:
+                h[lo:hi], y[lo:hi] = oracle.ffn_rows(xp[lo:hi], *expert(int(e)))
         y_sh = None if sh_b is None else oracle.ffn_rows(z, *sh_b)[1]
         out = oracle.combine(y, cs["row_of_assign"], w, y_sh)
         if w_upp_b is not None:
@@ -276,9 +287,35 @@ def shared_expert_overlap(cfg, inp, w, bufs, ws, flush, stream, n, dev) -> dict:
             "stream": "shared expert on an auxiliary stream, forked after the latent down-projection"}
 
 
+def fp8_accuracy(cfg, inp, bufs, dev) -> dict:
+    """What FP8 dispatch changes: the layer output against the bf16 layer on the same inputs
+    (relative Frobenius error, tokens whose expert set differs = 0 since routing precedes the
+    dispatch) and the dispatch payload."""
+    from routing_dispatch_grouped_top_b200 import binding as B
+    c16 = cfg.with_(fp8_dispatch=False)
+    d16 = B.dims_of(c16)
+    w16 = B.pack_layer_weights(d16, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"],
+                               inp["w_dp"], inp["w_upp"], shared=inp["shared"])
+    b16 = B.alloc_layer_buffers(d16, dev)
+    ws16 = B.make_workspace(d16, dev)
+    B.moe_layer_forward(inp["x"], w16, d16, b16, ws16)
+    torch.cuda.synchronize()
+    key = "final_out" if cfg.d_model else "out"
+    a, b = bufs[key].double(), b16[key].double()
+    rel = float(torch.linalg.norm(a - b) / torch.linalg.norm(b))
+    rel_h = float(torch.linalg.norm(bufs["h"].double() - b16["h"].double()) / torch.linalg.norm(b16["h"].double()))
+    same_routing = bool(torch.equal(bufs["topk_ids"], b16["topk_ids"]))
+    del w16, b16, ws16
+    torch.cuda.empty_cache()
+    return {"out_rel_frob_vs_bf16_layer": rel, "h_rel_frob_vs_bf16_layer": rel_h, "same_routing": same_routing,
+            "dispatch_bytes": cfg.dispatch_bytes_actual(), "bf16_dispatch_bytes": cfg.dispatch_bytes(2),
+            "format": "E4M3 codes, one fp32 scale per token (amax/448); gate/up weights E4M3 per output feature"}
+
+
 def config_dict(cfg, world: int) -> dict:
     return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K, "F": cfg.F, "P": cfg.P,
             "d_model": cfg.d_model, "group_limit": cfg.group_limit, "F_shared": cfg.F_shared,
+            "fp8_dispatch": cfg.fp8_dispatch,
             "parallelism": f"replicas{world}",
             "l2": "flushed (256 MiB write) before every timed step, outside its events"}
 
@@ -316,6 +353,8 @@ def main():
         cfg = cfg.with_(**{k: int(v)})
     if args.shape:
         cfg = cfg.with_(name=f"{cfg.name}_reshaped_" + "_".join(args.shape).replace("=", ""))
+    if args.fp8_dispatch:
+        cfg = cfg.with_(fp8_dispatch=True, name=f"{cfg.name}_fp8_dispatch")
     if args.shared_expert:
         cfg = cfg.with_(F_shared=args.shared_expert, name=f"{cfg.name}_shared_expert_Fs{args.shared_expert}")
     if args.impl == "reference":
@@ -392,6 +431,7 @@ def main():
     torch.cuda.synchronize()
     stage_ms = [[ev[j].elapsed_time(ev[j + 1]) for ev in events] for j in range(n_ev - 1)]
     shared_diag = shared_expert_overlap(cfg, inp, w, bufs, ws, flush, stream, n_diag, dev) if cfg.F_shared else None
+    fp8_diag = fp8_accuracy(cfg, inp, bufs, dev) if cfg.fp8_dispatch else None
 
     # End to end through the host-buffer entry point: every step copies its x from pinned host
     # memory and its output back, inside the timed region.  Steps alternate between two streams,
@@ -446,10 +486,13 @@ def main():
         n_touched = int((bufs["counts"] > 0).sum().item())
         T, H, F, TK = cfg.T, cfg.H, cfg.F, cfg.TK
         # algorithmic work per launch: (flops, HBM bytes)
+        fp8 = cfg.fp8_dispatch
+        xb = 1 if fp8 else 2            # bytes per dispatched activation element and gate/up weight
         work = {
-            "gate_up": (4 * H * F * TK, 2 * H * F * 2 * n_touched + TK * H * 2 + TK * F * 2),
+            "gate_up": (4 * H * F * TK, 2 * H * F * xb * n_touched + TK * H * xb + TK * F * 2
+                        + (2 * F * 4 * n_touched + TK * 4 if fp8 else 0)),
             "down": (2 * H * F * TK, H * F * 2 * n_touched + TK * F * 2 + TK * H * 2),
-            "permute": (0, T * H * 2 + TK * H * 2 + TK * (4 + 8 + 16)),
+            "permute": (0, T * H * 2 + TK * H * xb + TK * (4 + 8 + 16) + (TK * 4 if fp8 else 0)),
             "combine": (0, TK * H * 2 + T * H * 2 + TK * 8),
             "gating": (2 * T * H * cfg.E * 3, T * H * 2 + 3 * cfg.E * H * 2 + T * cfg.E * 4),
             "route": (0, T * cfg.E * 4 + TK * 8),
@@ -458,18 +501,22 @@ def main():
         fl, by = work[dominant]
         # the gate/up time comes from the timed region itself
         t_s = (gate_up_ms_timed if dominant == "gate_up" else stage_mean[dominant]) / 1e3
-        hbm_time, tc_time = by / (peaks["hbm"] * 1e9), fl / (bf16_peak * 1e12)
+        # E4M3 gate/up: the measured bf16 peak times the nominal dense fp8 / bf16 ratio (4.5 / 2.25)
+        tc_peak = 2.0 * bf16_peak if (fp8 and dominant == "gate_up") else bf16_peak
+        hbm_time, tc_time = by / (peaks["hbm"] * 1e9), fl / (tc_peak * 1e12)
         if hbm_time >= tc_time:
             roof = {"bound": "hbm", "achieved": by / t_s / 1e9, "peak": peaks["hbm"], "unit": "GB/s"}
         else:
-            roof = {"bound": "tensor", "achieved": fl / t_s / 1e12, "peak": bf16_peak, "unit": "TFLOP/s"}
+            roof = {"bound": "tensor", "achieved": fl / t_s / 1e12, "peak": tc_peak, "unit": "TFLOP/s"}
         roof["frac"] = roof["achieved"] / roof["peak"]
         roof["traffic"] = kernel_traffic(cfg.name, dominant)
         roof["kernel"] = dominant
         roof["algorithmic_bytes"] = by
         roof["algorithmic_flops"] = fl
         roof["peak_source"] = (f"{peaks['source']} " + ("HBM copy" if roof["bound"] == "hbm" else
-                                                         f"bf16 {'sustained' if long_run else 'burst'}"))
+                                                         f"bf16 {'sustained' if long_run else 'burst'}"
+                                                         + (" x 2 (nominal fp8/bf16)" if tc_peak != bf16_peak
+                                                            else "")))
         roof["timing"] = ("CUDA events around every gate/up launch of the timed steps" if dominant == "gate_up"
                           else "CUDA events of the per-stage pass")
         ffn_ms = stage_mean["gate_up"] + stage_mean["down"]
@@ -490,11 +537,12 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "e4m3 gate/up, bf16 elsewhere" if fp8 else "bf16", "data": "synthetic",
             "config": config_dict(cfg, world),
             "roofline": roof,
             "stages_ms": stage_mean,
             **({"shared_expert": shared_diag} if shared_diag else {}),
+            **({"fp8_dispatch": fp8_diag} if fp8_diag else {}),
             "fractions": frac,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": cfg.T * d_in * 2,
                     "d2h_bytes_per_step": cfg.T * d_in * 2},

@@ -63,6 +63,9 @@ typedef struct moe_dims {
                            needs P <= MOE_MAX_LIMITED_GROUPS and K <= M * E / P */
   int32_t F_shared;     /* 0, or the width of a shared expert that every token passes through
                            (a multiple of 8) */
+  int32_t fp8_dispatch; /* 0, or 1: the layer dispatches E4M3 rows with per-token scales and
+                           runs gate/up on E4M3 weights (moe_permute_fp8,
+                           moe_grouped_gate_up_fp8); needs H % 16 == 0 */
 } moe_dims;
 
 typedef enum moe_status {
@@ -256,6 +259,49 @@ moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w
                             const moe_dims* d, void* y, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* FP8 dispatch: E4M3 rows with one fp32 scale per row, gate/up on E4M3,     */
+/* bf16 down projection and combine.  A runtime may quantize the outbound   */
+/* activation, carry its scales, compute in the other format and return at  */
+/* higher precision (WideEP essay, "Top-k multiplies traffic. Locality      */
+/* subtracts it."); the change alters values, so it belongs to the bucket   */
+/* that needs a task-level evaluation before release ("Three Parameter      */
+/* Counts...", "Which optimizations need a task-level gate").                */
+/* Format: E4M3 (sign, 4 exponent bits with bias 7, 3 mantissa bits; largest */
+/* finite 448; no infinities; 0x7F / 0xFF are NaN).                          */
+/* ------------------------------------------------------------------------- */
+
+/* Per-row quantization of x [rows][cols] bf16:
+ *   scales[r] = amax_r / 448 (fp32 division; 1 when row r is all zero),
+ *   q[r][c]   = E4M3 code of fp32(x[r][c]) / scales[r] (fp32 division, round to nearest
+ *               even, saturating to +-448).
+ * q [rows][cols] uint8, scales [rows] fp32.  cols must be a multiple of 16.  One-time
+ * preparation of the gate and up weights ([E*F] rows of H each). */
+moe_status moe_quantize_fp8_rows(const void* x, int64_t rows, int32_t cols, void* q, float* scales,
+                                 void* stream);
+
+/* FP8 dispatch: each token t is quantized once as by moe_quantize_fp8_rows and its codes and
+ * scale land at the rows r = row_of_assign[t*K+k] of its K assignments: xq[r][:] (uint8
+ * [TK][H]) and xs[r] (fp32 [TK]), T*K*H + 4*T*K bytes in all (half the bf16 payload plus
+ * the scales).  Metadata as moe_permute.  H must be a multiple of 16. */
+moe_status moe_permute_fp8(const void* x, const int32_t* row_of_assign, const int32_t* topk_ids,
+                           const float* topk_w, const moe_dims* d, void* xq, float* xs,
+                           int32_t* meta_token, int32_t* meta_slot, float* meta_w,
+                           int32_t* meta_local_expert, void* stream);
+
+/* Gate/up + SwiGLU on E4M3 rows.  For every expert e and row r in [offsets[e], offsets[e+1]):
+ *   g = xs[r] * s_gate[e][f] * sum_k val(xq[r][k]) * val(wq_gate[e][f][k]),
+ *   u = xs[r] * s_up[e][f]   * sum_k val(xq[r][k]) * val(wq_up[e][f][k]),
+ *   h[r][f] = bf16( silu(g) * u ),
+ * E4M3 x E4M3 tensor-core products accumulated in fp32.  xq [TK][H] uint8, xs [TK] fp32 (from
+ * moe_permute_fp8); wq_gate, wq_up [E][F][H] uint8 and s_gate, s_up [E][F] fp32 (from
+ * moe_quantize_fp8_rows on the bf16 weights); h [TK][F] bf16, consumed by moe_grouped_down.
+ * H a multiple of 16.  Offsets are checked as in moe_grouped_ffn. */
+moe_status moe_grouped_gate_up_fp8(const void* xq, const float* xs, const int32_t* offsets,
+                                   const void* wq_gate, const void* wq_up, const float* s_gate,
+                                   const float* s_up, const moe_dims* d, void* h, void* ws,
+                                   size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* S6  Combine: unpermute + weighted sum                                     */
 /* Every expert output goes back to its token and the K outputs are summed */
 /* with the routing weights (WideEP essay, "The router writes a network     */
@@ -312,6 +358,10 @@ typedef struct moe_layer_weights {
   const void*  w_shared_gate; /* shared expert (F_shared > 0): [F_shared][H] bf16    */
   const void*  w_shared_up;   /* [F_shared][H] bf16                                  */
   const void*  w_shared_down; /* [H][F_shared] bf16                                  */
+  const void*  w_gate_q;    /* fp8_dispatch: [E][F][H] E4M3 codes of w_gate   */
+  const void*  w_up_q;      /* fp8_dispatch: [E][F][H] E4M3 codes of w_up     */
+  const float* s_gate;      /* fp8_dispatch: [E][F] fp32 scales of w_gate_q   */
+  const float* s_up;        /* fp8_dispatch: [E][F] fp32 scales of w_up_q     */
 } moe_layer_weights;
 
 typedef struct moe_layer_buffers {
@@ -341,6 +391,8 @@ typedef struct moe_layer_buffers {
                                runs alongside the routed path                */
   void*    fork_event;      /* with aux_stream: two cudaEvent_t created by the */
   void*    join_event;      /* caller (timing disabled is fine)              */
+  void*    xq;              /* fp8_dispatch: [TK][H] uint8 dispatched codes (xp unused) */
+  float*   xs;              /* fp8_dispatch: [TK] fp32 row scales            */
 } moe_layer_buffers;
 
 /* Number of stage boundaries recorded when stage events are given. */
@@ -348,7 +400,9 @@ typedef struct moe_layer_buffers {
 
 /* Runs every step on `stream` in pipeline order: [latent down-projection] ->
  * gating -> route -> count/scan -> permute -> gate/up+SwiGLU -> down -> combine
- * -> [latent up-projection] -> skew statistics.  With d->F_shared > 0 the shared
+ * -> [latent up-projection] -> skew statistics.  With d->fp8_dispatch the permute is
+ * moe_permute_fp8 (into b->xq, b->xs; b->xp may be NULL) and gate/up runs on
+ * w->w_gate_q / w->w_up_q with their scales.  With d->F_shared > 0 the shared
  * expert (gate/up+SwiGLU and down over all T tokens of the routed activations) runs
  * on b->aux_stream, forked after the routed activations are ready and joined before
  * the combine, or on `stream` when aux_stream is NULL.  x: [T][d_in] bf16 with

@@ -33,11 +33,11 @@ class MoEError(RuntimeError):
 class moe_dims(C.Structure):
     _fields_ = [("T", C.c_int64), ("H", C.c_int32), ("E", C.c_int32), ("K", C.c_int32), ("F", C.c_int32),
                 ("P", C.c_int32), ("renormalize", C.c_int32), ("d_model", C.c_int32), ("group_limit", C.c_int32),
-                ("F_shared", C.c_int32)]
+                ("F_shared", C.c_int32), ("fp8_dispatch", C.c_int32)]
 
 
 _W_FIELDS = ("w_g_split", "bias", "w_gate", "w_up", "w_down", "w_dp", "w_upp", "w_gate_up", "w_shared_gate",
-             "w_shared_up", "w_shared_down")
+             "w_shared_up", "w_shared_down", "w_gate_q", "w_up_q", "s_gate", "s_up")
 
 
 class moe_layer_weights(C.Structure):
@@ -46,7 +46,8 @@ class moe_layer_weights(C.Structure):
 
 _BUF_FIELDS = ("z", "logits", "topk_ids", "topk_w", "counts", "offsets", "part_counts", "part_offsets",
                "row_of_assign", "assign_of_row", "xp", "meta_token", "meta_slot", "meta_w", "meta_local_expert",
-               "h", "y", "out", "final_out", "skew", "h_shared", "y_shared", "aux_stream", "fork_event", "join_event")
+               "h", "y", "out", "final_out", "skew", "h_shared", "y_shared", "aux_stream", "fork_event", "join_event",
+               "xq", "xs")
 
 
 class moe_layer_buffers(C.Structure):
@@ -72,6 +73,9 @@ _SIGS = {
     "moe_packed_gate_up_bytes": (_SZ, [_DP]),
     "moe_pack_gate_up": (C.c_int, [_VP, _VP, _DP, _VP, _VP]),
     "moe_grouped_gate_up_packed": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
+    "moe_quantize_fp8_rows": (C.c_int, [_VP, _I64, _I32, _VP, _VP, _VP]),
+    "moe_permute_fp8": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "moe_grouped_gate_up_fp8": (C.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
     "moe_combine": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP]),
     "moe_skew_stats": (C.c_int, [_VP, _DP, _VP, _VP]),
     "moe_p95": (C.c_double, [C.POINTER(C.c_float), C.c_int]),
@@ -107,14 +111,15 @@ def _check(fn: str, status: int):
         raise MoEError(fn, status, lib().moe_status_str(status).decode())
 
 
-def dims(T, H, E, K, F, P=1, renormalize=True, d_model=0, group_limit=0, F_shared=0) -> moe_dims:
+def dims(T, H, E, K, F, P=1, renormalize=True, d_model=0, group_limit=0, F_shared=0,
+         fp8_dispatch=False) -> moe_dims:
     return moe_dims(int(T), int(H), int(E), int(K), int(F), int(P), int(bool(renormalize)), int(d_model or 0),
-                    int(group_limit or 0), int(F_shared or 0))
+                    int(group_limit or 0), int(F_shared or 0), int(bool(fp8_dispatch)))
 
 
 def dims_of(cfg, T=None) -> moe_dims:
     return dims(cfg.T if T is None else T, cfg.H, cfg.E, cfg.K, cfg.F, cfg.P, cfg.renormalize, cfg.d_model or 0,
-                cfg.group_limit or 0, cfg.F_shared or 0)
+                cfg.group_limit or 0, cfg.F_shared or 0, cfg.fp8_dispatch)
 
 
 def _stream(stream) -> int:
@@ -226,6 +231,47 @@ def moe_permute(x, row_of_assign, topk_ids, topk_w, d: moe_dims, xp, meta_token=
         _ptr(meta_local_expert, torch.int32, "meta_local_expert", TK), _stream(stream)))
 
 
+def moe_quantize_fp8_rows(x, q, scales, stream=None):
+    """Per-row E4M3 codes (uint8, x's shape) and fp32 scales of the bf16 rows of x."""
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    if tuple(q.shape) != tuple(x.shape) or scales.numel() < rows:
+        raise ValueError("shape mismatch")
+    _check("moe_quantize_fp8_rows", lib().moe_quantize_fp8_rows(
+        _ptr(x, torch.bfloat16, "x"), rows, cols, _ptr(q, torch.uint8, "q"), _ptr(scales, torch.float32, "scales"),
+        _stream(stream)))
+
+
+def quantize_fp8(x, stream=None):
+    """(codes, scales) of x [..., cols] bf16, allocated here."""
+    q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+    s = torch.empty(x.shape[:-1], dtype=torch.float32, device=x.device)
+    moe_quantize_fp8_rows(x, q, s, stream)
+    return q, s
+
+
+def moe_permute_fp8(x, row_of_assign, topk_ids, topk_w, d: moe_dims, xq, xs, meta_token=None, meta_slot=None,
+                    meta_w=None, meta_local_expert=None, stream=None):
+    TK = d.T * d.K
+    _check("moe_permute_fp8", lib().moe_permute_fp8(
+        _ptr(x, torch.bfloat16, "x", d.T * d.H), _ptr(row_of_assign, torch.int32, "row_of_assign", TK),
+        _ptr(topk_ids, torch.int32, "topk_ids", TK), _ptr(topk_w, torch.float32, "topk_w", TK), C.byref(d),
+        _ptr(xq, torch.uint8, "xq", TK * d.H), _ptr(xs, torch.float32, "xs", TK),
+        _ptr(meta_token, torch.int32, "meta_token", TK), _ptr(meta_slot, torch.int32, "meta_slot", TK),
+        _ptr(meta_w, torch.float32, "meta_w", TK), _ptr(meta_local_expert, torch.int32, "meta_local_expert", TK),
+        _stream(stream)))
+
+
+def moe_grouped_gate_up_fp8(xq, xs, offsets, wq_gate, wq_up, s_gate, s_up, d: moe_dims, h, ws, stream=None):
+    TK = d.T * d.K
+    _check("moe_grouped_gate_up_fp8", lib().moe_grouped_gate_up_fp8(
+        _ptr(xq, torch.uint8, "xq", TK * d.H), _ptr(xs, torch.float32, "xs", TK),
+        _ptr(offsets, torch.int32, "offsets", d.E + 1), _ptr(wq_gate, torch.uint8, "wq_gate", d.E * d.F * d.H),
+        _ptr(wq_up, torch.uint8, "wq_up", d.E * d.F * d.H), _ptr(s_gate, torch.float32, "s_gate", d.E * d.F),
+        _ptr(s_up, torch.float32, "s_up", d.E * d.F), C.byref(d), _ptr(h, torch.bfloat16, "h", TK * d.F),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
 def moe_grouped_ffn(xp, offsets, w_gate, w_up, w_down, d: moe_dims, h, y, ws, stream=None):
     TK = d.T * d.K
     _check("moe_grouped_ffn", lib().moe_grouped_ffn(
@@ -317,12 +363,14 @@ def alloc_layer_buffers(d: moe_dims, device="cuda", meta=True) -> dict:
     b = dict(z=e((T, d.H), bf) if d.d_model else None, logits=e((T, d.E), f32), topk_ids=e((T, d.K), i32),
              topk_w=e((T, d.K), f32), counts=e((d.E,), i32), offsets=e((d.E + 1,), i32), part_counts=e((d.P,), i32),
              part_offsets=e((d.P + 1,), i32), row_of_assign=e((TK,), i32), assign_of_row=e((TK,), i32),
-             xp=e((TK, d.H), bf), meta_token=e((TK,), i32) if meta else None,
+             xp=None if d.fp8_dispatch else e((TK, d.H), bf), meta_token=e((TK,), i32) if meta else None,
              meta_slot=e((TK,), i32) if meta else None, meta_w=e((TK,), f32) if meta else None,
              meta_local_expert=e((TK,), i32) if meta else None, h=e((TK, d.F), bf), y=e((TK, d.H), bf),
              out=e((T, d.H), bf), final_out=e((T, d.d_model), bf) if d.d_model else None, skew=e((1,), f32),
              h_shared=e((T, d.F_shared), bf) if d.F_shared else None,
-             y_shared=e((T, d.H), bf) if d.F_shared else None)
+             y_shared=e((T, d.H), bf) if d.F_shared else None,
+             xq=e((TK, d.H), torch.uint8) if d.fp8_dispatch else None,
+             xs=e((TK,), f32) if d.fp8_dispatch else None)
     return b
 
 
@@ -368,7 +416,10 @@ def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, 
                        pack_gate_up_weights=None, shared=None) -> dict:
     """One-time weight preparation: router split into three bf16 planes and, when
     ``pack_gate_up_weights`` (default: H >= PACK_GATE_UP_MIN_H), gate/up interleaved for the
-    packed gate/up GEMM."""
+    packed gate/up GEMM.  With ``d.fp8_dispatch`` the gate and up weights are quantized to
+    E4M3 per output feature instead."""
+    if d.fp8_dispatch:
+        pack_gate_up_weights = False
     if pack_gate_up_weights is None:
         pack_gate_up_weights = (d.H >= PACK_GATE_UP_MIN_H and
                                 d.T * d.K >= PACK_GATE_UP_MIN_ROWS_PER_EXPERT * d.E)
@@ -387,8 +438,12 @@ def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, 
     if d.F_shared:
         for name, t in (("w_shared_gate", sg), ("w_shared_up", su), ("w_shared_down", sd)):
             _ptr(t, torch.bfloat16, name, d.F_shared * d.H)
+    q = dict(w_gate_q=None, s_gate=None, w_up_q=None, s_up=None)
+    if d.fp8_dispatch:
+        q["w_gate_q"], q["s_gate"] = quantize_fp8(w_gate, stream)
+        q["w_up_q"], q["s_up"] = quantize_fp8(w_up, stream)
     return dict(w_g_split=split, bias=bias, w_gate=w_gate, w_up=w_up, w_down=w_down, w_dp=w_dp, w_upp=w_upp,
-                w_gate_up=w_gu, w_shared_gate=sg, w_shared_up=su, w_shared_down=sd)
+                w_gate_up=w_gu, w_shared_gate=sg, w_shared_up=su, w_shared_down=sd, **q)
 
 
 def moe_layer_forward(x, weights: dict, d: moe_dims, buffers: dict, ws, stage_events=None, stream=None):

@@ -26,6 +26,7 @@ class MoEConfig:
     d_model: Optional[int] = None       # latent layer: model width before the down-projection
     group_limit: int = 0                # node-limited routing: experts from the M best partitions
     F_shared: int = 0                   # width of a shared expert every token passes through (0: none)
+    fp8_dispatch: bool = False          # E4M3 dispatch with per-token scales, E4M3 gate/up weights
     seed: int = 0
 
     @property
@@ -53,6 +54,10 @@ class MoEConfig:
     def dispatch_bytes(self, b: int = 2) -> int:
         """T x K x H x b: activation payload of one dispatch (no padding)."""
         return self.T * self.K * self.H * b
+
+    def dispatch_bytes_actual(self) -> int:
+        """Bytes the dispatch writes: bf16 rows, or E4M3 rows plus one fp32 scale per row."""
+        return self.dispatch_bytes(1) + 4 * self.TK if self.fp8_dispatch else self.dispatch_bytes(2)
 
     def expert_weight_bytes(self, b: int = 2) -> int:
         return 3 * self.H * self.F * self.E * b

@@ -54,6 +54,8 @@ moe_status check_dims(const moe_dims* d) {
   if (d->group_limit > 0 && d->P > MOE_MAX_LIMITED_GROUPS) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (d->F_shared < 0) return MOE_ERR_INVALID_ARG;
   if (d->F_shared % 8 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (d->fp8_dispatch != 0 && d->fp8_dispatch != 1) return MOE_ERR_INVALID_ARG;
+  if (d->fp8_dispatch && d->H % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (d->T * static_cast<long long>(d->K) > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED_SHAPE;
   return MOE_OK;
 }
@@ -195,6 +197,42 @@ moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_
                                     meta_token, meta_slot, meta_w, meta_local_expert, as_stream(stream)));
 }
 
+moe_status moe_quantize_fp8_rows(const void* x, int64_t rows, int32_t cols, void* q, float* scales, void* stream) {
+  if (rows < 0 || cols < 16) return MOE_ERR_INVALID_ARG;
+  if (cols % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (!device_ok()) return MOE_ERR_NO_DEVICE;
+  if (rows == 0) return MOE_OK;
+  if (!x || !q || !scales || !aligned16(x) || !aligned16(q)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_quantize_fp8_rows(x, rows, cols, q, scales, as_stream(stream)));
+}
+
+moe_status moe_permute_fp8(const void* x, const int32_t* row_of_assign, const int32_t* topk_ids,
+                           const float* topk_w, const moe_dims* d, void* xq, float* xs, int32_t* meta_token,
+                           int32_t* meta_slot, float* meta_w, int32_t* meta_local_expert, void* stream) {
+  MOE_TRY(common_checks(d));
+  if (d->H % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (d->T == 0) return MOE_OK;
+  if (!x || !row_of_assign || !xq || !xs || (meta_w && !topk_w) || (meta_local_expert && !topk_ids))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(xq)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_permute_fp8(x, row_of_assign, topk_ids, topk_w, d->T, d->H, d->E, d->K, d->P, xq, xs,
+                                        meta_token, meta_slot, meta_w, meta_local_expert, as_stream(stream)));
+}
+
+moe_status moe_grouped_gate_up_fp8(const void* xq, const float* xs, const int32_t* offsets, const void* wq_gate,
+                                   const void* wq_up, const float* s_gate, const float* s_up, const moe_dims* d,
+                                   void* h, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(common_checks(d));
+  MOE_TRY(check_ws(ws, ws_bytes, d));
+  if (d->H % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
+  if (d->T == 0) return MOE_OK;
+  if (!xq || !xs || !offsets || !wq_gate || !wq_up || !s_gate || !s_up || !h) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(wq_gate) || !aligned16(wq_up)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(gemm_gate_up_fp8(xq, xs, offsets, wq_gate, wq_up, s_gate, s_up, d->E,
+                                      d->T * static_cast<long long>(d->K), d->H, d->F, h, ws_status(ws),
+                                      as_stream(stream)));
+}
+
 moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up,
                                const moe_dims* d, void* h, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(common_checks(d));
@@ -288,14 +326,18 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   MOE_TRY(check_ws(ws, ws_bytes, d));
   if (!x || !w || !b) return MOE_ERR_INVALID_ARG;
   const bool latent = d->d_model > 0;
-  if (!w->w_g_split || !w->w_down || (!w->w_gate_up && (!w->w_gate || !w->w_up))) return MOE_ERR_INVALID_ARG;
+  const bool fp8 = d->fp8_dispatch != 0;
+  if (!w->w_g_split || !w->w_down) return MOE_ERR_INVALID_ARG;
+  if (!fp8 && !w->w_gate_up && (!w->w_gate || !w->w_up)) return MOE_ERR_INVALID_ARG;
+  if (fp8 && (!w->w_gate_q || !w->w_up_q || !w->s_gate || !w->s_up || !b->xq || !b->xs)) return MOE_ERR_INVALID_ARG;
+  if (fp8 && (!aligned16(w->w_gate_q) || !aligned16(w->w_up_q) || !aligned16(b->xq))) return MOE_ERR_INVALID_ARG;
   if (latent && (!w->w_dp || !w->w_upp || !b->z || !b->final_out)) return MOE_ERR_INVALID_ARG;
   const bool shared = d->F_shared > 0;
   if (shared && (!w->w_shared_gate || !w->w_shared_up || !w->w_shared_down || !b->h_shared || !b->y_shared))
     return MOE_ERR_INVALID_ARG;
   if (shared && b->aux_stream && (!b->fork_event || !b->join_event)) return MOE_ERR_INVALID_ARG;
   if (!b->logits || !b->topk_ids || !b->topk_w || !b->counts || !b->offsets || !b->part_counts ||
-      !b->part_offsets || !b->row_of_assign || !b->assign_of_row || !b->xp || !b->h || !b->y || !b->out)
+      !b->part_offsets || !b->row_of_assign || !b->assign_of_row || (!fp8 && !b->xp) || !b->h || !b->y || !b->out)
     return MOE_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   auto mark = [&](int i) -> moe_status {
@@ -332,11 +374,18 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   MOE_CUDA(launch_count_scan(b->topk_ids, TK, d->E, d->P, b->counts, b->offsets, b->part_counts, b->part_offsets,
                              b->row_of_assign, b->assign_of_row, b->skew, scan_ws(ws, d), s));
   MOE_TRY(mark(4));
-  MOE_CUDA(launch_permute(routed, b->row_of_assign, b->topk_ids, b->topk_w, T, d->H, d->E, d->K, d->P, b->xp,
-                          b->meta_token, b->meta_slot, b->meta_w, b->meta_local_expert, s));
+  if (fp8)
+    MOE_CUDA(launch_permute_fp8(routed, b->row_of_assign, b->topk_ids, b->topk_w, T, d->H, d->E, d->K, d->P, b->xq,
+                                b->xs, b->meta_token, b->meta_slot, b->meta_w, b->meta_local_expert, s));
+  else
+    MOE_CUDA(launch_permute(routed, b->row_of_assign, b->topk_ids, b->topk_w, T, d->H, d->E, d->K, d->P, b->xp,
+                            b->meta_token, b->meta_slot, b->meta_w, b->meta_local_expert, s));
   MOE_TRY(mark(5));
   if (T > 0) {
-    if (w->w_gate_up)
+    if (fp8)
+      MOE_CUDA(gemm_gate_up_fp8(b->xq, b->xs, b->offsets, w->w_gate_q, w->w_up_q, w->s_gate, w->s_up, d->E, TK, d->H,
+                                d->F, b->h, status, s));
+    else if (w->w_gate_up)
       MOE_CUDA(gemm_gate_up_packed(b->xp, b->offsets, w->w_gate_up, d->E, TK, d->H, d->F, b->h, status, s));
     else
       MOE_CUDA(gemm_gate_up(b->xp, b->offsets, w->w_gate, w->w_up, d->E, TK, d->H, d->F, b->h, status, s));

@@ -13,6 +13,8 @@
 // item space is (token, vector) flattened, so consecutive threads touch
 // consecutive 16-byte pieces of one row (coalesced on both sides), and each
 // thread keeps several independent items in flight.
+#include <cuda_fp8.h>
+
 #include <algorithm>
 
 #include "device.cuh"
@@ -196,6 +198,112 @@ __global__ void pack_gate_up_kernel(const uint4* __restrict__ wg, const uint4* _
   }
 }
 
+// ---------------------------------------------------------------------------
+// FP8 (E4M3) rows with one fp32 scale per row.  Low-precision dispatch quantizes the
+// outbound activation and carries its scales (WideEP essay, "Top-k multiplies traffic.
+// Locality subtracts it.").  s = amax / 448 (1 for an all-zero row), code = E4M3 of x / s
+// (IEEE fp32 division, round to nearest even, saturating): both are decided in fp32.
+// One block per row: the first pass reduces |x| to amax, the second (an L1/L2 hit)
+// converts 8 values per 16-byte vector into one 8-byte store per destination row.
+// ---------------------------------------------------------------------------
+constexpr int kQuantThreads = 128;
+constexpr float kE4M3Max = 448.0f;
+
+__device__ __forceinline__ float block_max(float v, float* s_red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) s_red[warp] = v;
+  __syncthreads();
+  float m = s_red[0];
+#pragma unroll
+  for (int w = 1; w < kQuantThreads / 32; ++w) m = fmaxf(m, s_red[w]);
+  __syncthreads();  // s_red is reused by the next row
+  return m;
+}
+
+__device__ __forceinline__ uint2 quantize8(const uint4 v, float s) {
+  const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+  uint32_t w[2] = {0u, 0u};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const float2 f = __bfloat1622float2(p[j]);
+    const uint32_t lo = __nv_cvt_float_to_fp8(__fdiv_rn(f.x, s), __NV_SATFINITE, __NV_E4M3);
+    const uint32_t hi = __nv_cvt_float_to_fp8(__fdiv_rn(f.y, s), __NV_SATFINITE, __NV_E4M3);
+    w[j >> 1] |= (lo | (hi << 8)) << (16 * (j & 1));
+  }
+  return make_uint2(w[0], w[1]);
+}
+
+__device__ __forceinline__ float row_amax(const uint4* __restrict__ xr, int vpr) {
+  float m = 0.0f;
+  for (int v = threadIdx.x; v < vpr; v += kQuantThreads) {
+    const uint4 u = xr[v];
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const float2 f = __bfloat1622float2(p[j]);
+      m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+    }
+  }
+  return m;
+}
+
+// Rows of x [rows][vpr * 8] -> q [rows][vpr * 8] codes, scales [rows].
+__global__ void __launch_bounds__(kQuantThreads) quantize_fp8_rows_kernel(const uint4* __restrict__ x, long long rows,
+                                                                           int vpr, uint2* __restrict__ q,
+                                                                           float* __restrict__ scales) {
+  __shared__ float s_red[kQuantThreads / 32];
+  for (long long r = blockIdx.x; r < rows; r += gridDim.x) {
+    const uint4* xr = x + r * vpr;
+    const float amax = block_max(row_amax(xr, vpr), s_red);
+    const float s = amax > 0.0f ? __fdiv_rn(amax, kE4M3Max) : 1.0f;
+    for (int v = threadIdx.x; v < vpr; v += kQuantThreads) q[r * vpr + v] = quantize8(xr[v], s);
+    if (threadIdx.x == 0) scales[r] = s;
+  }
+}
+
+// FP8 dispatch: token t quantized once, its codes and scale stored at the rows of its K
+// assignments; routing metadata as in permute_kernel.
+__global__ void __launch_bounds__(kQuantThreads) permute_fp8_kernel(
+    const uint4* __restrict__ x, const int32_t* __restrict__ roa, const int32_t* __restrict__ ids,
+    const float* __restrict__ w, long long T, int vpr, int E, int K, int P, uint2* __restrict__ xq,
+    float* __restrict__ xs, int32_t* __restrict__ meta_token, int32_t* __restrict__ meta_slot,
+    float* __restrict__ meta_w, int32_t* __restrict__ meta_local) {
+  pdl_wait();  // row_of_assign comes from the count/scan kernel
+  pdl_launch_dependents();
+  __shared__ float s_red[kQuantThreads / 32];
+  __shared__ int s_row[MOE_MAX_K];
+  const long long TK = T * K;
+  const int epp = E / P;
+  for (long long t = blockIdx.x; t < T; t += gridDim.x) {
+    if (threadIdx.x < K) {
+      const long long a = t * K + threadIdx.x;
+      const int r = __ldg(roa + a);
+      const bool ok = static_cast<unsigned long long>(r) < static_cast<unsigned long long>(TK);
+      s_row[threadIdx.x] = ok ? r : -1;
+      if (ok) {
+        if (meta_token) meta_token[r] = static_cast<int>(t);
+        if (meta_slot) meta_slot[r] = threadIdx.x;
+        if (meta_w) meta_w[r] = __ldg(w + a);
+        if (meta_local) meta_local[r] = __ldg(ids + a) % epp;
+      }
+    }
+    const uint4* xr = x + t * vpr;
+    const float amax = block_max(row_amax(xr, vpr), s_red);  // its barriers also publish s_row
+    const float s = amax > 0.0f ? __fdiv_rn(amax, kE4M3Max) : 1.0f;
+    if (threadIdx.x < K && s_row[threadIdx.x] >= 0) xs[s_row[threadIdx.x]] = s;
+    for (int v = threadIdx.x; v < vpr; v += kQuantThreads) {
+      const uint2 c = quantize8(xr[v], s);
+      for (int k = 0; k < K; ++k) {
+        const int r = s_row[k];
+        if (r >= 0) xq[static_cast<long long>(r) * vpr + v] = c;
+      }
+    }
+    __syncthreads();  // s_row is rewritten for the next token
+  }
+}
+
 int copy_blocks(long long items) {
   const long long want = (items + kCopyThreads - 1) / kCopyThreads;
   return static_cast<int>(std::max<long long>(1, std::min<long long>(want, 8LL * num_sms())));
@@ -211,6 +319,25 @@ cudaError_t launch_permute(const void* x, const int32_t* roa, const int32_t* ids
   return launch_pdl(permute_kernel, dim3(copy_blocks(T * vpr / 2)), dim3(kCopyThreads), 0, s,
                     reinterpret_cast<const uint4*>(x), roa, ids, w, T, vpr, E, K, P, reinterpret_cast<uint4*>(xp),
                     meta_token, meta_slot, meta_w, meta_local);
+}
+
+cudaError_t launch_quantize_fp8_rows(const void* x, long long rows, int cols, void* q, float* scales,
+                                     cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<long long>(rows, 16LL * num_sms()));
+  quantize_fp8_rows_kernel<<<blocks, kQuantThreads, 0, s>>>(reinterpret_cast<const uint4*>(x), rows, cols / 8,
+                                                            reinterpret_cast<uint2*>(q), scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_fp8(const void* x, const int32_t* roa, const int32_t* ids, const float* w, long long T,
+                               int H, int E, int K, int P, void* xq, float* xs, int32_t* meta_token,
+                               int32_t* meta_slot, float* meta_w, int32_t* meta_local, cudaStream_t s) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = static_cast<int>(std::min<long long>(T, 16LL * num_sms()));
+  return launch_pdl(permute_fp8_kernel, dim3(blocks), dim3(kQuantThreads), 0, s, reinterpret_cast<const uint4*>(x),
+                    roa, ids, w, T, H / 8, E, K, P, reinterpret_cast<uint2*>(xq), xs, meta_token, meta_slot, meta_w,
+                    meta_local);
 }
 
 cudaError_t launch_combine(const void* y, const int32_t* roa, const float* w, const void* shared, long long T, int H,

@@ -77,6 +77,14 @@ struct Cfg<kEpiSwiGLUPacked> {
   static constexpr int NA = 2, NT = 256, STAGES = 3, FEAT = 128;
   static constexpr bool SEP = true;
 };
+// SwiGLU on E4M3 operands (FP8 dispatch): the same tile as the bf16 SwiGLU, each stage
+// carrying 128 K-elements (one 128-byte swizzle atom of 8-bit codes) instead of 64, so a
+// stage holds twice the MMA work.
+template <>
+struct Cfg<kEpiSwiGLUFp8> {
+  static constexpr int NA = 2, NT = 128, STAGES = 4, FEAT = 128;
+  static constexpr bool SEP = true;
+};
 // Plain bf16 output (down projection, latent projections).
 template <>
 struct Cfg<kEpiBF16> {
@@ -110,6 +118,12 @@ struct Layout {
 struct Tile {
   int g, n0, row0, nvalid, nround;
 };
+
+// K elements per stage: one 128-byte swizzle atom per operand row.
+template <int EPI>
+constexpr int stage_k() {
+  return EPI == kEpiSwiGLUFp8 ? 128 : kBK;
+}
 
 // silu(g) * u = g u / (1 + e^-g) with the fast exponential and divide (2 MUFU ops):
 // for g -> -inf the denominator overflows and the result is 0, for g -> +inf it is g u.
@@ -202,7 +216,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.offsets ? args.G : 1;
   const int NFT = (args.N + C::FEAT - 1) / C::FEAT;
-  const int KB = (args.Kd + kBK - 1) / kBK;
+  constexpr int KS = stage_k<EPI>();
+  const int KB = (args.Kd + KS - 1) / KS;
 
   // Set-up that reads no global input runs before the wait on the previous kernel.
   __shared__ int s_bad;
@@ -270,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           uint8_t* st = ring + stage * L::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
-          const int kx = kb * kBK;
+          const int kx = kb * KS;
           if constexpr (EPI == kEpiBF16 || EPI == kEpiSwiGLUPacked) {
             // both 128-row weight tiles in one 256-row box (packed rows are 2 per feature)
             tma_load_3d(st, &tmA0, &full[stage], kx, (EPI == kEpiSwiGLUPacked) ? 2 * tl.n0 : tl.n0, tl.g);
@@ -316,7 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           break;
         }
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(kBM, tl.nround);
+        const uint32_t idesc =
+            (EPI == kEpiSwiGLUFp8) ? idesc_e4m3_f32(kBM, tl.nround) : idesc_bf16_f32(kBM, tl.nround);
         const uint32_t d0 = tmem_base + acc * L::kAccCols;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) {
@@ -326,15 +342,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t sa = smem_u32(ring + stage * L::kStageBytes);
           const uint32_t sb = sa + NA * kABytes;
+          // four MMAs per 128-byte atom: K = 16 bf16 or 32 E4M3 elements (32 bytes) each
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk) {
+          for (int kk = 0; kk < 4; ++kk) {
             const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
 #pragma unroll
             for (int i = 0; i < NA; ++i) {
               const uint64_t adesc = sw128_kmajor_desc(sa + i * kABytes + kk * 32);
               const uint32_t d = d0 + (C::SEP ? i * NT : 0);
               const uint32_t accumulate = (kb > 0 || kk > 0 || (!C::SEP && i > 0)) ? 1u : 0u;
-              umma_bf16(d, adesc, bdesc, idesc, accumulate);
+              if constexpr (EPI == kEpiSwiGLUFp8) umma_e4m3(d, adesc, bdesc, idesc, accumulate);
+              else umma_bf16(d, adesc, bdesc, idesc, accumulate);
             }
           }
           umma_commit(&empty[stage]);  // frees the stage once these MMAs have read it
@@ -412,12 +430,20 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int f = tl.n0 + q * 32 + lane;
       const bool f_ok = f < args.N;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
+      float sg = 1.0f, su = 1.0f;  // FP8: per-feature weight scales of this thread's output feature
+      if constexpr (EPI == kEpiSwiGLUFp8) {
+        if (f_ok) {
+          const long long fi = static_cast<long long>(tl.g) * args.N + f;
+          sg = __ldg(args.scale_a0 + fi);
+          su = __ldg(args.scale_a1 + fi);
+        }
+      }
       for (int j0 = 0; j0 < tl.nvalid; j0 += 32) {
         uint32_t r0[32];
         tmem_ld_32cols(tbase + j0, r0);
         const int jn = min(32, tl.nvalid - j0);
         const long long row0 = static_cast<long long>(tl.row0) + j0;
-        if constexpr (EPI == kEpiSwiGLU) {
+        if constexpr (EPI == kEpiSwiGLU || EPI == kEpiSwiGLUFp8) {
           uint32_t r1[32];
           tmem_ld_32cols(tbase + NT + j0, r1);
           tmem_wait_ld();
@@ -426,8 +452,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
               if (j < jn) {
-                out[(row0 + j) * args.ldo + f] =
-                    __float2bfloat16_rn(silu_mul(__uint_as_float(r0[j]), __uint_as_float(r1[j])));
+                float g = __uint_as_float(r0[j]), u = __uint_as_float(r1[j]);
+                if constexpr (EPI == kEpiSwiGLUFp8) {
+                  const float sx = __ldg(args.scale_b + row0 + j);  // same address in every lane
+                  g *= sx * sg;
+                  u *= sx * su;
+                }
+                out[(row0 + j) * args.ldo + f] = __float2bfloat16_rn(silu_mul(g, u));
               }
             }
           }
@@ -784,34 +815,38 @@ EncodeTiledFn encoder() {
   return fn;
 }
 
-// bf16 tensor [d2][d1][d0] (d0 contiguous), box {64, box1, 1}, 128-byte swizzle.
-bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1) {
+// Tensor [d2][d1][d0] (d0 contiguous) of bf16 (elem = 2) or 8-bit codes (elem = 1), box
+// {128 bytes of d0, box1, 1}, 128-byte swizzle.
+bool map_bf16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box1,
+                 int elem = 2) {
   EncodeTiledFn enc = encoder();
   if (!enc) return false;
   const cuuint64_t dims[3] = {d0, d1, d2};
-  const cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
-  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kBK), box1, 1};
+  const cuuint64_t strides[2] = {d0 * elem, d0 * d1 * elem};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), box1, 1};
   const cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+  return enc(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 3,
+             const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool map_bf16_2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t box1) {
+bool map_bf16_2d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1, uint32_t box1, int elem = 2) {
   EncodeTiledFn enc = encoder();
   if (!enc) return false;
   const cuuint64_t dims[2] = {d0, d1};
-  const cuuint64_t strides[1] = {d0 * 2};
-  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kBK), box1};
+  const cuuint64_t strides[1] = {d0 * elem};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem), box1};
   const cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, es,
+  return enc(m, elem == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+             const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-bool map_token_boxes(BoxMaps* m, const void* base, uint64_t d0, uint64_t rows) {
+bool map_token_boxes(BoxMaps* m, const void* base, uint64_t d0, uint64_t rows, int elem = 2) {
   for (int i = 0; i < kNumBoxes; ++i)
-    if (!map_bf16_2d(&m->box[i], base, d0, rows, 256u >> i)) return false;
+    if (!map_bf16_2d(&m->box[i], base, d0, rows, 256u >> i, elem)) return false;
   return true;
 }
 
@@ -860,6 +895,7 @@ int gemm_smem_bytes(int epi) {
     case kEpiSwiGLU: return Layout<kEpiSwiGLU>::kSmemBytes;
     case kEpiSwiGLUPacked: return Layout<kEpiSwiGLUPacked>::kSmemBytes;
     case kEpiBF16: return Layout<kEpiBF16>::kSmemBytes;
+    case kEpiSwiGLUFp8: return Layout<kEpiSwiGLUFp8>::kSmemBytes;
     default: return Layout<kEpiF32>::kSmemBytes;
   }
 }
@@ -900,6 +936,21 @@ cudaError_t gemm_gate_up_packed(const void* xp, const int32_t* offsets, const vo
   return launch<kEpiSwiGLUPacked>(a0, a0, a0, b, args,
                                   tile_bound(rows, E, Cfg<kEpiSwiGLUPacked>::NT, F, Cfg<kEpiSwiGLUPacked>::FEAT),
                                   stream);
+}
+
+// FP8 dispatch: gate/up on E4M3 codes; g and u are scaled by the row's and the feature's
+// scales in the epilogue (both factor out of the K sum), h is bf16 as in gemm_gate_up.
+cudaError_t gemm_gate_up_fp8(const void* xq, const float* xs, const int32_t* offsets, const void* wq_gate,
+                             const void* wq_up, const float* s_gate, const float* s_up, int E, long long rows, int H,
+                             int F, void* h, int* status, cudaStream_t stream) {
+  GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status, s_gate, s_up, xs};
+  CUtensorMap a0, a1;
+  BoxMaps b;
+  if (!map_token_boxes(&b, xq, H, rows, 1) || !map_bf16_3d(&a0, wq_gate, H, F, E, kBM, 1) ||
+      !map_bf16_3d(&a1, wq_up, H, F, E, kBM, 1))
+    return cudaErrorInvalidValue;
+  return launch<kEpiSwiGLUFp8>(a0, a1, a1, b, args,
+                               tile_bound(rows, E, Cfg<kEpiSwiGLUFp8>::NT, F, Cfg<kEpiSwiGLUFp8>::FEAT), stream);
 }
 
 // y = h Wd^T per expert group.

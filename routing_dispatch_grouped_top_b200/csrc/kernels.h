@@ -6,7 +6,7 @@
 
 namespace moe {
 
-enum Epi : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2, kEpiSwiGLUPacked = 3 };
+enum Epi : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2, kEpiSwiGLUPacked = 3, kEpiSwiGLUFp8 = 4 };
 
 struct GemmArgs {
   const int32_t* offsets;  // [G + 1] device row offsets of the groups, or nullptr: one group of M rows
@@ -18,6 +18,9 @@ struct GemmArgs {
   long long ldo;           // output row stride in elements
   const float* bias;       // kEpiF32 only: [N] or nullptr
   int* status;             // device status word (MOE_DEV_* bits)
+  const float* scale_a0;   // kEpiSwiGLUFp8: per-feature scales of the gate weights [G][N]
+  const float* scale_a1;   //                per-feature scales of the up weights [G][N]
+  const float* scale_b;    //                per-row scales of the token operand [M]
 };
 
 int num_sms();             // SM count of the current device (cached per device)
@@ -49,6 +52,10 @@ cudaError_t launch_pack_gate_up(const void* w_gate, const void* w_up, int E, int
                                 cudaStream_t stream);
 cudaError_t gemm_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, int E, long long rows,
                                 int H, int F, void* h, int* status, cudaStream_t stream);
+// h = silu(s_x s_g (xq Wg_q^T)) * (s_x s_u (xq Wu_q^T)) on E4M3 operands.
+cudaError_t gemm_gate_up_fp8(const void* xq, const float* xs, const int32_t* offsets, const void* wq_gate,
+                             const void* wq_up, const float* s_gate, const float* s_up, int E, long long rows, int H,
+                             int F, void* h, int* status, cudaStream_t stream);
 cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down, int E, long long rows, int H,
                       int F, void* y, int* status, cudaStream_t stream);
 cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd, void* out, int* status,
@@ -76,6 +83,11 @@ cudaError_t launch_skew(const int32_t* counts, int E, float* ratio, cudaStream_t
 cudaError_t launch_permute(const void* x, const int32_t* row_of_assign, const int32_t* ids, const float* w,
                            long long T, int H, int E, int K, int P, void* xp, int32_t* meta_token,
                            int32_t* meta_slot, float* meta_w, int32_t* meta_local, cudaStream_t stream);
+cudaError_t launch_quantize_fp8_rows(const void* x, long long rows, int cols, void* q, float* scales,
+                                     cudaStream_t stream);
+cudaError_t launch_permute_fp8(const void* x, const int32_t* row_of_assign, const int32_t* ids, const float* w,
+                               long long T, int H, int E, int K, int P, void* xq, float* xs, int32_t* meta_token,
+                               int32_t* meta_slot, float* meta_w, int32_t* meta_local, cudaStream_t stream);
 cudaError_t launch_combine(const void* y, const int32_t* row_of_assign, const float* w, const void* shared,
                            long long T, int H, int K, void* out, cudaStream_t stream);
 cudaError_t launch_pack_router(const float* w_g, int H, int E, void* w_split, cudaStream_t stream);

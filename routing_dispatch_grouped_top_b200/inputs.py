@@ -160,6 +160,20 @@ def random_bf16(shape, seed: int = 0, std: float = 1.0, device="cpu") -> torch.T
     return _randn(shape, std, g, device, torch.bfloat16)
 
 
+def random_e4m3_codes(shape, seed: int = 0, spread: float = 64.0) -> torch.Tensor:
+    """uint8 E4M3 bit patterns of N(0, spread^2) draws clamped to +-448 (torch's own float8
+    conversion); no NaN codes."""
+    g = _gen("cpu", seed)
+    v = (torch.randn(shape, generator=g) * spread).clamp_(-448.0, 448.0)
+    return v.to(torch.float8_e4m3fn).view(torch.uint8)
+
+
+def random_scales(n: int, seed: int = 0, lo: float = 2.0 ** -9, hi: float = 2.0 ** -5) -> torch.Tensor:
+    """fp32 row scales, log-uniform in [lo, hi]."""
+    g = _gen("cpu", seed)
+    return torch.exp(torch.empty(n).uniform_(float(np.log(lo)), float(np.log(hi)), generator=g)).to(torch.float32)
+
+
 def random_counts(E: int, total: int, seed: int = 0, zipf_s=None, zero_frac: float = 0.0):
     """Per-expert row counts summing to ``total`` (some forced to zero if zero_frac > 0)."""
     g = _gen("cpu", seed)

@@ -118,6 +118,12 @@ SMALL = [
                               F_shared=384),
     LATENT_896E.with_(name="latent_shared_expert_T40_D512_H256_E64_Fs128", T=40, d_model=512, H=256, E=64, F=128,
                       P=8, F_shared=128),
+    QWEN3_30B_A3B_PREFILL.with_(name="qwen3_shape_fp8_dispatch_T256_H512_F384", T=256, H=512, F=384,
+                                fp8_dispatch=True),
+    DEEPSEEK_R1_PREFILL.with_(name="r1_shape_fp8_dispatch_T64_H1024_F256_E64", T=64, H=1024, F=256, E=64,
+                              fp8_dispatch=True),
+    LATENT_896E.with_(name="latent_fp8_dispatch_T48_D1024_H256_E112_P8", T=48, d_model=1024, H=256, E=112, F=128,
+                      P=8, fp8_dispatch=True),
 ]
 
 
@@ -136,7 +142,7 @@ def test_layer_matches_oracle(cfg):
                              bias=None if cpu_in["bias"] is None else cpu_in["bias"].numpy(),
                              w_dp_bits=None if cpu_in["w_dp"] is None else bits(cpu_in["w_dp"]),
                              w_upp_bits=None if cpu_in["w_upp"] is None else bits(cpu_in["w_upp"]),
-                             group_limit=cfg.group_limit, shared=shared)
+                             group_limit=cfg.group_limit, shared=shared, fp8=cfg.fp8_dispatch)
     latent = bool(cfg.d_model)
     if shared is not None and not latent:
         check_bf16("h_shared", bits(g["h_shared"]), r["h_shared"])
@@ -163,7 +169,10 @@ def test_layer_matches_oracle(cfg):
     if order_safe.all():
         for k in ("counts", "offsets", "part_counts", "part_offsets", "row_of_assign", "assign_of_row"):
             assert np.array_equal(cpu(g[k]), r[k]), k
-        if not latent:
+        if cfg.fp8_dispatch and not latent:
+            assert np.array_equal(cpu(g["xq"]), r["xq"])
+            assert np.array_equal(cpu(g["xs"]).view(np.uint32), r["xs"].view(np.uint32))
+        elif not latent:
             assert np.array_equal(bits(g["xp"]), r["xp"])
         for key, mk in (("meta_token", "token"), ("meta_slot", "slot"), ("meta_local_expert", "local_expert")):
             assert np.array_equal(cpu(g[key]), r["meta"][mk]), key
@@ -231,7 +240,8 @@ def test_layer_stage_events_are_recorded():
 # Full workloads: sampled tokens + size-independent properties
 # ---------------------------------------------------------------------------
 
-FULL = [QWEN3_30B_A3B_PREFILL, DEEPSEEK_R1_PREFILL, DEEPSEEK_R1_DECODE, LATENT_896E]
+FULL = [QWEN3_30B_A3B_PREFILL, DEEPSEEK_R1_PREFILL, DEEPSEEK_R1_DECODE, LATENT_896E,
+        DEEPSEEK_R1_PREFILL.with_(name=DEEPSEEK_R1_PREFILL.name + "_fp8_dispatch", fp8_dispatch=True)]
 HOST_EXPERT_BUDGET = 2.5e9   # bytes of expert weights copied to the host for the oracle
 
 
@@ -248,9 +258,15 @@ def test_full_size_sampled(cfg):
     routed = g["z"] if latent else inp["x"]
     roa = g["row_of_assign"].long()
     tok = torch.arange(T * K, device=DEV) // K
-    assert torch.equal(g["xp"][roa].view(torch.int16), routed[tok].view(torch.int16))
+    fp8 = cfg.fp8_dispatch
+    if fp8:   # every copy of a token carries the same codes and scale
+        first = roa.view(T, K)[:, :1].expand(T, K).reshape(-1)
+        assert torch.equal(g["xq"][roa], g["xq"][first]) and torch.equal(g["xs"][roa], g["xs"][first])
+        assert g["xq"].numel() + 4 * g["xs"].numel() == oracle.dispatch_bytes_fp8(T, K, H)
+    else:
+        assert torch.equal(g["xp"][roa].view(torch.int16), routed[tok].view(torch.int16))
+        assert g["xp"].numel() * 2 == oracle.dispatch_bytes(T, K, H, 2)
     assert torch.equal(g["meta_token"][roa].long(), tok)
-    assert g["xp"].numel() * 2 == oracle.dispatch_bytes(T, K, H, 2)
     # sampled tokens through the oracle
     rng = np.random.default_rng(cfg.T + cfg.E)
     cand = rng.permutation(T)[:256]
@@ -275,6 +291,8 @@ def test_full_size_sampled(cfg):
     # FFN + combine for sampled tokens with an unambiguous expert set, within a host-memory budget
     per_expert = 3 * H * F * 2
     max_experts = max(K, int(HOST_EXPERT_BUDGET // per_expert))
+    if cfg.fp8_dispatch:
+        max_experts = min(max_experts, 2 * K)    # the oracle quantizes each expert's weights on the host
     chosen, experts = [], set()
     for i in np.nonzero(set_safe)[0]:
         need = experts | set(ids_ref[i].tolist())
@@ -286,6 +304,15 @@ def test_full_size_sampled(cfg):
             break
     assert chosen, "no unambiguous sampled token"
     wcache = {e: (bits(inp["w_gate"][e]), bits(inp["w_up"][e]), bits(inp["w_down"][e])) for e in sorted(experts)}
+    if fp8:   # the oracle quantizes the sampled tokens and the experts' gate/up weights itself
+        zq, zs = oracle.quantize_rows_fp8(z_rows)
+        rows0 = torch.from_numpy(cpu(g["row_of_assign"]).reshape(T, K)[cand, 0].astype(np.int64)).to(DEV)
+        assert np.array_equal(cpu(g["xq"][rows0]), zq)
+        assert np.array_equal(cpu(g["xs"][rows0]).view(np.uint32), zs.view(np.uint32))
+        wq = {}
+        for e, (wg_, wu_, wd_) in wcache.items():
+            (qg, sg), (qu, su) = oracle.quantize_rows_fp8(wg_), oracle.quantize_rows_fp8(wu_)
+            wq[e] = (qg, sg, qu, su, wd_)
     ga = cpu(g["row_of_assign"]).reshape(T, K)
     gh, gy, gout = [], [], []
     rh, ry, rout = [], [], []
@@ -294,7 +321,10 @@ def test_full_size_sampled(cfg):
         acc = np.zeros(H)
         for k in range(K):
             e = int(ids_ref[i, k])
-            h_, y_ = oracle.ffn_rows(z_rows[i:i + 1], *wcache[e])
+            if fp8:
+                h_, y_ = oracle.ffn_rows_fp8(zq[i:i + 1], zs[i:i + 1], *wq[e])
+            else:
+                h_, y_ = oracle.ffn_rows(z_rows[i:i + 1], *wcache[e])
             rh.append(h_[0])
             ry.append(y_[0])
             acc += float(w_ref[i, k]) * oracle.bf16_bits_to_f64(y_)[0]

@@ -266,6 +266,87 @@ def test_grouped_ffn_matches_oracle(E, H, F, rows, zipf, zf, packed):
     check_bf16("y", bits(y), ry)
 
 
+# ---------------------------------------------------------------------------
+# FP8 dispatch: E4M3 codes with per-row scales, gate/up on E4M3
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("rows,cols", [(300, 256), (64, 7168), (7, 16), (129, 2064), (1, 48), (0, 32)])
+def test_quantize_fp8_rows_matches_oracle_bit_exact(rows, cols):
+    x = inputs.random_bf16((rows, cols), seed=rows + cols)
+    if rows:
+        # rows over many magnitudes, one all-zero row, one row of a single nonzero element
+        x = x * torch.exp(torch.linspace(-20.0, 12.0, rows)).to(torch.bfloat16)[:, None]
+        x[rows // 2] = 0
+        x[-1, :] = 0
+        x[-1, cols // 3] = -3.0
+    q = torch.full((rows, cols), 0x55, dtype=torch.uint8, device=DEV)
+    sc = torch.full((rows,), -1.0, dtype=torch.float32, device=DEV)
+    B.moe_quantize_fp8_rows(x.to(DEV), q, sc)
+    torch.cuda.synchronize()
+    rq, rs = oracle.quantize_rows_fp8(bits(x))
+    assert np.array_equal(cpu(q), rq)
+    assert np.array_equal(cpu(sc).view(np.uint32), rs.view(np.uint32))
+
+
+@pytest.mark.parametrize("T,H,E,K,P", [(300, 256, 16, 4, 4), (1, 16, 4, 1, 1), (64, 7168, 256, 8, 8),
+                                       (1000, 2048, 128, 8, 1), (33, 80, 6, 6, 3), (0, 64, 8, 2, 1)])
+def test_permute_fp8_matches_oracle_bit_exact(T, H, E, K, P):
+    x = inputs.random_bf16((T, H), seed=T + H)
+    ids = inputs.random_topk_ids(T, E, K, seed=T + E) if T else torch.zeros((0, K), dtype=torch.int32)
+    w = inputs.random_weights(T, K, seed=5)
+    cs = oracle.count_scan(ids.numpy(), E, P)
+    roa = torch.from_numpy(cs["row_of_assign"])
+    d = B.dims(T=T, H=H, E=E, K=K, F=8, P=P, fp8_dispatch=True)
+    TK = T * K
+    xq = torch.full((TK, H), 0x55, dtype=torch.uint8, device=DEV)
+    xs = torch.full((TK,), -1.0, dtype=torch.float32, device=DEV)
+    meta = [torch.full((TK,), -1, dtype=dt, device=DEV) for dt in (torch.int32, torch.int32, torch.float32, torch.int32)]
+    B.moe_permute_fp8(x.to(DEV), roa.to(DEV), ids.to(DEV), w.to(DEV), d, xq, xs, *meta)
+    torch.cuda.synchronize()
+    rq, rs = oracle.dispatch_fp8(bits(x), cs["row_of_assign"], K)
+    assert np.array_equal(cpu(xq), rq)
+    assert np.array_equal(cpu(xs).view(np.uint32), rs.view(np.uint32))
+    assert xq.numel() + 4 * xs.numel() == oracle.dispatch_bytes_fp8(T, K, H)
+    _, rmeta = oracle.permute(bits(x), cs["row_of_assign"], ids.numpy(), w.numpy(), E, P)
+    for got, key in zip(meta, ("token", "slot", "w", "local_expert")):
+        assert np.array_equal(cpu(got), rmeta[key]), key
+
+
+FP8_FFN_CASES = [  # E, H, F, rows, zipf, zero_frac
+    (8, 256, 512, 300, None, 0.25), (4, 208, 200, 260, None, 0.0), (16, 2048, 768, 2000, 1.1, 0.2),
+    (3, 64, 136, 1, None, 0.0), (32, 512, 256, 700, 2.0, 0.3), (1, 1024, 384, 513, None, 0.0),
+    (8, 7168, 256, 300, None, 0.0),
+]
+
+
+@pytest.mark.parametrize("E,H,F,rows,zipf,zf", FP8_FFN_CASES)
+def test_grouped_gate_up_fp8_matches_oracle(E, H, F, rows, zipf, zf):
+    counts = inputs.random_counts(E, rows, seed=E + rows, zipf_s=zipf, zero_frac=zf)
+    off = np.zeros(E + 1, np.int32)
+    off[1:] = np.cumsum(counts.numpy())
+    xq = inputs.random_e4m3_codes((rows, H), seed=1)
+    xs = inputs.random_scales(rows, seed=2)
+    wgq = inputs.random_e4m3_codes((E, F, H), seed=3)
+    wuq = inputs.random_e4m3_codes((E, F, H), seed=4)
+    # weight scales ~ 1/(64 sqrt(H)) keep g and u of order one
+    sg = inputs.random_scales(E * F, seed=5, lo=0.5 / (64 * H ** 0.5), hi=2.0 / (64 * H ** 0.5)).reshape(E, F)
+    su = inputs.random_scales(E * F, seed=6, lo=0.5 / (64 * H ** 0.5), hi=2.0 / (64 * H ** 0.5)).reshape(E, F)
+    d = B.dims(T=rows, H=H, E=E, K=1, F=F, fp8_dispatch=True)
+    ws = B.make_workspace(d)
+    h = torch.zeros((rows, F), dtype=torch.bfloat16, device=DEV)
+    B.moe_grouped_gate_up_fp8(xq.to(DEV), xs.to(DEV), torch.from_numpy(off).to(DEV), wgq.to(DEV), wuq.to(DEV),
+                              sg.to(DEV), su.to(DEV), d, h, ws)
+    assert B.read_device_status(ws) == 0
+    wd = np.zeros((E, 8, F), np.uint16)      # h only: the down projection is the bf16 kernel
+    rh = np.zeros((rows, F), np.uint16)
+    for e in range(E):
+        lo, hi = int(off[e]), int(off[e + 1])
+        if hi > lo:
+            rh[lo:hi], _ = oracle.ffn_rows_fp8(xq.numpy()[lo:hi], xs.numpy()[lo:hi], wgq.numpy()[e], sg.numpy()[e],
+                                               wuq.numpy()[e], su.numpy()[e], wd[e])
+    check_bf16("h", bits(h), rh)
+
+
 def test_pack_gate_up_layout():
     # packed rows [128 j, 128 j + 64) = gate rows [64 j, +64), next 64 = up rows; padding rows zero
     E, H, F = 3, 16, 136
