@@ -404,25 +404,23 @@ def _weights_struct(w: dict) -> moe_layer_weights:
     return moe_layer_weights(*[(w[n].data_ptr() if w.get(n) is not None else None) for n in _W_FIELDS])
 
 
-# Packed gate/up weights (256 x 256 tiles, single-buffered accumulators) measured faster
-# than the separate-weight kernel in the layer only with a long reduction and prefill-sized
-# expert batches (H = 7168, 256 rows per expert: 5.0 vs 5.3 ms); slower at H = 2048 and for
-# decode (few rows per expert).  Pack when both hold.
-PACK_GATE_UP_MIN_H = 4096
-PACK_GATE_UP_MIN_ROWS_PER_EXPERT = 64
+# Packed gate/up weights (one 256-row box of interleaved gate/up rows per stage, with a
+# shared-memory exchange in the epilogue) measured slower than the separate-weight kernel
+# with 256-token tiles and eight epilogue warps on every workload (DeepSeek-R1-shaped
+# layer: 4.23 vs 3.81 ms), so layers use the separate weights unless asked otherwise.
+PACK_GATE_UP_BY_DEFAULT = False
 
 
 def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, w_upp=None, stream=None,
                        pack_gate_up_weights=None, shared=None) -> dict:
     """One-time weight preparation: router split into three bf16 planes and, when
-    ``pack_gate_up_weights`` (default: H >= PACK_GATE_UP_MIN_H), gate/up interleaved for the
+    ``pack_gate_up_weights`` (default: PACK_GATE_UP_BY_DEFAULT), gate/up interleaved for the
     packed gate/up GEMM.  With ``d.fp8_dispatch`` the gate and up weights are quantized to
     E4M3 per output feature instead."""
     if d.fp8_dispatch:
         pack_gate_up_weights = False
     if pack_gate_up_weights is None:
-        pack_gate_up_weights = (d.H >= PACK_GATE_UP_MIN_H and
-                                d.T * d.K >= PACK_GATE_UP_MIN_ROWS_PER_EXPERT * d.E)
+        pack_gate_up_weights = PACK_GATE_UP_BY_DEFAULT
     split = torch.empty((3, d.E, d.H), dtype=torch.bfloat16, device=w_g.device)
     moe_pack_router(w_g.contiguous(), d, split, stream)
     for name, t, n in (("w_gate", w_gate, d.E * d.F * d.H), ("w_up", w_up, d.E * d.F * d.H),

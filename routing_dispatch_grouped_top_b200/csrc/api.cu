@@ -25,8 +25,10 @@ int num_sms() {
 namespace {
 
 // Workspace: [0] status word, [64] grid-barrier count, [128] grid-barrier
-// generation, [256 ...) per-block expert histograms of the count/scan kernel.
+// generation, [160 + 16 s) the GEMM tile schedule of call site s (s < 6), [256 ...)
+// per-block expert histograms of the count/scan kernel.
 constexpr size_t kWsHeader = 256;
+enum SchedSlot : int { kSchedGating = 0, kSchedGateUp, kSchedDown, kSchedDense, kSchedSharedGateUp, kSchedSharedDown };
 
 bool device_ok() {
   static int cache[64] = {0};  // 0 unknown, 1 ok, -1 not sm_100
@@ -67,6 +69,7 @@ size_t ws_bytes_for(const moe_dims* d) {
 }
 
 int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
+int* ws_sched(void* ws, SchedSlot s) { return reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(ws) + 160 + 16 * s); }
 
 ScanWorkspace scan_ws(void* ws, const moe_dims* d) {
   uint8_t* p = reinterpret_cast<uint8_t*>(ws);
@@ -161,7 +164,8 @@ moe_status moe_gating(const void* x, const void* w_g_split, const float* bias, c
   if (d->T == 0) return MOE_OK;
   if (!x || !w_g_split || !logits) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_g_split)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(gemm_gating(x, w_g_split, bias, d->T, d->H, d->E, logits, ws_status(ws), as_stream(stream)));
+  return cuda_status(gemm_gating(x, w_g_split, bias, d->T, d->H, d->E, logits, ws_status(ws),
+                                 ws_sched(ws, kSchedGating), as_stream(stream)));
 }
 
 moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids, float* topk_w, void* stream) {
@@ -230,7 +234,7 @@ moe_status moe_grouped_gate_up_fp8(const void* xq, const float* xs, const int32_
   if (!aligned16(xq) || !aligned16(wq_gate) || !aligned16(wq_up)) return MOE_ERR_INVALID_ARG;
   return cuda_status(gemm_gate_up_fp8(xq, xs, offsets, wq_gate, wq_up, s_gate, s_up, d->E,
                                       d->T * static_cast<long long>(d->K), d->H, d->F, h, ws_status(ws),
-                                      as_stream(stream)));
+                                      ws_sched(ws, kSchedGateUp), as_stream(stream)));
 }
 
 moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up,
@@ -241,7 +245,7 @@ moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const voi
   if (!xp || !offsets || !w_gate || !w_up || !h) return MOE_ERR_INVALID_ARG;
   if (!aligned16(xp) || !aligned16(w_gate) || !aligned16(w_up)) return MOE_ERR_INVALID_ARG;
   return cuda_status(gemm_gate_up(xp, offsets, w_gate, w_up, d->E, d->T * static_cast<long long>(d->K), d->H,
-                                  d->F, h, ws_status(ws), as_stream(stream)));
+                                  d->F, h, ws_status(ws), ws_sched(ws, kSchedGateUp), as_stream(stream)));
 }
 
 size_t moe_packed_gate_up_bytes(const moe_dims* d) {
@@ -264,7 +268,7 @@ moe_status moe_grouped_gate_up_packed(const void* xp, const int32_t* offsets, co
   if (!xp || !offsets || !w_gu || !h) return MOE_ERR_INVALID_ARG;
   if (!aligned16(xp) || !aligned16(w_gu)) return MOE_ERR_INVALID_ARG;
   return cuda_status(gemm_gate_up_packed(xp, offsets, w_gu, d->E, d->T * static_cast<long long>(d->K), d->H, d->F,
-                                         h, ws_status(ws), as_stream(stream)));
+                                         h, ws_status(ws), ws_sched(ws, kSchedGateUp), as_stream(stream)));
 }
 
 moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w_down, const moe_dims* d, void* y,
@@ -275,7 +279,7 @@ moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w
   if (!h || !offsets || !w_down || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(h) || !aligned16(w_down)) return MOE_ERR_INVALID_ARG;
   return cuda_status(gemm_down(h, offsets, w_down, d->E, d->T * static_cast<long long>(d->K), d->H, d->F, y,
-                               ws_status(ws), as_stream(stream)));
+                               ws_status(ws), ws_sched(ws, kSchedDown), as_stream(stream)));
 }
 
 moe_status moe_grouped_ffn(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up,
@@ -316,7 +320,7 @@ moe_status moe_dense(const void* a, const void* w, int64_t M, int32_t N, int32_t
   if (ws_bytes < kWsHeader || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_WORKSPACE;
   if (!aligned16(a) || !aligned16(w)) return MOE_ERR_INVALID_ARG;
   if (M == 0) return MOE_OK;
-  return cuda_status(gemm_dense(a, w, M, N, Kd, out, ws_status(ws), as_stream(stream)));
+  return cuda_status(gemm_dense(a, w, M, N, Kd, out, ws_status(ws), ws_sched(ws, kSchedDense), as_stream(stream)));
 }
 
 moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const moe_dims* d,
@@ -350,7 +354,7 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   MOE_TRY(mark(0));
   const void* routed = x;
   if (latent) {
-    if (T > 0) MOE_CUDA(gemm_dense(x, w->w_dp, T, d->H, d->d_model, b->z, status, s));
+    if (T > 0) MOE_CUDA(gemm_dense(x, w->w_dp, T, d->H, d->d_model, b->z, status, ws_sched(ws, kSchedDense), s));
     routed = b->z;
   }
   MOE_TRY(mark(1));
@@ -363,11 +367,14 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
       MOE_CUDA(cudaStreamWaitEvent(sh, reinterpret_cast<cudaEvent_t>(b->fork_event), 0));
     }
     MOE_CUDA(gemm_gate_up(routed, nullptr, w->w_shared_gate, w->w_shared_up, 1, T, d->H, d->F_shared, b->h_shared,
-                          status, sh));
-    MOE_CUDA(gemm_down(b->h_shared, nullptr, w->w_shared_down, 1, T, d->H, d->F_shared, b->y_shared, status, sh));
+                          status, ws_sched(ws, kSchedSharedGateUp), sh));
+    MOE_CUDA(gemm_down(b->h_shared, nullptr, w->w_shared_down, 1, T, d->H, d->F_shared, b->y_shared, status,
+                       ws_sched(ws, kSchedSharedDown), sh));
     if (b->aux_stream) MOE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(b->join_event), sh));
   }
-  if (T > 0) MOE_CUDA(gemm_gating(routed, w->w_g_split, w->bias, T, d->H, d->E, b->logits, status, s));
+  if (T > 0)
+    MOE_CUDA(gemm_gating(routed, w->w_g_split, w->bias, T, d->H, d->E, b->logits, status, ws_sched(ws, kSchedGating),
+                         s));
   MOE_TRY(mark(2));
   MOE_CUDA(launch_route(b->logits, T, d->E, d->K, d->renormalize, d->P, d->group_limit, b->topk_ids, b->topk_w, s));
   MOE_TRY(mark(3));
@@ -384,21 +391,25 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   if (T > 0) {
     if (fp8)
       MOE_CUDA(gemm_gate_up_fp8(b->xq, b->xs, b->offsets, w->w_gate_q, w->w_up_q, w->s_gate, w->s_up, d->E, TK, d->H,
-                                d->F, b->h, status, s));
+                                d->F, b->h, status, ws_sched(ws, kSchedGateUp), s));
     else if (w->w_gate_up)
-      MOE_CUDA(gemm_gate_up_packed(b->xp, b->offsets, w->w_gate_up, d->E, TK, d->H, d->F, b->h, status, s));
+      MOE_CUDA(gemm_gate_up_packed(b->xp, b->offsets, w->w_gate_up, d->E, TK, d->H, d->F, b->h, status,
+                                   ws_sched(ws, kSchedGateUp), s));
     else
-      MOE_CUDA(gemm_gate_up(b->xp, b->offsets, w->w_gate, w->w_up, d->E, TK, d->H, d->F, b->h, status, s));
+      MOE_CUDA(gemm_gate_up(b->xp, b->offsets, w->w_gate, w->w_up, d->E, TK, d->H, d->F, b->h, status,
+                            ws_sched(ws, kSchedGateUp), s));
   }
   MOE_TRY(mark(6));
-  if (T > 0) MOE_CUDA(gemm_down(b->h, b->offsets, w->w_down, d->E, TK, d->H, d->F, b->y, status, s));
+  if (T > 0)
+    MOE_CUDA(gemm_down(b->h, b->offsets, w->w_down, d->E, TK, d->H, d->F, b->y, status, ws_sched(ws, kSchedDown), s));
   MOE_TRY(mark(7));
   if (shared && T > 0 && b->aux_stream)
     MOE_CUDA(cudaStreamWaitEvent(s, reinterpret_cast<cudaEvent_t>(b->join_event), 0));
   MOE_CUDA(launch_combine(b->y, b->row_of_assign, b->topk_w, shared ? b->y_shared : nullptr, T, d->H, d->K,
                           b->out, s));
   MOE_TRY(mark(8));
-  if (latent && T > 0) MOE_CUDA(gemm_dense(b->out, w->w_upp, T, d->d_model, d->H, b->final_out, status, s));
+  if (latent && T > 0)
+    MOE_CUDA(gemm_dense(b->out, w->w_upp, T, d->d_model, d->H, b->final_out, status, ws_sched(ws, kSchedDense), s));
   MOE_TRY(mark(9));
   return MOE_OK;
 }

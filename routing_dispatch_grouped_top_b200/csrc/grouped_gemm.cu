@@ -45,9 +45,11 @@ constexpr int kNumBoxes = 5;
 struct BoxMaps {
   CUtensorMap box[kNumBoxes];  // box[i] is (256 >> i) rows x 64 columns
 };
-constexpr int kThreads = 192;
+constexpr int kThreads = 192;            // CTA-pair kernel: producer, MMA and 4 epilogue warps
 constexpr int kEpiThreads = 128;
+constexpr int kMaxThreads = 320;         // single-CTA kernel with 8 epilogue warps
 constexpr int kMaxGroups = MOE_MAX_E;
+constexpr int kRing = 8;                 // tile ids in flight from the producer to the MMA and epilogue warps
 
 template <int EPI>
 struct Cfg;
@@ -64,9 +66,18 @@ struct Cfg;
 // single-buffered, which measured 15-30 % faster than 128 x 256 on every workload.  For
 // SwiGLU the same widening was slower (its epilogue is heavier and no longer overlapped),
 // so it keeps 128 x (128 gate + 128 up) tiles with double-buffered accumulators.
+// Build-time tuning: token columns of the separate-weight SwiGLU tiles (128: double-buffered
+// accumulators, 4 stages; 256: single-buffered, 3 stages) and epilogue warps (4 or 8: two
+// warps per TMEM lane quadrant split a tile's token chunks).
+#ifndef MOE_SWIGLU_NT
+#define MOE_SWIGLU_NT 256
+#endif
+#ifndef MOE_EPI_WARPS
+#define MOE_EPI_WARPS 8
+#endif
 template <>
 struct Cfg<kEpiSwiGLU> {
-  static constexpr int NA = 2, NT = 128, STAGES = 4, FEAT = 128;
+  static constexpr int NA = 2, NT = MOE_SWIGLU_NT, STAGES = NT == 256 ? 3 : 4, FEAT = 128, EW = MOE_EPI_WARPS;
   static constexpr bool SEP = true;
 };
 // SwiGLU on packed weights: one 256-row box holds two 128-row weight tiles, each
@@ -74,7 +85,7 @@ struct Cfg<kEpiSwiGLU> {
 // (lanes 0-63) and up (lanes 64-127) meet through a shared-memory swap in the epilogue.
 template <>
 struct Cfg<kEpiSwiGLUPacked> {
-  static constexpr int NA = 2, NT = 256, STAGES = 3, FEAT = 128;
+  static constexpr int NA = 2, NT = 256, STAGES = 3, FEAT = 128, EW = 4;
   static constexpr bool SEP = true;
 };
 // SwiGLU on E4M3 operands (FP8 dispatch): the same tile as the bf16 SwiGLU, each stage
@@ -82,25 +93,28 @@ struct Cfg<kEpiSwiGLUPacked> {
 // stage holds twice the MMA work.
 template <>
 struct Cfg<kEpiSwiGLUFp8> {
-  static constexpr int NA = 2, NT = 128, STAGES = 4, FEAT = 128;
+  static constexpr int NA = 2, NT = MOE_SWIGLU_NT, STAGES = NT == 256 ? 3 : 4, FEAT = 128, EW = MOE_EPI_WARPS;
   static constexpr bool SEP = true;
 };
 // Plain bf16 output (down projection, latent projections).
 template <>
 struct Cfg<kEpiBF16> {
-  static constexpr int NA = 2, NT = 256, STAGES = 3, FEAT = 256;
+  static constexpr int NA = 2, NT = 256, STAGES = 3, FEAT = 256, EW = MOE_EPI_WARPS;
   static constexpr bool SEP = true;
 };
 // fp32 output: three bf16 weight planes accumulated into one fp32 accumulator.
 template <>
 struct Cfg<kEpiF32> {
-  static constexpr int NA = 3, NT = 128, STAGES = 3, FEAT = 128;
+  static constexpr int NA = 3, NT = 128, STAGES = 3, FEAT = 128, EW = 4;
   static constexpr bool SEP = false;
 };
 
 template <int EPI>
 struct Layout {
   using C = Cfg<EPI>;
+  static constexpr int kThr = 64 + 32 * C::EW;  // producer warp, MMA warp, epilogue warps
+  static_assert(C::EW == 4 || C::EW == 8, "one or two epilogue warps per TMEM lane quadrant");
+  static_assert(kThr <= kMaxThreads, "block size");
   static constexpr int kBBytes = C::NT * 128;
   static constexpr int kStageBytes = C::NA * kABytes + kBBytes;
   static constexpr int kAccCols = C::SEP ? C::NA * C::NT : C::NT;
@@ -108,7 +122,9 @@ struct Layout {
   static constexpr uint32_t kTmemCols = kNumAcc * kAccCols;
   static constexpr int kExchFloats = 2 * 16 * 64;  // SwiGLU swap of one 32-token chunk, both directions
   static constexpr int kExchBytes = (EPI == kEpiSwiGLUPacked) ? 2 * kExchFloats * 4 : 0;  // double-buffered
-  static constexpr int kBarBytes = 8 * (2 * C::STAGES + 5) + 16;
+  // barriers: full/empty per stage, tmem full/empty x2, drain, tile ring full/empty; then the
+  // TMEM address, the abort flag and the ring's tile ids
+  static constexpr int kBarBytes = (8 * (2 * C::STAGES + 5 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
   static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
   static constexpr int kSmemBytes = 1024 + C::STAGES * kStageBytes + kExchBytes + kBarBytes + kTableBytes;
   static_assert(kTmemCols == 128 || kTmemCols == 256 || kTmemCols == 512, "TMEM allocation must be a power of two");
@@ -158,7 +174,8 @@ __device__ __forceinline__ Tile decode_tile(int t, const int* s_pre, const int* 
 // s_pre[g] = sum_{g' < g} ceil(cnt_g' / NT) * NFT for g = 0..G (block-wide scan).
 __device__ void build_tile_table(int* s_pre, const int* s_off, int G, int NT, int NFT, int* s_warp) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int seg = (G + kThreads - 1) / kThreads;
+  const int nthreads = blockDim.x;
+  const int seg = (G + nthreads - 1) / nthreads;
   const int b = min(G, tid * seg), e = min(G, b + seg);
   int local = 0;
   for (int g = b; g < e; ++g) local += ((s_off[g + 1] - s_off[g] + NT - 1) / NT) * NFT;
@@ -172,7 +189,7 @@ __device__ void build_tile_table(int* s_pre, const int* s_off, int G, int NT, in
   __syncthreads();
   if (tid == 0) {
     int run = 0;
-    for (int w = 0; w < kThreads / 32; ++w) {
+    for (int w = 0; w < nthreads / 32; ++w) {
       const int v = s_warp[w];
       s_warp[w] = run;
       run += v;
@@ -189,7 +206,7 @@ __device__ void build_tile_table(int* s_pre, const int* s_off, int G, int NT, in
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kMaxThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                         const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ BoxMaps tmB,
                         const GemmArgs args) {
@@ -206,12 +223,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* rfull = drain + 1;       // tile ring: the producer publishes each tile id it takes
+  uint64_t* rempty = rfull + kRing;  // released by the MMA thread and every epilogue warp
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rempty + kRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* ring_tile = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(smem + STAGES * L::kStageBytes + L::kExchBytes + L::kBarBytes);
   int* s_pre = s_off + (kMaxGroups + 1);
-  __shared__ int s_warp_sums[kThreads / 32];
+  __shared__ int s_warp_sums[kMaxThreads / 32];
   (void)exch;
+  constexpr int kEpiThr = 32 * C::EW;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = args.offsets ? args.G : 1;
@@ -229,9 +250,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], kEpiThreads);
+      mbar_init(&tempty[a], kEpiThr);
     }
     mbar_init(drain, 1);
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], 1 + C::EW);
+    }
     *abort_flag = 0;
     mbar_init_fence();
   }
@@ -247,18 +272,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   pdl_wait();  // offsets and the token operand come from earlier kernels
   pdl_launch_dependents();
   __syncthreads();
-  for (int i = threadIdx.x; i <= G; i += kThreads)
+  for (int i = threadIdx.x; i <= G; i += L::kThr)
     s_off[i] = args.offsets ? __ldg(args.offsets + i) : (i == 0 ? 0 : args.M);
   __syncthreads();
   // Offsets must be non-decreasing inside [0, M]; otherwise no tile runs.
-  for (int i = threadIdx.x; i <= G; i += kThreads) {
+  for (int i = threadIdx.x; i <= G; i += L::kThr) {
     const bool bad = s_off[i] < 0 || s_off[i] > args.M || (i > 0 && s_off[i] < s_off[i - 1]);
     if (bad) s_bad = 1;
   }
   __syncthreads();
   if (s_bad) {
     if (threadIdx.x == 0) report(args.status, MOE_DEV_BAD_INDEX);
-    for (int i = threadIdx.x; i <= G; i += kThreads) s_off[i] = 0;
+    for (int i = threadIdx.x; i <= G; i += L::kThr) s_off[i] = 0;
   }
   __syncthreads();
   build_tile_table(s_pre, s_off, G, NT, NFT, s_warp_sums);  // ends with __syncthreads
@@ -266,6 +291,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_pre[G];
 
+  static_assert(EPI != kEpiSwiGLUPacked || C::EW == 4, "the packed epilogue pairs warps q and q + 2");
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -275,7 +301,22 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) pend[s] = false, pend_phase[s] = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+      uint32_t rs = 0, rphase = 0;
+      for (;;) {
+        // Dynamic schedule: the next unclaimed tile of the launch (tiles differ in their token
+        // count, so a fixed round-robin leaves some SMs with much more work than others).
+        if (!mbar_wait(&rempty[rs], rphase ^ 1u, abort_flag, args.status)) {
+          ok = false;
+          break;
+        }
+        const int t = atomicAdd(&args.sched[0], 1);
+        ring_tile[rs] = t < total ? t : -1;
+        mbar_arrive(&rfull[rs]);
+        if (++rs == kRing) {
+          rs = 0;
+          rphase ^= 1u;
+        }
+        if (t >= total) break;
         const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
         const uint32_t bytes = NA * kABytes + tl.nround * 128;
         for (int kb = 0; kb < KB; ++kb) {
@@ -312,6 +353,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             phase ^= 1u;
           }
         }
+        if (!ok) break;
       }
       if (!ok) {  // let the copies already issued land before the CTA exits
 #pragma unroll
@@ -322,9 +364,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0, rs = 0, rphase = 0;
       bool ok = true;
-      for (int t = blockIdx.x; ok && t < total; t += gridDim.x) {
+      for (;;) {
+        if (!mbar_wait(&rfull[rs], rphase, abort_flag, args.status)) {
+          ok = false;
+          break;
+        }
+        const int t = ring_tile[rs];
+        mbar_arrive(&rempty[rs]);
+        if (++rs == kRing) {
+          rs = 0;
+          rphase ^= 1u;
+        }
+        if (t < 0) break;
         const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) {
           ok = false;
@@ -376,8 +429,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;  // TMEM lanes [32q, 32q + 32) are visible to this warp
-    uint32_t acc = 0, acc_phase = 0, chunk = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
+    // With 8 epilogue warps, two share each lane quadrant and take alternate 32-token chunks.
+    constexpr int kSplit = C::EW / 4;
+    const int part = (warp - 2) >> 2;
+    uint32_t acc = 0, acc_phase = 0, chunk = 0, rs = 0, rphase = 0;
+    for (;;) {
+      if (!mbar_wait(&rfull[rs], rphase, abort_flag, args.status)) break;
+      const int t = ring_tile[rs];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&rempty[rs]);
+      if (++rs == kRing) {
+        rs = 0;
+        rphase ^= 1u;
+      }
+      if (t < 0) break;
       const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
@@ -405,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (is_gate) to_up[j * 64 + fi] = __uint_as_float(r[16 + j]);
               else to_gate[j * 64 + fi] = __uint_as_float(r[j]);
             }
-            named_bar_sync(1, kEpiThreads);
+            named_bar_sync(1, kEpiThr);
             if (f < args.N) {
               const long long row0 = static_cast<long long>(tl.row0) + j0 + jbase;
 #pragma unroll
@@ -430,7 +495,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int f = tl.n0 + q * 32 + lane;
       const bool f_ok = f < args.N;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
-      float sg = 1.0f, su = 1.0f;  // FP8: per-feature weight scales of this thread's output feature
+      float sg = 1.0f, su = 1.0f;
+      (void)part;  // FP8: per-feature weight scales of this thread's output feature
       if constexpr (EPI == kEpiSwiGLUFp8) {
         if (f_ok) {
           const long long fi = static_cast<long long>(tl.g) * args.N + f;
@@ -438,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           su = __ldg(args.scale_a1 + fi);
         }
       }
-      for (int j0 = 0; j0 < tl.nvalid; j0 += 32) {
+      for (int j0 = 32 * part; j0 < tl.nvalid; j0 += 32 * kSplit) {
         uint32_t r0[32];
         tmem_ld_32cols(tbase + j0, r0);
         const int jn = min(32, tl.nvalid - j0);
@@ -506,6 +572,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc(tmem_base, L::kTmemCols);
+  }
+  // The last CTA to finish rewinds the schedule for the next launch on this slot (every CTA
+  // has claimed its last tile before it counts itself done).
+  if (threadIdx.x == 0) {
+    __threadfence();
+    if (atomicAdd(&args.sched[1], 1) == static_cast<int>(gridDim.x) - 1) {
+      atomicExch(&args.sched[0], 0);
+      atomicExch(&args.sched[1], 0);
+    }
   }
 }
 
@@ -863,7 +938,7 @@ cudaError_t launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   if (attr_err != cudaSuccess) return attr_err;
   if (tile_bound <= 0) return cudaSuccess;
   const int grid = static_cast<int>(std::min<long long>(num_sms(), tile_bound));
-  return launch_pdl(grouped_gemm_kernel<EPI>, dim3(grid), dim3(kThreads), L::kSmemBytes, stream, a0, a1, a2, b, args);
+  return launch_pdl(grouped_gemm_kernel<EPI>, dim3(grid), dim3(L::kThr), L::kSmemBytes, stream, a0, a1, a2, b, args);
 }
 
 template <int EPI>
@@ -909,8 +984,8 @@ int gemm_smem_bytes(int epi) {
 
 // h = silu(xp Wg^T) * (xp Wu^T) per expert group.
 cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
-                         long long rows, int H, int F, void* h, int* status, cudaStream_t stream) {
-  GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status};
+                         long long rows, int H, int F, void* h, int* status, int* sched, cudaStream_t stream) {
+  GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status, nullptr, nullptr, nullptr, sched};
   CUtensorMap a0, a1;
   BoxMaps b;
   if (!map_token_boxes(&b, xp, H, rows)) return cudaErrorInvalidValue;
@@ -926,8 +1001,8 @@ long long packed_gate_up_rows(int F) { return 2LL * ((F + 63) / 64 * 64); }
 
 // Same result as gemm_gate_up, from weights packed by launch_pack_gate_up.
 cudaError_t gemm_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, int E, long long rows,
-                                int H, int F, void* h, int* status, cudaStream_t stream) {
-  GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status};
+                                int H, int F, void* h, int* status, int* sched, cudaStream_t stream) {
+  GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status, nullptr, nullptr, nullptr, sched};
   CUtensorMap a0;
   BoxMaps b;
   if (!map_bf16_3d(&a0, w_gu, H, static_cast<uint64_t>(packed_gate_up_rows(F)), E, 256) ||
@@ -942,8 +1017,8 @@ cudaError_t gemm_gate_up_packed(const void* xp, const int32_t* offsets, const vo
 // scales in the epilogue (both factor out of the K sum), h is bf16 as in gemm_gate_up.
 cudaError_t gemm_gate_up_fp8(const void* xq, const float* xs, const int32_t* offsets, const void* wq_gate,
                              const void* wq_up, const float* s_gate, const float* s_up, int E, long long rows, int H,
-                             int F, void* h, int* status, cudaStream_t stream) {
-  GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status, s_gate, s_up, xs};
+                             int F, void* h, int* status, int* sched, cudaStream_t stream) {
+  GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status, s_gate, s_up, xs, sched};
   CUtensorMap a0, a1;
   BoxMaps b;
   if (!map_token_boxes(&b, xq, H, rows, 1) || !map_bf16_3d(&a0, wq_gate, H, F, E, kBM, 1) ||
@@ -955,8 +1030,8 @@ cudaError_t gemm_gate_up_fp8(const void* xq, const float* xs, const int32_t* off
 
 // y = h Wd^T per expert group.
 cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down, int E, long long rows, int H,
-                      int F, void* y, int* status, cudaStream_t stream) {
-  GemmArgs args{offsets, E, static_cast<int>(rows), H, F, y, H, nullptr, status};
+                      int F, void* y, int* status, int* sched, cudaStream_t stream) {
+  GemmArgs args{offsets, E, static_cast<int>(rows), H, F, y, H, nullptr, status, nullptr, nullptr, nullptr, sched};
   CUtensorMap a0;
   BoxMaps b;
   if (!map_bf16_3d(&a0, w_down, F, H, E, MOE_GEMM_PAIR ? kBM : 256) || !map_token_boxes(&b, h, F, rows))
@@ -968,12 +1043,12 @@ cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down,
 
 // out[M][N] = a[M][Kd] w[N][Kd]^T, bf16 out.
 cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd, void* out, int* status,
-                       cudaStream_t stream) {
+                       int* sched, cudaStream_t stream) {
   CUtensorMap a0;
   BoxMaps b;
   if (!map_bf16_3d(&a0, w, Kd, N, 1, MOE_GEMM_PAIR ? kBM : 256) || !map_token_boxes(&b, a, Kd, M))
     return cudaErrorInvalidValue;
-  GemmArgs args{nullptr, 1, static_cast<int>(M), N, Kd, out, N, nullptr, status};
+  GemmArgs args{nullptr, 1, static_cast<int>(M), N, Kd, out, N, nullptr, status, nullptr, nullptr, nullptr, sched};
   if (MOE_GEMM_PAIR)
     return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(M, 1, PairLayout<kEpiBF16>::NT, N, 256), stream);
   return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(M, 1, Cfg<kEpiBF16>::NT, N, Cfg<kEpiBF16>::FEAT), stream);
@@ -981,11 +1056,11 @@ cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd,
 
 // logits[T][E] = x[T][H] (hi + mid + lo)^T (+ bias), fp32 out; w_split is [3][E][H] bf16.
 cudaError_t gemm_gating(const void* x, const void* w_split, const float* bias, long long T, int H, int E,
-                        float* logits, int* status, cudaStream_t stream) {
+                        float* logits, int* status, int* sched, cudaStream_t stream) {
   CUtensorMap a0;
   BoxMaps b;
   if (!map_bf16_3d(&a0, w_split, H, E, 3, kBM) || !map_token_boxes(&b, x, H, T)) return cudaErrorInvalidValue;
-  GemmArgs args{nullptr, 1, static_cast<int>(T), E, H, logits, E, bias, status};
+  GemmArgs args{nullptr, 1, static_cast<int>(T), E, H, logits, E, bias, status, nullptr, nullptr, nullptr, sched};
   return launch<kEpiF32>(a0, a0, a0, b, args, tile_bound(T, 1, Cfg<kEpiF32>::NT, E, kBM), stream);
 }
 

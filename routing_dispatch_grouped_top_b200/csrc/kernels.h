@@ -21,6 +21,7 @@ struct GemmArgs {
   const float* scale_a0;   // kEpiSwiGLUFp8: per-feature scales of the gate weights [G][N]
   const float* scale_a1;   //                per-feature scales of the up weights [G][N]
   const float* scale_b;    //                per-row scales of the token operand [M]
+  int* sched;              // two device ints {next tile, finished CTAs}, zero between launches
 };
 
 int num_sms();             // SM count of the current device (cached per device)
@@ -45,23 +46,23 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 int gemm_smem_bytes(int epi);
 
 cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
-                         long long rows, int H, int F, void* h, int* status, cudaStream_t stream);
+                         long long rows, int H, int F, void* h, int* status, int* sched, cudaStream_t stream);
 // Gate and up weights interleaved in 64-row blocks ([E][2 Fp][H], Fp = F rounded up to 64).
 long long packed_gate_up_rows(int F);
 cudaError_t launch_pack_gate_up(const void* w_gate, const void* w_up, int E, int H, int F, void* w_gu,
                                 cudaStream_t stream);
 cudaError_t gemm_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, int E, long long rows,
-                                int H, int F, void* h, int* status, cudaStream_t stream);
+                                int H, int F, void* h, int* status, int* sched, cudaStream_t stream);
 // h = silu(s_x s_g (xq Wg_q^T)) * (s_x s_u (xq Wu_q^T)) on E4M3 operands.
 cudaError_t gemm_gate_up_fp8(const void* xq, const float* xs, const int32_t* offsets, const void* wq_gate,
                              const void* wq_up, const float* s_gate, const float* s_up, int E, long long rows, int H,
-                             int F, void* h, int* status, cudaStream_t stream);
+                             int F, void* h, int* status, int* sched, cudaStream_t stream);
 cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down, int E, long long rows, int H,
-                      int F, void* y, int* status, cudaStream_t stream);
+                      int F, void* y, int* status, int* sched, cudaStream_t stream);
 cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd, void* out, int* status,
-                       cudaStream_t stream);
+                       int* sched, cudaStream_t stream);
 cudaError_t gemm_gating(const void* x, const void* w_split, const float* bias, long long T, int H, int E,
-                        float* logits, int* status, cudaStream_t stream);
+                        float* logits, int* status, int* sched, cudaStream_t stream);
 
 cudaError_t launch_route(const float* logits, long long T, int E, int K, int renormalize, int P, int group_limit,
                          int32_t* ids, float* w, cudaStream_t stream);
