@@ -21,7 +21,9 @@
  *
  * Conventions for every call:
  *  - Pointers are DEVICE pointers unless the name ends in _host.  bf16 data is
- *    passed as raw IEEE bfloat16 (void*), row-major, densely packed.
+ *    passed as raw IEEE bfloat16 (void*), row-major, densely packed.  Activation,
+ *    weight and output matrices (bf16 or E4M3 rows) must start on a 16-byte boundary:
+ *    the kernels move them in 16-byte pieces (MOE_ERR_INVALID_ARG otherwise).
  *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call only
  *    enqueues work and returns; none synchronizes with the host except
  *    moe_read_device_status.

@@ -231,7 +231,7 @@ moe_status moe_grouped_gate_up_fp8(const void* xq, const float* xs, const int32_
   if (d->H % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (d->T == 0) return MOE_OK;
   if (!xq || !xs || !offsets || !wq_gate || !wq_up || !s_gate || !s_up || !h) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(xq) || !aligned16(wq_gate) || !aligned16(wq_up)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(wq_gate) || !aligned16(wq_up) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
   return cuda_status(gemm_gate_up_fp8(xq, xs, offsets, wq_gate, wq_up, s_gate, s_up, d->E,
                                       d->T * static_cast<long long>(d->K), d->H, d->F, h, ws_status(ws),
                                       ws_sched(ws, kSchedGateUp), as_stream(stream)));
@@ -243,7 +243,7 @@ moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const voi
   MOE_TRY(check_ws(ws, ws_bytes, d));
   if (d->T == 0) return MOE_OK;
   if (!xp || !offsets || !w_gate || !w_up || !h) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(xp) || !aligned16(w_gate) || !aligned16(w_up)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xp) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
   return cuda_status(gemm_gate_up(xp, offsets, w_gate, w_up, d->E, d->T * static_cast<long long>(d->K), d->H,
                                   d->F, h, ws_status(ws), ws_sched(ws, kSchedGateUp), as_stream(stream)));
 }
@@ -266,7 +266,7 @@ moe_status moe_grouped_gate_up_packed(const void* xp, const int32_t* offsets, co
   MOE_TRY(check_ws(ws, ws_bytes, d));
   if (d->T == 0) return MOE_OK;
   if (!xp || !offsets || !w_gu || !h) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(xp) || !aligned16(w_gu)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(xp) || !aligned16(w_gu) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
   return cuda_status(gemm_gate_up_packed(xp, offsets, w_gu, d->E, d->T * static_cast<long long>(d->K), d->H, d->F,
                                          h, ws_status(ws), ws_sched(ws, kSchedGateUp), as_stream(stream)));
 }
@@ -277,7 +277,7 @@ moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w
   MOE_TRY(check_ws(ws, ws_bytes, d));
   if (d->T == 0) return MOE_OK;
   if (!h || !offsets || !w_down || !y) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(h) || !aligned16(w_down)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h) || !aligned16(w_down) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
   return cuda_status(gemm_down(h, offsets, w_down, d->E, d->T * static_cast<long long>(d->K), d->H, d->F, y,
                                ws_status(ws), ws_sched(ws, kSchedDown), as_stream(stream)));
 }
@@ -318,7 +318,7 @@ moe_status moe_dense(const void* a, const void* w, int64_t M, int32_t N, int32_t
   if (!a || !w || !out || !ws || M < 0 || N < 8 || Kd < 8) return MOE_ERR_INVALID_ARG;
   if (N % 8 != 0 || Kd % 8 != 0 || M > 0x7fffffffLL) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (ws_bytes < kWsHeader || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_WORKSPACE;
-  if (!aligned16(a) || !aligned16(w)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(a) || !aligned16(w) || !aligned16(out)) return MOE_ERR_INVALID_ARG;
   if (M == 0) return MOE_OK;
   return cuda_status(gemm_dense(a, w, M, N, Kd, out, ws_status(ws), ws_sched(ws, kSchedDense), as_stream(stream)));
 }
@@ -343,6 +343,12 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   if (!b->logits || !b->topk_ids || !b->topk_w || !b->counts || !b->offsets || !b->part_counts ||
       !b->part_offsets || !b->row_of_assign || !b->assign_of_row || (!fp8 && !b->xp) || !b->h || !b->y || !b->out)
     return MOE_ERR_INVALID_ARG;
+  // every bf16 row buffer is read or written in 16-byte pieces
+  for (const void* p : {x, static_cast<const void*>(b->xp), static_cast<const void*>(b->h), static_cast<const void*>(b->y),
+                        static_cast<const void*>(b->out), static_cast<const void*>(b->z),
+                        static_cast<const void*>(b->final_out), static_cast<const void*>(b->h_shared),
+                        static_cast<const void*>(b->y_shared)})
+    if (p && !aligned16(p)) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
   auto mark = [&](int i) -> moe_status {
     if (stage_events && stage_events[i])

@@ -121,7 +121,9 @@ struct Layout {
   static constexpr int kNumAcc = (2 * kAccCols <= 512) ? 2 : 1;
   static constexpr uint32_t kTmemCols = kNumAcc * kAccCols;
   static constexpr int kExchFloats = 2 * 16 * 64;  // SwiGLU swap of one 32-token chunk, both directions
-  static constexpr int kExchBytes = (EPI == kEpiSwiGLUPacked) ? 2 * kExchFloats * 4 : 0;  // double-buffered
+  static constexpr int kExchBytes = (EPI == kEpiSwiGLUPacked) ? 2 * kExchFloats * 4  // double-buffered
+                                    // bf16 outputs: one 32 x 32 transpose tile per epilogue warp
+                                    : (EPI == kEpiF32 ? 0 : C::EW * 32 * 32 * 2);
   // barriers: full/empty per stage, tmem full/empty x2, drain, tile ring full/empty; then the
   // TMEM address, the abort flag and the ring's tile ids
   static constexpr int kBarBytes = (8 * (2 * C::STAGES + 5 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
@@ -495,6 +497,26 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       const int f = tl.n0 + q * 32 + lane;
       const bool f_ok = f < args.N;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
+      // bf16 outputs leave through a per-warp 32 x 32 transpose in shared memory: the thread
+      // of feature f holds 32 tokens, a token row needs 32 consecutive features, so each
+      // lane then writes whole 16-byte pieces of rows (four per 32-token chunk) instead of
+      // 32 scattered 2-byte values.
+      __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(exch) + (warp - 2) * 32 * 32;
+      __nv_bfloat16* outb = reinterpret_cast<__nv_bfloat16*>(args.out);
+      auto store_rows = [&](const float (&v)[32], int fbase, long long row0, int jn) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) stg[j * 32 + lane] = __float2bfloat16_rn(v[j]);
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = 8 * i + (lane >> 2), c = 8 * (lane & 3);
+          if (j < jn && fbase + c < args.N)
+            *reinterpret_cast<uint4*>(outb + (row0 + j) * args.ldo + fbase + c) =
+                *reinterpret_cast<const uint4*>(stg + j * 32 + c);
+        }
+        __syncwarp();
+      };
+      (void)store_rows;
       float sg = 1.0f, su = 1.0f;
       (void)part;  // FP8: per-feature weight scales of this thread's output feature
       if constexpr (EPI == kEpiSwiGLUFp8) {
@@ -512,40 +534,34 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         if constexpr (EPI == kEpiSwiGLU || EPI == kEpiSwiGLUFp8) {
           uint32_t r1[32];
           tmem_ld_32cols(tbase + NT + j0, r1);
+          float sx = 1.0f;  // FP8: row scale of token j0 + lane, handed to the other lanes below
+          if constexpr (EPI == kEpiSwiGLUFp8) sx = lane < jn ? __ldg(args.scale_b + row0 + lane) : 0.0f;
           tmem_wait_ld();
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.out);
-          if (f_ok) {
+          float h[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              if (j < jn) {
-                float g = __uint_as_float(r0[j]), u = __uint_as_float(r1[j]);
-                if constexpr (EPI == kEpiSwiGLUFp8) {
-                  const float sx = __ldg(args.scale_b + row0 + j);  // same address in every lane
-                  g *= sx * sg;
-                  u *= sx * su;
-                }
-                out[(row0 + j) * args.ldo + f] = __float2bfloat16_rn(silu_mul(g, u));
-              }
+          for (int j = 0; j < 32; ++j) {
+            float g = __uint_as_float(r0[j]), u = __uint_as_float(r1[j]);
+            if constexpr (EPI == kEpiSwiGLUFp8) {
+              const float sj = __shfl_sync(0xffffffffu, sx, j);
+              g *= sj * sg;
+              u *= sj * su;
             }
+            h[j] = silu_mul(g, u);
           }
+          store_rows(h, tl.n0 + q * 32, row0, jn);
         } else if constexpr (EPI == kEpiBF16) {
           tmem_wait_ld();
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.out);
-          if (f_ok) {
+          float v[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < jn) out[(row0 + j) * args.ldo + f] = __float2bfloat16_rn(__uint_as_float(r0[j]));
-          }
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
+          store_rows(v, tl.n0 + q * 32, row0, jn);
           if constexpr (C::SEP) {  // wide tile: second accumulator = features n0 + 128 ..
             uint32_t r1[32];
             tmem_ld_32cols(tbase + NT + j0, r1);
             tmem_wait_ld();
-            const int f1 = f + kBM;
-            if (f1 < args.N) {
 #pragma unroll
-              for (int j = 0; j < 32; ++j)
-                if (j < jn) out[(row0 + j) * args.ldo + f1] = __float2bfloat16_rn(__uint_as_float(r1[j]));
-            }
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r1[j]);
+            store_rows(v, tl.n0 + kBM + q * 32, row0, jn);
           }
         } else {
           tmem_wait_ld();
