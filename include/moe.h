@@ -253,6 +253,13 @@ moe_status moe_grouped_gate_up_packed(const void* xp, const int32_t* offsets, co
                                       const moe_dims* d, void* h, void* ws, size_t ws_bytes,
                                       void* stream);
 
+/* Process-wide tuning of the grouped GEMMs (not part of the method): groups with at least
+ * `rows` rows on average (default 64) run on the CTA-pair kernel, in which the two SMs of a
+ * cluster share each token tile (tcgen05 cta_group::2); smaller groups, and every call when
+ * `rows` < 0, run on the single-CTA kernel.  Both give the same results up to fp32
+ * accumulation order.  Takes effect for launches enqueued after the call. */
+void moe_set_pair_min_rows(int32_t rows);
+
 /* The two halves of moe_grouped_ffn as separate launches (S4 and S5). */
 moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const void* w_gate,
                                const void* w_up, const moe_dims* d, void* h, void* ws,

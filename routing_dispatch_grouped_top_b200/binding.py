@@ -73,6 +73,7 @@ _SIGS = {
     "moe_packed_gate_up_bytes": (_SZ, [_DP]),
     "moe_pack_gate_up": (C.c_int, [_VP, _VP, _DP, _VP, _VP]),
     "moe_grouped_gate_up_packed": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
+    "moe_set_pair_min_rows": (None, [_I32]),
     "moe_quantize_fp8_rows": (C.c_int, [_VP, _I64, _I32, _VP, _VP, _VP]),
     "moe_permute_fp8": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_grouped_gate_up_fp8": (C.c_int, [_VP, _VP, _VP, _VP, _VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
@@ -229,6 +230,11 @@ def moe_permute(x, row_of_assign, topk_ids, topk_w, d: moe_dims, xp, meta_token=
         _ptr(xp, torch.bfloat16, "xp", TK * d.H), _ptr(meta_token, torch.int32, "meta_token", TK),
         _ptr(meta_slot, torch.int32, "meta_slot", TK), _ptr(meta_w, torch.float32, "meta_w", TK),
         _ptr(meta_local_expert, torch.int32, "meta_local_expert", TK), _stream(stream)))
+
+
+def set_pair_min_rows(rows: int):
+    """Average rows per group from which the grouped GEMMs use the CTA-pair kernel (< 0: never)."""
+    lib().moe_set_pair_min_rows(int(rows))
 
 
 def moe_quantize_fp8_rows(x, q, scales, stream=None):

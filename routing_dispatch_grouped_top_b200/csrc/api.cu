@@ -201,6 +201,8 @@ moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_
                                     meta_token, meta_slot, meta_w, meta_local_expert, as_stream(stream)));
 }
 
+void moe_set_pair_min_rows(int32_t rows) { set_pair_min_rows(rows); }
+
 moe_status moe_quantize_fp8_rows(const void* x, int64_t rows, int32_t cols, void* q, float* scales, void* stream) {
   if (rows < 0 || cols < 16) return MOE_ERR_INVALID_ARG;
   if (cols % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;

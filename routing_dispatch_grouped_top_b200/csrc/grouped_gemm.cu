@@ -27,6 +27,7 @@
 // then token chunk: CTAs working at the same time share weight and token tiles
 // through L2, so each expert's weights cross HBM about once.
 #include <algorithm>
+#include <atomic>
 #include <mutex>
 
 #include "device.cuh"
@@ -97,9 +98,12 @@ struct Cfg<kEpiSwiGLUFp8> {
   static constexpr bool SEP = true;
 };
 // Plain bf16 output (down projection, latent projections).
+#ifndef MOE_BF16_NT
+#define MOE_BF16_NT 256
+#endif
 template <>
 struct Cfg<kEpiBF16> {
-  static constexpr int NA = 2, NT = 256, STAGES = 3, FEAT = 256, EW = MOE_EPI_WARPS;
+  static constexpr int NA = 2, NT = MOE_BF16_NT, STAGES = NT == 256 ? 3 : 4, FEAT = 256, EW = MOE_EPI_WARPS;
   static constexpr bool SEP = true;
 };
 // fp32 output: three bf16 weight planes accumulated into one fp32 accumulator.
@@ -146,6 +150,25 @@ constexpr int stage_k() {
 // silu(g) * u = g u / (1 + e^-g) with the fast exponential and divide (2 MUFU ops):
 // for g -> -inf the denominator overflows and the result is 0, for g -> +inf it is g u.
 __device__ __forceinline__ float silu_mul(float g, float u) { return __fdividef(g * u, 1.0f + __expf(-g)); }
+
+// bf16 outputs leave through a per-warp 32 x 32 transpose in shared memory: the thread of
+// feature fbase + lane holds v[j] for tokens row0 + j, a token row wants 32 consecutive
+// features, so each lane then writes whole 16-byte pieces of rows (four per 32-token chunk)
+// instead of 32 scattered 2-byte values.  Rows j >= jn and features >= N are not written.
+__device__ __forceinline__ void store_rows32(__nv_bfloat16* stg, int lane, const float (&v)[32],
+                                             __nv_bfloat16* out, long long ldo, int N, int fbase, long long row0,
+                                             int jn) {
+#pragma unroll
+  for (int j = 0; j < 32; ++j) stg[j * 32 + lane] = __float2bfloat16_rn(v[j]);
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = 8 * i + (lane >> 2), c = 8 * (lane & 3);
+    if (j < jn && fbase + c < N)
+      *reinterpret_cast<uint4*>(out + (row0 + j) * ldo + fbase + c) = *reinterpret_cast<const uint4*>(stg + j * 32 + c);
+  }
+  __syncwarp();
+}
 
 // Tile t -> (group, weight tile, token chunk).  s_pre[g] = first tile of group g.  A group of
 // cnt rows is cut into ceil(cnt / NT) balanced chunks of a multiple of ROUND rows; a weight
@@ -497,24 +520,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       const int f = tl.n0 + q * 32 + lane;
       const bool f_ok = f < args.N;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
-      // bf16 outputs leave through a per-warp 32 x 32 transpose in shared memory: the thread
-      // of feature f holds 32 tokens, a token row needs 32 consecutive features, so each
-      // lane then writes whole 16-byte pieces of rows (four per 32-token chunk) instead of
-      // 32 scattered 2-byte values.
-      __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(exch) + (warp - 2) * 32 * 32;
+      __nv_bfloat16* stg = reinterpret_cast<__nv_bfloat16*>(exch) + (warp - 2) * 32 * 32;  // transpose tile
       __nv_bfloat16* outb = reinterpret_cast<__nv_bfloat16*>(args.out);
       auto store_rows = [&](const float (&v)[32], int fbase, long long row0, int jn) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) stg[j * 32 + lane] = __float2bfloat16_rn(v[j]);
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int j = 8 * i + (lane >> 2), c = 8 * (lane & 3);
-          if (j < jn && fbase + c < args.N)
-            *reinterpret_cast<uint4*>(outb + (row0 + j) * args.ldo + fbase + c) =
-                *reinterpret_cast<const uint4*>(stg + j * 32 + c);
-        }
-        __syncwarp();
+        store_rows32(stg, lane, v, outb, args.ldo, args.N, fbase, row0, jn);
       };
       (void)store_rows;
       float sg = 1.0f, su = 1.0f;
@@ -601,125 +610,166 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 }
 
 // ---------------------------------------------------------------------------
-// CTA-pair kernel (cta_group::2): one M = 256 x N (<= 256) MMA per K-step spans the
-// two SMs of a cluster.  Each CTA stages its own 128 weight rows and N/2 token rows
-// (32 KB per stage, 6 stages), so shared-memory traffic per MMA cycle is two thirds of
-// the single-CTA tiles'; the token tile crosses L2 once per pair.  The leader CTA
-// (rank 0) issues the MMAs; both CTAs' TMA loads complete on the leader's "full"
-// barrier, the leader's commits release both CTAs' "empty" and "tmem full" barriers,
-// and both CTAs' epilogues release the leader's "tmem empty" barrier.
-//   SwiGLU: CTA r holds gate rows [f0 + 64 r, +64) over up rows of the same features,
-//           so TMEM lanes 0-63 are gate and 64-127 up; the epilogue warps swap halves of
-//           each 32-token chunk through shared memory (warp q and q + 2 own the gate and
-//           up of the same features).  128 output features per pair tile.
-//   bf16:   CTA r holds weight rows [n0 + 128 r, +128).  256 output features per pair tile.
+// CTA-pair kernel (cta_group::2).  The two SMs of a cluster share one tile of 256 (SwiGLU)
+// or 512 (bf16) output features x N <= 256 tokens.  Each CTA stages its own 128 rows of
+// each of the two weight operands and half of the token rows; the pair MMA (M = 256,
+// issued by the leader, rank 0) reads both token halves, so a token tile crosses L2 once
+// per pair and each SM fills 48 KB of shared memory per K-step instead of the single-CTA
+// tile's 64 KB for the same MMA work per SM.
+//   SwiGLU: CTA r holds gate and up rows [n0 + 128 r, +128): gate and up accumulate in
+//           separate TMEM columns of the same lanes, so no exchange between warps.
+//   bf16:   CTA r holds rows [n0 + 128 r, +128) and [n0 + 256 + 128 r, +128).
+// Both CTAs' TMA loads of a stage complete on the leader's "full" barrier; the leader's
+// commits release both CTAs' "empty" and "tmem full" barriers; both CTAs' epilogue warps
+// release the leader's "tmem empty" barrier.  The leader's producer claims tiles from the
+// launch's counter and publishes each id to both CTAs through a ring in shared memory (the
+// peer's slot written over the cluster), which both CTAs' consumers release.
 // ---------------------------------------------------------------------------
-
 template <int EPI>
 struct PairLayout {
-  static constexpr int NT = 256;                      // token columns per tile (MMA N)
-  static constexpr int STAGES = 6;
-  static constexpr int kFeat = (EPI == kEpiSwiGLU) ? 128 : 256;
-  static constexpr int kABytes = 128 * kBK * 2;       // this CTA's 128 weight rows
-  static constexpr int kBBytes = (NT / 2) * 128;      // this CTA's token rows
-  static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr uint32_t kAccCols = NT;
-  static constexpr uint32_t kTmemCols = 2 * kAccCols;
-  static constexpr int kExchFloats = 2 * 16 * 64;     // one chunk: 16 tokens x 64 features, each direction
-  static constexpr int kExchBytes = (EPI == kEpiSwiGLU) ? 2 * kExchFloats * 4 : 0;  // double-buffered
-  static constexpr int kBarBytes = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int NT = 256;                                // tokens per pair tile (MMA N)
+  static constexpr int STAGES = 4;
+  static constexpr int EW = 8;                                  // epilogue warps per CTA
+  static constexpr int kThr = 64 + 32 * EW;
+  static constexpr int FEAT = (EPI == kEpiBF16) ? 512 : 256;    // output features per pair tile
+  static constexpr int kAPair = 2 * kABytes;                    // this CTA's two 128-row weight boxes
+  static constexpr int kBBytes = (NT / 2) * 128;                // this CTA's token rows
+  static constexpr int kStageBytes = kAPair + kBBytes;
+  static constexpr uint32_t kTmemCols = 2 * NT;                 // two accumulators, single-buffered
+  static constexpr int kStgBytes = EW * 32 * 32 * 2;
+  static constexpr int kBarBytes = (8 * (2 * STAGES + 3 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
   static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
-  static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kExchBytes + kBarBytes + kTableBytes;
+  static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kStgBytes + kBarBytes + kTableBytes;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
+  static_assert(kThr <= kMaxThreads, "block size");
 };
 
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                      const __grid_constant__ BoxMaps tmB, const GemmArgs args) {
   using L = PairLayout<EPI>;
-  constexpr int NT = L::NT, STAGES = L::STAGES;
+  constexpr int NT = L::NT, STAGES = L::STAGES, EW = L::EW;
+  constexpr int KS = stage_k<EPI>();
+  static_assert(EPI == kEpiSwiGLU || EPI == kEpiSwiGLUFp8 || EPI == kEpiBF16, "pair epilogues");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
-  float* exch = reinterpret_cast<float*>(smem + STAGES * L::kStageBytes);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::kStageBytes + L::kExchBytes);
+  __nv_bfloat16* stg_all = reinterpret_cast<__nv_bfloat16*>(smem + STAGES * L::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::kStageBytes + L::kStgBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* tempty = tfull + 1;
+  uint64_t* drain = tempty + 1;
+  uint64_t* rfull = drain + 1;
+  uint64_t* rempty = rfull + kRing;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rempty + kRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  int* s_off = reinterpret_cast<int*>(smem + STAGES * L::kStageBytes + L::kExchBytes + L::kBarBytes);
+  volatile int* ring_tile = reinterpret_cast<volatile int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(smem + STAGES * L::kStageBytes + L::kStgBytes + L::kBarBytes);
   int* s_pre = s_off + (kMaxGroups + 1);
-  __shared__ int s_warp_sums[kThreads / 32];
+  __shared__ int s_warp_sums[kMaxThreads / 32];
   __shared__ int s_bad;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
-  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
   const int G = args.offsets ? args.G : 1;
-  const int NFT = (args.N + L::kFeat - 1) / L::kFeat;
-  const int KB = (args.Kd + kBK - 1) / kBK;
+  const int NFT = (args.N + L::FEAT - 1) / L::FEAT;
+  const int KB = (args.Kd + KS - 1) / KS;
 
-  if (threadIdx.x == 0) s_bad = 0;
-  pdl_wait();
-  __syncthreads();
-  for (int i = threadIdx.x; i <= G; i += kThreads)
-    s_off[i] = args.offsets ? __ldg(args.offsets + i) : (i == 0 ? 0 : args.M);
-  __syncthreads();
-  for (int i = threadIdx.x; i <= G; i += kThreads) {
-    const bool bad = s_off[i] < 0 || s_off[i] > args.M || (i > 0 && s_off[i] < s_off[i - 1]);
-    if (bad) s_bad = 1;
-  }
-  __syncthreads();
-  if (s_bad) {
-    if (threadIdx.x == 0 && rank == 0) report(args.status, MOE_DEV_BAD_INDEX);
-    for (int i = threadIdx.x; i <= G; i += kThreads) s_off[i] = 0;
-  }
+  // Set-up that reads no global input runs before the wait on the previous kernel.
   if (threadIdx.x == 0) {
+    s_bad = 0;
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
-      mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 2 * (kEpiThreads / 32));  // one arrival per epilogue warp of each CTA
-    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 2 * EW);  // every epilogue warp of both CTAs
     mbar_init(drain, 1);
+    for (int r = 0; r < kRing; ++r) {
+      mbar_init(&rfull[r], 1);
+      mbar_init(&rempty[r], 2 + 2 * EW);  // leader MMA + leader epilogue, peer producer + peer epilogue
+    }
     *abort_flag = 0;
     mbar_init_fence();
   }
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmA0);
     tma_prefetch_map(&tmA1);
+    for (int i = 1; i < kNumBoxes; ++i) tma_prefetch_map(&tmB.box[i]);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, L::kTmemCols);
     tmem_relinquish_pair();
     tc_fence_before();
   }
+  pdl_wait();  // offsets and the token operand come from earlier kernels
+  pdl_launch_dependents();
+  __syncthreads();
+  for (int i = threadIdx.x; i <= G; i += L::kThr)
+    s_off[i] = args.offsets ? __ldg(args.offsets + i) : (i == 0 ? 0 : args.M);
+  __syncthreads();
+  for (int i = threadIdx.x; i <= G; i += L::kThr) {
+    const bool bad = s_off[i] < 0 || s_off[i] > args.M || (i > 0 && s_off[i] < s_off[i - 1]);
+    if (bad) s_bad = 1;
+  }
+  __syncthreads();
+  if (s_bad) {
+    if (threadIdx.x == 0 && rank == 0) report(args.status, MOE_DEV_BAD_INDEX);
+    for (int i = threadIdx.x; i <= G; i += L::kThr) s_off[i] = 0;
+  }
   __syncthreads();
   build_tile_table(s_pre, s_off, G, NT, NFT, s_warp_sums);  // ends with __syncthreads
-  cluster_sync();  // both CTAs' barriers exist before any remote arrival
+  cluster_sync();  // both CTAs' barriers exist before any access over the cluster
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_pre[G];
   const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
+  const uint32_t rempty_leader = mapa_shared(smem_u32(rempty), 0);
+  const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
+      const uint32_t rfull_peer = mapa_shared(smem_u32(rfull), 1);
+      const uint32_t ring_peer = mapa_shared(smem_u32(const_cast<int*>(ring_tile)), 1);
+      uint32_t stage = 0, phase = 0, rs = 0, rphase = 0;
       uint32_t pend_phase[STAGES];
       bool pend[STAGES];
 #pragma unroll
       for (int s = 0; s < STAGES; ++s) pend[s] = false, pend_phase[s] = 0;
       bool ok = true;
-      for (int t = pair; ok && t < total; t += npairs) {
-        const Tile tl = decode_tile<NT, 32, L::kFeat>(t, s_pre, s_off, G);
-        const int half = tl.nround >> 1;
+      for (;;) {
+        int t;
+        if (rank == 0) {
+          if (!mbar_wait_cluster(&rempty[rs], rphase ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          const int claimed = atomicAdd(&args.sched[0], 1);
+          t = claimed < total ? claimed : -1;
+          ring_tile[rs] = t;
+          st_shared_cluster(ring_peer + 4 * rs, t);
+          mbar_arrive(&rfull[rs]);
+          mbar_arrive_cluster(rfull_peer + 8 * rs);
+        } else {
+          if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          t = ring_tile[rs];
+          mbar_arrive_cluster(rempty_leader + 8 * rs);
+        }
+        if (++rs == kRing) {
+          rs = 0;
+          rphase ^= 1u;
+        }
+        if (t < 0) break;
+        const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
+        const int half = tl.nround >> 1;  // token rows staged by each CTA (a multiple of 16)
+        const int rbase = tl.row0 + static_cast<int>(rank) * half;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
             ok = false;
@@ -727,22 +777,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           uint8_t* st = ring + stage * L::kStageBytes;
           const uint32_t bar = full_leader + stage * 8;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kABytes + half * 128));
-          const int kx = kb * kBK;
-          if constexpr (EPI == kEpiSwiGLU) {
-            const int fr = tl.n0 + 64 * static_cast<int>(rank);
-            tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);             // gate rows -> lanes 0..63
-            tma_load_3d_pair(st + L::kABytes / 2, &tmA1, bar, kx, fr, tl.g);  // up rows -> lanes 64..127
-          } else {
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kAPair + half * 128));
+          const int kx = kb * KS;
+          if constexpr (EPI == kEpiBF16) {
             tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
+            tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
+          } else {
+            const int fr = tl.n0 + 128 * static_cast<int>(rank);
+            tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
+            tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
           }
-          const int rbase = tl.row0 + static_cast<int>(rank) * half;
           int r = 0;
 #pragma unroll
           for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
             const int rows = 256 >> i;
             if (half & rows) {
-              tma_load_2d_pair(st + L::kABytes + r * 128, &tmB.box[i], bar, kx, rbase + r);
+              tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
               r += rows;
             }
           }
@@ -753,6 +803,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             phase ^= 1u;
           }
         }
+        if (!ok) break;
       }
       if (!ok) {
         if (rank == 0) {
@@ -771,17 +822,28 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     if (lane == 0 && rank == 0) {
       const uint32_t empty_peer = mapa_shared(smem_u32(empty), 1);
       const uint32_t tfull_peer = mapa_shared(smem_u32(tfull), 1);
-      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0;
+      uint32_t stage = 0, phase = 0, acc_phase = 0, rs = 0, rphase = 0;
       bool ok = true;
-      for (int t = pair; ok && t < total; t += npairs) {
-        const Tile tl = decode_tile<NT, 32, L::kFeat>(t, s_pre, s_off, G);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) {
+      for (;;) {
+        if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) {
+          ok = false;
+          break;
+        }
+        const int t = ring_tile[rs];
+        mbar_arrive(&rempty[rs]);
+        if (++rs == kRing) {
+          rs = 0;
+          rphase ^= 1u;
+        }
+        if (t < 0) break;
+        const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
+        if (!mbar_wait(tempty, acc_phase ^ 1u, abort_flag, args.status)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t idesc = idesc_bf16_f32(256, tl.nround);
-        const uint32_t d = tmem_base + acc * L::kAccCols;
+        const uint32_t idesc =
+            (EPI == kEpiSwiGLUFp8) ? idesc_e4m3_f32(256, tl.nround) : idesc_bf16_f32(256, tl.nround);
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) {
             ok = false;
@@ -789,11 +851,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
           const uint32_t sa = smem_u32(ring + stage * L::kStageBytes);
-          const uint32_t sb = sa + L::kABytes;
+          const uint32_t sb = sa + L::kAPair;
 #pragma unroll
-          for (int kk = 0; kk < kBK / 16; ++kk)
-            umma_bf16_pair(d, sw128_kmajor_desc(sa + kk * 32), sw128_kmajor_desc(sb + kk * 32), idesc,
-                           (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
+#pragma unroll
+            for (int i = 0; i < 2; ++i) {
+              const uint64_t adesc = sw128_kmajor_desc(sa + i * kABytes + kk * 32);
+              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
+              if constexpr (EPI == kEpiSwiGLUFp8) umma_e4m3_pair(tmem_base + i * NT, adesc, bdesc, idesc, acc);
+              else umma_bf16_pair(tmem_base + i * NT, adesc, bdesc, idesc, acc);
+            }
+          }
           umma_commit_pair(smem_u32(&empty[stage]));  // both CTAs' stage buffers are free again
           umma_commit_pair(empty_peer + stage * 8);
           if (++stage == STAGES) {
@@ -802,10 +871,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         if (!ok) break;
-        umma_commit_pair(smem_u32(&tfull[acc]));
-        umma_commit_pair(tfull_peer + acc * 8);
-        acc ^= 1u;
-        if (acc == 0) acc_phase ^= 1u;
+        umma_commit_pair(smem_u32(tfull));
+        umma_commit_pair(tfull_peer);
+        acc_phase ^= 1u;
       }
       if (!ok) {
         umma_commit_pair(smem_u32(drain));
@@ -814,65 +882,75 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;  // TMEM lanes [32q, 32q + 32)
-    const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
-    uint32_t acc = 0, acc_phase = 0, chunk = 0;
-    for (int t = pair; t < total; t += npairs) {
-      const Tile tl = decode_tile<NT, 32, L::kFeat>(t, s_pre, s_off, G);
-      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
+    const int q = warp & 3;               // TMEM lanes [32q, 32q + 32)
+    const int part = (warp - 2) >> 2;     // two warps per lane quadrant take alternate chunks
+    __nv_bfloat16* stg = stg_all + (warp - 2) * 32 * 32;
+    __nv_bfloat16* outb = reinterpret_cast<__nv_bfloat16*>(args.out);
+    uint32_t acc_phase = 0, rs = 0, rphase = 0;
+    for (;;) {
+      if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) break;
+      const int t = ring_tile[rs];
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(&rempty[rs]);
+        else mbar_arrive_cluster(rempty_leader + 8 * rs);
+      }
+      if (++rs == kRing) {
+        rs = 0;
+        rphase ^= 1u;
+      }
+      if (t < 0) break;
+      const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
+      if (!mbar_wait(tfull, acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
-      for (int j0 = 0; j0 < tl.nvalid; j0 += 32, ++chunk) {
-        uint32_t r[32];
-        tmem_ld_32cols(tbase + j0, r);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const int fa = tl.n0 + 128 * static_cast<int>(rank) + 32 * q;  // this warp's first feature
+      float sg = 1.0f, su = 1.0f;
+      if constexpr (EPI == kEpiSwiGLUFp8) {
+        if (fa + lane < args.N) {
+          const long long fi = static_cast<long long>(tl.g) * args.N + fa + lane;
+          sg = __ldg(args.scale_a0 + fi);
+          su = __ldg(args.scale_a1 + fi);
+        }
+      }
+      for (int j0 = 32 * part; j0 < tl.nvalid; j0 += 64) {
+        const int jn = min(32, tl.nvalid - j0);
+        const long long row0 = static_cast<long long>(tl.row0) + j0;
+        uint32_t r0[32], r1[32];
+        tmem_ld_32cols(tbase + j0, r0);
+        tmem_ld_32cols(tbase + NT + j0, r1);
+        float sx = 1.0f;
+        if constexpr (EPI == kEpiSwiGLUFp8) sx = lane < jn ? __ldg(args.scale_b + row0 + lane) : 0.0f;
         tmem_wait_ld();
-        if constexpr (EPI == kEpiSwiGLU) {
-          // warps q < 2 own gate of features fi, warps q >= 2 own up of the same fi
-          const int fi = 32 * (q & 1) + lane;
-          const bool is_gate = q < 2;
-          float* xb = exch + (chunk & 1) * L::kExchFloats;
-          float* to_up = xb;                 // gate of tokens 16..31, read by the up owner
-          float* to_gate = xb + 16 * 64;     // up of tokens 0..15, read by the gate owner
+        float v[32];
+        if constexpr (EPI == kEpiBF16) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            if (is_gate) to_up[j * 64 + fi] = __uint_as_float(r[16 + j]);
-            else to_gate[j * 64 + fi] = __uint_as_float(r[j]);
-          }
-          named_bar_sync(1, kEpiThreads);
-          const int f = tl.n0 + 64 * static_cast<int>(rank) + fi;
-          const int jbase = is_gate ? 0 : 16;
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.out);
-          if (f < args.N) {
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
+          store_rows32(stg, lane, v, outb, args.ldo, args.N, fa, row0, jn);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              const int tok = j0 + jbase + j;
-              if (tok < tl.nvalid) {
-                const float g = is_gate ? __uint_as_float(r[j]) : to_up[j * 64 + fi];
-                const float u = is_gate ? to_gate[j * 64 + fi] : __uint_as_float(r[16 + j]);
-                out[static_cast<long long>(tl.row0 + tok) * args.ldo + f] = __float2bfloat16_rn(silu_mul(g, u));
-              }
-            }
-          }
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r1[j]);
+          store_rows32(stg, lane, v, outb, args.ldo, args.N, fa + 256, row0, jn);
         } else {
-          const int f = tl.n0 + 128 * static_cast<int>(rank) + q * 32 + lane;
-          const int jn = min(32, tl.nvalid - j0);
-          __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.out);
-          if (f < args.N) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j)
-              if (j < jn)
-                out[static_cast<long long>(tl.row0 + j0 + j) * args.ldo + f] = __float2bfloat16_rn(__uint_as_float(r[j]));
+          for (int j = 0; j < 32; ++j) {
+            float g = __uint_as_float(r0[j]), u = __uint_as_float(r1[j]);
+            if constexpr (EPI == kEpiSwiGLUFp8) {
+              const float sj = __shfl_sync(0xffffffffu, sx, j);
+              g *= sj * sg;
+              u *= sj * su;
+            }
+            v[j] = silu_mul(g, u);
           }
+          store_rows32(stg, lane, v, outb, args.ldo, args.N, fa, row0, jn);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (rank == 0) mbar_arrive(&tempty[acc]);
-        else mbar_arrive_cluster(tempty_leader + acc * 8);
+        if (rank == 0) mbar_arrive(tempty);
+        else mbar_arrive_cluster(tempty_leader);
       }
-      acc ^= 1u;
-      if (acc == 0) acc_phase ^= 1u;
+      acc_phase ^= 1u;
     }
   }
 
@@ -882,6 +960,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
     tc_fence_after();
     tmem_dealloc_pair(tmem_base, L::kTmemCols);
+  }
+  if (threadIdx.x == 0) {  // the last CTA rewinds the schedule for the next launch on this slot
+    __threadfence();
+    if (atomicAdd(&args.sched[1], 1) == static_cast<int>(gridDim.x) - 1) {
+      atomicExch(&args.sched[0], 0);
+      atomicExch(&args.sched[1], 0);
+    }
   }
 }
 
@@ -970,8 +1055,7 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const BoxM
   if (attr_err != cudaSuccess) return attr_err;
   if (tile_bound <= 0) return cudaSuccess;
   const int pairs = static_cast<int>(std::min<long long>(num_sms() / 2, tile_bound));
-  pair_gemm_kernel<EPI><<<2 * pairs, kThreads, L::kSmemBytes, stream>>>(a0, a1, b, args);
-  return cudaGetLastError();
+  return launch_pdl(pair_gemm_kernel<EPI>, dim3(2 * pairs), dim3(L::kThr), L::kSmemBytes, stream, a0, a1, b, args);
 }
 
 long long tile_bound(long long rows, int groups, int NT, int N, int feat) {
@@ -991,12 +1075,24 @@ int gemm_smem_bytes(int epi) {
   }
 }
 
-// The CTA-pair kernel is correct (it passes the same parity tests when built with
-// MOE_GEMM_PAIR=1) and faster on long-K dense shapes, but slower than the single-CTA
-// kernel on the layer workloads measured so far, so the single-CTA kernel is the default.
+// The CTA-pair kernel serves groups of at least MOE_PAIR_MIN_ROWS rows on average (its
+// token tiles are cut in multiples of 32 rows and split between the two SMs); smaller
+// groups (decode) and the fp32 gating use the single-CTA kernel.  MOE_GEMM_PAIR=0 builds
+// the single-CTA kernel only.
 #ifndef MOE_GEMM_PAIR
-#define MOE_GEMM_PAIR 0
+#define MOE_GEMM_PAIR 1
 #endif
+#ifndef MOE_PAIR_MIN_ROWS
+#define MOE_PAIR_MIN_ROWS 64
+#endif
+static std::atomic<int> g_pair_min_rows{MOE_PAIR_MIN_ROWS};
+static bool use_pair(long long rows, int groups) {
+  const int min_rows = g_pair_min_rows.load(std::memory_order_relaxed);
+  return MOE_GEMM_PAIR && min_rows >= 0 && num_sms() >= 2 &&
+         rows >= static_cast<long long>(min_rows) * std::max(groups, 1);
+}
+
+void set_pair_min_rows(int rows) { g_pair_min_rows.store(rows, std::memory_order_relaxed); }
 
 // h = silu(xp Wg^T) * (xp Wu^T) per expert group.
 cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
@@ -1005,11 +1101,11 @@ cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_g
   CUtensorMap a0, a1;
   BoxMaps b;
   if (!map_token_boxes(&b, xp, H, rows)) return cudaErrorInvalidValue;
-  if (MOE_GEMM_PAIR) {
-    if (!map_bf16_3d(&a0, w_gate, H, F, E, 64) || !map_bf16_3d(&a1, w_up, H, F, E, 64)) return cudaErrorInvalidValue;
-    return launch_pair<kEpiSwiGLU>(a0, a1, b, args, tile_bound(rows, E, PairLayout<kEpiSwiGLU>::NT, F, 128), stream);
-  }
   if (!map_bf16_3d(&a0, w_gate, H, F, E, kBM) || !map_bf16_3d(&a1, w_up, H, F, E, kBM)) return cudaErrorInvalidValue;
+  if (use_pair(rows, E))
+    return launch_pair<kEpiSwiGLU>(a0, a1, b, args,
+                                   tile_bound(rows, E, PairLayout<kEpiSwiGLU>::NT, F, PairLayout<kEpiSwiGLU>::FEAT),
+                                   stream);
   return launch<kEpiSwiGLU>(a0, a1, a1, b, args, tile_bound(rows, E, Cfg<kEpiSwiGLU>::NT, F, Cfg<kEpiSwiGLU>::FEAT), stream);
 }
 
@@ -1040,6 +1136,9 @@ cudaError_t gemm_gate_up_fp8(const void* xq, const float* xs, const int32_t* off
   if (!map_token_boxes(&b, xq, H, rows, 1) || !map_bf16_3d(&a0, wq_gate, H, F, E, kBM, 1) ||
       !map_bf16_3d(&a1, wq_up, H, F, E, kBM, 1))
     return cudaErrorInvalidValue;
+  if (use_pair(rows, E))
+    return launch_pair<kEpiSwiGLUFp8>(
+        a0, a1, b, args, tile_bound(rows, E, PairLayout<kEpiSwiGLUFp8>::NT, F, PairLayout<kEpiSwiGLUFp8>::FEAT), stream);
   return launch<kEpiSwiGLUFp8>(a0, a1, a1, b, args,
                                tile_bound(rows, E, Cfg<kEpiSwiGLUFp8>::NT, F, Cfg<kEpiSwiGLUFp8>::FEAT), stream);
 }
@@ -1050,10 +1149,12 @@ cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down,
   GemmArgs args{offsets, E, static_cast<int>(rows), H, F, y, H, nullptr, status, nullptr, nullptr, nullptr, sched};
   CUtensorMap a0;
   BoxMaps b;
-  if (!map_bf16_3d(&a0, w_down, F, H, E, MOE_GEMM_PAIR ? kBM : 256) || !map_token_boxes(&b, h, F, rows))
+  const bool pair = use_pair(rows, E);
+  if (!map_bf16_3d(&a0, w_down, F, H, E, pair ? kBM : 256) || !map_token_boxes(&b, h, F, rows))
     return cudaErrorInvalidValue;
-  if (MOE_GEMM_PAIR)
-    return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(rows, E, PairLayout<kEpiBF16>::NT, H, 256), stream);
+  if (pair)
+    return launch_pair<kEpiBF16>(a0, a0, b, args,
+                                 tile_bound(rows, E, PairLayout<kEpiBF16>::NT, H, PairLayout<kEpiBF16>::FEAT), stream);
   return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(rows, E, Cfg<kEpiBF16>::NT, H, Cfg<kEpiBF16>::FEAT), stream);
 }
 
@@ -1062,11 +1163,13 @@ cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd,
                        int* sched, cudaStream_t stream) {
   CUtensorMap a0;
   BoxMaps b;
-  if (!map_bf16_3d(&a0, w, Kd, N, 1, MOE_GEMM_PAIR ? kBM : 256) || !map_token_boxes(&b, a, Kd, M))
+  const bool pair = use_pair(M, 1);
+  if (!map_bf16_3d(&a0, w, Kd, N, 1, pair ? kBM : 256) || !map_token_boxes(&b, a, Kd, M))
     return cudaErrorInvalidValue;
   GemmArgs args{nullptr, 1, static_cast<int>(M), N, Kd, out, N, nullptr, status, nullptr, nullptr, nullptr, sched};
-  if (MOE_GEMM_PAIR)
-    return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(M, 1, PairLayout<kEpiBF16>::NT, N, 256), stream);
+  if (pair)
+    return launch_pair<kEpiBF16>(a0, a0, b, args, tile_bound(M, 1, PairLayout<kEpiBF16>::NT, N, PairLayout<kEpiBF16>::FEAT),
+                                 stream);
   return launch<kEpiBF16>(a0, a0, a0, b, args, tile_bound(M, 1, Cfg<kEpiBF16>::NT, N, Cfg<kEpiBF16>::FEAT), stream);
 }
 

@@ -44,6 +44,8 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 int gemm_smem_bytes(int epi);
+// Average rows per group from which the grouped GEMMs use the CTA-pair kernel (< 0: never).
+void set_pair_min_rows(int rows);
 
 cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
                          long long rows, int H, int F, void* h, int* status, int* sched, cudaStream_t stream);

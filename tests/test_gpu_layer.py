@@ -38,6 +38,15 @@ def bits(t):
     return inputs.to_bits(t)
 
 
+@pytest.fixture(params=["single_cta", "cta_pair"])
+def gemm_kernel(request):
+    """Runs a layer once with every grouped GEMM on the single-CTA kernel and once on the
+    CTA-pair kernel (default rule: pair from 64 rows per expert)."""
+    B.set_pair_min_rows(-1 if request.param == "single_cta" else 0)
+    yield request.param
+    B.set_pair_min_rows(64)
+
+
 def cpu(t):
     return t.detach().cpu().numpy()
 
@@ -128,7 +137,7 @@ SMALL = [
 
 
 @pytest.mark.parametrize("cfg", SMALL, ids=lambda c: c.name)
-def test_layer_matches_oracle(cfg):
+def test_layer_matches_oracle(cfg, gemm_kernel):
     inp = inputs.make_layer(cfg, DEV)
     # both gate/up paths: separate weights for two layers, packed weights for the others;
     # the shared expert on its own stream in one layer and in line in the other

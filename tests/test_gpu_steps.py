@@ -26,6 +26,17 @@ def bits(t):
     return inputs.to_bits(t)
 
 
+PAIR_DEFAULT_MIN_ROWS = 64
+
+
+@pytest.fixture(params=["single_cta", "cta_pair"])
+def gemm_kernel(request):
+    """Runs a GEMM test once on the single-CTA kernel and once on the CTA-pair kernel."""
+    B.set_pair_min_rows(-1 if request.param == "single_cta" else 0)
+    yield request.param
+    B.set_pair_min_rows(PAIR_DEFAULT_MIN_ROWS)
+
+
 def cpu(t):
     return t.detach().cpu().numpy()
 
@@ -247,7 +258,7 @@ def ffn_inputs(E, H, F, rows, zipf, zero_frac, seed=0):
 
 @pytest.mark.parametrize("packed", [False, True], ids=["separate", "packed"])
 @pytest.mark.parametrize("E,H,F,rows,zipf,zf", FFN_CASES)
-def test_grouped_ffn_matches_oracle(E, H, F, rows, zipf, zf, packed):
+def test_grouped_ffn_matches_oracle(E, H, F, rows, zipf, zf, packed, gemm_kernel):
     off, xp, wg, wu, wd = ffn_inputs(E, H, F, rows, zipf, zf)
     d = B.dims(T=rows, H=H, E=E, K=1, F=F)
     ws = B.make_workspace(d)
@@ -320,7 +331,7 @@ FP8_FFN_CASES = [  # E, H, F, rows, zipf, zero_frac
 
 
 @pytest.mark.parametrize("E,H,F,rows,zipf,zf", FP8_FFN_CASES)
-def test_grouped_gate_up_fp8_matches_oracle(E, H, F, rows, zipf, zf):
+def test_grouped_gate_up_fp8_matches_oracle(E, H, F, rows, zipf, zf, gemm_kernel):
     counts = inputs.random_counts(E, rows, seed=E + rows, zipf_s=zipf, zero_frac=zf)
     off = np.zeros(E + 1, np.int32)
     off[1:] = np.cumsum(counts.numpy())
@@ -364,7 +375,7 @@ def test_pack_gate_up_layout():
             assert int(rows[:, n:].view(torch.int16).abs().sum()) == 0
 
 
-def test_grouped_down_alone_matches_oracle():
+def test_grouped_down_alone_matches_oracle(gemm_kernel):
     E, H, F, rows = 12, 1024, 512, 900
     counts = inputs.random_counts(E, rows, seed=4, zero_frac=0.2)
     off = np.concatenate([[0], np.cumsum(counts.numpy())]).astype(np.int32)
@@ -452,7 +463,7 @@ def test_gating_matches_oracle(T, H, E, bias):
 
 
 @pytest.mark.parametrize("M,Kd,N", [(300, 1024, 256), (64, 7168, 2048), (257, 2048, 7168), (3, 72, 40)])
-def test_dense_projection_matches_oracle(M, Kd, N):
+def test_dense_projection_matches_oracle(M, Kd, N, gemm_kernel):
     a = inputs.random_bf16((M, Kd), seed=M)
     w = inputs.random_bf16((N, Kd), seed=N, std=Kd ** -0.5)
     out = torch.zeros((M, N), dtype=torch.bfloat16, device=DEV)
