@@ -617,27 +617,38 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 // per pair and each SM fills 48 KB of shared memory per K-step instead of the single-CTA
 // tile's 64 KB for the same MMA work per SM.
 //   SwiGLU: CTA r holds gate and up rows [n0 + 128 r, +128): gate and up accumulate in
-//           separate TMEM columns of the same lanes, so no exchange between warps.
-//   bf16:   CTA r holds rows [n0 + 128 r, +128) and [n0 + 256 + 128 r, +128).
+//           separate TMEM columns of the same lanes, so no exchange between warps; the two
+//           accumulators fill TMEM, so the epilogue of a tile runs between main loops.
+//   bf16:   CTA r holds rows [n0 + 128 r, +128) and [n0 + 256 + 128 r, +128) (NA = 2).
+//           Built with MOE_PAIR_BF16_NA=1 it holds one weight operand with a double-buffered
+//           accumulator (the epilogue then overlaps the next main loop); that measured
+//           slower on the down projections (Qwen3 layer 164 vs 142 us), since each K-step
+//           carries half the MMA work for the same synchronisation.
 // Both CTAs' TMA loads of a stage complete on the leader's "full" barrier; the leader's
 // commits release both CTAs' "empty" and "tmem full" barriers; both CTAs' epilogue warps
 // release the leader's "tmem empty" barrier.  The leader's producer claims tiles from the
 // launch's counter and publishes each id to both CTAs through a ring in shared memory (the
 // peer's slot written over the cluster), which both CTAs' consumers release.
 // ---------------------------------------------------------------------------
+#ifndef MOE_PAIR_BF16_NA
+#define MOE_PAIR_BF16_NA 2
+#endif
 template <int EPI>
 struct PairLayout {
   static constexpr int NT = 256;                                // tokens per pair tile (MMA N)
-  static constexpr int STAGES = 4;
+  static constexpr int NA = (EPI == kEpiBF16) ? MOE_PAIR_BF16_NA : 2;  // weight operands (accumulators)
+  static constexpr int STAGES = (NA == 1) ? 6 : 4;
   static constexpr int EW = 8;                                  // epilogue warps per CTA
   static constexpr int kThr = 64 + 32 * EW;
-  static constexpr int FEAT = (EPI == kEpiBF16) ? 512 : 256;    // output features per pair tile
-  static constexpr int kAPair = 2 * kABytes;                    // this CTA's two 128-row weight boxes
+  static constexpr int FEAT = (EPI == kEpiBF16) ? 256 * NA : 256;  // output features per pair tile
+  static constexpr int kAPair = NA * kABytes;                   // this CTA's 128-row weight boxes
   static constexpr int kBBytes = (NT / 2) * 128;                // this CTA's token rows
   static constexpr int kStageBytes = kAPair + kBBytes;
-  static constexpr uint32_t kTmemCols = 2 * NT;                 // two accumulators, single-buffered
+  static constexpr uint32_t kAccCols = NA * NT;                 // one tile's accumulators
+  static constexpr int kNumAcc = (NA == 1) ? 2 : 1;             // TMEM buffers
+  static constexpr uint32_t kTmemCols = kNumAcc * kAccCols;
   static constexpr int kStgBytes = EW * 32 * 32 * 2;
-  static constexpr int kBarBytes = (8 * (2 * STAGES + 3 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
+  static constexpr int kBarBytes = (8 * (2 * STAGES + 5 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
   static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
   static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kStgBytes + kBarBytes + kTableBytes;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -649,9 +660,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                      const __grid_constant__ BoxMaps tmB, const GemmArgs args) {
   using L = PairLayout<EPI>;
-  constexpr int NT = L::NT, STAGES = L::STAGES, EW = L::EW;
+  constexpr int NT = L::NT, NA = L::NA, STAGES = L::STAGES, EW = L::EW;
   constexpr int KS = stage_k<EPI>();
   static_assert(EPI == kEpiSwiGLU || EPI == kEpiSwiGLUFp8 || EPI == kEpiBF16, "pair epilogues");
+  static_assert(L::kTmemCols == 512, "TMEM allocation");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -660,8 +672,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::kStageBytes + L::kStgBytes);
   uint64_t* empty = full + STAGES;
   uint64_t* tfull = empty + STAGES;
-  uint64_t* tempty = tfull + 1;
-  uint64_t* drain = tempty + 1;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
   uint64_t* rfull = drain + 1;
   uint64_t* rempty = rfull + kRing;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rempty + kRing);
@@ -685,8 +697,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(tfull, 1);
-    mbar_init(tempty, 2 * EW);  // every epilogue warp of both CTAs
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 2 * EW);  // every epilogue warp of both CTAs
+    }
     mbar_init(drain, 1);
     for (int r = 0; r < kRing; ++r) {
       mbar_init(&rfull[r], 1);
@@ -781,7 +795,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
           const int kx = kb * KS;
           if constexpr (EPI == kEpiBF16) {
             tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
-            tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
+            if constexpr (NA == 2)
+              tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
           } else {
             const int fr = tl.n0 + 128 * static_cast<int>(rank);
             tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
@@ -822,7 +837,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     if (lane == 0 && rank == 0) {
       const uint32_t empty_peer = mapa_shared(smem_u32(empty), 1);
       const uint32_t tfull_peer = mapa_shared(smem_u32(tfull), 1);
-      uint32_t stage = 0, phase = 0, acc_phase = 0, rs = 0, rphase = 0;
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0, rs = 0, rphase = 0;
       bool ok = true;
       for (;;) {
         if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) {
@@ -837,10 +852,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         }
         if (t < 0) break;
         const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
-        if (!mbar_wait(tempty, acc_phase ^ 1u, abort_flag, args.status)) {
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) {
           ok = false;
           break;
         }
+        const uint32_t d0 = tmem_base + acc * L::kAccCols;
         tc_fence_after();
         const uint32_t idesc =
             (EPI == kEpiSwiGLUFp8) ? idesc_e4m3_f32(256, tl.nround) : idesc_bf16_f32(256, tl.nround);
@@ -856,11 +872,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
 #pragma unroll
-            for (int i = 0; i < 2; ++i) {
+            for (int i = 0; i < NA; ++i) {
               const uint64_t adesc = sw128_kmajor_desc(sa + i * kABytes + kk * 32);
-              const uint32_t acc = (kb > 0 || kk > 0) ? 1u : 0u;
-              if constexpr (EPI == kEpiSwiGLUFp8) umma_e4m3_pair(tmem_base + i * NT, adesc, bdesc, idesc, acc);
-              else umma_bf16_pair(tmem_base + i * NT, adesc, bdesc, idesc, acc);
+              const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+              if constexpr (EPI == kEpiSwiGLUFp8) umma_e4m3_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
+              else umma_bf16_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
             }
           }
           umma_commit_pair(smem_u32(&empty[stage]));  // both CTAs' stage buffers are free again
@@ -871,9 +887,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
           }
         }
         if (!ok) break;
-        umma_commit_pair(smem_u32(tfull));
-        umma_commit_pair(tfull_peer);
-        acc_phase ^= 1u;
+        umma_commit_pair(smem_u32(&tfull[acc]));
+        umma_commit_pair(tfull_peer + acc * 8);
+        if (++acc == L::kNumAcc) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
       }
       if (!ok) {
         umma_commit_pair(smem_u32(drain));
@@ -886,7 +905,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     const int part = (warp - 2) >> 2;     // two warps per lane quadrant take alternate chunks
     __nv_bfloat16* stg = stg_all + (warp - 2) * 32 * 32;
     __nv_bfloat16* outb = reinterpret_cast<__nv_bfloat16*>(args.out);
-    uint32_t acc_phase = 0, rs = 0, rphase = 0;
+    uint32_t acc = 0, acc_phase = 0, rs = 0, rphase = 0;
     for (;;) {
       if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) break;
       const int t = ring_tile[rs];
@@ -901,9 +920,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
       }
       if (t < 0) break;
       const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
-      if (!mbar_wait(tfull, acc_phase, abort_flag, args.status)) break;
+      if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
-      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+      const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
       const int fa = tl.n0 + 128 * static_cast<int>(rank) + 32 * q;  // this warp's first feature
       float sg = 1.0f, su = 1.0f;
       if constexpr (EPI == kEpiSwiGLUFp8) {
@@ -918,7 +937,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         const long long row0 = static_cast<long long>(tl.row0) + j0;
         uint32_t r0[32], r1[32];
         tmem_ld_32cols(tbase + j0, r0);
-        tmem_ld_32cols(tbase + NT + j0, r1);
+        if constexpr (NA == 2) tmem_ld_32cols(tbase + NT + j0, r1);
         float sx = 1.0f;
         if constexpr (EPI == kEpiSwiGLUFp8) sx = lane < jn ? __ldg(args.scale_b + row0 + lane) : 0.0f;
         tmem_wait_ld();
@@ -927,9 +946,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
           store_rows32(stg, lane, v, outb, args.ldo, args.N, fa, row0, jn);
+          if constexpr (NA == 2) {
 #pragma unroll
-          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r1[j]);
-          store_rows32(stg, lane, v, outb, args.ldo, args.N, fa + 256, row0, jn);
+            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r1[j]);
+            store_rows32(stg, lane, v, outb, args.ldo, args.N, fa + 256, row0, jn);
+          } else {
+            (void)r1;
+          }
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -947,10 +970,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) {
-        if (rank == 0) mbar_arrive(tempty);
-        else mbar_arrive_cluster(tempty_leader);
+        if (rank == 0) mbar_arrive(&tempty[acc]);
+        else mbar_arrive_cluster(tempty_leader + acc * 8);
       }
-      acc_phase ^= 1u;
+      if (++acc == L::kNumAcc) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
     }
   }
 
