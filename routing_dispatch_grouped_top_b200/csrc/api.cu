@@ -62,10 +62,27 @@ moe_status check_dims(const moe_dims* d) {
   return MOE_OK;
 }
 
-size_t ws_bytes_for(const moe_dims* d) {
+// The split gating reduction keeps its partial logits after the histograms.  The workspace
+// is sized for a 148-SM B200; a device with fewer SMs uses fewer splits.
+constexpr int kSizingSms = 148;
+
+size_t hist_bytes(const moe_dims* d) {
   const long long TK = d->T * static_cast<long long>(d->K);
-  const size_t hist = static_cast<size_t>(scan_max_blocks(TK)) * d->E * sizeof(int);
-  return kWsHeader + (hist + 255) / 256 * 256;
+  return (static_cast<size_t>(scan_max_blocks(TK)) * d->E * sizeof(int) + 255) / 256 * 256;
+}
+
+int gating_split_count(const moe_dims* d) {
+  return std::min(gating_splits(d->T, d->H, d->E, num_sms()), gating_splits(d->T, d->H, d->E, kSizingSms));
+}
+
+size_t ws_bytes_for(const moe_dims* d) {
+  const int S = gating_splits(d->T, d->H, d->E, kSizingSms);
+  const size_t partials = S > 1 ? static_cast<size_t>(S) * d->T * d->E * sizeof(float) : 0;
+  return kWsHeader + hist_bytes(d) + partials;
+}
+
+float* ws_partials(void* ws, const moe_dims* d) {
+  return reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsHeader + hist_bytes(d));
 }
 
 int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
@@ -164,16 +181,22 @@ moe_status moe_gating(const void* x, const void* w_g_split, const float* bias, c
   if (d->T == 0) return MOE_OK;
   if (!x || !w_g_split || !logits) return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(w_g_split)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(gemm_gating(x, w_g_split, bias, d->T, d->H, d->E, logits, ws_status(ws),
-                                 ws_sched(ws, kSchedGating), as_stream(stream)));
+  const int S = gating_split_count(d);
+  if (S <= 1)
+    return cuda_status(gemm_gating(x, w_g_split, bias, d->T, d->H, d->E, logits, 1, ws_status(ws),
+                                   ws_sched(ws, kSchedGating), as_stream(stream)));
+  float* partials = ws_partials(ws, d);
+  MOE_CUDA(gemm_gating(x, w_g_split, bias, d->T, d->H, d->E, partials, S, ws_status(ws), ws_sched(ws, kSchedGating),
+                       as_stream(stream)));
+  return cuda_status(launch_sum_partials(partials, S, d->T * static_cast<long long>(d->E), logits, as_stream(stream)));
 }
 
 moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids, float* topk_w, void* stream) {
   MOE_TRY(common_checks(d));
   if (d->T == 0) return MOE_OK;
   if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_route(logits, d->T, d->E, d->K, d->renormalize, d->P, d->group_limit, topk_ids, topk_w,
-                                  as_stream(stream)));
+  return cuda_status(launch_route(logits, 1, nullptr, d->T, d->E, d->K, d->renormalize, d->P, d->group_limit,
+                                  topk_ids, topk_w, as_stream(stream)));
 }
 
 moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* counts, int32_t* offsets,
@@ -380,11 +403,16 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
                        ws_sched(ws, kSchedSharedDown), sh));
     if (b->aux_stream) MOE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(b->join_event), sh));
   }
+  // Gating with a split reduction leaves partial logits in the workspace; the route kernel adds
+  // them in split order and writes the logits buffer.
+  const int nsplit = gating_split_count(d);
+  float* gate_out = nsplit > 1 ? ws_partials(ws, d) : b->logits;
   if (T > 0)
-    MOE_CUDA(gemm_gating(routed, w->w_g_split, w->bias, T, d->H, d->E, b->logits, status, ws_sched(ws, kSchedGating),
-                         s));
+    MOE_CUDA(gemm_gating(routed, w->w_g_split, w->bias, T, d->H, d->E, gate_out, nsplit, status,
+                         ws_sched(ws, kSchedGating), s));
   MOE_TRY(mark(2));
-  MOE_CUDA(launch_route(b->logits, T, d->E, d->K, d->renormalize, d->P, d->group_limit, b->topk_ids, b->topk_w, s));
+  MOE_CUDA(launch_route(gate_out, nsplit, b->logits, T, d->E, d->K, d->renormalize, d->P, d->group_limit, b->topk_ids,
+                        b->topk_w, s));
   MOE_TRY(mark(3));
   MOE_CUDA(launch_count_scan(b->topk_ids, TK, d->E, d->P, b->counts, b->offsets, b->part_counts, b->part_offsets,
                              b->row_of_assign, b->assign_of_row, b->skew, scan_ws(ws, d), s));

@@ -314,7 +314,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   build_tile_table(s_pre, s_off, G, NT, NFT, s_warp_sums);  // ends with __syncthreads
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  const int total = s_pre[G];
+  // Split reduction (fp32 gating only): tile t covers output tile t / S and K-steps
+  // [ks KB / S, (ks + 1) KB / S) of split ks = t % S; the host keeps S <= KB.
+  const int S = (EPI == kEpiF32 && args.ksplit > 1) ? args.ksplit : 1;
+  const int total = s_pre[G] * S;
 
   static_assert(EPI != kEpiSwiGLUPacked || C::EW == 4, "the packed epilogue pairs warps q and q + 2");
   if (warp == 0) {
@@ -342,9 +345,10 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           rphase ^= 1u;
         }
         if (t >= total) break;
-        const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
+        const int tb = t / S, ks = t - tb * S;
+        const Tile tl = decode_tile<NT, 16, C::FEAT>(tb, s_pre, s_off, G);
         const uint32_t bytes = NA * kABytes + tl.nround * 128;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = ks * KB / S; kb < (ks + 1) * KB / S; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
@@ -403,7 +407,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           rphase ^= 1u;
         }
         if (t < 0) break;
-        const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
+        const int tb = t / S, ks = t - tb * S;
+        const int kb_lo = ks * KB / S, kb_hi = (ks + 1) * KB / S;
+        const Tile tl = decode_tile<NT, 16, C::FEAT>(tb, s_pre, s_off, G);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) {
           ok = false;
           break;
@@ -412,7 +418,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const uint32_t idesc =
             (EPI == kEpiSwiGLUFp8) ? idesc_e4m3_f32(kBM, tl.nround) : idesc_bf16_f32(kBM, tl.nround);
         const uint32_t d0 = tmem_base + acc * L::kAccCols;
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = kb_lo; kb < kb_hi; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) {
             ok = false;
             break;
@@ -428,7 +434,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
             for (int i = 0; i < NA; ++i) {
               const uint64_t adesc = sw128_kmajor_desc(sa + i * kABytes + kk * 32);
               const uint32_t d = d0 + (C::SEP ? i * NT : 0);
-              const uint32_t accumulate = (kb > 0 || kk > 0 || (!C::SEP && i > 0)) ? 1u : 0u;
+              const uint32_t accumulate = (kb > kb_lo || kk > 0 || (!C::SEP && i > 0)) ? 1u : 0u;
               if constexpr (EPI == kEpiSwiGLUFp8) umma_e4m3(d, adesc, bdesc, idesc, accumulate);
               else umma_bf16(d, adesc, bdesc, idesc, accumulate);
             }
@@ -468,7 +474,8 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         rphase ^= 1u;
       }
       if (t < 0) break;
-      const Tile tl = decode_tile<NT, 16, C::FEAT>(t, s_pre, s_off, G);
+      const int tb = t / S, ks = t - tb * S;
+      const Tile tl = decode_tile<NT, 16, C::FEAT>(tb, s_pre, s_off, G);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
       if constexpr (EPI == kEpiSwiGLUPacked) {
@@ -574,9 +581,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           }
         } else {
           tmem_wait_ld();
-          float* out = reinterpret_cast<float*>(args.out);
+          float* out = reinterpret_cast<float*>(args.out) + ks * args.split_stride;
           if (f_ok) {
-            const float b = args.bias ? __ldg(args.bias + f) : 0.0f;
+            const float b = (args.bias && ks == 0) ? __ldg(args.bias + f) : 0.0f;
 #pragma unroll
             for (int j = 0; j < 32; ++j)
               if (j < jn) out[(row0 + j) * args.ldo + f] = __uint_as_float(r0[j]) + b;
@@ -1200,13 +1207,27 @@ cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd,
 }
 
 // logits[T][E] = x[T][H] (hi + mid + lo)^T (+ bias), fp32 out; w_split is [3][E][H] bf16.
+// Splits of the gating reduction: enough work units to fill the SMs when the output has few
+// tiles (Qwen3 layer: 32 tiles of 128 tokens x 128 experts over 148 SMs -> 4 splits), at least
+// 4 K-steps per split, at most 8 splits.
+int gating_splits(long long T, int H, int E, int sms) {
+  const long long units = ((T + 127) / 128) * ((E + 127) / 128);
+  const int KB = (H + kBK - 1) / kBK;
+  if (units <= 0) return 1;
+  long long s = sms / units;
+  s = std::min<long long>(s, std::min(8, KB / 4));
+  return static_cast<int>(std::max<long long>(1, s));
+}
+
 cudaError_t gemm_gating(const void* x, const void* w_split, const float* bias, long long T, int H, int E,
-                        float* logits, int* status, int* sched, cudaStream_t stream) {
+                        float* logits, int ksplit, int* status, int* sched, cudaStream_t stream) {
   CUtensorMap a0;
   BoxMaps b;
   if (!map_bf16_3d(&a0, w_split, H, E, 3, kBM) || !map_token_boxes(&b, x, H, T)) return cudaErrorInvalidValue;
-  GemmArgs args{nullptr, 1, static_cast<int>(T), E, H, logits, E, bias, status, nullptr, nullptr, nullptr, sched};
-  return launch<kEpiF32>(a0, a0, a0, b, args, tile_bound(T, 1, Cfg<kEpiF32>::NT, E, kBM), stream);
+  const int S = std::max(1, ksplit);
+  GemmArgs args{nullptr, 1, static_cast<int>(T), E, H, logits, E, bias, status, nullptr, nullptr, nullptr, sched,
+                S, T * E};
+  return launch<kEpiF32>(a0, a0, a0, b, args, tile_bound(T, 1, Cfg<kEpiF32>::NT, E, kBM) * S, stream);
 }
 
 }  // namespace moe

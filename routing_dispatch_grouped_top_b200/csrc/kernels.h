@@ -22,6 +22,8 @@ struct GemmArgs {
   const float* scale_a1;   //                per-feature scales of the up weights [G][N]
   const float* scale_b;    //                per-row scales of the token operand [M]
   int* sched;              // two device ints {next tile, finished CTAs}, zero between launches
+  int ksplit;              // kEpiF32: reduction split into this many partial outputs (0 or 1: none)
+  long long split_stride;  // elements between the partial outputs of consecutive splits
 };
 
 int num_sms();             // SM count of the current device (cached per device)
@@ -63,11 +65,17 @@ cudaError_t gemm_down(const void* h, const int32_t* offsets, const void* w_down,
                       int F, void* y, int* status, int* sched, cudaStream_t stream);
 cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd, void* out, int* status,
                        int* sched, cudaStream_t stream);
+// logits (ksplit <= 1), or ksplit partial sums at logits + s * T * E whose sum in order
+// s = 0, 1, ... is the logits (bias in partial 0).  gating_splits picks ksplit.
 cudaError_t gemm_gating(const void* x, const void* w_split, const float* bias, long long T, int H, int E,
-                        float* logits, int* status, int* sched, cudaStream_t stream);
+                        float* logits, int ksplit, int* status, int* sched, cudaStream_t stream);
+int gating_splits(long long T, int H, int E, int sms);
+cudaError_t launch_sum_partials(const float* partials, int nsplit, long long n, float* out, cudaStream_t stream);
 
-cudaError_t launch_route(const float* logits, long long T, int E, int K, int renormalize, int P, int group_limit,
-                         int32_t* ids, float* w, cudaStream_t stream);
+// With nsplit > 1 the logits are the in-order sum of nsplit partial planes (T * E apart) starting
+// at `logits`; the kernel writes that sum to `logits_out` as well.
+cudaError_t launch_route(const float* logits, int nsplit, float* logits_out, long long T, int E, int K,
+                         int renormalize, int P, int group_limit, int32_t* ids, float* w, cudaStream_t stream);
 
 // Count/scan workspace: status word, grid-barrier words, per-block histograms.
 struct ScanWorkspace {

@@ -40,7 +40,8 @@ __device__ __forceinline__ float key_value(uint32_t k) {
 constexpr int kRouteWarps = 8;
 
 template <int VPL>
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, long long T, int E, int K,
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int nsplit,
+                                                    float* __restrict__ logits_out, long long T, int E, int K,
                                                     int renormalize, int P, int M, int32_t* __restrict__ ids,
                                                     float* __restrict__ w) {
   // node-limited routing: best expert key of each group, then the kept groups (per warp)
@@ -62,7 +63,12 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
       const int e = lane + 32 * i;
       key[i] = 0ull;
       if (e < E) {
-        const float v = __ldg(row + e);
+        float v = __ldg(row + e);
+        if (nsplit > 1) {  // split gating reduction: partial sums added in split order
+          const long long plane = T * E;
+          for (int p = 1; p < nsplit; ++p) v += __ldg(row + p * plane + e);
+          logits_out[t * E + e] = v;
+        }
         key[i] = (static_cast<unsigned long long>(order_key(v)) << 32) | static_cast<uint32_t>(~e);
       }
     }
@@ -137,8 +143,9 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
     if (renormalize) {
       den = num;
     } else {
-      const float* r = row;
-      for (int e = lane; e < E; e += 32) den += expf(__ldg(r + e) - top);
+      // the lane reads back only the logits it summed itself (same e = lane + 32 i)
+      const float* r = nsplit > 1 ? logits_out + t * E : row;
+      for (int e = lane; e < E; e += 32) den += expf(r[e] - top);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
@@ -150,11 +157,24 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 }
 
 template <int VPL>
-cudaError_t launch_route_vpl(const float* logits, long long T, int E, int K, int renorm, int P, int M, int32_t* ids,
-                             float* w, cudaStream_t s) {
+cudaError_t launch_route_vpl(const float* logits, int nsplit, float* logits_out, long long T, int E, int K,
+                             int renorm, int P, int M, int32_t* ids, float* w, cudaStream_t s) {
   const long long blocks = std::min<long long>((T + kRouteWarps - 1) / kRouteWarps, 64LL * num_sms());
   return launch_pdl(route_kernel<VPL>, dim3(static_cast<unsigned>(std::max<long long>(blocks, 1))),
-                    dim3(32 * kRouteWarps), 0, s, logits, T, E, K, renorm, P, M, ids, w);
+                    dim3(32 * kRouteWarps), 0, s, logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w);
+}
+
+// out[i] = sum_{p < nsplit} partials[p * n + i], added in order p = 0, 1, ...
+__global__ void sum_partials_kernel(const float* __restrict__ partials, int nsplit, long long n,
+                                    float* __restrict__ out) {
+  pdl_wait();
+  pdl_launch_dependents();
+  for (long long i = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    float v = partials[i];
+    for (int p = 1; p < nsplit; ++p) v += partials[p * n + i];
+    out[i] = v;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -351,16 +371,24 @@ size_t scan_smem_bytes(int E) { return static_cast<size_t>(E * 2 + 1 + kScanWarp
 
 }  // namespace
 
-cudaError_t launch_route(const float* logits, long long T, int E, int K, int renorm, int P, int M, int32_t* ids,
+cudaError_t launch_sum_partials(const float* partials, int nsplit, long long n, float* out, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  const long long blocks = std::min<long long>((n + 255) / 256, 8LL * num_sms());
+  return launch_pdl(sum_partials_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s, partials, nsplit, n,
+                    out);
+}
+
+cudaError_t launch_route(const float* logits, int nsplit, float* logits_out, long long T, int E, int K, int renorm,
+                         int P, int M, int32_t* ids,
                          float* w, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int vpl = (E + 31) / 32;
-  if (vpl <= 1) return launch_route_vpl<1>(logits, T, E, K, renorm, P, M, ids, w, s);
-  if (vpl <= 2) return launch_route_vpl<2>(logits, T, E, K, renorm, P, M, ids, w, s);
-  if (vpl <= 4) return launch_route_vpl<4>(logits, T, E, K, renorm, P, M, ids, w, s);
-  if (vpl <= 8) return launch_route_vpl<8>(logits, T, E, K, renorm, P, M, ids, w, s);
-  if (vpl <= 16) return launch_route_vpl<16>(logits, T, E, K, renorm, P, M, ids, w, s);
-  return launch_route_vpl<32>(logits, T, E, K, renorm, P, M, ids, w, s);
+  if (vpl <= 1) return launch_route_vpl<1>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
+  if (vpl <= 2) return launch_route_vpl<2>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
+  if (vpl <= 4) return launch_route_vpl<4>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
+  if (vpl <= 8) return launch_route_vpl<8>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
+  if (vpl <= 16) return launch_route_vpl<16>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
+  return launch_route_vpl<32>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
 }
 
 int scan_max_blocks(long long TK) {
