@@ -640,17 +640,22 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 #ifndef MOE_PAIR_BF16_NA
 #define MOE_PAIR_BF16_NA 2
 #endif
+#ifndef MOE_PAIR_BF16_KA
+#define MOE_PAIR_BF16_KA 2
+#endif
 template <int EPI>
 struct PairLayout {
   static constexpr int NT = 256;                                // tokens per pair tile (MMA N)
   static constexpr int NA = (EPI == kEpiBF16) ? MOE_PAIR_BF16_NA : 2;  // weight operands (accumulators)
-  static constexpr int STAGES = (NA == 1) ? 6 : 4;
+  static constexpr int KA = (NA == 1) ? MOE_PAIR_BF16_KA : 1;   // 128-byte K atoms per stage
+  static constexpr int STAGES = (NA == 1) ? 6 / KA : 4;
   static constexpr int EW = 8;                                  // epilogue warps per CTA
   static constexpr int kThr = 64 + 32 * EW;
   static constexpr int FEAT = (EPI == kEpiBF16) ? 256 * NA : 256;  // output features per pair tile
-  static constexpr int kAPair = NA * kABytes;                   // this CTA's 128-row weight boxes
-  static constexpr int kBBytes = (NT / 2) * 128;                // this CTA's token rows
-  static constexpr int kStageBytes = kAPair + kBBytes;
+  static constexpr int kAPair = NA * kABytes;                   // this CTA's 128-row weight boxes (one atom)
+  static constexpr int kBBytes = (NT / 2) * 128;                // this CTA's token rows (one atom)
+  static constexpr int kAtomBytes = kAPair + kBBytes;
+  static constexpr int kStageBytes = KA * kAtomBytes;
   static constexpr uint32_t kAccCols = NA * NT;                 // one tile's accumulators
   static constexpr int kNumAcc = (NA == 1) ? 2 : 1;             // TMEM buffers
   static constexpr uint32_t kTmemCols = kNumAcc * kAccCols;
@@ -695,7 +700,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int G = args.offsets ? args.G : 1;
   const int NFT = (args.N + L::FEAT - 1) / L::FEAT;
-  const int KB = (args.Kd + KS - 1) / KS;
+  const int KB = (args.Kd + KS * L::KA - 1) / (KS * L::KA);  // stages of KA atoms along K
 
   // Set-up that reads no global input runs before the wait on the previous kernel.
   if (threadIdx.x == 0) {
@@ -796,26 +801,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
             ok = false;
             break;
           }
-          uint8_t* st = ring + stage * L::kStageBytes;
           const uint32_t bar = full_leader + stage * 8;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kAPair + half * 128));
-          const int kx = kb * KS;
-          if constexpr (EPI == kEpiBF16) {
-            tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
-            if constexpr (NA == 2)
-              tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
-          } else {
-            const int fr = tl.n0 + 128 * static_cast<int>(rank);
-            tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
-            tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
-          }
-          int r = 0;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * L::KA * (L::kAPair + half * 128));
 #pragma unroll
-          for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
-            const int rows = 256 >> i;
-            if (half & rows) {
-              tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
-              r += rows;
+          for (int a = 0; a < L::KA; ++a) {  // a K atom beyond Kd reads the zero fill
+            uint8_t* st = ring + stage * L::kStageBytes + a * L::kAtomBytes;
+            const int kx = (kb * L::KA + a) * KS;
+            if constexpr (EPI == kEpiBF16) {
+              tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
+              if constexpr (NA == 2)
+                tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
+            } else {
+              const int fr = tl.n0 + 128 * static_cast<int>(rank);
+              tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
+              tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
+            }
+            int r = 0;
+#pragma unroll
+            for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
+              const int rows = 256 >> i;
+              if (half & rows) {
+                tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
+                r += rows;
+              }
             }
           }
           pend[stage] = true;
@@ -873,17 +881,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(ring + stage * L::kStageBytes);
-          const uint32_t sb = sa + L::kAPair;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
+          for (int a = 0; a < L::KA; ++a) {
+            const uint32_t sa = smem_u32(ring + stage * L::kStageBytes + a * L::kAtomBytes);
+            const uint32_t sb = sa + L::kAPair;
 #pragma unroll
-            for (int i = 0; i < NA; ++i) {
-              const uint64_t adesc = sw128_kmajor_desc(sa + i * kABytes + kk * 32);
-              const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
-              if constexpr (EPI == kEpiSwiGLUFp8) umma_e4m3_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
-              else umma_bf16_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
+#pragma unroll
+              for (int i = 0; i < NA; ++i) {
+                const uint64_t adesc = sw128_kmajor_desc(sa + i * kABytes + kk * 32);
+                const uint32_t accum = (kb > 0 || a > 0 || kk > 0) ? 1u : 0u;
+                if constexpr (EPI == kEpiSwiGLUFp8) umma_e4m3_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
+                else umma_bf16_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
+              }
             }
           }
           umma_commit_pair(smem_u32(&empty[stage]));  // both CTAs' stage buffers are free again
