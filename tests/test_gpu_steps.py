@@ -358,6 +358,27 @@ def test_grouped_gate_up_fp8_matches_oracle(E, H, F, rows, zipf, zf, gemm_kernel
     check_bf16("h", bits(h), rh)
 
 
+def test_grouped_gemm_schedule_rewinds_across_many_launches(gemm_kernel):
+    # every launch claims tiles from the workspace's per-call-site counter and the last CTA
+    # rewinds it: 40 launches in a row on one workspace give the same result every time
+    off, xp, wg, wu, wd = ffn_inputs(16, 512, 384, 3000, 1.1, 0.1, seed=3)
+    d = B.dims(T=3000, H=512, E=16, K=1, F=384)
+    ws = B.make_workspace(d)
+    offd, xpd, wgd, wud, wdd = (torch.from_numpy(off).to(DEV), xp.to(DEV), wg.to(DEV), wu.to(DEV), wd.to(DEV))
+    h = torch.zeros((3000, 384), dtype=torch.bfloat16, device=DEV)
+    y = torch.zeros((3000, 512), dtype=torch.bfloat16, device=DEV)
+    B.moe_grouped_ffn(xpd, offd, wgd, wud, wdd, d, h, y, ws)
+    first = y.clone()
+    for _ in range(40):
+        y.zero_()
+        B.moe_grouped_ffn(xpd, offd, wgd, wud, wdd, d, h, y, ws)
+    torch.cuda.synchronize()
+    assert B.read_device_status(ws) == 0
+    assert torch.equal(y.view(torch.int16), first.view(torch.int16))
+    sched = ws[160:256].view(torch.int32).cpu()
+    assert int(sched.abs().sum()) == 0          # every counter rewound to zero
+
+
 def test_pack_gate_up_layout():
     # packed rows [128 j, 128 j + 64) = gate rows [64 j, +64), next 64 = up rows; padding rows zero
     E, H, F = 3, 16, 136
