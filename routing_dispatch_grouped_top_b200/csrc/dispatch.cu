@@ -24,8 +24,20 @@ namespace moe {
 
 namespace {
 
+#ifndef MOE_COPY_UNROLL
+#define MOE_COPY_UNROLL 4
+#endif
+// Grid of the copy kernels: up to this many 256-thread blocks per SM.  Measured on B200 (Qwen3 /
+// DeepSeek-R1 layers): 8 -> 16 raised permute from 74 to 80 % and combine from 79 to 84 % of the
+// HBM copy bandwidth; 4, 32, and 2 or 8 loads in flight per thread were no better.
+#ifndef MOE_COPY_BLOCKS_PER_SM
+#define MOE_COPY_BLOCKS_PER_SM 16
+#endif
+#ifndef MOE_COMBINE_KC
+#define MOE_COMBINE_KC 4
+#endif
 constexpr int kCopyThreads = 256;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = MOE_COPY_UNROLL;   // independent 16-byte loads in flight per thread
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
@@ -306,7 +318,8 @@ __global__ void __launch_bounds__(kQuantThreads) permute_fp8_kernel(
 
 int copy_blocks(long long items) {
   const long long want = (items + kCopyThreads - 1) / kCopyThreads;
-  return static_cast<int>(std::max<long long>(1, std::min<long long>(want, 8LL * num_sms())));
+  return static_cast<int>(
+      std::max<long long>(1, std::min<long long>(want, static_cast<long long>(MOE_COPY_BLOCKS_PER_SM) * num_sms())));
 }
 
 }  // namespace
@@ -348,8 +361,9 @@ cudaError_t launch_combine(const void* y, const int32_t* roa, const float* w, co
   if (K <= 2)
     return launch_pdl(combine_kernel<2>, dim3(blocks), dim3(kCopyThreads), 0, s, reinterpret_cast<const uint4*>(y),
                       roa, w, reinterpret_cast<const uint4*>(shared), T, vpr, K, reinterpret_cast<uint4*>(out));
-  return launch_pdl(combine_kernel<4>, dim3(blocks), dim3(kCopyThreads), 0, s, reinterpret_cast<const uint4*>(y),
-                    roa, w, reinterpret_cast<const uint4*>(shared), T, vpr, K, reinterpret_cast<uint4*>(out));
+  return launch_pdl(combine_kernel<MOE_COMBINE_KC>, dim3(blocks), dim3(kCopyThreads), 0, s,
+                    reinterpret_cast<const uint4*>(y), roa, w, reinterpret_cast<const uint4*>(shared), T, vpr, K,
+                    reinterpret_cast<uint4*>(out));
 }
 
 cudaError_t launch_pack_gate_up(const void* w_gate, const void* w_up, int E, int H, int F, void* w_gu,
