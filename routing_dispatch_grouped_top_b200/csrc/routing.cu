@@ -239,6 +239,8 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
   for (int e = tid; e < E; e += kScanThreads) s_hist[e] = 0;
   for (int i = tid; i < kScanWarps * E; i += kScanThreads) s_wcnt[i] = 0;
   if (tid == 0) s_bad = 0;
+  pdl_wait();  // the expert ids come from the route kernel
+  pdl_launch_dependents();
   __syncthreads();
 
   // phase 1
@@ -421,10 +423,22 @@ cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, in
   unsigned int* bc = ws.bar_count;
   unsigned int* bg = ws.bar_gen;
   int* status = ws.status;
-  void* args[] = {&ids, &TKi, &E, &P, &chunki, &counts, &offsets, &part_counts, &part_offsets,
-                  &row_of_assign, &assign_of_row, &skew, &block_counts, &bc, &bg, &status};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<void*>(count_scan_kernel), dim3(blocks), dim3(kScanThreads),
-                                     args, smem, s);
+  // Cooperative (the grid barrier needs every block resident) and programmatic: the blocks may
+  // start while the route kernel drains and wait for it in griddepcontrol.wait.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(kScanThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr2[2];
+  attr2[0].id = cudaLaunchAttributeCooperative;
+  attr2[0].val.cooperative = 1;
+  attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr2[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr2;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, count_scan_kernel, ids, TKi, E, P, chunki, counts, offsets, part_counts,
+                            part_offsets, row_of_assign, assign_of_row, skew, block_counts, bc, bg, status);
 }
 
 cudaError_t launch_skew(const int32_t* counts, int E, float* ratio, cudaStream_t s) {
