@@ -16,16 +16,21 @@
 // costs nothing.  The instruction descriptor carries N, so it is chosen per
 // tile at run time.
 //
-// Roles (192 threads, one CTA per SM, persistent over a static tile order):
-//   warp 0      TMA producer: weight tile(s) 128 x 64 and token boxes (16..256) x 64,
-//               128-byte swizzle, into a STAGES-deep ring of shared memory;
+// Roles (persistent, one CTA per SM; two kernels, single-CTA and CTA-pair):
+//   warp 0      TMA producer: claims the next tile of the launch from a counter in
+//               the workspace (the last CTA rewinds it), publishes its id through a
+//               ring of tile ids in shared memory, and streams weight boxes of 128 or
+//               256 rows and token boxes of 16..256 rows (128-byte swizzle) into a
+//               STAGES-deep ring of shared memory;
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer;
-//   warps 2..5  epilogue: tcgen05.ld of the fp32 accumulator (each warp reads
-//               the TMEM lane quadrant warp % 4), activation, masked stores.
-// Accumulators are double-buffered in TMEM so the epilogue of tile i overlaps
-// the main loop of tile i + 1.  Tiles are ordered group-major, then weight tile,
-// then token chunk: CTAs working at the same time share weight and token tiles
-// through L2, so each expert's weights cross HBM about once.
+//   warps 2..   epilogue: tcgen05.ld of the fp32 accumulator (warp w reads the TMEM
+//               lane quadrant w % 4; with eight warps two share a quadrant and take
+//               alternate 32-token chunks), activation, and bf16 rows written through a
+//               per-warp shared-memory transpose as 16-byte pieces.
+// Tiles are numbered group-major, then weight tile, then token chunk, and claimed in
+// that order: CTAs working at the same time share weight and token tiles through L2,
+// so each expert's weights cross HBM about once, and SMs that draw short tiles take
+// more of them.
 #include <algorithm>
 #include <atomic>
 #include <mutex>
@@ -46,8 +51,6 @@ constexpr int kNumBoxes = 5;
 struct BoxMaps {
   CUtensorMap box[kNumBoxes];  // box[i] is (256 >> i) rows x 64 columns
 };
-constexpr int kThreads = 192;            // CTA-pair kernel: producer, MMA and 4 epilogue warps
-constexpr int kEpiThreads = 128;
 constexpr int kMaxThreads = 320;         // single-CTA kernel with 8 epilogue warps
 constexpr int kMaxGroups = MOE_MAX_E;
 constexpr int kRing = 8;                 // tile ids in flight from the producer to the MMA and epilogue warps
