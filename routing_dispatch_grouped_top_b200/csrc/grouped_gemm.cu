@@ -1222,14 +1222,14 @@ cudaError_t gemm_dense(const void* a, const void* w, long long M, int N, int Kd,
 
 // logits[T][E] = x[T][H] (hi + mid + lo)^T (+ bias), fp32 out; w_split is [3][E][H] bf16.
 // Splits of the gating reduction: enough work units to fill the SMs when the output has few
-// tiles (Qwen3 layer: 32 tiles of 128 tokens x 128 experts over 148 SMs -> 4 splits), at least
-// 4 K-steps per split, at most 8 splits.
+// tiles (Qwen3 layer: 32 tiles of 128 tokens x 128 experts over 148 SMs -> 4 splits; a
+// DeepSeek-R1 decode step: 2 tiles -> 28 splits), at least 4 K-steps per split, at most 32.
 int gating_splits(long long T, int H, int E, int sms) {
   const long long units = ((T + 127) / 128) * ((E + 127) / 128);
   const int KB = (H + kBK - 1) / kBK;
   if (units <= 0) return 1;
   long long s = sms / units;
-  s = std::min<long long>(s, std::min(8, KB / 4));
+  s = std::min<long long>(s, std::min(32, KB / 4));
   return static_cast<int>(std::max<long long>(1, s));
 }
 
