@@ -57,6 +57,29 @@ def test_argument_errors_are_synchronous(lib):
         assert lib.moe_status_str(s)
 
 
+def test_option_fields_are_validated_on_the_host(lib):
+    ok = dict(T=8, H=64, E=8, K=2, F=64, P=4)
+    assert binding.workspace_bytes(binding.dims(**ok, fp8_dispatch=True)) > 0
+    fp8_odd = binding.dims(T=8, H=72, E=8, K=2, F=64, fp8_dispatch=True)     # E4M3 rows need H % 16 == 0
+    assert lib.moe_route(None, C.byref(fp8_odd), None, None, None) == 2
+    bad_flag = binding.dims(**ok)
+    bad_flag.fp8_dispatch = 2
+    assert lib.moe_route(None, C.byref(bad_flag), None, None, None) == 1
+    assert binding.workspace_bytes(binding.dims(**ok, group_limit=5)) == 0      # M > P
+    assert binding.workspace_bytes(binding.dims(**dict(ok, K=5), group_limit=1)) == 0  # K > M * E / P
+    assert binding.workspace_bytes(binding.dims(**ok, F_shared=12)) == 0       # F_shared % 8 != 0
+
+
+def test_gating_partials_enlarge_the_workspace(lib):
+    # a layer whose router output has few tiles splits the gating reduction and keeps the
+    # partial logits in the workspace (Qwen3 layer: 4 splits of T x E fp32)
+    from routing_dispatch_grouped_top_b200.config import QWEN3_30B_A3B_PREFILL as q
+    d = binding.dims_of(q)
+    d_r1 = binding.dims_of(ALL["deepseek_r1_prefill_T8192_H7168_E256_K8_F2048_P8"])
+    assert binding.workspace_bytes(d) >= 4 * q.T * q.E * 4
+    assert binding.workspace_bytes(d_r1) < q.T * q.E * 4 * 4   # 128 router tiles: no split
+
+
 @pytest.mark.parametrize("n", [1, 2, 19, 20, 21, 100, 101])
 def test_p95_host_helper_matches_oracle(lib, n):
     r = np.random.default_rng(n).uniform(1, 6, n).astype(np.float32)
