@@ -99,9 +99,10 @@ typedef enum moe_status {
  * time.  Returns 0 for an invalid shape. */
 size_t moe_workspace_bytes(const moe_dims* d);
 
-/* Clears the workspace's status word and the count/scan kernel's grid-barrier
- * counters (an async memset on `stream`).  Call once after allocating the
- * workspace, and again after a device-side error has been reported. */
+/* Clears the workspace's 256-byte header: the status word, the count/scan kernel's
+ * grid-barrier counters and the grouped GEMMs' tile-schedule counters (an async memset
+ * on `stream`).  Call once after allocating the workspace, and again after a
+ * device-side error has been reported. */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronizes `stream`, then copies the workspace status word to *status
@@ -126,7 +127,9 @@ moe_status moe_pack_router(const float* w_g, const moe_dims* d, void* w_g_split,
 /* logits[t][e] = sum_h x[t][h] * W_g[h][e] (+ bias[e]), fp32 out [T][E].
  * x: [T][H] bf16.  w_g_split: from moe_pack_router.  bias: [E] fp32 or NULL.
  * Tensor-core products of the exact bf16 x with the three bf16 planes,
- * accumulated in fp32. */
+ * accumulated in fp32.  When [T][E] has few 128 x 128 tiles the reduction over H is
+ * split (up to 32 parts) into partial logits in the workspace, added in split order;
+ * the workspace of moe_workspace_bytes(d) bytes holds them. */
 moe_status moe_gating(const void* x, const void* w_g_split, const float* bias,
                       const moe_dims* d, float* logits, void* ws, size_t ws_bytes, void* stream);
 
@@ -232,8 +235,9 @@ moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_
  * it is read on the device, so launch shapes never depend on the counts.
  * Experts with no rows cost nothing.  H and F must be multiples of 8.  Offsets
  * that decrease or leave [0, TK] set MOE_DEV_BAD_INDEX and the call computes
- * nothing.  The GEMM calls use only the workspace's status word; any workspace
- * of moe_workspace_bytes(d) bytes serves (moe_dense needs 256 bytes). */
+ * nothing.  The GEMM calls use only the workspace's 256-byte header (status word and
+ * tile-schedule counters); any workspace of moe_workspace_bytes(d) bytes serves
+ * (moe_dense needs 256 bytes). */
 moe_status moe_grouped_ffn(const void* xp, const int32_t* offsets, const void* w_gate,
                            const void* w_up, const void* w_down, const moe_dims* d,
                            void* h, void* y, void* ws, size_t ws_bytes, void* stream);
