@@ -125,6 +125,12 @@ moe_status check_ws(const void* ws, size_t ws_bytes, const moe_dims* d) {
   return MOE_OK;
 }
 
+// The grouped GEMMs use only the workspace header (status word and tile-schedule counters).
+moe_status check_ws_header(const void* ws, size_t ws_bytes) {
+  if (!ws || ws_bytes < kWsHeader || reinterpret_cast<uintptr_t>(ws) % 256 != 0) return MOE_ERR_WORKSPACE;
+  return MOE_OK;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -252,7 +258,7 @@ moe_status moe_grouped_gate_up_fp8(const void* xq, const float* xs, const int32_
                                    const void* wq_up, const float* s_gate, const float* s_up, const moe_dims* d,
                                    void* h, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(common_checks(d));
-  MOE_TRY(check_ws(ws, ws_bytes, d));
+  MOE_TRY(check_ws_header(ws, ws_bytes));
   if (d->H % 16 != 0) return MOE_ERR_UNSUPPORTED_SHAPE;
   if (d->T == 0) return MOE_OK;
   if (!xq || !xs || !offsets || !wq_gate || !wq_up || !s_gate || !s_up || !h) return MOE_ERR_INVALID_ARG;
@@ -265,7 +271,7 @@ moe_status moe_grouped_gate_up_fp8(const void* xq, const float* xs, const int32_
 moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up,
                                const moe_dims* d, void* h, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(common_checks(d));
-  MOE_TRY(check_ws(ws, ws_bytes, d));
+  MOE_TRY(check_ws_header(ws, ws_bytes));
   if (d->T == 0) return MOE_OK;
   if (!xp || !offsets || !w_gate || !w_up || !h) return MOE_ERR_INVALID_ARG;
   if (!aligned16(xp) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
@@ -288,7 +294,7 @@ moe_status moe_pack_gate_up(const void* w_gate, const void* w_up, const moe_dims
 moe_status moe_grouped_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, const moe_dims* d,
                                       void* h, void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(common_checks(d));
-  MOE_TRY(check_ws(ws, ws_bytes, d));
+  MOE_TRY(check_ws_header(ws, ws_bytes));
   if (d->T == 0) return MOE_OK;
   if (!xp || !offsets || !w_gu || !h) return MOE_ERR_INVALID_ARG;
   if (!aligned16(xp) || !aligned16(w_gu) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
@@ -299,7 +305,7 @@ moe_status moe_grouped_gate_up_packed(const void* xp, const int32_t* offsets, co
 moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w_down, const moe_dims* d, void* y,
                             void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(common_checks(d));
-  MOE_TRY(check_ws(ws, ws_bytes, d));
+  MOE_TRY(check_ws_header(ws, ws_bytes));
   if (d->T == 0) return MOE_OK;
   if (!h || !offsets || !w_down || !y) return MOE_ERR_INVALID_ARG;
   if (!aligned16(h) || !aligned16(w_down) || !aligned16(y)) return MOE_ERR_INVALID_ARG;
