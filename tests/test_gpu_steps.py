@@ -379,6 +379,23 @@ def test_grouped_gemm_schedule_rewinds_across_many_launches(gemm_kernel):
     assert int(sched.abs().sum()) == 0          # every counter rewound to zero
 
 
+def test_grouped_gemms_run_on_a_header_only_workspace():
+    # the GEMM calls use only the 256-byte workspace header (status, tile-schedule counters)
+    off, xp, wg, wu, wd = ffn_inputs(4, 256, 128, 300, None, 0.0, seed=7)
+    d = B.dims(T=300, H=256, E=4, K=1, F=128)
+    ws = torch.empty(256, dtype=torch.uint8, device=DEV)
+    B.workspace_init(ws)
+    h = torch.zeros((300, 128), dtype=torch.bfloat16, device=DEV)
+    y = torch.zeros((300, 256), dtype=torch.bfloat16, device=DEV)
+    B.moe_grouped_ffn(xp.to(DEV), torch.from_numpy(off).to(DEV), wg.to(DEV), wu.to(DEV), wd.to(DEV), d, h, y, ws)
+    assert B.read_device_status(ws) == 0
+    rh, ry = oracle.grouped_ffn(bits(xp), off, bits(wg), bits(wu), bits(wd))
+    check_bf16("y", bits(y), ry)
+    with pytest.raises(B.MoEError):
+        B.moe_grouped_ffn(xp.to(DEV), torch.from_numpy(off).to(DEV), wg.to(DEV), wu.to(DEV), wd.to(DEV), d, h, y,
+                          ws[:128])
+
+
 def test_pack_gate_up_layout():
     # packed rows [128 j, 128 j + 64) = gate rows [64 j, +64), next 64 = up rows; padding rows zero
     E, H, F = 3, 16, 136
