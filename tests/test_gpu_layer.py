@@ -215,6 +215,31 @@ def test_layer_matches_oracle(cfg, gemm_kernel):
     assert float(g["skew"].item()) == pytest.approx(oracle.skew_ratio(cpu(g["counts"])), rel=1e-6)
 
 
+def test_layer_with_no_tokens_enqueues_nothing_and_reports_ok():
+    cfg = TINY.with_(name="no_tokens", T=0)
+    d = B.dims_of(cfg)
+    inp = inputs.make_layer(TINY, DEV)
+    w = B.pack_layer_weights(d, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"])
+    bufs = B.alloc_layer_buffers(d)
+    ws = B.make_workspace(d)
+    B.moe_layer_forward(torch.empty((0, cfg.H), dtype=torch.bfloat16, device=DEV), w, d, bufs, ws)
+    assert B.read_device_status(ws) == 0
+    assert torch.equal(bufs["offsets"].cpu(), torch.zeros(cfg.E + 1, dtype=torch.int32))
+    assert float(bufs["skew"].item()) == 0.0
+
+
+def test_layer_with_a_single_expert_is_one_dense_ffn():
+    # E = K = 1: every token goes to the one expert with weight 1, so the layer is that expert's FFN
+    cfg = TINY.with_(name="single_expert", T=200, E=1, K=1, P=1)
+    inp = inputs.make_layer(cfg, DEV)
+    g = run_gpu_layer(cfg, inp)
+    assert torch.equal(g["topk_ids"].cpu(), torch.zeros((cfg.T, 1), dtype=torch.int32))
+    assert torch.all(g["topk_w"] == 1.0)
+    assert torch.equal(g["row_of_assign"].cpu(), torch.arange(cfg.T, dtype=torch.int32))
+    h, y = oracle.ffn_rows(bits(inp["x"]), bits(inp["w_gate"][0]), bits(inp["w_up"][0]), bits(inp["w_down"][0]))
+    check_bf16("out", bits(g["out"]), y)
+
+
 def test_layer_forward_host_io_matches_device_call():
     cfg = TINY.with_(T=200, name="tiny_T200")
     inp = inputs.make_layer(cfg, DEV)
