@@ -411,7 +411,9 @@ typedef struct moe_layer_buffers {
 /* Number of stage boundaries recorded when stage events are given. */
 #define MOE_NUM_STAGE_EVENTS 10
 
-/* Runs every step on `stream` in pipeline order: [latent down-projection] ->
+/* With d->T = 0 only counts, offsets, part_counts, part_offsets (all set to zero) and skew
+ * (set to 0) are written; the other pointers may be NULL.
+ * Runs every step on `stream` in pipeline order: [latent down-projection] ->
  * gating -> route -> count/scan -> permute -> gate/up+SwiGLU -> down -> combine
  * -> [latent up-projection] -> skew statistics.  With d->fp8_dispatch the permute is
  * moe_permute_fp8 (into b->xq, b->xs; b->xp may be NULL) and gate/up runs on

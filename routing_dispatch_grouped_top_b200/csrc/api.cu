@@ -359,6 +359,15 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
                              void* stream) {
   MOE_TRY(common_checks(d));
   MOE_TRY(check_ws(ws, ws_bytes, d));
+  if (d->T == 0) {
+    // No tokens: only the per-expert outputs exist, all zero (count/scan of no assignments).
+    if (!b || !b->counts || !b->offsets || !b->part_counts || !b->part_offsets) return MOE_ERR_INVALID_ARG;
+    cudaStream_t s0 = as_stream(stream);
+    for (int i = 0; stage_events && i < MOE_NUM_STAGE_EVENTS; ++i)
+      if (stage_events[i]) MOE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(stage_events[i]), s0));
+    return cuda_status(launch_count_scan(nullptr, 0, d->E, d->P, b->counts, b->offsets, b->part_counts,
+                                         b->part_offsets, nullptr, nullptr, b->skew, scan_ws(ws, d), s0));
+  }
   if (!x || !w || !b) return MOE_ERR_INVALID_ARG;
   const bool latent = d->d_model > 0;
   const bool fp8 = d->fp8_dispatch != 0;
@@ -460,6 +469,7 @@ moe_status moe_layer_forward_host(const void* x_host, void* x_dev, const moe_lay
                                   const moe_layer_buffers* b, void* ws, size_t ws_bytes, void* out_host,
                                   void* stream) {
   MOE_TRY(common_checks(d));
+  if (d->T == 0) return moe_layer_forward(x_dev, w, d, b, ws, ws_bytes, nullptr, stream);
   if (!x_host || !x_dev || !out_host || !b) return MOE_ERR_INVALID_ARG;
   const bool latent = d->d_model > 0;
   const size_t d_in = latent ? d->d_model : d->H;
