@@ -328,7 +328,7 @@ def run_reference(args, cfg):
     steps = []
     for _ in range(args.warmup):
         cpu_oracle_rate(cfg, 0.0)
-    rates = [cpu_oracle_rate(cfg, max(1.0, args.cpu_seconds / max(args.steps, 1))) for _ in range(args.steps)]
+    rates = [cpu_oracle_rate(cfg, max(0.5, args.cpu_seconds / max(args.steps, 1))) for _ in range(args.steps)]
     val = statistics.mean(r["value"] for r in rates)
     cb = dict(rates[-1])
     cb["value"] = val
