@@ -64,12 +64,12 @@ struct Cfg;
 // FEAT output features per tile.  Accumulators are double-buffered in TMEM when two fit
 // in its 512 columns (the epilogue of one tile then overlaps the next tile's main loop).
 //
-// Measured on B200: the per-SM rate at which TMA can fill shared memory, not the MMA,
-// bounds these kernels; a 128 x 256 tile needs 48 KB per 542 MMA cycles.  The bf16
-// kernel therefore uses 256 x 256 tiles (two 128-row weight tiles, 42 B per MMA cycle),
-// single-buffered, which measured 15-30 % faster than 128 x 256 on every workload.  For
-// SwiGLU the same widening was slower (its epilogue is heavier and no longer overlapped),
-// so it keeps 128 x (128 gate + 128 up) tiles with double-buffered accumulators.
+// Measured on B200: the MMA itself runs at its full rate (128 cycles per 128 x 256 x 16
+// bf16 MMA, with a commit every 8), and the shared-memory fill per MMA cycle is what these
+// kernels trade against the TMEM budget: 256-token tiles (two 128-row weight tiles and a
+// 256-row token tile per stage, single-buffered accumulators) beat 128-token tiles with
+// double-buffered accumulators on every layer workload once the epilogue stores were
+// vectorised (Qwen3 gate/up 253 -> 214 us).
 // Build-time tuning: token columns of the separate-weight SwiGLU tiles (128: double-buffered
 // accumulators, 4 stages; 256: single-buffered, 3 stages) and epilogue warps (4 or 8: two
 // warps per TMEM lane quadrant split a tile's token chunks).
