@@ -156,10 +156,24 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
 
 
+def code_fingerprint(path: str) -> str:
+    """sha256[:12] of a CUDA source with its // comments and blank lines removed: a comment
+    edit keeps the fingerprint, any change to the code changes it."""
+    import hashlib
+    lines = []
+    for ln in open(path, encoding="utf-8"):
+        cut = ln.find("//")
+        if cut >= 0 and ln[:cut].count('"') % 2 == 0:
+            ln = ln[:cut]
+        ln = ln.rstrip()
+        if ln:
+            lines.append(ln)
+    return hashlib.sha256("\n".join(lines).encode()).hexdigest()[:12]
+
+
 def kernel_traffic(workload: str, stage: str):
     """DRAM bytes per launch of one kernel from a committed ncu summary, or None when the
-    kernel source changed since the counters were taken (the summary records its hash)."""
-    import hashlib
+    kernel's code changed since the counters were taken (the summary records its fingerprint)."""
     path = os.path.join(ROOT, "profiles", "dram_traffic.txt")
     if not os.path.exists(path):
         return None
@@ -169,8 +183,7 @@ def kernel_traffic(workload: str, stage: str):
             src = os.path.join(ROOT, "routing_dispatch_grouped_top_b200", "csrc", f[3].split(":")[0])
             if not os.path.exists(src):
                 return None
-            h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:12]
-            return float(f[2]) if h == f[3].split(":")[1] else None
+            return float(f[2]) if code_fingerprint(src) == f[3].split(":")[1] else None
     return None
 
 
