@@ -132,7 +132,7 @@ def f64_to_bf16_bits(v) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------
-# Step S0: gating logits   [WideEP/router]: "computes the gating scores"
+# Step S0: gating logits   [WideEP/router]: the sending rank scores every expert per token
 # ----------------------------------------------------------------------------
 
 def gating_logits(x_bits, w_g, bias=None) -> np.ndarray:
