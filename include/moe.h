@@ -273,9 +273,9 @@ moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w
 
 /* ------------------------------------------------------------------------- */
 /* FP8 dispatch: E4M3 rows with one fp32 scale per row, gate/up on E4M3,     */
-/* bf16 down projection and combine.  A runtime may quantize the outbound   */
-/* activation, carry its scales, compute in the other format and return at  */
-/* higher precision (WideEP essay, "Top-k multiplies traffic. Locality      */
+/* bf16 down projection and combine.  The rows sent to the experts may be  */
+/* narrowed to a low-precision format with their scales alongside and the   */
+/* result widened again (WideEP essay, "Top-k multiplies traffic. Locality  */
 /* subtracts it."); the change alters values, so it belongs to the bucket   */
 /* that needs a task-level evaluation before release ("Three Parameter      */
 /* Counts...", "Which optimizations need a task-level gate").                */

@@ -38,8 +38,8 @@ and section:
   "Definition" and "Current Synthesis": experts receive a narrower, projected
   hidden state.
 * [ParamCounts/layout]  "Three Parameter Counts...", section "Halving top-k is
-  a network change first": DeepSeek-V3's node-limited routing bounds how many
-  nodes (expert groups) one token's experts may span.
+  a network change first": in DeepSeek-V3 the set of nodes (expert groups) a
+  token's experts may come from is capped by the trained router itself.
 
 Readings where the pages are silent:
 

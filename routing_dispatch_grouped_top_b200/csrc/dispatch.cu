@@ -211,8 +211,8 @@ __global__ void pack_gate_up_kernel(const uint4* __restrict__ wg, const uint4* _
 }
 
 // ---------------------------------------------------------------------------
-// FP8 (E4M3) rows with one fp32 scale per row.  Low-precision dispatch quantizes the
-// outbound activation and carries its scales (WideEP essay, "Top-k multiplies traffic.
+// FP8 (E4M3) rows with one fp32 scale per row.  Low-precision dispatch narrows each row sent
+// to the experts and sends its scale with it (WideEP essay, "Top-k multiplies traffic.
 // Locality subtracts it.").  s = amax / 448 (1 for an all-zero row), code = E4M3 of x / s
 // (IEEE fp32 division, round to nearest even, saturating): both are decided in fp32.
 // One block per row: the first pass reduces |x| to amax, the second (an L1/L2 hit)
