@@ -18,68 +18,102 @@ namespace moe {
 namespace {
 
 // ---------------------------------------------------------------------------
-// Top-K: one warp per token.  Each lane holds logits e = lane + 32 i.  A logit
-// becomes a 64-bit key: high word = order-preserving image of the float (NaN ->
-// 0, the lowest; -0.0 folded into +0.0), low word = ~e so that equal values
-// prefer the lower expert id.  K rounds of (lane-local max, warp max by
-// butterfly shuffles, the winner's slot is cleared).
+// Top-K: one warp per token.  Lane l owns experts e = l + 32 i (i < VPL).  Each
+// logit becomes a 32-bit order key: the order-preserving image of the float
+// (-0.0 folded into +0.0), 1 for NaN (below every number) and 0 for an empty or
+// retired slot.  The warp keeps the keys of its token in shared memory and each
+// lane its best (key, i), ties to the lower i.  A round takes the warp maximum of
+// the lanes' best keys and, among the lanes holding it, the lowest expert id
+// (two warp reductions), so equal values prefer the lower expert id.  The winner's
+// slot is cleared and its owner's best is rebuilt by the whole warp: lane j reads
+// the owner's slot j, two more reductions give the new best.  Slot w + 32 j is
+// only ever read or written by lane j during the rounds.
 // ---------------------------------------------------------------------------
 
 __device__ __forceinline__ uint32_t order_key(float v) {
-  if (v != v) return 0u;   // NaN ranks below every number
+  if (v != v) return 1u;    // NaN ranks below every number, above an empty slot
   if (v == 0.0f) v = 0.0f;  // -0.0 == +0.0
   const uint32_t u = __float_as_uint(v);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);  // -inf -> 0x007fffff > 1
 }
 
 __device__ __forceinline__ float key_value(uint32_t k) {
-  if (k == 0u) return __uint_as_float(0x7fc00000u);
+  if (k <= 1u) return __uint_as_float(0x7fc00000u);
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
 }
 
-constexpr int kRouteWarps = 8;
+// Warps per block: the per-warp key rows grow with VPL.
+constexpr int route_warps(int vpl) { return vpl <= 8 ? 8 : 4; }
 
 template <int VPL>
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int nsplit,
-                                                    float* __restrict__ logits_out, long long T, int E, int K,
-                                                    int renormalize, int P, int M, int32_t* __restrict__ ids,
-                                                    float* __restrict__ w) {
+__global__ void __launch_bounds__(32 * route_warps(VPL)) route_kernel(
+    const float* __restrict__ logits, int nsplit, float* __restrict__ logits_out, long long T, int E, int K,
+    int renormalize, int P, int M, int32_t* __restrict__ ids, float* __restrict__ w) {
+  constexpr int W = route_warps(VPL);
+  constexpr unsigned kFull = 0xffffffffu;
+  __shared__ uint32_t s_key[W][32 * VPL];
   // node-limited routing: best expert key of each group, then the kept groups (per warp)
-  __shared__ unsigned long long s_gkey[kRouteWarps][MOE_MAX_LIMITED_GROUPS];
-  __shared__ unsigned char s_kept[kRouteWarps][MOE_MAX_LIMITED_GROUPS];
+  __shared__ unsigned long long s_gkey[W][MOE_MAX_LIMITED_GROUPS];
+  __shared__ unsigned char s_kept[W][MOE_MAX_LIMITED_GROUPS];
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
   const bool limited = M > 0 && M < P;
   const int epp = E / P;
+  uint32_t* sk = s_key[wib];
   pdl_wait();  // logits come from the previous kernel
   pdl_launch_dependents();
-  const long long warps = static_cast<long long>(gridDim.x) * (blockDim.x >> 5);
-  for (long long t = static_cast<long long>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T;
-       t += warps) {
+  const long long warps = static_cast<long long>(gridDim.x) * W;
+  for (long long t = static_cast<long long>(blockIdx.x) * W + wib; t < T; t += warps) {
     const float* row = logits + t * E;
-    unsigned long long key[VPL];
+    float v[VPL];
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
       const int e = lane + 32 * i;
-      key[i] = 0ull;
-      if (e < E) {
-        float v = __ldg(row + e);
-        if (nsplit > 1) {  // split gating reduction: partial sums added in split order
-          const long long plane = T * E;
-          for (int p = 1; p < nsplit; ++p) v += __ldg(row + p * plane + e);
-          logits_out[t * E + e] = v;
+      v[i] = (e < E) ? __ldg(row + e) : 0.0f;
+    }
+    if (nsplit > 1) {
+      // Split gating reduction: partial sums added in split order.  The loads of
+      // kSplitBatch splits are issued before their additions so that their
+      // latencies overlap (fewer splits per batch when each lane already holds
+      // many experts); the additions keep the order p = 1, 2, ...
+      constexpr int kSplitBatch = VPL <= 4 ? 4 : (VPL <= 8 ? 2 : 1);
+      const long long plane = T * E;
+      for (int p0 = 1; p0 < nsplit; p0 += kSplitBatch) {
+        float part[kSplitBatch][VPL];
+#pragma unroll
+        for (int q = 0; q < kSplitBatch; ++q) {
+#pragma unroll
+          for (int i = 0; i < VPL; ++i) {
+            const int e = lane + 32 * i;
+            part[q][i] = (p0 + q < nsplit && e < E) ? __ldg(row + (p0 + q) * plane + e) : 0.0f;
+          }
         }
-        key[i] = (static_cast<unsigned long long>(order_key(v)) << 32) | static_cast<uint32_t>(~e);
+#pragma unroll
+        for (int q = 0; q < kSplitBatch; ++q) {
+          if (p0 + q < nsplit) {
+#pragma unroll
+            for (int i = 0; i < VPL; ++i) v[i] += part[q][i];
+          }
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) logits_out[t * E + e] = v[i];
       }
     }
-    // Every real candidate has key > 0 (low word ~e != 0), padding has key 0.
+    uint32_t hk[VPL];
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) hk[i] = (lane + 32 * i < E) ? order_key(v[i]) : 0u;
     if (limited) {
+      // group key = (order key, ~e): a group ranks by its best expert, ties to the lower id
       for (int g = lane; g < P; g += 32) s_gkey[wib][g] = 0ull;
       __syncwarp();
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < E) atomicMax(&s_gkey[wib][e / epp], key[i]);
+        if (e < E)
+          atomicMax(&s_gkey[wib][e / epp], (static_cast<unsigned long long>(hk[i]) << 32) | static_cast<uint32_t>(~e));
       }
       __syncwarp();
       // M rounds of warp arg-max over the group keys; lane owns groups lane + 32 j
@@ -97,7 +131,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
         for (int j = 0; j < GPL; ++j) best = gk[j] > best ? gk[j] : best;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
-          const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+          const unsigned long long other = __shfl_xor_sync(kFull, best, o);
           best = other > best ? other : best;
         }
 #pragma unroll
@@ -112,32 +146,39 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < E && !s_kept[wib][e / epp]) key[i] = 0ull;  // experts of dropped groups leave the race
+        if (e < E && !s_kept[wib][e / epp]) hk[i] = 0u;  // experts of dropped groups leave the race
       }
-      __syncwarp();
     }
+    // Every real candidate has key >= 1; empty slots have 0.  K <= number of candidates.
+    uint32_t bh = 0u;
+    int bi = 0;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      sk[lane + 32 * i] = hk[i];
+      if (hk[i] > bh) bh = hk[i], bi = i;
+    }
+    __syncwarp();
     int my_id = 0;
-    float my_val = 0.0f;
+    uint32_t my_key = 0u;
     for (int k = 0; k < K; ++k) {
-      unsigned long long best = 0ull;
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) best = key[i] > best ? key[i] : best;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
-        best = other > best ? other : best;
+      const uint32_t m = __reduce_max_sync(kFull, bh);
+      const int e = __reduce_min_sync(kFull, bh == m ? lane + 32 * bi : 0x7fffffff);
+      if (lane == k) my_id = e, my_key = m;
+      // retire e; the owner's best is rebuilt over its remaining slots
+      const int owner = e & 31;
+      uint32_t x = 0u;
+      if (lane < VPL) {
+        x = sk[owner + 32 * lane];
+        if (owner + 32 * lane == e) sk[e] = x = 0u;
       }
-      const int e = static_cast<int>(~static_cast<uint32_t>(best));
-      // Keys are unique (the low word is the id): the owner of the winner retires it.
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) key[i] = (key[i] == best) ? 0ull : key[i];
-      if (lane == k) {
-        my_id = e;
-        my_val = key_value(static_cast<uint32_t>(best >> 32));
-      }
+      const uint32_t nm = __reduce_max_sync(kFull, x);
+      const int ni = __reduce_min_sync(kFull, (lane < VPL && x == nm) ? lane : 0x7fffffff);
+      if (lane == owner) bh = nm, bi = ni;
     }
+    __syncwarp();  // the next token's keys overwrite this token's slots
+    const float my_val = key_value(my_key);
     // Weights: exp(l_k - l_top) / (sum over the K selected, or over all E).
-    const float top = __shfl_sync(0xffffffffu, my_val, 0);
+    const float top = __shfl_sync(kFull, my_val, 0);
     const float num = (lane < K) ? expf(my_val - top) : 0.0f;
     float den = 0.0f;
     if (renormalize) {
@@ -148,7 +189,7 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
       for (int e = lane; e < E; e += 32) den += expf(r[e] - top);
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
+    for (int o = 16; o > 0; o >>= 1) den += __shfl_xor_sync(kFull, den, o);
     if (lane < K) {
       ids[t * K + lane] = my_id;
       w[t * K + lane] = num / den;
@@ -159,9 +200,10 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
 template <int VPL>
 cudaError_t launch_route_vpl(const float* logits, int nsplit, float* logits_out, long long T, int E, int K,
                              int renorm, int P, int M, int32_t* ids, float* w, cudaStream_t s) {
-  const long long blocks = std::min<long long>((T + kRouteWarps - 1) / kRouteWarps, 64LL * num_sms());
-  return launch_pdl(route_kernel<VPL>, dim3(static_cast<unsigned>(std::max<long long>(blocks, 1))),
-                    dim3(32 * kRouteWarps), 0, s, logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w);
+  constexpr int W = route_warps(VPL);
+  const long long blocks = std::min<long long>((T + W - 1) / W, 64LL * num_sms());
+  return launch_pdl(route_kernel<VPL>, dim3(static_cast<unsigned>(std::max<long long>(blocks, 1))), dim3(32 * W), 0,
+                    s, logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w);
 }
 
 // out[i] = sum_{p < nsplit} partials[p * n + i], added in order p = 0, 1, ...
@@ -255,18 +297,40 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
 
   if (!grid_barrier(bar_count, bar_gen, gridDim.x, status, &s_ok)) return;
 
-  // phase 2: column sums over blocks
+  // phase 2: column sums over blocks.  The block_counts rows start 16-byte aligned (the
+  // workspace is 256-byte aligned), so with E % 4 == 0 a thread sums four experts per
+  // 16-byte load and keeps eight loads in flight.
   int my_max = 0;
-  for (int e = tid; e < E; e += kScanThreads) {
-    int before = 0, total = 0;
-    for (int bb = 0; bb < static_cast<int>(gridDim.x); ++bb) {
-      const int c = __ldcg(block_counts + static_cast<long long>(bb) * E + e);
-      before += (bb < b) ? c : 0;
-      total += c;
+  const int nb = static_cast<int>(gridDim.x);
+  if ((E & 3) == 0) {
+    const int E4 = E >> 2;
+    for (int q = tid; q < E4; q += kScanThreads) {
+      const int4* col = reinterpret_cast<const int4*>(block_counts) + q;
+      int4 before = make_int4(0, 0, 0, 0), total = make_int4(0, 0, 0, 0);
+#pragma unroll 8
+      for (int bb = 0; bb < nb; ++bb) {
+        const int4 c = __ldcg(col + static_cast<long long>(bb) * E4);
+        if (bb < b) before.x += c.x, before.y += c.y, before.z += c.z, before.w += c.w;
+        total.x += c.x, total.y += c.y, total.z += c.z, total.w += c.w;
+      }
+      const int e = 4 * q;
+      s_hist[e] = before.x, s_hist[e + 1] = before.y, s_hist[e + 2] = before.z, s_hist[e + 3] = before.w;
+      s_off[e] = total.x, s_off[e + 1] = total.y, s_off[e + 2] = total.z, s_off[e + 3] = total.w;
+      my_max = max(my_max, max(max(total.x, total.y), max(total.z, total.w)));
     }
-    s_hist[e] = before;
-    s_off[e] = total;
-    my_max = max(my_max, total);
+  } else {
+    for (int e = tid; e < E; e += kScanThreads) {
+      int before = 0, total = 0;
+#pragma unroll 8
+      for (int bb = 0; bb < nb; ++bb) {
+        const int c = __ldcg(block_counts + static_cast<long long>(bb) * E + e);
+        before += (bb < b) ? c : 0;
+        total += c;
+      }
+      s_hist[e] = before;
+      s_off[e] = total;
+      my_max = max(my_max, total);
+    }
   }
   __syncthreads();
   // exclusive scan of s_off[0..E) in place (E <= 1024: 4 per thread)

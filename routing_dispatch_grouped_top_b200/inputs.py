@@ -127,6 +127,16 @@ def special_logits(T: int, E: int, seed: int = 0) -> torch.Tensor:
     return pool[idx]
 
 
+def nan_heavy_logits(T: int, E: int, frac: float = 0.8, seed: int = 0) -> torch.Tensor:
+    """Gaussian logits with a fraction `frac` replaced by NaN and every fifth row all NaN,
+    so that the top-K reaches into (and ties among) NaNs."""
+    g = _gen("cpu", seed)
+    l = torch.randn((T, E), generator=g, dtype=torch.float32)
+    drop = torch.rand((T, E), generator=g) < frac
+    drop[::5] = True
+    return torch.where(drop, torch.full_like(l, float("nan")), l)
+
+
 def quantized_logits(T: int, E: int, levels: int = 4, seed: int = 0) -> torch.Tensor:
     """Logits drawn from a few integer levels: every row is full of exact ties."""
     g = _gen("cpu", seed)

@@ -49,7 +49,8 @@ ROUTE_CASES = [  # T, E, K, renormalize, generator
     (300, 8, 2, True, "random"), (257, 128, 8, True, "random"), (100, 256, 8, False, "random"),
     (77, 896, 16, True, "random"), (64, 33, 5, True, "quantized"), (50, 1024, 32, True, "random"),
     (129, 64, 6, True, "special"), (40, 1000, 7, False, "quantized"), (1, 5, 5, True, "random"),
-    (0, 16, 4, True, "random"), (4096, 128, 8, True, "random"),
+    (0, 16, 4, True, "random"), (4096, 128, 8, True, "random"), (64, 64, 8, True, "nan_heavy"),
+    (40, 896, 16, False, "nan_heavy"), (33, 1024, 32, True, "nan_heavy"),
 ]
 
 
@@ -60,6 +61,8 @@ def test_route_matches_oracle(T, E, K, renorm, gen):
         l = inputs.random_logits(T, E, seed=seed, scale=2.0)
     elif gen == "quantized":
         l = inputs.quantized_logits(T, E, levels=5, seed=seed)
+    elif gen == "nan_heavy":
+        l = inputs.nan_heavy_logits(T, E, seed=seed)
     else:
         l = inputs.special_logits(T, E, seed=seed)
     d = B.dims(T=T, H=8, E=E, K=K, F=8, renormalize=renorm)
@@ -71,7 +74,7 @@ def test_route_matches_oracle(T, E, K, renorm, gen):
         return
     rid, rw = oracle.route(l.numpy(), K, renorm)
     assert np.array_equal(cpu(ids), rid)
-    if gen == "special":
+    if gen in ("special", "nan_heavy"):
         sel = np.take_along_axis(l.numpy(), rid, axis=1)
         ok_rows = np.all(np.isfinite(sel), axis=1) & np.all(np.isfinite(l.numpy()) | renorm, axis=1)
         np.testing.assert_allclose(cpu(w)[ok_rows], rw[ok_rows], atol=WEIGHT_ABS, rtol=0)
@@ -84,7 +87,7 @@ def test_route_matches_oracle(T, E, K, renorm, gen):
 LIMITED_CASES = [  # T, E, K, P, M, renormalize, generator
     (300, 256, 8, 8, 4, True, "random"), (200, 896, 16, 64, 8, True, "random"), (100, 16, 3, 4, 2, True, "quantized"),
     (129, 64, 6, 16, 3, False, "special"), (77, 1024, 8, 256, 4, True, "random"), (50, 32, 4, 32, 4, True, "random"),
-    (64, 48, 5, 6, 1, True, "quantized"),
+    (64, 48, 5, 6, 1, True, "quantized"), (60, 256, 8, 8, 4, True, "nan_heavy"),
 ]
 
 
@@ -93,7 +96,8 @@ def test_route_limited_matches_oracle(T, E, K, P, M, renorm, gen):
     seed = T + E + M
     l = {"random": lambda: inputs.random_logits(T, E, seed=seed, scale=2.0),
          "quantized": lambda: inputs.quantized_logits(T, E, levels=4, seed=seed),
-         "special": lambda: inputs.special_logits(T, E, seed=seed)}[gen]()
+         "special": lambda: inputs.special_logits(T, E, seed=seed),
+         "nan_heavy": lambda: inputs.nan_heavy_logits(T, E, seed=seed)}[gen]()
     d = B.dims(T=T, H=8, E=E, K=K, F=8, P=P, renormalize=renorm, group_limit=M)
     ids = torch.full((T, K), -7, dtype=torch.int32, device=DEV)
     w = torch.empty((T, K), dtype=torch.float32, device=DEV)
@@ -101,7 +105,7 @@ def test_route_limited_matches_oracle(T, E, K, P, M, renorm, gen):
     torch.cuda.synchronize()
     rid, rw = oracle.route_limited(l.numpy(), K, P, M, renorm)
     assert np.array_equal(cpu(ids), rid)
-    if gen != "special":
+    if gen not in ("special", "nan_heavy"):
         np.testing.assert_allclose(cpu(w), rw, atol=WEIGHT_ABS, rtol=0)
 
 
