@@ -51,9 +51,10 @@ __global__ void __launch_bounds__(32 * route_warps(VPL)) route_kernel(
     int renormalize, int P, int M, int32_t* __restrict__ ids, float* __restrict__ w) {
   constexpr int W = route_warps(VPL);
   constexpr unsigned kFull = 0xffffffffu;
-  __shared__ uint32_t s_key[W][32 * VPL];
-  // node-limited routing: best expert key of each group, then the kept groups (per warp)
-  __shared__ unsigned long long s_gkey[W][MOE_MAX_LIMITED_GROUPS];
+  __shared__ alignas(16) uint32_t s_key[W][32 * VPL];
+  // node-limited routing: each group's best key and expert, and the groups kept (per warp)
+  __shared__ uint32_t s_gh[W][MOE_MAX_LIMITED_GROUPS];
+  __shared__ int s_ge[W][MOE_MAX_LIMITED_GROUPS];
   __shared__ unsigned char s_kept[W][MOE_MAX_LIMITED_GROUPS];
   const int lane = threadIdx.x & 31;
   const int wib = threadIdx.x >> 5;
@@ -104,60 +105,71 @@ __global__ void __launch_bounds__(32 * route_warps(VPL)) route_kernel(
     }
     uint32_t hk[VPL];
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) hk[i] = (lane + 32 * i < E) ? order_key(v[i]) : 0u;
+    for (int i = 0; i < VPL; ++i) {
+      hk[i] = (lane + 32 * i < E) ? order_key(v[i]) : 0u;
+      sk[lane + 32 * i] = hk[i];
+    }
+    __syncwarp();
     if (limited) {
-      // group key = (order key, ~e): a group ranks by its best expert, ties to the lower id
-      for (int g = lane; g < P; g += 32) s_gkey[wib][g] = 0ull;
-      __syncwarp();
-#pragma unroll
-      for (int i = 0; i < VPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E)
-          atomicMax(&s_gkey[wib][e / epp], (static_cast<unsigned long long>(hk[i]) << 32) | static_cast<uint32_t>(~e));
-      }
-      __syncwarp();
-      // M rounds of warp arg-max over the group keys; lane owns groups lane + 32 j
-      constexpr int GPL = MOE_MAX_LIMITED_GROUPS / 32;
-      unsigned long long gk[GPL];
-#pragma unroll
-      for (int j = 0; j < GPL; ++j) {
-        const int g = lane + 32 * j;
-        gk[j] = g < P ? s_gkey[wib][g] : 0ull;
-        if (g < P) s_kept[wib][g] = 0;
-      }
-      for (int m = 0; m < M; ++m) {
-        unsigned long long best = 0ull;
-#pragma unroll
-        for (int j = 0; j < GPL; ++j) best = gk[j] > best ? gk[j] : best;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-          const unsigned long long other = __shfl_xor_sync(kFull, best, o);
-          best = other > best ? other : best;
-        }
-#pragma unroll
-        for (int j = 0; j < GPL; ++j) {
-          if (gk[j] == best && best != 0ull) {  // keys are unique: the owner marks its group kept
-            s_kept[wib][lane + 32 * j] = 1;
-            gk[j] = 0ull;
+      // A group ranks by its best expert under the same order (higher key, then lower id).
+      // Lane l owns groups l, l + 32, ... and scans their experts from shared memory; then
+      // M rounds of the two warp reductions keep the best groups.
+      uint32_t* gh = s_gh[wib];
+      int* ge = s_ge[wib];
+      for (int g = lane; g < P; g += 32) {
+        const int e0 = g * epp;
+        uint32_t bh = 0u;
+        int be = e0;
+        if ((epp & 3) == 0) {  // 16-byte aligned runs of 4 keys (e0 % 4 == 0)
+          const uint4* q = reinterpret_cast<const uint4*>(sk + e0);
+          for (int c = 0; c < (epp >> 2); ++c) {
+            const uint4 h4 = q[c];
+            const int e = e0 + 4 * c;
+            if (h4.x > bh) bh = h4.x, be = e;
+            if (h4.y > bh) bh = h4.y, be = e + 1;
+            if (h4.z > bh) bh = h4.z, be = e + 2;
+            if (h4.w > bh) bh = h4.w, be = e + 3;
+          }
+        } else {
+          for (int e = e0; e < e0 + epp; ++e) {
+            const uint32_t h = sk[e];
+            if (h > bh) bh = h, be = e;
           }
         }
+        gh[g] = bh;
+        ge[g] = be;
+        s_kept[wib][g] = 0;
+      }
+      for (int m = 0; m < M; ++m) {
+        uint32_t bh = 0u;
+        int be = 0x7fffffff;
+        for (int g = lane; g < P; g += 32) {
+          const uint32_t h = gh[g];
+          if (h > bh || (h == bh && ge[g] < be)) bh = h, be = ge[g];
+        }
+        const uint32_t top = __reduce_max_sync(kFull, bh);
+        const int e = __reduce_min_sync(kFull, bh == top ? be : 0x7fffffff);
+        const int g = e / epp;  // every group not yet kept holds a candidate (key >= 1)
+        if (lane == (g & 31)) {
+          s_kept[wib][g] = 1;
+          gh[g] = 0u;
+        }
       }
       __syncwarp();
 #pragma unroll
       for (int i = 0; i < VPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < E && !s_kept[wib][e / epp]) hk[i] = 0u;  // experts of dropped groups leave the race
+        if (e < E && !s_kept[wib][e / epp]) hk[i] = 0u, sk[e] = 0u;  // dropped groups leave the race
       }
+      __syncwarp();
     }
     // Every real candidate has key >= 1; empty slots have 0.  K <= number of candidates.
     uint32_t bh = 0u;
     int bi = 0;
 #pragma unroll
     for (int i = 0; i < VPL; ++i) {
-      sk[lane + 32 * i] = hk[i];
       if (hk[i] > bh) bh = hk[i], bi = i;
     }
-    __syncwarp();
     int my_id = 0;
     uint32_t my_key = 0u;
     for (int k = 0; k < K; ++k) {
