@@ -50,8 +50,8 @@ Readings where the pages are silent:
   E followed by renormalising the top-K); with ``renormalize=False`` the weight
   is the plain softmax over all E at the selected experts.
 * Order of rows inside one expert: stable (assignment a = t*K + k ascending).
-* Shared expert [ParamCounts/dashboard: DeepSeekMoE-style shared experts run on every
-  token whatever the router says; InferenceX review claim IX2-0406 lists the shared
+* Shared expert [ParamCounts/dashboard: a shared expert in the DeepSeekMoE manner
+  processes all tokens, independent of routing; InferenceX review claim IX2-0406 lists the shared
   expert among the replicated non-expert weights]: a SwiGLU FFN of its own width on
   every token, rounded like a routed expert, added with weight 1 in the combine:
   out[t] = bf16( sum_k w[t,k] y[row(t,k)] + s[t] ).
