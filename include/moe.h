@@ -323,8 +323,8 @@ moe_status moe_grouped_gate_up_fp8(const void* xq, const float* xs, const int32_
 
 /* out[t][:] = bf16( sum_{k<K} topk_w[t][k] * y[row_of_assign[t*K+k]][:] + shared[t][:] ),
  * accumulated in fp32 in slot order.  y [TK][H] bf16, out [T][H] bf16; shared: [T][H] bf16
- * output of a shared expert (added with weight 1: shared experts run on every token
- * regardless of the router, "Three Parameter Counts...", "What the utilization dashboard
+ * output of a shared expert (added with weight 1: a shared expert sees every token and
+ * takes no routing weight, "Three Parameter Counts...", "What the utilization dashboard
  * smooths away"), or NULL. */
 moe_status moe_combine(const void* y, const int32_t* row_of_assign, const float* topk_w,
                        const void* shared, const moe_dims* d, void* out, void* stream);
