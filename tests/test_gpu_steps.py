@@ -50,7 +50,8 @@ ROUTE_CASES = [  # T, E, K, renormalize, generator
     (77, 896, 16, True, "random"), (64, 33, 5, True, "quantized"), (50, 1024, 32, True, "random"),
     (129, 64, 6, True, "special"), (40, 1000, 7, False, "quantized"), (1, 5, 5, True, "random"),
     (0, 16, 4, True, "random"), (4096, 128, 8, True, "random"), (64, 64, 8, True, "nan_heavy"),
-    (40, 896, 16, False, "nan_heavy"), (33, 1024, 32, True, "nan_heavy"),
+    (40, 896, 16, False, "nan_heavy"), (33, 1024, 32, True, "nan_heavy"), (10, 1, 1, True, "random"),
+    (17, 32, 32, True, "quantized"), (9, 64, 32, False, "special"), (5, 1024, 32, True, "quantized"),
 ]
 
 
@@ -88,6 +89,7 @@ LIMITED_CASES = [  # T, E, K, P, M, renormalize, generator
     (300, 256, 8, 8, 4, True, "random"), (200, 896, 16, 64, 8, True, "random"), (100, 16, 3, 4, 2, True, "quantized"),
     (129, 64, 6, 16, 3, False, "special"), (77, 1024, 8, 256, 4, True, "random"), (50, 32, 4, 32, 4, True, "random"),
     (64, 48, 5, 6, 1, True, "quantized"), (60, 256, 8, 8, 4, True, "nan_heavy"),
+    (40, 12, 3, 4, 3, True, "quantized"), (30, 60, 9, 20, 3, True, "special"), (25, 128, 16, 8, 7, True, "nan_heavy"),
 ]
 
 
