@@ -1,8 +1,8 @@
 // api.cu - the C ABI of libmoe_b200 (declared in include/moe.h): argument
 // checks, workspace layout and the order of the layer's launches.
 #include <algorithm>
+#include <atomic>
 #include <cmath>
-#include <mutex>
 #include <vector>
 
 #include "device.cuh"
@@ -11,15 +11,27 @@
 namespace moe {
 
 int num_sms() {
-  static int cache[64] = {0};
+  static std::atomic<int> cache[kMaxDevices] = {};
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
-    int n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 148;
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = n > 0 ? n : 148;
+    n = n > 0 ? n : 148;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
+}
+
+cudaError_t smem_attr_once(const void* func, int bytes, std::atomic<int>* done) {
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return err;
+  const bool tracked = dev >= 0 && dev < kMaxDevices;
+  if (tracked && done[dev].load(std::memory_order_acquire)) return cudaSuccess;
+  err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (err == cudaSuccess && tracked) done[dev].store(1, std::memory_order_release);
+  return err;
 }
 
 namespace {
@@ -31,16 +43,18 @@ constexpr size_t kWsHeader = 256;
 enum SchedSlot : int { kSchedGating = 0, kSchedGateUp, kSchedDown, kSchedDense, kSchedSharedGateUp, kSchedSharedDown };
 
 bool device_ok() {
-  static int cache[64] = {0};  // 0 unknown, 1 ok, -1 not sm_100
+  static std::atomic<int> cache[kMaxDevices] = {};  // 0 unknown, 1 ok, -1 not sm_100
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
-  if (cache[dev] == 0) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return false;
+  int ok = cache[dev].load(std::memory_order_relaxed);
+  if (ok == 0) {
     int major = 0, minor = 0;
     cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
     cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
-    cache[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    ok = (major == 10 && minor == 0) ? 1 : -1;
+    cache[dev].store(ok, std::memory_order_relaxed);
   }
-  return cache[dev] == 1;
+  return ok == 1;
 }
 
 moe_status check_dims(const moe_dims* d) {

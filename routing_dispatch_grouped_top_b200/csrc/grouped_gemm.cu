@@ -1077,12 +1077,9 @@ template <int EPI>
 cudaError_t launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorMap& a2, const BoxMaps& b,
                    const GemmArgs& args, long long tile_bound, cudaStream_t stream) {
   using L = Layout<EPI>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    L::kSmemBytes);
-  });
+  static std::atomic<int> attr_done[kMaxDevices] = {};
+  const cudaError_t attr_err =
+      smem_attr_once(reinterpret_cast<const void*>(grouped_gemm_kernel<EPI>), L::kSmemBytes, attr_done);
   if (attr_err != cudaSuccess) return attr_err;
   if (tile_bound <= 0) return cudaSuccess;
   const int grid = static_cast<int>(std::min<long long>(num_sms(), tile_bound));
@@ -1093,12 +1090,9 @@ template <int EPI>
 cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const BoxMaps& b, const GemmArgs& args,
                         long long tile_bound, cudaStream_t stream) {
   using L = PairLayout<EPI>;
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(pair_gemm_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    L::kSmemBytes);
-  });
+  static std::atomic<int> attr_done[kMaxDevices] = {};
+  const cudaError_t attr_err =
+      smem_attr_once(reinterpret_cast<const void*>(pair_gemm_kernel<EPI>), L::kSmemBytes, attr_done);
   if (attr_err != cudaSuccess) return attr_err;
   if (tile_bound <= 0) return cudaSuccess;
   const int pairs = static_cast<int>(std::min<long long>(num_sms() / 2, tile_bound));

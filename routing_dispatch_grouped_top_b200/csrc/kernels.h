@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace moe {
 
 enum Epi : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2, kEpiSwiGLUPacked = 3, kEpiSwiGLUFp8 = 4 };
@@ -27,6 +29,13 @@ struct GemmArgs {
 };
 
 int num_sms();             // SM count of the current device (cached per device)
+
+// Raises `func`'s dynamic shared-memory limit to `bytes` on the current device, once per
+// device: a function attribute belongs to the device's context, so a process that drives
+// several GPUs sets it on each.  `done` is the caller's per-device flag table
+// (kMaxDevices entries, zero-initialised).
+constexpr int kMaxDevices = 64;
+cudaError_t smem_attr_once(const void* func, int bytes, std::atomic<int>* done);
 
 // Launches `kernel` with programmatic stream serialization, so that it may begin while
 // the previous kernel on the stream drains (the kernel calls pdl_wait before reading).

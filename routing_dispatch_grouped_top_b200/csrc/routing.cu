@@ -8,7 +8,6 @@
 #include <cuda/atomic>
 
 #include <algorithm>
-#include <mutex>
 
 #include "device.cuh"
 #include "kernels.h"
@@ -478,12 +477,9 @@ cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, in
                               int32_t* part_counts, int32_t* part_offsets, int32_t* row_of_assign,
                               int32_t* assign_of_row, float* skew, const ScanWorkspace& ws, cudaStream_t s) {
   const size_t smem = scan_smem_bytes(E);
-  static std::once_flag once;
-  static cudaError_t attr = cudaSuccess;
-  std::call_once(once, [] {
-    attr = cudaFuncSetAttribute(count_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                static_cast<int>(scan_smem_bytes(MOE_MAX_E)));
-  });
+  static std::atomic<int> attr_done[kMaxDevices] = {};
+  const cudaError_t attr = smem_attr_once(reinterpret_cast<const void*>(count_scan_kernel),
+                                          static_cast<int>(scan_smem_bytes(MOE_MAX_E)), attr_done);
   if (attr != cudaSuccess) return attr;
   int occ = 0;
   cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, count_scan_kernel, kScanThreads, smem);
