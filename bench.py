@@ -32,7 +32,7 @@ from routing_dispatch_grouped_top_b200 import inputs  # noqa: E402
 
 METRIC = "MoE layer tokens/s; grouped-GEMM % of bf16 peak; permute/combine % of HBM BW"
 UNIT = "tokens/s"
-DEFAULT_CONFIG = "qwen3"       # Qwen3-30B-A3B-shaped prefill layer
+DEFAULT_CONFIG = "r1_prefill"  # DeepSeek-R1-shaped prefill layer: the largest single-GPU workload
 FLUSH_BYTES = 256 << 20
 E2E_LANES = 3
 
@@ -187,12 +187,19 @@ def kernel_traffic(workload: str, stage: str):
     return None
 
 
-def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 16):
+def oracle_sample_tokens(cfg) -> int:
+    """Tokens per oracle sample: 16 for the small layers, fewer for the wide ones, so that one
+    sample (its K experts' weights made on the host, then the float64 layer) stays within seconds."""
+    return max(1, min(16, int(1.5e9 // (6 * cfg.H * cfg.F * cfg.K))))
+
+
+def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 0):
     """The oracle (as it stands) on bounded samples of the workload: tokens/s on the host."""
     import numpy as np
     from threadpoolctl import threadpool_info
 
     import oracle
+    seed_tokens = seed_tokens or oracle_sample_tokens(cfg)
     # Only the experts the sample needs are materialised on the host.
     x_all = inputs.make_tokens(cfg, "cpu")
     w_g, bias = inputs.make_router(cfg, "cpu")
@@ -346,7 +353,8 @@ def run_reference(args, cfg):
     cb = dict(rates[-1])
     cb["value"] = val
     line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1000.0 * 16 / val, "higher_is_better": True,
+            "warmup": args.warmup, "ms_per_step": 1000.0 * oracle_sample_tokens(cfg) / val,
+            "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "impl": "reference", "config": config_dict(cfg, ws),
             "cpu_baseline": cb, "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
@@ -495,11 +503,15 @@ def main():
 
     if rank == 0:
         peaks = measured_peaks()
+        clocks = clk.summary()
         names = ["latent_down", "gating", "route", "count_scan", "permute", "gate_up", "down", "combine",
                  "latent_up_and_skew"]
         stage_mean = {n: statistics.mean(v) for n, v in zip(names, stage_ms)}
-        long_run = total_ms > 1000.0
-        bf16_peak = peaks["bf16_sustained"] if long_run else peaks["bf16"]
+        # The burst bf16 peak is a GEMM timed alone at full clock; the sustained one a GEMM loop
+        # held under the 1 kW power cap.  A timed region longer than a second, or one whose clock
+        # record shows the power cap, is compared with the sustained figure.
+        sustained = total_ms > 1000.0 or "sw_power_cap" in clocks["reasons"]
+        bf16_peak = peaks["bf16_sustained"] if sustained else peaks["bf16"]
         n_touched = int((bufs["counts"] > 0).sum().item())
         T, H, F, TK = cfg.T, cfg.H, cfg.F, cfg.TK
         # algorithmic work per launch: (flops, HBM bytes)
@@ -531,7 +543,7 @@ def main():
         roof["algorithmic_bytes"] = by
         roof["algorithmic_flops"] = fl
         roof["peak_source"] = (f"{peaks['source']} " + ("HBM copy" if roof["bound"] == "hbm" else
-                                                         f"bf16 {'sustained' if long_run else 'burst'}"
+                                                         f"bf16 {'sustained' if sustained else 'burst'}"
                                                          + (" x 2 (nominal fp8/bf16)" if tc_peak != bf16_peak
                                                             else "")))
         roof["timing"] = ("CUDA events around every gate/up launch of the timed steps" if dominant == "gate_up"
@@ -546,7 +558,10 @@ def main():
             frac[n]["frac_hbm"] = frac[n]["gbs"] / peaks["hbm"]
             if frac[n]["tflops"]:
                 frac[n]["frac_bf16"] = frac[n]["tflops"] / bf16_peak
+                frac[n]["frac_bf16_burst"] = frac[n]["tflops"] / peaks["bf16"]
         frac["grouped_ffn"] = {"ms": ffn_ms, "tflops": ffn_tflops, "frac_bf16": ffn_tflops / bf16_peak,
+                               "frac_bf16_burst": ffn_tflops / peaks["bf16"],
+                               "bf16_peak": "sustained" if sustained else "burst",
                                "gbs": ffn_bytes / (ffn_ms / 1e3) / 1e9,
                                "frac_hbm": ffn_bytes / (ffn_ms / 1e3) / 1e9 / peaks["hbm"],
                                "roofline_ms": 1e3 * max(ffn_bytes / (peaks["hbm"] * 1e9),
@@ -564,7 +579,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": UNIT, "streams": E2E_LANES, "h2d_bytes_per_step": cfg.T * d_in * 2,
                     "d2h_bytes_per_step": cfg.T * d_in * 2},
             "gpu_launches": (7 + (2 if cfg.d_model else 0) + (2 if cfg.F_shared else 0)) * args.steps,
-            "clocks": clk.summary(),
+            "clocks": clocks,
             "skew_max_over_mean": float(bufs["skew"].item()),
         }
         if not args.no_cpu_baseline and world == 1:

@@ -99,10 +99,11 @@ typedef enum moe_status {
  * time.  Returns 0 for an invalid shape. */
 size_t moe_workspace_bytes(const moe_dims* d);
 
-/* Clears the workspace's 256-byte header: the status word, the count/scan kernel's
- * grid-barrier counters and the grouped GEMMs' tile-schedule counters (an async memset
- * on `stream`).  Call once after allocating the workspace, and again after a
- * device-side error has been reported. */
+/* Clears the whole workspace (an async memset of ws_bytes on `stream`): the status word,
+ * the count/scan state (its block ticket, done counter, look-back flags and expert totals)
+ * and the grouped GEMMs' tile-schedule counters.  The kernels leave that state at zero
+ * after every call, so this is needed once after allocating the workspace, and again after
+ * a device-side error has been reported or a call failed part-way. */
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /* Synchronizes `stream`, then copies the workspace status word to *status
@@ -165,9 +166,13 @@ moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids,
  *   row_of_assign[TK]: row of assignment a in the expert-major buffer, a stable
  *     counting sort (rows of one expert keep increasing a),
  *   assign_of_row[TK]: its inverse.
- * An id outside [0, E) sets MOE_DEV_BAD_INDEX; such assignments are given no row
- * and the outputs are then unspecified.  Uses the workspace (grid barrier and
- * per-block histograms). */
+ * Two launches: an expert histogram of the ids, then one pass over the assignments in
+ * up to 128 chunks with a decoupled look-back scan across the chunks (each chunk's
+ * counts are published and added up by its successors; no grid-wide barrier).  Uses the
+ * workspace (expert totals, per-chunk count rows, look-back flags and counters).
+ * An id outside [0, E) sets MOE_DEV_BAD_INDEX and gets row -1; a look-back wait that runs
+ * out (2 s) sets MOE_DEV_TIMEOUT.  Either way offsets[E] is set to -1 (a bad-offsets
+ * marker that the grouped GEMMs refuse) and the other outputs are unspecified. */
 moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* counts,
                           int32_t* offsets, int32_t* part_counts, int32_t* part_offsets,
                           int32_t* row_of_assign, int32_t* assign_of_row,
@@ -181,19 +186,19 @@ moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* c
  * this call; it exists for callers that cannot allocate device memory: a plugin inside
  * a host framework that owns every device allocation, or a real-time loop that may not
  * call cudaMalloc/cudaFree, which can also synchronize the device, once it runs).
- * Same arguments and results as moe_count_scan minus the workspace.  The scratch is a
- * fixed device array inside the library: 256 bytes of status and grid-barrier words
- * plus one E-entry int32 histogram per block (ceil(T*K / 1024) blocks, at most 1024),
- * at most MOE_NOALLOC_SCRATCH_BYTES in all; larger shapes return
- * MOE_ERR_UNSUPPORTED_SHAPE (with E = 1024 up to T*K = 261 120 assignments).
- * The call allocates nothing: it clears the scratch's status and barrier words with
- * an async memset on `stream`, then launches the count/scan kernel.  The first call on
- * a device looks up the scratch's device address once (with that device current);
- * make that first call before any stream capture.  All calls share the one scratch
- * and it keeps the last call's contents, so calls that overlap on the GPU (other
- * streams, other host threads) race: serialize them.  Device-side conditions are not
- * reported back (no workspace to read): an id outside [0, E) shows up as row -1 in
- * row_of_assign. */
+ * Same arguments, results and status codes as moe_count_scan minus the workspace.  The
+ * scratch is a fixed device array inside the library holding the count/scan state:
+ * 768 bytes of counters and flags, the E expert totals and two int32 rows of E per chunk
+ * (ceil(T*K / 256) chunks, at most 128), at most MOE_NOALLOC_SCRATCH_BYTES in all; larger
+ * shapes return MOE_ERR_UNSUPPORTED_SHAPE (only E >= 1020 with T*K > 32 512 exceed it).  The call allocates nothing: it clears the scratch's counters, flags
+ * and totals with an async memset on `stream`, then launches the two count/scan kernels.
+ * The first call on a device looks up the scratch's device address once (with that
+ * device current); make that first call before any stream capture.  All calls share the
+ * one scratch and it keeps the last call's contents, so calls that overlap on the GPU
+ * (other streams, other host threads) race: serialize them.  Device-side conditions
+ * have no status word to go to (no workspace): an id outside [0, E) shows up as row -1 in
+ * row_of_assign, and a call that met one, or whose look-back wait ran out, leaves
+ * offsets[E] = -1. */
 moe_status moe_count_scan_noalloc(const int32_t* topk_ids, const moe_dims* d, int32_t* counts,
                                   int32_t* offsets, int32_t* part_counts, int32_t* part_offsets,
                                   int32_t* row_of_assign, int32_t* assign_of_row, void* stream);
@@ -241,21 +246,6 @@ moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_
 moe_status moe_grouped_ffn(const void* xp, const int32_t* offsets, const void* w_gate,
                            const void* w_up, const void* w_down, const moe_dims* d,
                            void* h, void* y, void* ws, size_t ws_bytes, void* stream);
-
-/* One-time weight preparation for the gate/up GEMM: interleaves w_gate and w_up
- * ([E][F][H] each) in blocks of 64 rows into w_gu [E][2 Fp][H] bf16, Fp = F rounded up
- * to a multiple of 64 (rows [128 j, 128 j + 64) = gate rows [64 j, 64 j + 64), the next 64
- * = the up rows of the same features, rows of features >= F zero).  Then one TMA box
- * carries gate and up of 128 features and the GEMM runs N = 256 MMAs.  Size in bytes:
- * moe_packed_gate_up_bytes(d).  Not part of the per-token path. */
-size_t moe_packed_gate_up_bytes(const moe_dims* d);
-moe_status moe_pack_gate_up(const void* w_gate, const void* w_up, const moe_dims* d, void* w_gu,
-                            void* stream);
-
-/* moe_grouped_gate_up on packed weights: identical h. */
-moe_status moe_grouped_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu,
-                                      const moe_dims* d, void* h, void* ws, size_t ws_bytes,
-                                      void* stream);
 
 /* Process-wide tuning of the grouped GEMMs (not part of the method): groups with at least
  * `rows` rows on average (default 64) run on the CTA-pair kernel, in which the two SMs of a
@@ -366,8 +356,6 @@ typedef struct moe_layer_weights {
   const void*  w_down;      /* [E][H][F] bf16                                */
   const void*  w_dp;        /* latent only: [H][d_model] bf16, else NULL     */
   const void*  w_upp;       /* latent only: [d_model][H] bf16, else NULL     */
-  const void*  w_gate_up;   /* optional: w_gate/w_up packed by moe_pack_gate_up;
-                               when set the layer uses it (w_gate/w_up may be NULL) */
   const void*  w_shared_gate; /* shared expert (F_shared > 0): [F_shared][H] bf16    */
   const void*  w_shared_up;   /* [F_shared][H] bf16                                  */
   const void*  w_shared_down; /* [H][F_shared] bf16                                  */

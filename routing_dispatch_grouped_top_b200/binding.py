@@ -36,7 +36,7 @@ class moe_dims(C.Structure):
                 ("F_shared", C.c_int32), ("fp8_dispatch", C.c_int32)]
 
 
-_W_FIELDS = ("w_g_split", "bias", "w_gate", "w_up", "w_down", "w_dp", "w_upp", "w_gate_up", "w_shared_gate",
+_W_FIELDS = ("w_g_split", "bias", "w_gate", "w_up", "w_down", "w_dp", "w_upp", "w_shared_gate",
              "w_shared_up", "w_shared_down", "w_gate_q", "w_up_q", "s_gate", "s_up")
 
 
@@ -70,9 +70,6 @@ _SIGS = {
     "moe_grouped_ffn": (C.c_int, [_VP, _VP, _VP, _VP, _VP, _DP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_gate_up": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_down": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
-    "moe_packed_gate_up_bytes": (_SZ, [_DP]),
-    "moe_pack_gate_up": (C.c_int, [_VP, _VP, _DP, _VP, _VP]),
-    "moe_grouped_gate_up_packed": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
     "moe_set_pair_min_rows": (None, [_I32]),
     "moe_quantize_fp8_rows": (C.c_int, [_VP, _I64, _I32, _VP, _VP, _VP]),
     "moe_permute_fp8": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
@@ -296,31 +293,6 @@ def moe_grouped_gate_up(xp, offsets, w_gate, w_up, d: moe_dims, h, ws, stream=No
         _stream(stream)))
 
 
-def packed_gate_up_bytes(d: moe_dims) -> int:
-    return int(lib().moe_packed_gate_up_bytes(C.byref(d)))
-
-
-def moe_pack_gate_up(w_gate, w_up, d: moe_dims, w_gu, stream=None):
-    n = d.E * d.F * d.H
-    _check("moe_pack_gate_up", lib().moe_pack_gate_up(
-        _ptr(w_gate, torch.bfloat16, "w_gate", n), _ptr(w_up, torch.bfloat16, "w_up", n), C.byref(d),
-        _ptr(w_gu, torch.bfloat16, "w_gu", packed_gate_up_bytes(d) // 2), _stream(stream)))
-
-
-def pack_gate_up(w_gate, w_up, d: moe_dims, stream=None) -> torch.Tensor:
-    w_gu = torch.empty(packed_gate_up_bytes(d) // 2, dtype=torch.bfloat16, device=w_gate.device)
-    moe_pack_gate_up(w_gate, w_up, d, w_gu, stream)
-    return w_gu
-
-
-def moe_grouped_gate_up_packed(xp, offsets, w_gu, d: moe_dims, h, ws, stream=None):
-    TK = d.T * d.K
-    _check("moe_grouped_gate_up_packed", lib().moe_grouped_gate_up_packed(
-        _ptr(xp, torch.bfloat16, "xp", TK * d.H), _ptr(offsets, torch.int32, "offsets", d.E + 1),
-        _ptr(w_gu, torch.bfloat16, "w_gu", packed_gate_up_bytes(d) // 2), C.byref(d),
-        _ptr(h, torch.bfloat16, "h", TK * d.F), _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
-
-
 def moe_grouped_down(h, offsets, w_down, d: moe_dims, y, ws, stream=None):
     TK = d.T * d.K
     _check("moe_grouped_down", lib().moe_grouped_down(
@@ -410,23 +382,10 @@ def _weights_struct(w: dict) -> moe_layer_weights:
     return moe_layer_weights(*[(w[n].data_ptr() if w.get(n) is not None else None) for n in _W_FIELDS])
 
 
-# Packed gate/up weights (one 256-row box of interleaved gate/up rows per stage, with a
-# shared-memory exchange in the epilogue) measured slower than the separate-weight kernel
-# with 256-token tiles and eight epilogue warps on every workload (DeepSeek-R1-shaped
-# layer: 4.23 vs 3.81 ms), so layers use the separate weights unless asked otherwise.
-PACK_GATE_UP_BY_DEFAULT = False
-
-
 def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, w_upp=None, stream=None,
-                       pack_gate_up_weights=None, shared=None) -> dict:
-    """One-time weight preparation: router split into three bf16 planes and, when
-    ``pack_gate_up_weights`` (default: PACK_GATE_UP_BY_DEFAULT), gate/up interleaved for the
-    packed gate/up GEMM.  With ``d.fp8_dispatch`` the gate and up weights are quantized to
-    E4M3 per output feature instead."""
-    if d.fp8_dispatch:
-        pack_gate_up_weights = False
-    if pack_gate_up_weights is None:
-        pack_gate_up_weights = PACK_GATE_UP_BY_DEFAULT
+                       shared=None) -> dict:
+    """One-time weight preparation: router split into three bf16 planes; with
+    ``d.fp8_dispatch`` the gate and up weights are also quantized to E4M3 per output feature."""
     split = torch.empty((3, d.E, d.H), dtype=torch.bfloat16, device=w_g.device)
     moe_pack_router(w_g.contiguous(), d, split, stream)
     for name, t, n in (("w_gate", w_gate, d.E * d.F * d.H), ("w_up", w_up, d.E * d.F * d.H),
@@ -437,7 +396,6 @@ def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, 
         _ptr(w_upp, torch.bfloat16, "w_upp", d.H * d.d_model)
     if bias is not None:
         _ptr(bias, torch.float32, "bias", d.E)
-    w_gu = pack_gate_up(w_gate, w_up, d, stream) if pack_gate_up_weights else None
     sg, su, sd = shared if shared is not None else (None, None, None)
     if d.F_shared:
         for name, t in (("w_shared_gate", sg), ("w_shared_up", su), ("w_shared_down", sd)):
@@ -447,7 +405,7 @@ def pack_layer_weights(d: moe_dims, w_g, bias, w_gate, w_up, w_down, w_dp=None, 
         q["w_gate_q"], q["s_gate"] = quantize_fp8(w_gate, stream)
         q["w_up_q"], q["s_up"] = quantize_fp8(w_up, stream)
     return dict(w_g_split=split, bias=bias, w_gate=w_gate, w_up=w_up, w_down=w_down, w_dp=w_dp, w_upp=w_upp,
-                w_gate_up=w_gu, w_shared_gate=sg, w_shared_up=su, w_shared_down=sd, **q)
+                w_shared_gate=sg, w_shared_up=su, w_shared_down=sd, **q)
 
 
 def moe_layer_forward(x, weights: dict, d: moe_dims, buffers: dict, ws, stage_events=None, stream=None):

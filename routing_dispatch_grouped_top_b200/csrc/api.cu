@@ -34,14 +34,6 @@ cudaError_t smem_attr_once(const void* func, int bytes, std::atomic<int>* done) 
   return err;
 }
 
-namespace {
-
-// Workspace: [0] status word, [64] grid-barrier count, [128] grid-barrier
-// generation, [160 + 16 s) the GEMM tile schedule of call site s (s < 6), [256 ...)
-// per-block expert histograms of the count/scan kernel.
-constexpr size_t kWsHeader = 256;
-enum SchedSlot : int { kSchedGating = 0, kSchedGateUp, kSchedDown, kSchedDense, kSchedSharedGateUp, kSchedSharedDown };
-
 bool device_ok() {
   static std::atomic<int> cache[kMaxDevices] = {};  // 0 unknown, 1 ok, -1 not sm_100
   int dev = 0;
@@ -76,14 +68,20 @@ moe_status check_dims(const moe_dims* d) {
   return MOE_OK;
 }
 
+namespace {
+
+// Workspace: the count/scan state (ScanWorkspace: [0] status word, [64, 160) the count/scan
+// ticket, done counter and failure flag, [256 ...) look-back flags, expert totals and per-block
+// rows), whose bytes [160 + 16 s, 176 + 16 s) hold the GEMM tile schedule of call site s
+// (s < 6); then the gating partials.
+constexpr size_t kWsHeader = 256;
+enum SchedSlot : int { kSchedGating = 0, kSchedGateUp, kSchedDown, kSchedDense, kSchedSharedGateUp, kSchedSharedDown };
+
 // The split gating reduction keeps its partial logits after the histograms.  The workspace
 // is sized for a 148-SM B200; a device with fewer SMs uses fewer splits.
 constexpr int kSizingSms = 148;
 
-size_t hist_bytes(const moe_dims* d) {
-  const long long TK = d->T * static_cast<long long>(d->K);
-  return (static_cast<size_t>(scan_max_blocks(TK)) * d->E * sizeof(int) + 255) / 256 * 256;
-}
+size_t scan_bytes(const moe_dims* d) { return scan_ws_bytes(d->T * static_cast<long long>(d->K), d->E); }
 
 int gating_split_count(const moe_dims* d) {
   return std::min(gating_splits(d->T, d->H, d->E, num_sms()), gating_splits(d->T, d->H, d->E, kSizingSms));
@@ -92,25 +90,18 @@ int gating_split_count(const moe_dims* d) {
 size_t ws_bytes_for(const moe_dims* d) {
   const int S = gating_splits(d->T, d->H, d->E, kSizingSms);
   const size_t partials = S > 1 ? static_cast<size_t>(S) * d->T * d->E * sizeof(float) : 0;
-  return kWsHeader + hist_bytes(d) + partials;
+  return scan_bytes(d) + partials;
 }
 
 float* ws_partials(void* ws, const moe_dims* d) {
-  return reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + kWsHeader + hist_bytes(d));
+  return reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(ws) + scan_bytes(d));
 }
 
 int* ws_status(void* ws) { return reinterpret_cast<int*>(ws); }
 int* ws_sched(void* ws, SchedSlot s) { return reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(ws) + 160 + 16 * s); }
 
 ScanWorkspace scan_ws(void* ws, const moe_dims* d) {
-  uint8_t* p = reinterpret_cast<uint8_t*>(ws);
-  ScanWorkspace s;
-  s.status = reinterpret_cast<int*>(p);
-  s.bar_count = reinterpret_cast<unsigned int*>(p + 64);
-  s.bar_gen = reinterpret_cast<unsigned int*>(p + 128);
-  s.block_counts = reinterpret_cast<int*>(p + kWsHeader);
-  s.max_blocks = scan_max_blocks(d->T * static_cast<long long>(d->K));
-  return s;
+  return scan_workspace(ws, d->T * static_cast<long long>(d->K), d->E);
 }
 
 moe_status cuda_status(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA; }
@@ -163,7 +154,7 @@ size_t moe_workspace_bytes(const moe_dims* d) {
 
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (!ws || ws_bytes < kWsHeader) return MOE_ERR_WORKSPACE;
-  MOE_CUDA(cudaMemsetAsync(ws, 0, kWsHeader, as_stream(stream)));
+  MOE_CUDA(cudaMemsetAsync(ws, 0, ws_bytes, as_stream(stream)));
   return MOE_OK;
 }
 
@@ -216,7 +207,7 @@ moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids, 
   if (d->T == 0) return MOE_OK;
   if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_route(logits, 1, nullptr, d->T, d->E, d->K, d->renormalize, d->P, d->group_limit,
-                                  topk_ids, topk_w, as_stream(stream)));
+                                  topk_ids, topk_w, nullptr, as_stream(stream)));
 }
 
 moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* counts, int32_t* offsets,
@@ -227,9 +218,11 @@ moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* c
   if (!counts || !offsets || !part_counts || !part_offsets || (d->T > 0 && (!topk_ids || !row_of_assign ||
                                                                            !assign_of_row)))
     return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_count_scan(topk_ids, d->T * static_cast<long long>(d->K), d->E, d->P, counts, offsets,
-                                       part_counts, part_offsets, row_of_assign, assign_of_row, nullptr,
-                                       scan_ws(ws, d), as_stream(stream)));
+  const long long TK = d->T * static_cast<long long>(d->K);
+  const ScanWorkspace sw = scan_ws(ws, d);
+  MOE_CUDA(launch_hist(topk_ids, TK, d->E, sw, as_stream(stream)));
+  return cuda_status(launch_count_scan(topk_ids, TK, d->E, d->P, counts, offsets, part_counts, part_offsets,
+                                       row_of_assign, assign_of_row, nullptr, sw, as_stream(stream)));
 }
 
 moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_t* topk_ids, const float* topk_w,
@@ -291,29 +284,6 @@ moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const voi
   if (!aligned16(xp) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
   return cuda_status(gemm_gate_up(xp, offsets, w_gate, w_up, d->E, d->T * static_cast<long long>(d->K), d->H,
                                   d->F, h, ws_status(ws), ws_sched(ws, kSchedGateUp), as_stream(stream)));
-}
-
-size_t moe_packed_gate_up_bytes(const moe_dims* d) {
-  if (check_dims(d) != MOE_OK) return 0;
-  return static_cast<size_t>(d->E) * static_cast<size_t>(packed_gate_up_rows(d->F)) * d->H * 2;
-}
-
-moe_status moe_pack_gate_up(const void* w_gate, const void* w_up, const moe_dims* d, void* w_gu, void* stream) {
-  MOE_TRY(common_checks(d));
-  if (!w_gate || !w_up || !w_gu) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(w_gate) || !aligned16(w_up) || !aligned16(w_gu)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_pack_gate_up(w_gate, w_up, d->E, d->H, d->F, w_gu, as_stream(stream)));
-}
-
-moe_status moe_grouped_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, const moe_dims* d,
-                                      void* h, void* ws, size_t ws_bytes, void* stream) {
-  MOE_TRY(common_checks(d));
-  MOE_TRY(check_ws_header(ws, ws_bytes));
-  if (d->T == 0) return MOE_OK;
-  if (!xp || !offsets || !w_gu || !h) return MOE_ERR_INVALID_ARG;
-  if (!aligned16(xp) || !aligned16(w_gu) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(gemm_gate_up_packed(xp, offsets, w_gu, d->E, d->T * static_cast<long long>(d->K), d->H, d->F,
-                                         h, ws_status(ws), ws_sched(ws, kSchedGateUp), as_stream(stream)));
 }
 
 moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w_down, const moe_dims* d, void* y,
@@ -386,7 +356,7 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
   const bool latent = d->d_model > 0;
   const bool fp8 = d->fp8_dispatch != 0;
   if (!w->w_g_split || !w->w_down) return MOE_ERR_INVALID_ARG;
-  if (!fp8 && !w->w_gate_up && (!w->w_gate || !w->w_up)) return MOE_ERR_INVALID_ARG;
+  if (!fp8 && (!w->w_gate || !w->w_up)) return MOE_ERR_INVALID_ARG;
   if (fp8 && (!w->w_gate_q || !w->w_up_q || !w->s_gate || !w->s_up || !b->xq || !b->xs)) return MOE_ERR_INVALID_ARG;
   if (fp8 && (!aligned16(w->w_gate_q) || !aligned16(w->w_up_q) || !aligned16(b->xq))) return MOE_ERR_INVALID_ARG;
   if (latent && (!w->w_dp || !w->w_upp || !b->z || !b->final_out)) return MOE_ERR_INVALID_ARG;
@@ -440,11 +410,12 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
     MOE_CUDA(gemm_gating(routed, w->w_g_split, w->bias, T, d->H, d->E, gate_out, nsplit, status,
                          ws_sched(ws, kSchedGating), s));
   MOE_TRY(mark(2));
+  const ScanWorkspace sw = scan_ws(ws, d);
   MOE_CUDA(launch_route(gate_out, nsplit, b->logits, T, d->E, d->K, d->renormalize, d->P, d->group_limit, b->topk_ids,
-                        b->topk_w, s));
+                        b->topk_w, sw.hist, s));
   MOE_TRY(mark(3));
   MOE_CUDA(launch_count_scan(b->topk_ids, TK, d->E, d->P, b->counts, b->offsets, b->part_counts, b->part_offsets,
-                             b->row_of_assign, b->assign_of_row, b->skew, scan_ws(ws, d), s));
+                             b->row_of_assign, b->assign_of_row, b->skew, sw, s));
   MOE_TRY(mark(4));
   if (fp8)
     MOE_CUDA(launch_permute_fp8(routed, b->row_of_assign, b->topk_ids, b->topk_w, T, d->H, d->E, d->K, d->P, b->xq,
@@ -457,9 +428,6 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
     if (fp8)
       MOE_CUDA(gemm_gate_up_fp8(b->xq, b->xs, b->offsets, w->w_gate_q, w->w_up_q, w->s_gate, w->s_up, d->E, TK, d->H,
                                 d->F, b->h, status, ws_sched(ws, kSchedGateUp), s));
-    else if (w->w_gate_up)
-      MOE_CUDA(gemm_gate_up_packed(b->xp, b->offsets, w->w_gate_up, d->E, TK, d->H, d->F, b->h, status,
-                                   ws_sched(ws, kSchedGateUp), s));
     else
       MOE_CUDA(gemm_gate_up(b->xp, b->offsets, w->w_gate, w->w_up, d->E, TK, d->H, d->F, b->h, status,
                             ws_sched(ws, kSchedGateUp), s));

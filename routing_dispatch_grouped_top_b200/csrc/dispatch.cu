@@ -187,29 +187,6 @@ __global__ void pack_router_kernel(const float* __restrict__ w_g, int H, int E, 
   }
 }
 
-// Gate/up weights [E][F][H] each -> [E][2 Fp][H], Fp = F rounded up to 64: packed rows
-// [128 j, 128 j + 64) are gate rows [64 j, 64 j + 64) and the next 64 are the up rows of
-// the same features; rows of features >= F are zero.  16-byte vectors over (row, vector).
-__global__ void pack_gate_up_kernel(const uint4* __restrict__ wg, const uint4* __restrict__ wu, int E, int F, int Fp,
-                                    int vpr, uint4* __restrict__ out) {
-  const long long n = static_cast<long long>(E) * 2 * Fp * vpr;
-  for (long long it = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; it < n;
-       it += static_cast<long long>(gridDim.x) * blockDim.x) {
-    const int v = static_cast<int>(it % vpr);
-    const long long prow = it / vpr;
-    const int e = static_cast<int>(prow / (2 * Fp));
-    const int pr = static_cast<int>(prow - static_cast<long long>(e) * 2 * Fp);
-    const int blk = pr >> 7, within = pr & 127;
-    const int f = 64 * blk + (within & 63);
-    uint4 val = make_uint4(0u, 0u, 0u, 0u);
-    if (f < F) {
-      const long long src = (static_cast<long long>(e) * F + f) * vpr + v;
-      val = within < 64 ? wg[src] : wu[src];
-    }
-    out[it] = val;
-  }
-}
-
 // ---------------------------------------------------------------------------
 // FP8 (E4M3) rows with one fp32 scale per row.  Low-precision dispatch narrows each row sent
 // to the experts and sends its scale with it (WideEP essay, "Top-k multiplies traffic.
@@ -364,16 +341,6 @@ cudaError_t launch_combine(const void* y, const int32_t* roa, const float* w, co
   return launch_pdl(combine_kernel<MOE_COMBINE_KC>, dim3(blocks), dim3(kCopyThreads), 0, s,
                     reinterpret_cast<const uint4*>(y), roa, w, reinterpret_cast<const uint4*>(shared), T, vpr, K,
                     reinterpret_cast<uint4*>(out));
-}
-
-cudaError_t launch_pack_gate_up(const void* w_gate, const void* w_up, int E, int H, int F, void* w_gu,
-                                cudaStream_t s) {
-  const int Fp = (F + 63) / 64 * 64;
-  const int vpr = H / 8;
-  pack_gate_up_kernel<<<copy_blocks(static_cast<long long>(E) * 2 * Fp * vpr), kCopyThreads, 0, s>>>(
-      reinterpret_cast<const uint4*>(w_gate), reinterpret_cast<const uint4*>(w_up), E, F, Fp, vpr,
-      reinterpret_cast<uint4*>(w_gu));
-  return cudaGetLastError();
 }
 
 cudaError_t launch_pack_router(const float* w_g, int H, int E, void* w_split, cudaStream_t s) {

@@ -84,14 +84,6 @@ struct Cfg<kEpiSwiGLU> {
   static constexpr int NA = 2, NT = MOE_SWIGLU_NT, STAGES = NT == 256 ? 3 : 4, FEAT = 128, EW = MOE_EPI_WARPS;
   static constexpr bool SEP = true;
 };
-// SwiGLU on packed weights: one 256-row box holds two 128-row weight tiles, each
-// [64 gate rows; the 64 up rows of the same features]; two N = 256 accumulators, so gate
-// (lanes 0-63) and up (lanes 64-127) meet through a shared-memory swap in the epilogue.
-template <>
-struct Cfg<kEpiSwiGLUPacked> {
-  static constexpr int NA = 2, NT = 256, STAGES = 3, FEAT = 128, EW = 4;
-  static constexpr bool SEP = true;
-};
 // SwiGLU on E4M3 operands (FP8 dispatch): the same tile as the bf16 SwiGLU, each stage
 // carrying 128 K-elements (one 128-byte swizzle atom of 8-bit codes) instead of 64, so a
 // stage holds twice the MMA work.
@@ -127,10 +119,8 @@ struct Layout {
   static constexpr int kAccCols = C::SEP ? C::NA * C::NT : C::NT;
   static constexpr int kNumAcc = (2 * kAccCols <= 512) ? 2 : 1;
   static constexpr uint32_t kTmemCols = kNumAcc * kAccCols;
-  static constexpr int kExchFloats = 2 * 16 * 64;  // SwiGLU swap of one 32-token chunk, both directions
-  static constexpr int kExchBytes = (EPI == kEpiSwiGLUPacked) ? 2 * kExchFloats * 4  // double-buffered
-                                    // bf16 outputs: one 32 x 32 transpose tile per epilogue warp
-                                    : (EPI == kEpiF32 ? 0 : C::EW * 32 * 32 * 2);
+  // bf16 outputs: one 32 x 32 transpose tile per epilogue warp
+  static constexpr int kExchBytes = EPI == kEpiF32 ? 0 : C::EW * 32 * 32 * 2;
   // barriers: full/empty per stage, tmem full/empty x2, drain, tile ring full/empty; then the
   // TMEM address, the abort flag and the ring's tile ids
   static constexpr int kBarBytes = (8 * (2 * C::STAGES + 5 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
@@ -322,7 +312,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
   const int S = (EPI == kEpiF32 && args.ksplit > 1) ? args.ksplit : 1;
   const int total = s_pre[G] * S;
 
-  static_assert(EPI != kEpiSwiGLUPacked || C::EW == 4, "the packed epilogue pairs warps q and q + 2");
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -359,9 +348,9 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
           uint8_t* st = ring + stage * L::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], bytes);
           const int kx = kb * KS;
-          if constexpr (EPI == kEpiBF16 || EPI == kEpiSwiGLUPacked) {
-            // both 128-row weight tiles in one 256-row box (packed rows are 2 per feature)
-            tma_load_3d(st, &tmA0, &full[stage], kx, (EPI == kEpiSwiGLUPacked) ? 2 * tl.n0 : tl.n0, tl.g);
+          if constexpr (EPI == kEpiBF16) {
+            // both 128-row weight tiles in one 256-row box
+            tma_load_3d(st, &tmA0, &full[stage], kx, tl.n0, tl.g);
           } else {
 #pragma unroll
             for (int i = 0; i < NA; ++i) {
@@ -481,52 +470,6 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       const Tile tl = decode_tile<NT, 16, C::FEAT>(tb, s_pre, s_off, G);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
-      if constexpr (EPI == kEpiSwiGLUPacked) {
-        // Accumulator i covers features n0 + 64 i + fi: gate in warps q < 2, up in warps q >= 2.
-        // The gate owner keeps tokens 0..15 of each 32-token chunk and hands 16..31 to the up
-        // owner, who hands back the up of tokens 0..15; each then finishes 16 tokens of h.
-        const int fi = 32 * (q & 1) + lane;
-        const bool is_gate = q < 2;
-        const int jbase = is_gate ? 0 : 16;
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(args.out);
-        const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
-#pragma unroll 1
-        for (int i = 0; i < NA; ++i) {
-          const int f = tl.n0 + 64 * i + fi;
-          for (int j0 = 0; j0 < tl.nvalid; j0 += 32, ++chunk) {
-            uint32_t r[32];
-            tmem_ld_32cols(tb + i * NT + j0, r);
-            tmem_wait_ld();
-            float* xb = exch + (chunk & 1) * L::kExchFloats;
-            float* to_up = xb;              // gate of tokens 16..31
-            float* to_gate = xb + 16 * 64;  // up of tokens 0..15
-#pragma unroll
-            for (int j = 0; j < 16; ++j) {
-              if (is_gate) to_up[j * 64 + fi] = __uint_as_float(r[16 + j]);
-              else to_gate[j * 64 + fi] = __uint_as_float(r[j]);
-            }
-            named_bar_sync(1, kEpiThr);
-            if (f < args.N) {
-              const long long row0 = static_cast<long long>(tl.row0) + j0 + jbase;
-#pragma unroll
-              for (int j = 0; j < 16; ++j) {
-                if (j0 + jbase + j < tl.nvalid) {
-                  const float g = is_gate ? __uint_as_float(r[j]) : to_up[j * 64 + fi];
-                  const float u = is_gate ? to_gate[j * 64 + fi] : __uint_as_float(r[16 + j]);
-                  out[(row0 + j) * args.ldo + f] = __float2bfloat16_rn(silu_mul(g, u));
-                }
-              }
-            }
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(&tempty[acc]);
-        if (++acc == L::kNumAcc) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
-        continue;
-      }
       const int f = tl.n0 + q * 32 + lane;
       const bool f_ok = f < args.N;
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
@@ -630,37 +573,25 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 //           separate TMEM columns of the same lanes, so no exchange between warps; the two
 //           accumulators fill TMEM, so the epilogue of a tile runs between main loops.
 //   bf16:   CTA r holds rows [n0 + 128 r, +128) and [n0 + 256 + 128 r, +128) (NA = 2).
-//           Built with MOE_PAIR_BF16_NA=1 it holds one weight operand with a double-buffered
-//           accumulator (the epilogue then overlaps the next main loop); that measured
-//           slower on the down projections (Qwen3 layer 164 vs 142 us), since each K-step
-//           carries half the MMA work for the same synchronisation.
 // Both CTAs' TMA loads of a stage complete on the leader's "full" barrier; the leader's
 // commits release both CTAs' "empty" and "tmem full" barriers; both CTAs' epilogue warps
 // release the leader's "tmem empty" barrier.  The leader's producer claims tiles from the
 // launch's counter and publishes each id to both CTAs through a ring in shared memory (the
 // peer's slot written over the cluster), which both CTAs' consumers release.
 // ---------------------------------------------------------------------------
-#ifndef MOE_PAIR_BF16_NA
-#define MOE_PAIR_BF16_NA 2
-#endif
-#ifndef MOE_PAIR_BF16_KA
-#define MOE_PAIR_BF16_KA 2
-#endif
 template <int EPI>
 struct PairLayout {
   static constexpr int NT = 256;                                // tokens per pair tile (MMA N)
-  static constexpr int NA = (EPI == kEpiBF16) ? MOE_PAIR_BF16_NA : 2;  // weight operands (accumulators)
-  static constexpr int KA = (NA == 1) ? MOE_PAIR_BF16_KA : 1;   // 128-byte K atoms per stage
-  static constexpr int STAGES = (NA == 1) ? 6 / KA : 4;
+  static constexpr int NA = 2;                                  // weight operands (accumulators)
+  static constexpr int STAGES = 4;
   static constexpr int EW = 8;                                  // epilogue warps per CTA
   static constexpr int kThr = 64 + 32 * EW;
-  static constexpr int FEAT = (EPI == kEpiBF16) ? 256 * NA : 256;  // output features per pair tile
+  static constexpr int FEAT = (EPI == kEpiBF16) ? 512 : 256;   // output features per pair tile
   static constexpr int kAPair = NA * kABytes;                   // this CTA's 128-row weight boxes (one atom)
   static constexpr int kBBytes = (NT / 2) * 128;                // this CTA's token rows (one atom)
-  static constexpr int kAtomBytes = kAPair + kBBytes;
-  static constexpr int kStageBytes = KA * kAtomBytes;
+  static constexpr int kStageBytes = kAPair + kBBytes;
   static constexpr uint32_t kAccCols = NA * NT;                 // one tile's accumulators
-  static constexpr int kNumAcc = (NA == 1) ? 2 : 1;             // TMEM buffers
+  static constexpr int kNumAcc = 1;                             // TMEM buffers
   static constexpr uint32_t kTmemCols = kNumAcc * kAccCols;
   static constexpr int kStgBytes = EW * 32 * 32 * 2;
   static constexpr int kBarBytes = (8 * (2 * STAGES + 5 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
@@ -703,7 +634,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
   const uint32_t rank = cluster_ctarank();
   const int G = args.offsets ? args.G : 1;
   const int NFT = (args.N + L::FEAT - 1) / L::FEAT;
-  const int KB = (args.Kd + KS * L::KA - 1) / (KS * L::KA);  // stages of KA atoms along K
+  const int KB = (args.Kd + KS - 1) / KS;  // K-steps (a K atom beyond Kd reads the zero fill)
 
   // Set-up that reads no global input runs before the wait on the previous kernel.
   if (threadIdx.x == 0) {
@@ -805,28 +736,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
             break;
           }
           const uint32_t bar = full_leader + stage * 8;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * L::KA * (L::kAPair + half * 128));
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kAPair + half * 128));
+          uint8_t* st = ring + stage * L::kStageBytes;
+          const int kx = kb * KS;
+          if constexpr (EPI == kEpiBF16) {
+            tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
+            tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
+          } else {
+            const int fr = tl.n0 + 128 * static_cast<int>(rank);
+            tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
+            tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
+          }
+          int r = 0;
 #pragma unroll
-          for (int a = 0; a < L::KA; ++a) {  // a K atom beyond Kd reads the zero fill
-            uint8_t* st = ring + stage * L::kStageBytes + a * L::kAtomBytes;
-            const int kx = (kb * L::KA + a) * KS;
-            if constexpr (EPI == kEpiBF16) {
-              tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
-              if constexpr (NA == 2)
-                tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
-            } else {
-              const int fr = tl.n0 + 128 * static_cast<int>(rank);
-              tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
-              tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
-            }
-            int r = 0;
-#pragma unroll
-            for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
-              const int rows = 256 >> i;
-              if (half & rows) {
-                tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
-                r += rows;
-              }
+          for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
+            const int rows = 256 >> i;
+            if (half & rows) {
+              tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
+              r += rows;
             }
           }
           pend[stage] = true;
@@ -884,20 +811,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
             break;
           }
           tc_fence_after();
+          const uint32_t sa = smem_u32(ring + stage * L::kStageBytes);
+          const uint32_t sb = sa + L::kAPair;
 #pragma unroll
-          for (int a = 0; a < L::KA; ++a) {
-            const uint32_t sa = smem_u32(ring + stage * L::kStageBytes + a * L::kAtomBytes);
-            const uint32_t sb = sa + L::kAPair;
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
 #pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
-#pragma unroll
-              for (int i = 0; i < NA; ++i) {
-                const uint64_t adesc = sw128_kmajor_desc(sa + i * kABytes + kk * 32);
-                const uint32_t accum = (kb > 0 || a > 0 || kk > 0) ? 1u : 0u;
-                if constexpr (EPI == kEpiSwiGLUFp8) umma_e4m3_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
-                else umma_bf16_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
-              }
+            for (int i = 0; i < NA; ++i) {
+              const uint64_t adesc = sw128_kmajor_desc(sa + i * kABytes + kk * 32);
+              const uint32_t accum = (kb > 0 || kk > 0) ? 1u : 0u;
+              if constexpr (EPI == kEpiSwiGLUFp8) umma_e4m3_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
+              else umma_bf16_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
             }
           }
           umma_commit_pair(smem_u32(&empty[stage]));  // both CTAs' stage buffers are free again
@@ -958,7 +882,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         const long long row0 = static_cast<long long>(tl.row0) + j0;
         uint32_t r0[32], r1[32];
         tmem_ld_32cols(tbase + j0, r0);
-        if constexpr (NA == 2) tmem_ld_32cols(tbase + NT + j0, r1);
+        tmem_ld_32cols(tbase + NT + j0, r1);
         float sx = 1.0f;
         if constexpr (EPI == kEpiSwiGLUFp8) sx = lane < jn ? __ldg(args.scale_b + row0 + lane) : 0.0f;
         tmem_wait_ld();
@@ -967,13 +891,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
           store_rows32(stg, lane, v, outb, args.ldo, args.N, fa, row0, jn);
-          if constexpr (NA == 2) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r1[j]);
-            store_rows32(stg, lane, v, outb, args.ldo, args.N, fa + 256, row0, jn);
-          } else {
-            (void)r1;
-          }
+          for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r1[j]);
+          store_rows32(stg, lane, v, outb, args.ldo, args.N, fa + 256, row0, jn);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -1109,7 +1029,6 @@ long long tile_bound(long long rows, int groups, int NT, int N, int feat) {
 int gemm_smem_bytes(int epi) {
   switch (epi) {
     case kEpiSwiGLU: return Layout<kEpiSwiGLU>::kSmemBytes;
-    case kEpiSwiGLUPacked: return Layout<kEpiSwiGLUPacked>::kSmemBytes;
     case kEpiBF16: return Layout<kEpiBF16>::kSmemBytes;
     case kEpiSwiGLUFp8: return Layout<kEpiSwiGLUFp8>::kSmemBytes;
     default: return Layout<kEpiF32>::kSmemBytes;
@@ -1148,22 +1067,6 @@ cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_g
                                    tile_bound(rows, E, PairLayout<kEpiSwiGLU>::NT, F, PairLayout<kEpiSwiGLU>::FEAT),
                                    stream);
   return launch<kEpiSwiGLU>(a0, a1, a1, b, args, tile_bound(rows, E, Cfg<kEpiSwiGLU>::NT, F, Cfg<kEpiSwiGLU>::FEAT), stream);
-}
-
-long long packed_gate_up_rows(int F) { return 2LL * ((F + 63) / 64 * 64); }
-
-// Same result as gemm_gate_up, from weights packed by launch_pack_gate_up.
-cudaError_t gemm_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, int E, long long rows,
-                                int H, int F, void* h, int* status, int* sched, cudaStream_t stream) {
-  GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status, nullptr, nullptr, nullptr, sched};
-  CUtensorMap a0;
-  BoxMaps b;
-  if (!map_bf16_3d(&a0, w_gu, H, static_cast<uint64_t>(packed_gate_up_rows(F)), E, 256) ||
-      !map_token_boxes(&b, xp, H, rows))
-    return cudaErrorInvalidValue;
-  return launch<kEpiSwiGLUPacked>(a0, a0, a0, b, args,
-                                  tile_bound(rows, E, Cfg<kEpiSwiGLUPacked>::NT, F, Cfg<kEpiSwiGLUPacked>::FEAT),
-                                  stream);
 }
 
 // FP8 dispatch: gate/up on E4M3 codes; g and u are scaled by the row's and the feature's

@@ -6,9 +6,11 @@
 
 #include <atomic>
 
+#include "../../include/moe.h"
+
 namespace moe {
 
-enum Epi : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2, kEpiSwiGLUPacked = 3, kEpiSwiGLUFp8 = 4 };
+enum Epi : int { kEpiSwiGLU = 0, kEpiBF16 = 1, kEpiF32 = 2, kEpiSwiGLUFp8 = 4 };
 
 struct GemmArgs {
   const int32_t* offsets;  // [G + 1] device row offsets of the groups, or nullptr: one group of M rows
@@ -29,6 +31,8 @@ struct GemmArgs {
 };
 
 int num_sms();             // SM count of the current device (cached per device)
+bool device_ok();          // the current device is an sm_100 (cached per device)
+moe_status check_dims(const moe_dims* d);  // the shape checks every entry point makes
 
 // Raises `func`'s dynamic shared-memory limit to `bytes` on the current device, once per
 // device: a function attribute belongs to the device's context, so a process that drives
@@ -60,12 +64,6 @@ void set_pair_min_rows(int rows);
 
 cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
                          long long rows, int H, int F, void* h, int* status, int* sched, cudaStream_t stream);
-// Gate and up weights interleaved in 64-row blocks ([E][2 Fp][H], Fp = F rounded up to 64).
-long long packed_gate_up_rows(int F);
-cudaError_t launch_pack_gate_up(const void* w_gate, const void* w_up, int E, int H, int F, void* w_gu,
-                                cudaStream_t stream);
-cudaError_t gemm_gate_up_packed(const void* xp, const int32_t* offsets, const void* w_gu, int E, long long rows,
-                                int H, int F, void* h, int* status, int* sched, cudaStream_t stream);
 // h = silu(s_x s_g (xq Wg_q^T)) * (s_x s_u (xq Wu_q^T)) on E4M3 operands.
 cudaError_t gemm_gate_up_fp8(const void* xq, const float* xs, const int32_t* offsets, const void* wq_gate,
                              const void* wq_up, const float* s_gate, const float* s_up, int E, long long rows, int H,
@@ -83,18 +81,36 @@ cudaError_t launch_sum_partials(const float* partials, int nsplit, long long n, 
 
 // With nsplit > 1 the logits are the in-order sum of nsplit partial planes (T * E apart) starting
 // at `logits`; the kernel writes that sum to `logits_out` as well.
+// With hist != nullptr every selected id is also added to hist[id] (the count/scan totals).
 cudaError_t launch_route(const float* logits, int nsplit, float* logits_out, long long T, int E, int K,
-                         int renormalize, int P, int group_limit, int32_t* ids, float* w, cudaStream_t stream);
+                         int renormalize, int P, int group_limit, int32_t* ids, float* w, int* hist,
+                         cudaStream_t stream);
 
-// Count/scan workspace: status word, grid-barrier words, per-block histograms.
+// Count/scan state inside a workspace (or the library's own scratch):
+//   [0] status word, [64] ticket, [96] done counter, [128] failure flag (the bytes 160-255
+//   belong to the GEMMs' tile schedules), [256] kScanMaxBlocks look-back flags, then
+//   hist[E], agg[nb][E] and inc[nb][E] (each 256-byte aligned).  The ticket, done counter,
+//   failure flag, flags and hist are zero between calls (the last block of every call clears
+//   them; the workspace starts zeroed).
+constexpr int kScanMaxBlocks = 128;
+inline size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 struct ScanWorkspace {
+  static constexpr size_t kFixedBytes = 256 + kScanMaxBlocks * sizeof(int);
   int* status;
-  unsigned int* bar_count;
-  unsigned int* bar_gen;
-  int* block_counts;   // [max_blocks][E]
-  int max_blocks;
+  int* ticket;
+  int* done;
+  int* fail;
+  int* flags;   // [kScanMaxBlocks]
+  int* hist;    // [E] expert totals of the call
+  int* agg;     // [nb][E] per-block counts
+  int* inc;     // [nb][E] per-block inclusive prefixes over blocks
 };
-int scan_max_blocks(long long TK);
+int scan_blocks(long long TK);                      // blocks (chunks) of one count/scan call
+size_t scan_ws_bytes(long long TK, int E);          // bytes of the state above
+ScanWorkspace scan_workspace(void* base, long long TK, int E);
+// hist[e] += #{a : ids[a] = e} (the caller's ids; the route kernel does this itself when given hist).
+cudaError_t launch_hist(const int32_t* ids, long long TK, int E, const ScanWorkspace& ws, cudaStream_t stream);
+// Needs ws.hist to hold the totals of ids (launch_hist or the route kernel, on the same stream before).
 cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, int32_t* counts, int32_t* offsets,
                               int32_t* part_counts, int32_t* part_offsets, int32_t* row_of_assign,
                               int32_t* assign_of_row, float* skew, const ScanWorkspace& ws, cudaStream_t stream);

@@ -5,8 +5,6 @@
 // router writes a network schedule").  Counts are per token-expert assignment
 // and the skew statistic is the busiest expert's load over the mean load
 // ("Three Parameter Counts...", "What the utilization dashboard smooths away").
-#include <cuda/atomic>
-
 #include <algorithm>
 
 #include "device.cuh"
@@ -47,7 +45,7 @@ constexpr int route_warps(int vpl) { return vpl <= 8 ? 8 : 4; }
 template <int VPL>
 __global__ void __launch_bounds__(32 * route_warps(VPL)) route_kernel(
     const float* __restrict__ logits, int nsplit, float* __restrict__ logits_out, long long T, int E, int K,
-    int renormalize, int P, int M, int32_t* __restrict__ ids, float* __restrict__ w) {
+    int renormalize, int P, int M, int32_t* __restrict__ ids, float* __restrict__ w, int* __restrict__ hist) {
   constexpr int W = route_warps(VPL);
   constexpr unsigned kFull = 0xffffffffu;
   __shared__ alignas(16) uint32_t s_key[W][32 * VPL];
@@ -204,17 +202,18 @@ __global__ void __launch_bounds__(32 * route_warps(VPL)) route_kernel(
     if (lane < K) {
       ids[t * K + lane] = my_id;
       w[t * K + lane] = num / den;
+      if (hist) atomicAdd(hist + my_id, 1);  // expert totals for the count/scan that follows
     }
   }
 }
 
 template <int VPL>
 cudaError_t launch_route_vpl(const float* logits, int nsplit, float* logits_out, long long T, int E, int K,
-                             int renorm, int P, int M, int32_t* ids, float* w, cudaStream_t s) {
+                             int renorm, int P, int M, int32_t* ids, float* w, int* hist, cudaStream_t s) {
   constexpr int W = route_warps(VPL);
   const long long blocks = std::min<long long>((T + W - 1) / W, 64LL * num_sms());
   return launch_pdl(route_kernel<VPL>, dim3(static_cast<unsigned>(std::max<long long>(blocks, 1))), dim3(32 * W), 0,
-                    s, logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w);
+                    s, logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, hist);
 }
 
 // out[i] = sum_{p < nsplit} partials[p * n + i], added in order p = 0, 1, ...
@@ -231,134 +230,106 @@ __global__ void sum_partials_kernel(const float* __restrict__ partials, int nspl
 }
 
 // ---------------------------------------------------------------------------
-// Count + scan + stable rank, one cooperative launch.
-//  phase 1: block b histograms its contiguous slice of assignments -> block_counts[b][e]
-//  grid barrier (bounded wait; all blocks are co-resident by the cooperative launch)
-//  phase 2: offsets[e] = sum of all counts of experts < e; base[b][e] = offsets[e] +
-//           counts of expert e in blocks < b.  Block 0 writes counts, offsets,
-//           partition counts/offsets and the skew ratio.
-//  phase 3: block b walks its slice in order, 256 assignments at a time; the rank of
-//           an assignment among equal ids = earlier warps' counts (shared) + its rank
-//           inside the warp (__match_any_sync); row = base + rank.
+// Count + scan + stable rank: a block-local histogram and a decoupled look-back scan.
+//
+// The expert totals come from a histogram taken before the scan: the route kernel adds
+// every id it writes to hist[E] (the layer path), or expert_hist_kernel counts a caller's
+// ids (moe_count_scan).  count_scan_kernel then makes one pass over the assignments in nb
+// chunks, one block per chunk, the chunk chosen by a ticket the block takes when it
+// starts (so a block only ever waits for blocks that are already running):
+//   1. block histogram of its chunk, kept per warp (warp w owns a contiguous slice);
+//   2. the block publishes its per-expert counts (flag AGG) and looks back over its
+//      predecessors: one warp reads 32 flags at a time, and the counts of the blocks up
+//      to the nearest one that has published an inclusive prefix (flag INC) are added to
+//      that prefix; then it publishes its own inclusive prefix (flag INC);
+//   3. row of assignment a with expert e = offsets[e] (exclusive scan of hist) + the
+//      counts of e in earlier blocks + in earlier warps of this block + the number of
+//      earlier assignments of e in this warp (__match_any_sync): rows of one expert keep
+//      increasing a, a stable counting sort;
+//   4. the last block to finish clears hist and the flags and rewinds the ticket and
+//      the done counter for the next call.
+// Every wait is bounded: a block that gives up sets MOE_DEV_TIMEOUT and scatters nothing.
+// A call that met an invalid id or a wait that ran out leaves offsets[E] = -1.
 // ---------------------------------------------------------------------------
 
 constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
-constexpr int kScanMinChunk = 1024;
+constexpr int kScanMinChunk = 256;
+constexpr int kLookWindow = 32;
+constexpr int kPerThreadE = MOE_MAX_E / kScanThreads;  // experts a thread scans and looks back for
+constexpr int kFlagAgg = 1, kFlagInc = 2;
 
-__device__ bool grid_barrier(unsigned int* count, unsigned int* gen, unsigned int nblocks, int* status,
-                             int* s_ok) {
+__device__ __forceinline__ int ld_acquire(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void st_release(int* p, int v) {
+  asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+// hist[e] += number of ids equal to e (ids outside [0, E) are skipped; count_scan reports them).
+__global__ void __launch_bounds__(kScanThreads) expert_hist_kernel(const int32_t* __restrict__ ids, long long TK,
+                                                                   int E, int* __restrict__ hist) {
+  extern __shared__ int s_h[];
+  for (int e = threadIdx.x; e < E; e += kScanThreads) s_h[e] = 0;
+  pdl_wait();
+  pdl_launch_dependents();
   __syncthreads();
-  if (threadIdx.x == 0) {
-    cuda::atomic_ref<unsigned int, cuda::thread_scope_device> c(*count), g(*gen);
-    const unsigned int my_gen = g.load(cuda::memory_order_acquire);
-    const unsigned int arrived = c.fetch_add(1u, cuda::memory_order_acq_rel);
-    int ok = 1;
-    if (arrived == nblocks - 1) {
-      c.store(0u, cuda::memory_order_relaxed);
-      g.fetch_add(1u, cuda::memory_order_release);
-    } else {
-      const uint64_t t0 = global_timer_ns();
-      unsigned int i = 0;
-      while (g.load(cuda::memory_order_acquire) == my_gen) {
-        if ((++i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
-          report(status, MOE_DEV_TIMEOUT);
-          ok = 0;
-          break;
-        }
-      }
-    }
-    *s_ok = ok;
+  const long long stride = static_cast<long long>(gridDim.x) * kScanThreads;
+  for (long long a = static_cast<long long>(blockIdx.x) * kScanThreads + threadIdx.x; a < TK; a += stride) {
+    const int e = __ldg(ids + a);
+    if (e >= 0 && e < E) atomicAdd(&s_h[e], 1);
   }
   __syncthreads();
-  return *s_ok != 0;
+  for (int e = threadIdx.x; e < E; e += kScanThreads)
+    if (s_h[e]) atomicAdd(hist + e, s_h[e]);
 }
 
 __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
-    const int32_t* __restrict__ ids, int TK, int E, int P, int chunk, int32_t* __restrict__ counts,
+    const int32_t* __restrict__ ids, int TK, int E, int P, int chunk, int nb, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int32_t* __restrict__ part_counts, int32_t* __restrict__ part_offsets,
     int32_t* __restrict__ row_of_assign, int32_t* __restrict__ assign_of_row, float* __restrict__ skew,
-    int* block_counts, unsigned int* bar_count, unsigned int* bar_gen, int* status) {
+    const ScanWorkspace ws) {
   extern __shared__ int sm[];
-  int* s_hist = sm;                    // [E]   this block's histogram, then its running base
-  int* s_off = s_hist + E;             // [E+1] global exclusive offsets
-  int* s_wcnt = s_off + E + 1;         // [kScanWarps][E] per-warp counts of one 256-slice
-  __shared__ int s_ok, s_bad, s_red[kScanWarps], s_max[kScanWarps];
+  int* s_run = sm;                        // [kScanWarps][E] warp counts, then each warp's next row
+  int* s_agg = s_run + kScanWarps * E;    // [E] this block's counts
+  int* s_off = s_agg + E;                 // [E + 1] exclusive scan of the totals
+  __shared__ int s_b, s_bad, s_ok, s_last, s_nwin, s_incpos, s_red[kScanWarps], s_max[kScanWarps];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int b = blockIdx.x;
-  const int lo = min(TK, b * chunk), hi = min(TK, lo + chunk);
-
-  for (int e = tid; e < E; e += kScanThreads) s_hist[e] = 0;
-  for (int i = tid; i < kScanWarps * E; i += kScanThreads) s_wcnt[i] = 0;
-  if (tid == 0) s_bad = 0;
-  pdl_wait();  // the expert ids come from the route kernel
+  for (int i = tid; i < kScanWarps * E; i += kScanThreads) s_run[i] = 0;
+  pdl_wait();  // the ids and the histogram come from the previous kernel
   pdl_launch_dependents();
-  __syncthreads();
-
-  // phase 1
-  for (int a = lo + tid; a < hi; a += kScanThreads) {
-    const int e = __ldg(ids + a);
-    if (e >= 0 && e < E) atomicAdd(&s_hist[e], 1);
-    else s_bad = 1;
+  if (tid == 0) {
+    s_b = atomicAdd(ws.ticket, 1);
+    s_bad = 0;
+    s_ok = s_b < nb;  // a ticket beyond the grid: the previous call on this workspace did not finish
+    if (!s_ok) report(ws.status, MOE_DEV_TIMEOUT);
   }
-  __syncthreads();
-  if (s_bad && tid == 0) report(status, MOE_DEV_BAD_INDEX);
-  for (int e = tid; e < E; e += kScanThreads) block_counts[static_cast<long long>(b) * E + e] = s_hist[e];
 
-  if (!grid_barrier(bar_count, bar_gen, gridDim.x, status, &s_ok)) return;
-
-  // phase 2: column sums over blocks.  The block_counts rows start 16-byte aligned (the
-  // workspace is 256-byte aligned), so with E % 4 == 0 a thread sums four experts per
-  // 16-byte load and keeps eight loads in flight.
+  // global exclusive offsets from the totals (up to 4 experts per thread)
   int my_max = 0;
-  const int nb = static_cast<int>(gridDim.x);
-  if ((E & 3) == 0) {
-    const int E4 = E >> 2;
-    for (int q = tid; q < E4; q += kScanThreads) {
-      const int4* col = reinterpret_cast<const int4*>(block_counts) + q;
-      int4 before = make_int4(0, 0, 0, 0), total = make_int4(0, 0, 0, 0);
-#pragma unroll 8
-      for (int bb = 0; bb < nb; ++bb) {
-        const int4 c = __ldcg(col + static_cast<long long>(bb) * E4);
-        if (bb < b) before.x += c.x, before.y += c.y, before.z += c.z, before.w += c.w;
-        total.x += c.x, total.y += c.y, total.z += c.z, total.w += c.w;
-      }
-      const int e = 4 * q;
-      s_hist[e] = before.x, s_hist[e + 1] = before.y, s_hist[e + 2] = before.z, s_hist[e + 3] = before.w;
-      s_off[e] = total.x, s_off[e + 1] = total.y, s_off[e + 2] = total.z, s_off[e + 3] = total.w;
-      my_max = max(my_max, max(max(total.x, total.y), max(total.z, total.w)));
-    }
-  } else {
-    for (int e = tid; e < E; e += kScanThreads) {
-      int before = 0, total = 0;
-#pragma unroll 8
-      for (int bb = 0; bb < nb; ++bb) {
-        const int c = __ldcg(block_counts + static_cast<long long>(bb) * E + e);
-        before += (bb < b) ? c : 0;
-        total += c;
-      }
-      s_hist[e] = before;
-      s_off[e] = total;
-      my_max = max(my_max, total);
-    }
-  }
-  __syncthreads();
-  // exclusive scan of s_off[0..E) in place (E <= 1024: 4 per thread)
   {
     const int per = (E + kScanThreads - 1) / kScanThreads;
     const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
     int local = 0;
-    for (int e = e0; e < e1; ++e) local += s_off[e];
+    for (int e = e0; e < e1; ++e) {
+      const int c = __ldcg(ws.hist + e);
+      s_off[e] = c;
+      local += c;
+      my_max = max(my_max, c);
+    }
     int incl = local;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    if (lane == 31) s_red[warp] = incl;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, o));
+    if (lane == 31) s_red[warp] = incl;
     if (lane == 0) s_max[warp] = my_max;
     __syncthreads();
     int wbase = 0, total = 0, mx = 0;
@@ -368,7 +339,6 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
       mx = max(mx, s_max[w]);
     }
     int run = wbase + incl - local;
-    __syncthreads();
     for (int e = e0; e < e1; ++e) {
       const int c = s_off[e];
       s_off[e] = run;
@@ -376,7 +346,7 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
     }
     if (tid == 0) s_off[E] = total;
     __syncthreads();
-    if (b == 0) {
+    if (s_b == 0) {  // the block holding ticket 0 writes the per-expert outputs
       for (int e = tid; e <= E; e += kScanThreads) {
         offsets[e] = s_off[e];
         if (e < E) counts[e] = s_off[e + 1] - s_off[e];
@@ -389,36 +359,170 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
       if (tid == 0 && skew) skew[0] = total > 0 ? static_cast<float>(mx) * static_cast<float>(E) / total : 0.0f;
     }
   }
-  for (int e = tid; e < E; e += kScanThreads) s_hist[e] += s_off[e];
-  __syncthreads();
 
-  // phase 3
+  const int b = s_b;
+  const bool active = s_ok;  // block-uniform
+  const int lo = min(TK, b * chunk), hi = min(TK, lo + chunk);
+  const int sub = ((chunk + kScanWarps - 1) / kScanWarps + 31) & ~31;
+  const int wlo = min(hi, lo + warp * sub), whi = min(hi, wlo + sub);
   const unsigned lt_mask = (1u << lane) - 1u;
-  for (int base = lo; base < hi; base += kScanThreads) {
-    const int a = base + tid;
-    int e = -1;
-    if (a < hi) {
-      e = __ldg(ids + a);
-      if (e < 0 || e >= E) e = -1;
-    }
-    const unsigned same = __match_any_sync(0xffffffffu, e);
-    const int leader = __ffs(same) - 1;
-    const int rank_in_warp = __popc(same & lt_mask);
-    if (e >= 0 && lane == leader) s_wcnt[warp * E + e] = __popc(same);
-    __syncthreads();
-    if (a < hi && e < 0) row_of_assign[a] = -1;  // an invalid id gets no row
-    if (e >= 0) {
-      int r = s_hist[e] + rank_in_warp;
-      for (int w = 0; w < warp; ++w) r += s_wcnt[w * E + e];
-      row_of_assign[a] = r;
-      assign_of_row[r] = a;
-    }
-    __syncthreads();
-    if (e >= 0 && lane == leader) {
-      atomicAdd(&s_hist[e], __popc(same));
-      s_wcnt[warp * E + e] = 0;
+  int excl[kPerThreadE];
+#pragma unroll
+  for (int j = 0; j < kPerThreadE; ++j) excl[j] = 0;
+
+  if (active) {
+    // 1. counts of this warp's slice
+    for (int base = wlo; base < whi; base += 32) {
+      const int a = base + lane;
+      int e = -1;
+      if (a < whi) {
+        e = __ldg(ids + a);
+        if (e < 0 || e >= E) {
+          e = -1;
+          s_bad = 1;
+        }
+      }
+      const unsigned same = __match_any_sync(0xffffffffu, e);
+      if (e >= 0 && lane == __ffs(same) - 1) s_run[warp * E + e] += __popc(same);
+      __syncwarp();
     }
     __syncthreads();
+    // per expert: counts of the earlier warps of the block, and the block's count, published
+    int* my_row = (b == 0 ? ws.inc : ws.agg) + static_cast<long long>(b) * E;
+    for (int e = tid; e < E; e += kScanThreads) {
+      int run = 0;
+#pragma unroll
+      for (int w = 0; w < kScanWarps; ++w) {
+        const int c = s_run[w * E + e];
+        s_run[w * E + e] = run;
+        run += c;
+      }
+      s_agg[e] = run;
+      __stcg(my_row + e, run);
+    }
+    __syncthreads();
+    if (tid == 0) {
+      __threadfence();
+      st_release(ws.flags + b, b == 0 ? kFlagInc : kFlagAgg);
+    }
+    // 2. look back over the predecessors, kLookWindow blocks at a time
+    int top = b - 1;
+    while (top >= 0) {
+      if (warp == 0) {
+        const int p = top - lane;
+        int f = 0;
+        bool ok = true;
+        if (p >= 0) {
+          f = ld_acquire(ws.flags + p);
+          if (f == 0) {
+            const uint64_t t0 = global_timer_ns();
+            unsigned int i = 0;
+            while ((f = ld_acquire(ws.flags + p)) == 0) {
+              if ((++i & 63u) == 0 && global_timer_ns() - t0 > kWaitLimitNs) {
+                ok = false;
+                break;
+              }
+            }
+          }
+        }
+        const unsigned okm = __ballot_sync(0xffffffffu, ok);
+        const unsigned incm = __ballot_sync(0xffffffffu, p >= 0 && f == kFlagInc);
+        if (lane == 0) {
+          if (okm != 0xffffffffu) {
+            s_ok = 0;
+            report(ws.status, MOE_DEV_TIMEOUT);
+          }
+          // lanes before the first INC carry counts (AGG); block 0 is INC, so a window that
+          // reaches it always ends in an INC
+          s_incpos = incm ? __ffs(incm) - 1 : -1;
+          s_nwin = incm ? __ffs(incm) : min(kLookWindow, top + 1);
+        }
+      }
+      __syncthreads();
+      if (!s_ok) break;
+      const int n = s_nwin, ip = s_incpos;
+#pragma unroll
+      for (int j = 0; j < kPerThreadE; ++j) {
+        const int e = tid + j * kScanThreads;
+        if (e < E) {
+          int acc = 0;
+          for (int i = 0; i < n; ++i) {
+            const int* src = (i == ip) ? ws.inc : ws.agg;
+            acc += __ldcg(src + static_cast<long long>(top - i) * E + e);
+          }
+          excl[j] += acc;
+        }
+      }
+      if (ip >= 0) break;
+      top -= kLookWindow;
+      __syncthreads();  // s_nwin and s_incpos are rewritten
+    }
+    __syncthreads();
+  }
+  if (active && s_ok) {
+    if (b > 0) {
+      for (int j = 0; j < kPerThreadE; ++j) {
+        const int e = tid + j * kScanThreads;
+        if (e < E) __stcg(ws.inc + static_cast<long long>(b) * E + e, excl[j] + s_agg[e]);
+      }
+      __syncthreads();
+      if (tid == 0) {
+        __threadfence();
+        st_release(ws.flags + b, kFlagInc);
+      }
+    }
+    // 3. each warp's first row per expert, then the rows of its slice in order
+#pragma unroll
+    for (int j = 0; j < kPerThreadE; ++j) {
+      const int e = tid + j * kScanThreads;
+      if (e < E) {
+        const int base = s_off[e] + excl[j];
+#pragma unroll
+        for (int w = 0; w < kScanWarps; ++w) s_run[w * E + e] += base;
+      }
+    }
+    __syncthreads();
+    for (int base = wlo; base < whi; base += 32) {
+      const int a = base + lane;
+      int e = -1;
+      if (a < whi) {
+        e = __ldg(ids + a);
+        if (e < 0 || e >= E) e = -1;
+      }
+      const unsigned same = __match_any_sync(0xffffffffu, e);
+      if (a < whi) {
+        if (e < 0) {
+          row_of_assign[a] = -1;  // an invalid id gets no row
+        } else {
+          const int r = s_run[warp * E + e] + __popc(same & lt_mask);
+          row_of_assign[a] = r;
+          assign_of_row[r] = a;
+        }
+      }
+      __syncwarp();
+      if (e >= 0 && lane == __ffs(same) - 1) s_run[warp * E + e] += __popc(same);
+      __syncwarp();
+    }
+  }
+
+  // 4. the last block rewinds the workspace for the next call
+  __syncthreads();
+  if (tid == 0) {
+    if (s_bad) report(ws.status, MOE_DEV_BAD_INDEX);
+    if (s_bad || !s_ok) atomicOr(ws.fail, 1);
+    __threadfence();
+    s_last = atomicAdd(ws.done, 1) == nb - 1;
+  }
+  __syncthreads();
+  if (s_last) {
+    __threadfence();
+    for (int e = tid; e < E; e += kScanThreads) ws.hist[e] = 0;
+    for (int p = tid; p < kScanMaxBlocks; p += kScanThreads) ws.flags[p] = 0;
+    if (tid == 0) {
+      if (atomicExch(ws.fail, 0)) offsets[E] = -1;  // after ticket 0's write: every block is done
+      *ws.ticket = 0;
+      *ws.done = 0;
+    }
   }
 }
 
@@ -444,7 +548,7 @@ __global__ void skew_kernel(const int32_t* __restrict__ counts, int E, float* ra
   }
 }
 
-size_t scan_smem_bytes(int E) { return static_cast<size_t>(E * 2 + 1 + kScanWarps * E) * sizeof(int); }
+size_t scan_smem_bytes(int E) { return static_cast<size_t>(kScanWarps * E + E + E + 1) * sizeof(int); }
 
 }  // namespace
 
@@ -456,61 +560,65 @@ cudaError_t launch_sum_partials(const float* partials, int nsplit, long long n, 
 }
 
 cudaError_t launch_route(const float* logits, int nsplit, float* logits_out, long long T, int E, int K, int renorm,
-                         int P, int M, int32_t* ids,
-                         float* w, cudaStream_t s) {
+                         int P, int M, int32_t* ids, float* w, int* hist, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int vpl = (E + 31) / 32;
-  if (vpl <= 1) return launch_route_vpl<1>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
-  if (vpl <= 2) return launch_route_vpl<2>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
-  if (vpl <= 4) return launch_route_vpl<4>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
-  if (vpl <= 8) return launch_route_vpl<8>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
-  if (vpl <= 16) return launch_route_vpl<16>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
-  return launch_route_vpl<32>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s);
+#define MOE_ROUTE(V) launch_route_vpl<V>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, hist, s)
+  if (vpl <= 1) return MOE_ROUTE(1);
+  if (vpl <= 2) return MOE_ROUTE(2);
+  if (vpl <= 4) return MOE_ROUTE(4);
+  if (vpl <= 8) return MOE_ROUTE(8);
+  if (vpl <= 16) return MOE_ROUTE(16);
+  return MOE_ROUTE(32);
+#undef MOE_ROUTE
 }
 
-int scan_max_blocks(long long TK) {
+int scan_blocks(long long TK) {
   const long long b = (TK + kScanMinChunk - 1) / kScanMinChunk;
-  return static_cast<int>(std::max<long long>(1, std::min<long long>(b, 1024)));
+  return static_cast<int>(std::max<long long>(1, std::min<long long>(b, kScanMaxBlocks)));
+}
+
+size_t scan_ws_bytes(long long TK, int E) {
+  const size_t rows = static_cast<size_t>(scan_blocks(TK)) * E * sizeof(int);
+  return ScanWorkspace::kFixedBytes + round256(static_cast<size_t>(E) * sizeof(int)) + 2 * round256(rows);
+}
+
+ScanWorkspace scan_workspace(void* base, long long TK, int E) {
+  uint8_t* p = static_cast<uint8_t*>(base);
+  ScanWorkspace w;
+  w.status = reinterpret_cast<int*>(p);
+  w.ticket = reinterpret_cast<int*>(p + 64);
+  w.done = reinterpret_cast<int*>(p + 96);
+  w.fail = reinterpret_cast<int*>(p + 128);
+  w.flags = reinterpret_cast<int*>(p + 256);
+  size_t off = ScanWorkspace::kFixedBytes;
+  w.hist = reinterpret_cast<int*>(p + off);
+  off += round256(static_cast<size_t>(E) * sizeof(int));
+  const size_t rows = round256(static_cast<size_t>(scan_blocks(TK)) * E * sizeof(int));
+  w.agg = reinterpret_cast<int*>(p + off);
+  w.inc = reinterpret_cast<int*>(p + off + rows);
+  return w;
+}
+
+cudaError_t launch_hist(const int32_t* ids, long long TK, int E, const ScanWorkspace& ws, cudaStream_t s) {
+  if (TK == 0) return cudaSuccess;
+  const long long blocks = std::min<long long>((TK + 4 * kScanThreads - 1) / (4 * kScanThreads), num_sms());
+  return launch_pdl(expert_hist_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kScanThreads),
+                    static_cast<size_t>(E) * sizeof(int), s, ids, TK, E, ws.hist);
 }
 
 cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, int32_t* counts, int32_t* offsets,
                               int32_t* part_counts, int32_t* part_offsets, int32_t* row_of_assign,
                               int32_t* assign_of_row, float* skew, const ScanWorkspace& ws, cudaStream_t s) {
-  const size_t smem = scan_smem_bytes(E);
   static std::atomic<int> attr_done[kMaxDevices] = {};
   const cudaError_t attr = smem_attr_once(reinterpret_cast<const void*>(count_scan_kernel),
                                           static_cast<int>(scan_smem_bytes(MOE_MAX_E)), attr_done);
   if (attr != cudaSuccess) return attr;
-  int occ = 0;
-  cudaError_t err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, count_scan_kernel, kScanThreads, smem);
-  if (err != cudaSuccess) return err;
-  const long long resident = static_cast<long long>(std::max(occ, 1)) * num_sms();
-  int blocks = static_cast<int>(std::min<long long>({static_cast<long long>(ws.max_blocks), resident,
-                                                     std::max<long long>(1, (TK + kScanMinChunk - 1) / kScanMinChunk)}));
-  blocks = std::max(blocks, 1);
-  long long chunk = (TK + blocks - 1) / blocks;
-  chunk = (chunk + kScanThreads - 1) / kScanThreads * kScanThreads;
-  int TKi = static_cast<int>(TK), chunki = static_cast<int>(std::max<long long>(chunk, kScanThreads));
-  int* block_counts = ws.block_counts;
-  unsigned int* bc = ws.bar_count;
-  unsigned int* bg = ws.bar_gen;
-  int* status = ws.status;
-  // Cooperative (the grid barrier needs every block resident) and programmatic: the blocks may
-  // start while the route kernel drains and wait for it in griddepcontrol.wait.
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(blocks);
-  cfg.blockDim = dim3(kScanThreads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr2[2];
-  attr2[0].id = cudaLaunchAttributeCooperative;
-  attr2[0].val.cooperative = 1;
-  attr2[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr2[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr2;
-  cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, count_scan_kernel, ids, TKi, E, P, chunki, counts, offsets, part_counts,
-                            part_offsets, row_of_assign, assign_of_row, skew, block_counts, bc, bg, status);
+  const int nb = scan_blocks(TK);
+  const long long chunk = (TK + nb - 1) / nb;
+  return launch_pdl(count_scan_kernel, dim3(nb), dim3(kScanThreads), scan_smem_bytes(E), s, ids,
+                    static_cast<int>(TK), E, P, static_cast<int>(chunk), nb, counts, offsets, part_counts,
+                    part_offsets, row_of_assign, assign_of_row, skew, ws);
 }
 
 cudaError_t launch_skew(const int32_t* counts, int E, float* ratio, cudaStream_t s) {

@@ -85,3 +85,14 @@ def test_p95_host_helper_matches_oracle(lib, n):
     r = np.random.default_rng(n).uniform(1, 6, n).astype(np.float32)
     assert binding.moe_p95(list(r)) == pytest.approx(oracle.p95_nearest_rank(r), abs=0)
     assert math.isnan(lib.moe_p95(None, 0))
+
+
+def test_noalloc_count_scan_returns_the_same_shape_codes(lib):
+    # the scratch-free call checks shapes exactly like moe_count_scan (checked before any device use)
+    for d, code in ((binding.dims(T=4, H=64, E=1025, K=2, F=64), 2),      # E > MOE_MAX_E
+                    (binding.dims(T=4, H=64, E=64, K=33, F=64), 2),       # K > MOE_MAX_K
+                    (binding.dims(T=1 << 30, H=64, E=64, K=8, F=64), 2),  # T*K beyond int32
+                    (binding.dims(T=4, H=64, E=8, K=9, F=64), 1)):        # K > E
+        a = lib.moe_count_scan(None, C.byref(d), None, None, None, None, None, None, None, 0, None)
+        b = lib.moe_count_scan_noalloc(None, C.byref(d), None, None, None, None, None, None, None)
+        assert a == b == code

@@ -125,6 +125,8 @@ SCAN_CASES = [  # T, E, K, P, zipf
     (64, 8, 2, 1, None), (300, 16, 4, 4, None), (1, 4, 4, 2, None), (0, 8, 2, 1, None),
     (128, 256, 8, 8, 1.1), (4096, 128, 8, 1, None), (8192, 256, 8, 8, None), (4096, 896, 16, 64, None),
     (3000, 1024, 3, 16, 2.0), (5000, 7, 7, 7, None), (20000, 64, 6, 4, 1.1),
+    # 128 chunks of 2048 assignments, four experts per thread in the look-back; all ids on one expert
+    (32768, 1024, 8, 8, 1.1), (32768, 64, 8, 4, None), (4000, 1, 1, 1, None),
 ]
 
 
@@ -177,22 +179,46 @@ def test_count_scan_flags_out_of_range_ids():
     flat = ids.numpy().reshape(-1)
     assert got["counts"].sum() == int(((flat >= 0) & (flat < 16)).sum())
     assert got["row_of_assign"][17 * 2 + 1] == -1 and got["row_of_assign"][100] == -1
+    assert got["offsets"][16] == -1          # the call is marked failed
 
 
-def test_count_scan_barrier_wait_times_out_and_reports():
-    # A grid-barrier counter that can never reach its target (set on the host):
-    # every block's bounded wait must give up, report MOE_DEV_TIMEOUT and return.
-    ids = inputs.random_topk_ids(4000, 32, 4, seed=9)
-    d = B.dims(T=4000, H=8, E=32, K=4, F=8)
+def test_count_scan_lookback_wait_times_out_and_reports():
+    # A block ticket counter that starts at 1 (set on the host): no block draws ticket 0, so
+    # the first chunk's flag is never published and every look-back that reaches it must
+    # give up after its bounded wait, report MOE_DEV_TIMEOUT and mark the call failed.
+    T, E, K = 4000, 32, 4
+    ids = inputs.random_topk_ids(T, E, K, seed=9)
+    d = B.dims(T=T, H=8, E=E, K=K, F=8)
     ws = B.make_workspace(d)
-    ws[64:68] = torch.tensor([0xF0, 0xFF, 0xFF, 0x7F], dtype=torch.uint8, device=DEV)
-    bufs = [torch.empty(n, dtype=torch.int32, device=DEV) for n in (32, 33, 1, 2, 16000, 16000)]
+    ws[64:68] = torch.tensor([1, 0, 0, 0], dtype=torch.uint8, device=DEV)
+    bufs = [torch.empty(n, dtype=torch.int32, device=DEV) for n in (E, E + 1, 1, 2, T * K, T * K)]
     B.moe_count_scan(ids.to(DEV), d, *bufs, ws)
     assert B.read_device_status(ws) & B.DEV_TIMEOUT
-    B.workspace_init(ws)   # the context stays usable: the next call works
+    assert int(bufs[1][E]) == -1
+    # the kernels rewound their state: the context stays usable and the next call works
+    B.workspace_init(ws)
     B.moe_count_scan(ids.to(DEV), d, *bufs, ws)
     assert B.read_device_status(ws) == 0
-    assert np.array_equal(cpu(bufs[4]), oracle.count_scan(ids.numpy(), 32)["row_of_assign"])
+    want = oracle.count_scan(ids.numpy(), E)
+    assert np.array_equal(cpu(bufs[4]), want["row_of_assign"])
+    assert np.array_equal(cpu(bufs[1]), want["offsets"])
+
+
+def test_count_scan_state_is_rewound_without_reinit():
+    # after a normal call the kernels leave ticket, flags and totals at zero: many calls of
+    # different sizes on one workspace (sized for the largest) stay exact
+    E, K, P = 64, 4, 4
+    d = B.dims(T=9000, H=8, E=E, K=K, F=8, P=P)
+    ws = B.make_workspace(d)
+    for i, T in enumerate((9000, 1, 300, 64, 9000, 0, 257)):
+        ids = inputs.random_topk_ids(T, E, K, seed=40 + i) if T else torch.zeros((0, K), dtype=torch.int32)
+        di = B.dims(T=T, H=8, E=E, K=K, F=8, P=P)
+        bufs = [torch.full((n,), -7, dtype=torch.int32, device=DEV) for n in (E, E + 1, P, P + 1, T * K, T * K)]
+        B.moe_count_scan(ids.to(DEV), di, *bufs, ws)
+        want = oracle.count_scan(ids.numpy(), E, P)
+        for k, a in zip(("counts", "offsets", "part_counts", "part_offsets", "row_of_assign", "assign_of_row"), bufs):
+            assert np.array_equal(cpu(a), want[k]), (T, k)
+    assert B.read_device_status(ws) == 0
 
 
 # ---------------------------------------------------------------------------
@@ -262,21 +288,15 @@ def ffn_inputs(E, H, F, rows, zipf, zero_frac, seed=0):
     return off, xp, wg, wu, wd
 
 
-@pytest.mark.parametrize("packed", [False, True], ids=["separate", "packed"])
 @pytest.mark.parametrize("E,H,F,rows,zipf,zf", FFN_CASES)
-def test_grouped_ffn_matches_oracle(E, H, F, rows, zipf, zf, packed, gemm_kernel):
+def test_grouped_ffn_matches_oracle(E, H, F, rows, zipf, zf, gemm_kernel):
     off, xp, wg, wu, wd = ffn_inputs(E, H, F, rows, zipf, zf)
     d = B.dims(T=rows, H=H, E=E, K=1, F=F)
     ws = B.make_workspace(d)
     h = torch.zeros((rows, F), dtype=torch.bfloat16, device=DEV)
     y = torch.zeros((rows, H), dtype=torch.bfloat16, device=DEV)
     offd = torch.from_numpy(off).to(DEV)
-    if packed:
-        w_gu = B.pack_gate_up(wg.to(DEV), wu.to(DEV), d)
-        B.moe_grouped_gate_up_packed(xp.to(DEV), offd, w_gu, d, h, ws)
-        B.moe_grouped_down(h, offd, wd.to(DEV), d, y, ws)
-    else:
-        B.moe_grouped_ffn(xp.to(DEV), offd, wg.to(DEV), wu.to(DEV), wd.to(DEV), d, h, y, ws)
+    B.moe_grouped_ffn(xp.to(DEV), offd, wg.to(DEV), wu.to(DEV), wd.to(DEV), d, h, y, ws)
     assert B.read_device_status(ws) == 0
     rh, ry = oracle.grouped_ffn(bits(xp), off, bits(wg), bits(wu), bits(wd))
     check_bf16("h", bits(h), rh)
@@ -400,23 +420,6 @@ def test_grouped_gemms_run_on_a_header_only_workspace():
     with pytest.raises(B.MoEError):
         B.moe_grouped_ffn(xp.to(DEV), torch.from_numpy(off).to(DEV), wg.to(DEV), wu.to(DEV), wd.to(DEV), d, h, y,
                           ws[:128])
-
-
-def test_pack_gate_up_layout():
-    # packed rows [128 j, 128 j + 64) = gate rows [64 j, +64), next 64 = up rows; padding rows zero
-    E, H, F = 3, 16, 136
-    wg = inputs.random_bf16((E, F, H), seed=1)
-    wu = inputs.random_bf16((E, F, H), seed=2)
-    d = B.dims(T=1, H=H, E=E, K=1, F=F)
-    w_gu = B.pack_gate_up(wg.to(DEV), wu.to(DEV), d).view(E, -1, H).cpu()
-    Fp = 192
-    assert w_gu.shape[1] == 2 * Fp
-    for j in range(Fp // 64):
-        for half, src in ((0, wg), (1, wu)):
-            rows = w_gu[:, 128 * j + 64 * half: 128 * j + 64 * half + 64]
-            n = max(0, min(64, F - 64 * j))
-            assert torch.equal(rows[:, :n].view(torch.int16), src[:, 64 * j: 64 * j + n].view(torch.int16))
-            assert int(rows[:, n:].view(torch.int16).abs().sum()) == 0
 
 
 def test_grouped_down_alone_matches_oracle(gemm_kernel):

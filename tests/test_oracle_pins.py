@@ -412,6 +412,52 @@ def test_layer_forward_tiny_is_consistent():
     assert np.array_equal(oracle.f64_to_bf16_bits(acc), r["out"][t])
 
 
+def test_latent_layer_routes_and_dispatches_z_and_projects_the_combined_output():
+    # "Latent MoE" (Definition, Current Synthesis): the experts see the narrower projected state z.
+    # With a permutation W_dp (not an involution), z = x[:, perm] exactly: the router must rank
+    # z W_g (routing on x gives other experts here) and the dispatched rows must be rows of z.
+    # With W_upp rows that add two columns of their input, final = bf16(out[:, a] + out[:, b]) of
+    # the combined output (one rounding); a projection applied to the expert rows before the
+    # combine rounds differently somewhere.
+    rng = np.random.default_rng(5)
+    T, D, E, K, F = 64, 8, 6, 2, 16
+    x = bf(rng.standard_normal((T, D)))
+    perm = np.array([3, 0, 6, 1, 7, 2, 5, 4])
+    w_dp = np.zeros((D, D))
+    w_dp[np.arange(D), perm] = 1.0
+    w_g = rng.standard_normal((D, E)).astype(np.float32)
+    wg = bf(rng.standard_normal((E, F, D)) * 0.5)
+    wu = bf(rng.standard_normal((E, F, D)) * 0.5)
+    wd = bf(rng.standard_normal((E, D, F)) * 0.25)
+    a_idx, b_idx = np.arange(D), (np.arange(D) + 3) % D
+    w_upp = np.zeros((D, D))
+    w_upp[np.arange(D), a_idx] = 1.0
+    w_upp[np.arange(D), b_idx] = 1.0
+    r = oracle.layer_forward(x, w_g, wg, wu, wd, K, 1, w_dp_bits=bf(w_dp), w_upp_bits=bf(w_upp))
+    z = x[:, perm]
+    assert np.array_equal(r["z"], z)
+
+    def topk_by_definition(l):
+        return np.array([sorted(range(E), key=lambda e: (-float(l[t, e]), e))[:K] for t in range(T)])
+
+    want = topk_by_definition((val(z) @ w_g.astype(np.float64)).astype(np.float32))
+    assert np.array_equal(r["topk_ids"], want)
+    assert not np.array_equal(topk_by_definition((val(x) @ w_g.astype(np.float64)).astype(np.float32)), want)
+    roa = r["row_of_assign"].reshape(T, K)
+    for t in range(T):
+        for k in range(K):
+            assert np.array_equal(r["xp"][roa[t, k]], z[t])
+    out = val(r["out"])
+    assert np.array_equal(r["final"], bf(out[:, a_idx] + out[:, b_idx]))
+    y, w = val(r["y"]), r["topk_w"].astype(np.float64)
+    early = np.zeros((T, D))
+    for t in range(T):
+        for k in range(K):
+            row = y[roa[t, k]]
+            early[t] += w[t, k] * val(bf(row[a_idx] + row[b_idx]))
+    assert not np.array_equal(bf(early), r["final"])
+
+
 # ---------------------------------------------------------------------------
 # Figures the pages print
 # ---------------------------------------------------------------------------
