@@ -426,6 +426,95 @@ moe_status moe_layer_forward_host(const void* x_host, void* x_dev, const moe_lay
                                   const moe_dims* d, const moe_layer_buffers* b, void* ws,
                                   size_t ws_bytes, void* out_host, void* stream);
 
+/* ------------------------------------------------------------------------- */
+/* Expert-parallel exchange across GPUs (one process per GPU, R ranks)       */
+/* The experts are split evenly over the ranks (WideEP essay, "896 experts  */
+/* across 64 ranks"; EP8 = 32 of 256 experts per GPU in the InferenceX v2   */
+/* review, claim IX2-0384); each rank routes its own tokens, counts what    */
+/* every destination receives, reserves the rows there and sends the        */
+/* activations; the experts' outputs come back to be weighted and summed    */
+/* (WideEP essay, "The router writes a network schedule"), about T*K*H*b    */
+/* bytes each way ("Top-k multiplies traffic. Locality subtracts it.").      */
+/*                                                                           */
+/* Protocol, per layer call with an epoch number that every rank increases  */
+/* in step (1, 2, ...):                                                      */
+/*   1. each rank: route and moe_count_scan of its T tokens with P = R (the */
+/*      partitions are the ranks: rank d owns experts [d*El, (d+1)*El),     */
+/*      El = E / R); every rank has the same T;                             */
+/*   2. all-gather of the E per-expert counts of every rank into C [R][E]   */
+/*      (the caller's collective, e.g. NCCL on the same stream);            */
+/*   3. moe_ep_plan (C on the device), moe_ep_dispatch;                     */
+/*   4. moe_ep_wait(phase 0); grouped gate/up and down on the received rows  */
+/*      (moe_grouped_ffn with recv_offsets, E = El local experts);           */
+/*   5. moe_ep_return; moe_ep_wait(phase 1); moe_combine on ret_y with the   */
+/*      rank's own row_of_assign and weights.                                */
+/* Rank d's receive buffer holds its experts' rows expert-major, then by    */
+/* source rank, then in the source's stable order: the single-GPU layout of */
+/* all ranks' tokens concatenated in rank order, restricted to its experts. */
+/* The transfers are plain 16-byte stores into the peers' memory (CUDA IPC   */
+/* mappings, NVLink), no TMA and no multicast; each kernel's last block     */
+/* publishes the epoch in every peer's signal pad with system-scope release */
+/* stores, and moe_ep_wait acquires them (2 s limit, then MOE_DEV_TIMEOUT). */
+/* Buffers: recv_x [cap][H] bf16 and recv_meta [cap][2] int32 (source rank, */
+/* source row) with cap = R*T*K (every assignment of every rank may land on */
+/* one rank: no capacity factor, no dropped tokens), ret_y [T*K][H] bf16,    */
+/* signal [2][R] int32 zeroed once; all four are read or written by peers.   */
+/* ------------------------------------------------------------------------- */
+
+#define MOE_EP_MAX_RANKS 64
+#define MOE_EP_IPC_HANDLE_BYTES 64
+
+/* Device addresses, valid in the calling process, of every rank's exchange buffers
+ * (entries [0, R); this rank's own buffers at index rank). */
+typedef struct moe_ep_peers {
+  void*    recv_x[MOE_EP_MAX_RANKS];
+  int32_t* recv_meta[MOE_EP_MAX_RANKS];
+  void*    ret_y[MOE_EP_MAX_RANKS];
+  int32_t* signal[MOE_EP_MAX_RANKS];
+} moe_ep_peers;
+
+/* Bytes of the EP workspace (status word and the two kernels' done counters), zeroed once
+ * with moe_workspace_init; one per rank, one stream at a time. */
+size_t moe_ep_workspace_bytes(void);
+
+/* From C [R][E] (device int32): send_base[E], the row of rank d = e / El's receive buffer at
+ * which this rank's rows of expert e start, and recv_offsets[El + 1], this rank's received
+ * rows per local expert (the grouped GEMM's offsets).  One block on `stream`. */
+moe_status moe_ep_plan(const int32_t* counts_all, int32_t R, int32_t rank, const moe_dims* d,
+                       int32_t* send_base, int32_t* recv_offsets, void* stream);
+/* The same plan computed on the host from a host copy of C (host pointers, no GPU). */
+moe_status moe_ep_plan_host(const int32_t* counts_all, int32_t R, int32_t rank, const moe_dims* d,
+                            int32_t* send_base, int32_t* recv_offsets);
+
+/* For every assignment a = t*K + k with expert e: row = send_base[e] + row_of_assign[a] -
+ * offsets[e] of rank e / El receives x[t] (recv_x) and (rank, row_of_assign[a])
+ * (recv_meta); then slot [0][rank] of every rank's signal pad gets `epoch`.  x [T][H] bf16;
+ * offsets from moe_count_scan.  A row outside [0, cap) is skipped and sets
+ * MOE_DEV_BAD_INDEX in the EP workspace. */
+moe_status moe_ep_dispatch(const void* x, const int32_t* row_of_assign, const int32_t* topk_ids,
+                           const int32_t* offsets, const int32_t* send_base, const moe_dims* d,
+                           int32_t R, int32_t rank, int64_t cap, const moe_ep_peers* peers,
+                           int32_t epoch, void* ep_ws, void* stream);
+
+/* Waits on the device until slots [phase][0..R) of this rank's signal pad hold at least
+ * `epoch` (phase 0: every source has dispatched; phase 1: every owner has returned). */
+moe_status moe_ep_wait(const int32_t* signal, int32_t R, int32_t phase, int32_t epoch, void* ep_ws,
+                       void* stream);
+
+/* For every received row j < recv_offsets[El]: y_recv[j] goes to row recv_meta[j].row of
+ * rank recv_meta[j].rank's ret_y; then slot [1][rank] of every signal pad gets `epoch`.
+ * y_recv [cap][H] bf16 (the grouped FFN's output on recv_x). */
+moe_status moe_ep_return(const void* y_recv, const int32_t* recv_meta, const int32_t* recv_offsets,
+                         const moe_dims* d, int32_t R, int32_t rank, int64_t cap,
+                         const moe_ep_peers* peers, int32_t epoch, void* ep_ws, void* stream);
+
+/* CUDA IPC plumbing for the peer addresses: export a handle (MOE_EP_IPC_HANDLE_BYTES) of the
+ * allocation holding dev_ptr and dev_ptr's offset in it; import opens a peer's handle in this
+ * process (*base, to close later) and returns base + offset; close releases an import. */
+moe_status moe_ep_ipc_export(const void* dev_ptr, void* handle, uint64_t* offset);
+moe_status moe_ep_ipc_import(const void* handle, uint64_t offset, void** base, void** dev_ptr);
+moe_status moe_ep_ipc_close(void* base);
+
 #ifdef __cplusplus
 }
 #endif

@@ -54,6 +54,15 @@ class moe_layer_buffers(C.Structure):
     _fields_ = [(n, C.c_void_p) for n in _BUF_FIELDS]
 
 
+MOE_EP_MAX_RANKS = 64
+MOE_EP_IPC_HANDLE_BYTES = 64
+
+
+class moe_ep_peers(C.Structure):
+    _fields_ = [("recv_x", C.c_void_p * MOE_EP_MAX_RANKS), ("recv_meta", C.c_void_p * MOE_EP_MAX_RANKS),
+                ("ret_y", C.c_void_p * MOE_EP_MAX_RANKS), ("signal", C.c_void_p * MOE_EP_MAX_RANKS)]
+
+
 _VP, _SZ, _I32, _I64 = C.c_void_p, C.c_size_t, C.c_int32, C.c_int64
 _DP = C.POINTER(moe_dims)
 _SIGS = {
@@ -82,6 +91,16 @@ _SIGS = {
                                     _SZ, C.POINTER(_VP), _VP]),
     "moe_layer_forward_host": (C.c_int, [_VP, _VP, C.POINTER(moe_layer_weights), _DP,
                                          C.POINTER(moe_layer_buffers), _VP, _SZ, _VP, _VP]),
+    "moe_ep_workspace_bytes": (_SZ, []),
+    "moe_ep_plan": (C.c_int, [_VP, _I32, _I32, _DP, _VP, _VP, _VP]),
+    "moe_ep_plan_host": (C.c_int, [_VP, _I32, _I32, _DP, _VP, _VP]),
+    "moe_ep_dispatch": (C.c_int, [_VP, _VP, _VP, _VP, _VP, _DP, _I32, _I32, _I64, C.POINTER(moe_ep_peers), _I32,
+                                  _VP, _VP]),
+    "moe_ep_wait": (C.c_int, [_VP, _I32, _I32, _I32, _VP, _VP]),
+    "moe_ep_return": (C.c_int, [_VP, _VP, _VP, _DP, _I32, _I32, _I64, C.POINTER(moe_ep_peers), _I32, _VP, _VP]),
+    "moe_ep_ipc_export": (C.c_int, [_VP, _VP, C.POINTER(C.c_uint64)]),
+    "moe_ep_ipc_import": (C.c_int, [_VP, C.c_uint64, C.POINTER(_VP), C.POINTER(_VP)]),
+    "moe_ep_ipc_close": (C.c_int, [_VP]),
 }
 EXPORTED = tuple(_SIGS)
 
@@ -436,3 +455,87 @@ def moe_layer_forward_host(x_host, x_dev, weights: dict, d: moe_dims, buffers: d
     _check("moe_layer_forward_host", lib().moe_layer_forward_host(
         x_host.data_ptr(), _ptr(x_dev, torch.bfloat16, "x_dev", d.T * d_in), C.byref(wst), C.byref(d),
         C.byref(bst), _ptr(ws, torch.uint8, "ws"), ws.numel(), out_host.data_ptr(), _stream(stream)))
+
+
+# ---------------------------------------------------------------------------
+# Expert-parallel exchange (include/moe.h, "Expert-parallel exchange across GPUs")
+# ---------------------------------------------------------------------------
+
+def ep_workspace(device="cuda") -> torch.Tensor:
+    ws = torch.empty(int(lib().moe_ep_workspace_bytes()), dtype=torch.uint8, device=device)
+    workspace_init(ws)
+    return ws
+
+
+def ep_peers(recv_x: Sequence[int], recv_meta: Sequence[int], ret_y: Sequence[int], signal: Sequence[int]) -> moe_ep_peers:
+    """Peer table from per-rank device addresses (ints valid in this process)."""
+    R = len(recv_x)
+    if not (len(recv_meta) == len(ret_y) == len(signal) == R) or R > MOE_EP_MAX_RANKS:
+        raise ValueError("one address per rank for each buffer")
+    p = moe_ep_peers()
+    for i in range(R):
+        p.recv_x[i], p.recv_meta[i], p.ret_y[i], p.signal[i] = recv_x[i], recv_meta[i], ret_y[i], signal[i]
+    return p
+
+
+def moe_ep_plan(counts_all, R: int, rank: int, d: moe_dims, send_base, recv_offsets, stream=None):
+    El = d.E // R
+    _check("moe_ep_plan", lib().moe_ep_plan(
+        _ptr(counts_all, torch.int32, "counts_all", R * d.E), R, rank, C.byref(d),
+        _ptr(send_base, torch.int32, "send_base", d.E), _ptr(recv_offsets, torch.int32, "recv_offsets", El + 1),
+        _stream(stream)))
+
+
+def moe_ep_plan_host(counts_all, R: int, rank: int, d: moe_dims):
+    """(send_base [E], recv_offsets [E/R + 1]) from a host int32 array C [R][E]; no GPU."""
+    import numpy as np
+    c = np.ascontiguousarray(np.asarray(counts_all, dtype=np.int32).reshape(R, d.E))
+    send_base = np.zeros(d.E, np.int32)
+    recv_off = np.zeros(d.E // R + 1, np.int32)
+    _check("moe_ep_plan_host", lib().moe_ep_plan_host(
+        c.ctypes.data_as(C.c_void_p), R, rank, C.byref(d), send_base.ctypes.data_as(C.c_void_p),
+        recv_off.ctypes.data_as(C.c_void_p)))
+    return send_base, recv_off
+
+
+def moe_ep_dispatch(x, row_of_assign, topk_ids, offsets, send_base, d: moe_dims, R: int, rank: int, cap: int,
+                    peers: moe_ep_peers, epoch: int, ep_ws, stream=None):
+    TK = d.T * d.K
+    _check("moe_ep_dispatch", lib().moe_ep_dispatch(
+        _ptr(x, torch.bfloat16, "x", d.T * d.H), _ptr(row_of_assign, torch.int32, "row_of_assign", TK),
+        _ptr(topk_ids, torch.int32, "topk_ids", TK), _ptr(offsets, torch.int32, "offsets", d.E + 1),
+        _ptr(send_base, torch.int32, "send_base", d.E), C.byref(d), R, rank, cap, C.byref(peers), epoch,
+        _ptr(ep_ws, torch.uint8, "ep_ws"), _stream(stream)))
+
+
+def moe_ep_wait(signal, R: int, phase: int, epoch: int, ep_ws, stream=None):
+    _check("moe_ep_wait", lib().moe_ep_wait(_ptr(signal, torch.int32, "signal", 2 * R), R, phase, epoch,
+                                            _ptr(ep_ws, torch.uint8, "ep_ws"), _stream(stream)))
+
+
+def moe_ep_return(y_recv, recv_meta, recv_offsets, d: moe_dims, R: int, rank: int, cap: int, peers: moe_ep_peers,
+                  epoch: int, ep_ws, stream=None):
+    _check("moe_ep_return", lib().moe_ep_return(
+        _ptr(y_recv, torch.bfloat16, "y_recv", cap * d.H), _ptr(recv_meta, torch.int32, "recv_meta", 2 * cap),
+        _ptr(recv_offsets, torch.int32, "recv_offsets", d.E // R + 1), C.byref(d), R, rank, cap, C.byref(peers),
+        epoch, _ptr(ep_ws, torch.uint8, "ep_ws"), _stream(stream)))
+
+
+def ep_ipc_export(t: torch.Tensor):
+    """(handle bytes, offset) naming tensor t's device memory for another process."""
+    h = (C.c_uint8 * MOE_EP_IPC_HANDLE_BYTES)()
+    off = C.c_uint64(0)
+    _check("moe_ep_ipc_export", lib().moe_ep_ipc_export(_ptr(t, name="tensor"), h, C.byref(off)))
+    return bytes(h), int(off.value)
+
+
+def ep_ipc_import(handle: bytes, offset: int):
+    """(base, address) of a peer's exported memory opened in this process."""
+    h = (C.c_uint8 * MOE_EP_IPC_HANDLE_BYTES).from_buffer_copy(handle)
+    base, ptr = C.c_void_p(), C.c_void_p()
+    _check("moe_ep_ipc_import", lib().moe_ep_ipc_import(h, offset, C.byref(base), C.byref(ptr)))
+    return int(base.value), int(ptr.value)
+
+
+def ep_ipc_close(base: int):
+    _check("moe_ep_ipc_close", lib().moe_ep_ipc_close(base))

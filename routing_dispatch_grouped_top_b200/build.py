@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 OUT = os.path.join(PKG, "libmoe_b200.so")
 BUILD = os.path.join(ROOT, "_build")
-SOURCES = ["api.cu", "routing.cu", "dispatch.cu", "grouped_gemm.cu", "noalloc.cu"]
+SOURCES = ["api.cu", "routing.cu", "dispatch.cu", "grouped_gemm.cu", "ep.cu", "noalloc.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
