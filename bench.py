@@ -193,84 +193,99 @@ def oracle_sample_tokens(cfg) -> int:
     return max(1, min(16, int(1.5e9 // (6 * cfg.H * cfg.F * cfg.K))))
 
 
+class OracleSampler:
+    """The oracle (as it stands) on bounded samples of the workload, for the host-side baseline.
+    The host copies of the tokens, router and latent weights are made once; each expert's
+    weights are made when a sample first needs them and kept (the 64 most recent)."""
+
+    def __init__(self, cfg, seed_tokens: int = 0):
+        import collections
+
+        import oracle
+        self.cfg, self.oracle = cfg, oracle
+        self.seed_tokens = seed_tokens or oracle_sample_tokens(cfg)
+        self.x_all = inputs.make_tokens(cfg, "cpu")
+        w_g, bias = inputs.make_router(cfg, "cpu")
+        w_dp, w_upp = inputs.make_latent(cfg, "cpu")
+        self.w_g = w_g.numpy()
+        self.bias = None if bias is None else bias.numpy()
+        self.w_dp = None if w_dp is None else inputs.to_bits(w_dp)
+        self.w_upp = None if w_upp is None else inputs.to_bits(w_upp)
+        sh = inputs.make_shared_expert(cfg, "cpu")
+        self.shared = None if sh is None else tuple(inputs.to_bits(t) for t in sh)
+        self.g = torch.Generator().manual_seed(cfg.seed + 5)
+        self.experts = collections.OrderedDict()
+
+    def expert(self, e):
+        cfg, oracle = self.cfg, self.oracle
+        if e in self.experts:
+            self.experts.move_to_end(e)
+            return self.experts[e]
+        ge = torch.Generator().manual_seed(10_000 + e)
+        F, H = cfg.F, cfg.H
+        wts = tuple(inputs.to_bits((torch.randn(s, generator=ge) * std).to(torch.bfloat16))
+                    for s, std in (((F, H), H ** -0.5), ((F, H), H ** -0.5), ((H, F), F ** -0.5)))
+        if cfg.fp8_dispatch:   # one-time weight preparation, like the GPU's
+            (qg, sg), (qu, su) = oracle.quantize_rows_fp8(wts[0]), oracle.quantize_rows_fp8(wts[1])
+            wts = (qg, sg, qu, su, wts[2])
+        self.experts[e] = wts
+        if len(self.experts) > 64:
+            self.experts.popitem(last=False)
+        return wts
+
+    def rate(self, seconds: float) -> dict:
+        """Tokens/s of the oracle over samples of seed_tokens random tokens, until `seconds` of
+        oracle compute have passed (at least one sample)."""
+        import numpy as np
+        from threadpoolctl import threadpool_info
+        cfg, oracle = self.cfg, self.oracle
+        n_tok = runs = 0
+        busy = 0.0                     # oracle compute time only (input preparation excluded)
+        while True:
+            idx = torch.randperm(cfg.T, generator=self.g)[:self.seed_tokens]
+            xs = inputs.to_bits(self.x_all[idx])
+            t0 = time.perf_counter()
+            z = oracle.dense_bf16(xs, self.w_dp) if self.w_dp is not None else xs
+            logits = oracle.gating_logits(z, self.w_g, self.bias)
+            if cfg.group_limit:
+                ids, w = oracle.route_limited(logits, cfg.K, cfg.P, cfg.group_limit, cfg.renormalize)
+            else:
+                ids, w = oracle.route(logits, cfg.K, cfg.renormalize)
+            cs = oracle.count_scan(ids, cfg.E, cfg.P)
+            xp, _ = oracle.permute(z, cs["row_of_assign"], ids, w, cfg.E, cfg.P)
+            busy += time.perf_counter() - t0
+            touched = [int(e) for e in np.nonzero(cs["counts"])[0]]
+            wts = {e: self.expert(e) for e in touched}    # weights made outside the clock
+            t0 = time.perf_counter()
+            off = cs["offsets"]
+            h = np.zeros((xp.shape[0], cfg.F), np.uint16)
+            y = np.zeros((xp.shape[0], cfg.H), np.uint16)
+            if cfg.fp8_dispatch:
+                xq, xsc = oracle.dispatch_fp8(z, cs["row_of_assign"], cfg.K)
+            for e in touched:
+                lo, hi = off[e], off[e + 1]
+                if cfg.fp8_dispatch:
+                    h[lo:hi], y[lo:hi] = oracle.ffn_rows_fp8(xq[lo:hi], xsc[lo:hi], *wts[e])
+                else:
+                    h[lo:hi], y[lo:hi] = oracle.ffn_rows(xp[lo:hi], *wts[e])
+            y_sh = None if self.shared is None else oracle.ffn_rows(z, *self.shared)[1]
+            out = oracle.combine(y, cs["row_of_assign"], w, y_sh)
+            if self.w_upp is not None:
+                oracle.dense_bf16(out, self.w_upp)
+            busy += time.perf_counter() - t0
+            n_tok += self.seed_tokens
+            runs += 1
+            if busy >= seconds:
+                break
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return dict(value=n_tok / busy, unit=UNIT, cores=int(threads), kind="oracle",
+                    sample=f"{runs} runs x {self.seed_tokens} random tokens of {cfg.name} through the whole layer "
+                           f"(numpy float64, {busy:.1f} s of oracle compute; weights prepared outside the clock)")
+
+
 def cpu_oracle_rate(cfg, seconds: float, seed_tokens: int = 0):
     """The oracle (as it stands) on bounded samples of the workload: tokens/s on the host."""
-    import numpy as np
-    from threadpoolctl import threadpool_info
-
-    import oracle
-    seed_tokens = seed_tokens or oracle_sample_tokens(cfg)
-    # Only the experts the sample needs are materialised on the host.
-    x_all = inputs.make_tokens(cfg, "cpu")
-    w_g, bias = inputs.make_router(cfg, "cpu")
-    w_dp, w_upp = inputs.make_latent(cfg, "cpu")
-    g = torch.Generator().manual_seed(cfg.seed + 5)
-    n_tok = 0
-    runs = 0
-    busy = 0.0                     # oracle compute time only (input preparation excluded)
-    expert_cache = {}
-
-    def expert(e):
-        if e not in expert_cache:
-            ge = torch.Generator().manual_seed(10_000 + e)
-            F, H = cfg.F, cfg.H
-            wts = tuple(inputs.to_bits((torch.randn(s, generator=ge) * std).to(torch.bfloat16))
-                        for s, std in (((F, H), H ** -0.5), ((F, H), H ** -0.5), ((H, F), F ** -0.5)))
-            if cfg.fp8_dispatch:   # one-time weight preparation, like the GPU's
-                (qg, sg), (qu, su) = oracle.quantize_rows_fp8(wts[0]), oracle.quantize_rows_fp8(wts[1])
-                wts = (qg, sg, qu, su, wts[2])
-            expert_cache[e] = wts
-        return expert_cache[e]
-
-    w_g_np = w_g.numpy()
-    bias_np = None if bias is None else bias.numpy()
-    w_dp_b = None if w_dp is None else inputs.to_bits(w_dp)
-    w_upp_b = None if w_upp is None else inputs.to_bits(w_upp)
-    sh = inputs.make_shared_expert(cfg, "cpu")
-    sh_b = None if sh is None else tuple(inputs.to_bits(t) for t in sh)
-    while True:
-        idx = torch.randperm(cfg.T, generator=g)[:seed_tokens]
-        xs = inputs.to_bits(x_all[idx])
-        t0 = time.perf_counter()
-        z = oracle.dense_bf16(xs, w_dp_b) if w_dp_b is not None else xs
-        logits = oracle.gating_logits(z, w_g_np, bias_np)
-        if cfg.group_limit:
-            ids, w = oracle.route_limited(logits, cfg.K, cfg.P, cfg.group_limit, cfg.renormalize)
-        else:
-            ids, w = oracle.route(logits, cfg.K, cfg.renormalize)
-        cs = oracle.count_scan(ids, cfg.E, cfg.P)
-        xp, _ = oracle.permute(z, cs["row_of_assign"], ids, w, cfg.E, cfg.P)
-        busy += time.perf_counter() - t0
-        for e in np.nonzero(cs["counts"])[0]:
-            expert(int(e))                 # materialise the weights outside the clock
-        t0 = time.perf_counter()
-        off = cs["offsets"]
-        h = np.zeros((xp.shape[0], cfg.F), np.uint16)
-        y = np.zeros((xp.shape[0], cfg.H), np.uint16)
-        if cfg.fp8_dispatch:
-            xq, xs = oracle.dispatch_fp8(z, cs["row_of_assign"], cfg.K)
-        for e in np.nonzero(cs["counts"])[0]:
-            lo, hi = off[e], off[e + 1]
-            if cfg.fp8_dispatch:
-                h[lo:hi], y[lo:hi] = oracle.ffn_rows_fp8(xq[lo:hi], xs[lo:hi], *expert(int(e)))
-            else:
-                h[lo:hi], y[lo:hi] = oracle.ffn_rows(xp[lo:hi], *expert(int(e)))
-        y_sh = None if sh_b is None else oracle.ffn_rows(z, *sh_b)[1]
-        out = oracle.combine(y, cs["row_of_assign"], w, y_sh)
-        if w_upp_b is not None:
-            oracle.dense_bf16(out, w_upp_b)
-        busy += time.perf_counter() - t0
-        n_tok += seed_tokens
-        runs += 1
-        if len(expert_cache) > 64:
-            expert_cache.clear()
-        if busy >= seconds:
-            break
-    el = busy
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return dict(value=n_tok / el, unit=UNIT, cores=int(threads), kind="oracle",
-                sample=f"{runs} runs x {seed_tokens} random tokens of {cfg.name} through the whole layer "
-                       f"(numpy float64, {el:.1f} s of oracle compute; weights prepared outside the clock)")
+    return OracleSampler(cfg, seed_tokens).rate(seconds)
 
 
 def shared_expert_overlap(cfg, inp, w, bufs, ws, flush, stream, n, dev) -> dict:
@@ -346,9 +361,10 @@ def run_reference(args, cfg):
     if rank != 0:
         return 0
     steps = []
+    sampler = OracleSampler(cfg)
     for _ in range(args.warmup):
-        cpu_oracle_rate(cfg, 0.0)
-    rates = [cpu_oracle_rate(cfg, max(0.5, args.cpu_seconds / max(args.steps, 1))) for _ in range(args.steps)]
+        sampler.rate(0.0)
+    rates = [sampler.rate(max(0.5, args.cpu_seconds / max(args.steps, 1))) for _ in range(args.steps)]
     val = statistics.mean(r["value"] for r in rates)
     cb = dict(rates[-1])
     cb["value"] = val

@@ -99,15 +99,14 @@ def test_ep_exchange_matches_the_oracle_layout_and_outputs(R, T, H, E, K, F):
             assert np.array_equal(meta[:, 1], [src_roa[a // (T * K)][a % (T * K)] for a in cs["assign_of_row"][lo:hi]])
             check_bf16(f"y_recv[{d}]", bits(r.y_recv[:n]), y_ref[lo:hi])
         # returned rows are bit copies of the owners' outputs; combine at each source
+        y_recv = [bits(r.y_recv) for r in ranks]
         for s, r in enumerate(ranks):
             ret = bits(r.ret_y)
             roa = r.row_of_assign.cpu().numpy()
             for a in range(T * K):
-                g = s * T * K + a                      # global assignment
-                row_g = cs["row_of_assign"][g]
+                row_g = cs["row_of_assign"][s * T * K + a]     # the assignment's row in the global layout
                 d = int(np.searchsorted(off, row_g, side="right") - 1) // El
-                j = row_g - off[d * El]
-                assert np.array_equal(ret[roa[a]], bits(ranks[d].y_recv[j]))
+                assert np.array_equal(ret[roa[a]], y_recv[d][row_g - off[d * El]])
             ref_out = oracle.combine(y_ref[cs["row_of_assign"][s * T * K:(s + 1) * T * K]], np.arange(T * K),
                                      wts[s * T:(s + 1) * T])
             check_bf16(f"out[{s}]", bits(outs[s]), ref_out)
