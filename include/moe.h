@@ -166,10 +166,11 @@ moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids,
  *   row_of_assign[TK]: row of assignment a in the expert-major buffer, a stable
  *     counting sort (rows of one expert keep increasing a),
  *   assign_of_row[TK]: its inverse.
- * Two launches: an expert histogram of the ids, then one pass over the assignments in
- * up to 128 chunks with a decoupled look-back scan across the chunks (each chunk's
- * counts are published and added up by its successors; no grid-wide barrier).  Uses the
- * workspace (expert totals, per-chunk count rows, look-back flags and counters).
+ * Two launches: one pass over the assignments in up to 128 chunks, block-local histograms
+ * with a decoupled look-back scan across the chunks (each chunk's counts are published and
+ * added up by its successors; no grid-wide barrier), which ranks every assignment within
+ * its expert and leaves the offsets; then the ranks become rows.  Uses the workspace
+ * (per-chunk count rows, look-back flags and counters).
  * An id outside [0, E) sets MOE_DEV_BAD_INDEX and gets row -1; a look-back wait that runs
  * out (2 s) sets MOE_DEV_TIMEOUT.  Either way offsets[E] is set to -1 (a bad-offsets
  * marker that the grouped GEMMs refuse) and the other outputs are unspecified. */
@@ -187,18 +188,18 @@ moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* c
  * a host framework that owns every device allocation, or a real-time loop that may not
  * call cudaMalloc/cudaFree, which can also synchronize the device, once it runs).
  * Same arguments, results and status codes as moe_count_scan minus the workspace.  The
- * scratch is a fixed device array inside the library holding the count/scan state:
- * 768 bytes of counters and flags, the E expert totals and two int32 rows of E per chunk
- * (ceil(T*K / 256) chunks, at most 128), at most MOE_NOALLOC_SCRATCH_BYTES in all; larger
- * shapes return MOE_ERR_UNSUPPORTED_SHAPE (only E >= 1020 with T*K > 32 512 exceed it).  The call allocates nothing: it clears the scratch's counters, flags
- * and totals with an async memset on `stream`, then launches the two count/scan kernels.
- * The first call on a device looks up the scratch's device address once (with that
- * device current); make that first call before any stream capture.  All calls share the
- * one scratch and it keeps the last call's contents, so calls that overlap on the GPU
- * (other streams, other host threads) race: serialize them.  Device-side conditions
- * have no status word to go to (no workspace): an id outside [0, E) shows up as row -1 in
- * row_of_assign, and a call that met one, or whose look-back wait ran out, leaves
- * offsets[E] = -1. */
+ * scratch is a fixed device array inside the library holding the count/scan state: 768
+ * bytes of counters and look-back flags and two int32 rows of E per chunk (ceil(T*K / 256)
+ * chunks, at most 128), at most MOE_NOALLOC_SCRATCH_BYTES in all; larger shapes return
+ * MOE_ERR_UNSUPPORTED_SHAPE (only E = 1024 with T*K > 32 512 exceeds it).  The call
+ * allocates nothing: it clears the scratch's counters and flags with an async memset on
+ * `stream`, then launches the count/scan kernel and the kernel that turns ranks into rows.
+ * The first call on a device looks up the scratch's device address once (with that device
+ * current); make that first call before any stream capture.  All calls share the one
+ * scratch and it keeps the last call's contents, so calls that overlap on the GPU (other
+ * streams, other host threads) race: serialize them.  Device-side conditions have no status
+ * word to go to (no workspace): an id outside [0, E) shows up as row -1 in row_of_assign,
+ * and a call that met one, or whose look-back wait ran out, leaves offsets[E] = -1. */
 moe_status moe_count_scan_noalloc(const int32_t* topk_ids, const moe_dims* d, int32_t* counts,
                                   int32_t* offsets, int32_t* part_counts, int32_t* part_offsets,
                                   int32_t* row_of_assign, int32_t* assign_of_row, void* stream);

@@ -207,7 +207,7 @@ moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids, 
   if (d->T == 0) return MOE_OK;
   if (!logits || !topk_ids || !topk_w) return MOE_ERR_INVALID_ARG;
   return cuda_status(launch_route(logits, 1, nullptr, d->T, d->E, d->K, d->renormalize, d->P, d->group_limit,
-                                  topk_ids, topk_w, nullptr, as_stream(stream)));
+                                  topk_ids, topk_w, as_stream(stream)));
 }
 
 moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* counts, int32_t* offsets,
@@ -219,10 +219,10 @@ moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* c
                                                                            !assign_of_row)))
     return MOE_ERR_INVALID_ARG;
   const long long TK = d->T * static_cast<long long>(d->K);
-  const ScanWorkspace sw = scan_ws(ws, d);
-  MOE_CUDA(launch_hist(topk_ids, TK, d->E, sw, as_stream(stream)));
-  return cuda_status(launch_count_scan(topk_ids, TK, d->E, d->P, counts, offsets, part_counts, part_offsets,
-                                       row_of_assign, assign_of_row, nullptr, sw, as_stream(stream)));
+  MOE_CUDA(launch_count_scan(topk_ids, TK, d->E, d->P, row_of_assign, counts, offsets, part_counts, part_offsets,
+                             nullptr, scan_ws(ws, d), as_stream(stream)));
+  return cuda_status(launch_scan_finalize(topk_ids, TK, d->E, offsets, row_of_assign, assign_of_row,
+                                          as_stream(stream)));
 }
 
 moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_t* topk_ids, const float* topk_w,
@@ -233,8 +233,10 @@ moe_status moe_permute(const void* x, const int32_t* row_of_assign, const int32_
   if (!x || !row_of_assign || !xp || (meta_w && !topk_w) || (meta_local_expert && !topk_ids))
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(xp)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_permute(x, row_of_assign, topk_ids, topk_w, d->T, d->H, d->E, d->K, d->P, xp,
-                                    meta_token, meta_slot, meta_w, meta_local_expert, as_stream(stream)));
+  // the rows are given: the kernel only reads row_of_assign
+  return cuda_status(launch_permute(x, const_cast<int32_t*>(row_of_assign), topk_ids, topk_w, d->T, d->H, d->E, d->K,
+                                    d->P, xp, meta_token, meta_slot, meta_w, meta_local_expert, nullptr, nullptr,
+                                    as_stream(stream)));
 }
 
 void moe_set_pair_min_rows(int32_t rows) { set_pair_min_rows(rows); }
@@ -257,8 +259,9 @@ moe_status moe_permute_fp8(const void* x, const int32_t* row_of_assign, const in
   if (!x || !row_of_assign || !xq || !xs || (meta_w && !topk_w) || (meta_local_expert && !topk_ids))
     return MOE_ERR_INVALID_ARG;
   if (!aligned16(x) || !aligned16(xq)) return MOE_ERR_INVALID_ARG;
-  return cuda_status(launch_permute_fp8(x, row_of_assign, topk_ids, topk_w, d->T, d->H, d->E, d->K, d->P, xq, xs,
-                                        meta_token, meta_slot, meta_w, meta_local_expert, as_stream(stream)));
+  return cuda_status(launch_permute_fp8(x, const_cast<int32_t*>(row_of_assign), topk_ids, topk_w, d->T, d->H, d->E,
+                                        d->K, d->P, xq, xs, meta_token, meta_slot, meta_w, meta_local_expert, nullptr,
+                                        nullptr, as_stream(stream)));
 }
 
 moe_status moe_grouped_gate_up_fp8(const void* xq, const float* xs, const int32_t* offsets, const void* wq_gate,
@@ -349,8 +352,8 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
     cudaStream_t s0 = as_stream(stream);
     for (int i = 0; stage_events && i < MOE_NUM_STAGE_EVENTS; ++i)
       if (stage_events[i]) MOE_CUDA(cudaEventRecord(reinterpret_cast<cudaEvent_t>(stage_events[i]), s0));
-    return cuda_status(launch_count_scan(nullptr, 0, d->E, d->P, b->counts, b->offsets, b->part_counts,
-                                         b->part_offsets, nullptr, nullptr, b->skew, scan_ws(ws, d), s0));
+    return cuda_status(launch_count_scan(nullptr, 0, d->E, d->P, nullptr, b->counts, b->offsets, b->part_counts,
+                                         b->part_offsets, b->skew, scan_ws(ws, d), s0));
   }
   if (!x || !w || !b) return MOE_ERR_INVALID_ARG;
   const bool latent = d->d_model > 0;
@@ -410,19 +413,22 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
     MOE_CUDA(gemm_gating(routed, w->w_g_split, w->bias, T, d->H, d->E, gate_out, nsplit, status,
                          ws_sched(ws, kSchedGating), s));
   MOE_TRY(mark(2));
-  const ScanWorkspace sw = scan_ws(ws, d);
   MOE_CUDA(launch_route(gate_out, nsplit, b->logits, T, d->E, d->K, d->renormalize, d->P, d->group_limit, b->topk_ids,
-                        b->topk_w, sw.hist, s));
+                        b->topk_w, s));
   MOE_TRY(mark(3));
-  MOE_CUDA(launch_count_scan(b->topk_ids, TK, d->E, d->P, b->counts, b->offsets, b->part_counts, b->part_offsets,
-                             b->row_of_assign, b->assign_of_row, b->skew, sw, s));
+  // count/scan leaves each assignment's rank within its expert in row_of_assign; the permute
+  // turns it into the row (offsets[e] + rank) and writes assign_of_row
+  MOE_CUDA(launch_count_scan(b->topk_ids, TK, d->E, d->P, b->row_of_assign, b->counts, b->offsets, b->part_counts,
+                             b->part_offsets, b->skew, scan_ws(ws, d), s));
   MOE_TRY(mark(4));
   if (fp8)
     MOE_CUDA(launch_permute_fp8(routed, b->row_of_assign, b->topk_ids, b->topk_w, T, d->H, d->E, d->K, d->P, b->xq,
-                                b->xs, b->meta_token, b->meta_slot, b->meta_w, b->meta_local_expert, s));
+                                b->xs, b->meta_token, b->meta_slot, b->meta_w, b->meta_local_expert, b->offsets,
+                                b->assign_of_row, s));
   else
     MOE_CUDA(launch_permute(routed, b->row_of_assign, b->topk_ids, b->topk_w, T, d->H, d->E, d->K, d->P, b->xp,
-                            b->meta_token, b->meta_slot, b->meta_w, b->meta_local_expert, s));
+                            b->meta_token, b->meta_slot, b->meta_w, b->meta_local_expert, b->offsets,
+                            b->assign_of_row, s));
   MOE_TRY(mark(5));
   if (T > 0) {
     if (fp8)

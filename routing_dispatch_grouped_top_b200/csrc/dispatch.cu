@@ -47,51 +47,69 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return v;
 }
 
-__global__ void __launch_bounds__(kCopyThreads) permute_kernel(
-    const uint4* __restrict__ x, const int32_t* __restrict__ roa, const int32_t* __restrict__ ids,
-    const float* __restrict__ w, long long T, int vpr, int E, int K, int P, uint4* __restrict__ xp,
-    int32_t* __restrict__ meta_token, int32_t* __restrict__ meta_slot, float* __restrict__ meta_w,
-    int32_t* __restrict__ meta_local) {
-  pdl_wait();  // row_of_assign comes from the count/scan kernel
-  pdl_launch_dependents();
-  const long long n_items = T * vpr;
-  const long long stride = static_cast<long long>(gridDim.x) * blockDim.x;
-  const long long tid = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (long long base = tid; base < n_items; base += stride * kUnroll) {
-    uint4 v[kUnroll];
-    long long tok[kUnroll];
-    int vec[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const long long it = base + u * stride;
-      tok[u] = it / vpr;
-      vec[u] = static_cast<int>(it - tok[u] * vpr);
-      if (it < n_items) v[u] = ld_stream(x + it);
+// Row of assignment a for the copy kernels: row_of_assign[a] as given, or, with rank_off
+// (the layer path), count/scan's rank of a within its expert turned into rank_off[e] + rank and
+// written back, with assign_of_row[row] = a.  Only the thread that owns a reads or writes
+// row_of_assign[a].  -1 for an assignment without a valid row.
+__device__ __forceinline__ int assignment_row(int32_t* roa, const int32_t* __restrict__ ids, long long a, long long TK,
+                                             int E, const int32_t* __restrict__ rank_off, int32_t* aor) {
+  int r = roa[a];
+  if (rank_off) {
+    const int e = __ldg(ids + a);
+    int row = -1;
+    if (r >= 0 && e >= 0 && e < E) {
+      const long long v = static_cast<long long>(__ldg(rank_off + e)) + r;
+      if (v >= 0 && v < TK) row = static_cast<int>(v);
     }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const long long it = base + u * stride;
-      if (it < n_items) {
-        const int32_t* r = roa + tok[u] * K;
-        for (int k = 0; k < K; ++k) {
-          const int row = __ldg(r + k);
-          if (static_cast<unsigned long long>(row) < static_cast<unsigned long long>(T * K))
-            xp[static_cast<long long>(row) * vpr + vec[u]] = v[u];
-        }
-      }
-    }
+    roa[a] = row;
+    if (row >= 0) aor[row] = static_cast<int>(a);
+    r = row;
   }
-  // routing metadata of every row
+  return (r >= 0 && r < TK) ? r : -1;
+}
+
+// One warp per token: lanes k < K find the rows of the token's K assignments (and write their
+// metadata), then the warp copies the token's row of 16-byte vectors to those K rows, kUnroll
+// loads in flight per lane; consecutive lanes touch consecutive vectors (coalesced both ways).
+__global__ void __launch_bounds__(kCopyThreads) permute_kernel(
+    const uint4* __restrict__ x, int32_t* roa, const int32_t* __restrict__ ids, const float* __restrict__ w,
+    long long T, int vpr, int E, int K, int P, uint4* __restrict__ xp, int32_t* __restrict__ meta_token,
+    int32_t* __restrict__ meta_slot, float* __restrict__ meta_w, int32_t* __restrict__ meta_local,
+    const int32_t* __restrict__ rank_off, int32_t* __restrict__ aor) {
+  pdl_wait();  // the ranks or rows come from the count/scan kernel
+  pdl_launch_dependents();
+  constexpr int kWarps = kCopyThreads / 32;
+  const int lane = threadIdx.x & 31;
   const long long TK = T * K;
   const int epp = E / P;
-  for (long long a = tid; a < TK; a += stride) {
-    const int r = __ldg(roa + a);
-    if (static_cast<unsigned long long>(r) >= static_cast<unsigned long long>(TK)) continue;
-    const int t = static_cast<int>(a / K);
-    if (meta_token) meta_token[r] = t;
-    if (meta_slot) meta_slot[r] = static_cast<int>(a - static_cast<long long>(t) * K);
-    if (meta_w) meta_w[r] = __ldg(w + a);
-    if (meta_local) meta_local[r] = __ldg(ids + a) % epp;
+  const long long nwarps = static_cast<long long>(gridDim.x) * kWarps;
+  for (long long t = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
+    int row = -1;
+    if (lane < K) {
+      const long long a = t * K + lane;
+      row = assignment_row(roa, ids, a, TK, E, rank_off, aor);
+      if (row >= 0) {
+        if (meta_token) meta_token[row] = static_cast<int>(t);
+        if (meta_slot) meta_slot[row] = lane;
+        if (meta_w) meta_w[row] = __ldg(w + a);
+        if (meta_local) meta_local[row] = __ldg(ids + a) % epp;
+      }
+    }
+    const uint4* src = x + t * vpr;
+    for (int v0 = lane; v0 < vpr; v0 += 32 * kUnroll) {
+      uint4 v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (v0 + 32 * u < vpr) v[u] = ld_stream(src + v0 + 32 * u);
+      for (int k = 0; k < K; ++k) {
+        const int rk = __shfl_sync(0xffffffffu, row, k);
+        if (rk < 0) continue;
+        uint4* dst = xp + static_cast<long long>(rk) * vpr + v0;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u)
+          if (v0 + 32 * u < vpr) dst[32 * u] = v[u];
+      }
+    }
   }
 }
 
@@ -255,10 +273,10 @@ __global__ void __launch_bounds__(kQuantThreads) quantize_fp8_rows_kernel(const 
 // FP8 dispatch: token t quantized once, its codes and scale stored at the rows of its K
 // assignments; routing metadata as in permute_kernel.
 __global__ void __launch_bounds__(kQuantThreads) permute_fp8_kernel(
-    const uint4* __restrict__ x, const int32_t* __restrict__ roa, const int32_t* __restrict__ ids,
-    const float* __restrict__ w, long long T, int vpr, int E, int K, int P, uint2* __restrict__ xq,
-    float* __restrict__ xs, int32_t* __restrict__ meta_token, int32_t* __restrict__ meta_slot,
-    float* __restrict__ meta_w, int32_t* __restrict__ meta_local) {
+    const uint4* __restrict__ x, int32_t* roa, const int32_t* __restrict__ ids, const float* __restrict__ w,
+    long long T, int vpr, int E, int K, int P, uint2* __restrict__ xq, float* __restrict__ xs,
+    int32_t* __restrict__ meta_token, int32_t* __restrict__ meta_slot, float* __restrict__ meta_w,
+    int32_t* __restrict__ meta_local, const int32_t* __restrict__ rank_off, int32_t* __restrict__ aor) {
   pdl_wait();  // row_of_assign comes from the count/scan kernel
   pdl_launch_dependents();
   __shared__ float s_red[kQuantThreads / 32];
@@ -268,9 +286,9 @@ __global__ void __launch_bounds__(kQuantThreads) permute_fp8_kernel(
   for (long long t = blockIdx.x; t < T; t += gridDim.x) {
     if (threadIdx.x < K) {
       const long long a = t * K + threadIdx.x;
-      const int r = __ldg(roa + a);
-      const bool ok = static_cast<unsigned long long>(r) < static_cast<unsigned long long>(TK);
-      s_row[threadIdx.x] = ok ? r : -1;
+      const int r = assignment_row(roa, ids, a, TK, E, rank_off, aor);
+      const bool ok = r >= 0;
+      s_row[threadIdx.x] = r;
       if (ok) {
         if (meta_token) meta_token[r] = static_cast<int>(t);
         if (meta_slot) meta_slot[r] = threadIdx.x;
@@ -301,14 +319,16 @@ int copy_blocks(long long items) {
 
 }  // namespace
 
-cudaError_t launch_permute(const void* x, const int32_t* roa, const int32_t* ids, const float* w, long long T,
-                           int H, int E, int K, int P, void* xp, int32_t* meta_token, int32_t* meta_slot,
-                           float* meta_w, int32_t* meta_local, cudaStream_t s) {
+cudaError_t launch_permute(const void* x, int32_t* roa, const int32_t* ids, const float* w, long long T, int H,
+                           int E, int K, int P, void* xp, int32_t* meta_token, int32_t* meta_slot, float* meta_w,
+                           int32_t* meta_local, const int32_t* rank_off, int32_t* aor, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int vpr = H / 8;
-  return launch_pdl(permute_kernel, dim3(copy_blocks(T * vpr / 2)), dim3(kCopyThreads), 0, s,
+  const long long blocks = std::min<long long>((T + kCopyThreads / 32 - 1) / (kCopyThreads / 32),
+                                               static_cast<long long>(MOE_COPY_BLOCKS_PER_SM) * num_sms());
+  return launch_pdl(permute_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kCopyThreads), 0, s,
                     reinterpret_cast<const uint4*>(x), roa, ids, w, T, vpr, E, K, P, reinterpret_cast<uint4*>(xp),
-                    meta_token, meta_slot, meta_w, meta_local);
+                    meta_token, meta_slot, meta_w, meta_local, rank_off, aor);
 }
 
 cudaError_t launch_quantize_fp8_rows(const void* x, long long rows, int cols, void* q, float* scales,
@@ -320,14 +340,15 @@ cudaError_t launch_quantize_fp8_rows(const void* x, long long rows, int cols, vo
   return cudaGetLastError();
 }
 
-cudaError_t launch_permute_fp8(const void* x, const int32_t* roa, const int32_t* ids, const float* w, long long T,
+cudaError_t launch_permute_fp8(const void* x, int32_t* roa, const int32_t* ids, const float* w, long long T,
                                int H, int E, int K, int P, void* xq, float* xs, int32_t* meta_token,
-                               int32_t* meta_slot, float* meta_w, int32_t* meta_local, cudaStream_t s) {
+                               int32_t* meta_slot, float* meta_w, int32_t* meta_local, const int32_t* rank_off,
+                               int32_t* aor, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int blocks = static_cast<int>(std::min<long long>(T, 16LL * num_sms()));
   return launch_pdl(permute_fp8_kernel, dim3(blocks), dim3(kQuantThreads), 0, s, reinterpret_cast<const uint4*>(x),
                     roa, ids, w, T, H / 8, E, K, P, reinterpret_cast<uint2*>(xq), xs, meta_token, meta_slot, meta_w,
-                    meta_local);
+                    meta_local, rank_off, aor);
 }
 
 cudaError_t launch_combine(const void* y, const int32_t* roa, const float* w, const void* shared, long long T, int H,

@@ -81,17 +81,15 @@ cudaError_t launch_sum_partials(const float* partials, int nsplit, long long n, 
 
 // With nsplit > 1 the logits are the in-order sum of nsplit partial planes (T * E apart) starting
 // at `logits`; the kernel writes that sum to `logits_out` as well.
-// With hist != nullptr every selected id is also added to hist[id] (the count/scan totals).
 cudaError_t launch_route(const float* logits, int nsplit, float* logits_out, long long T, int E, int K,
-                         int renormalize, int P, int group_limit, int32_t* ids, float* w, int* hist,
-                         cudaStream_t stream);
+                         int renormalize, int P, int group_limit, int32_t* ids, float* w, cudaStream_t stream);
 
 // Count/scan state inside a workspace (or the library's own scratch):
 //   [0] status word, [64] ticket, [96] done counter, [128] failure flag (the bytes 160-255
 //   belong to the GEMMs' tile schedules), [256] kScanMaxBlocks look-back flags, then
-//   hist[E], agg[nb][E] and inc[nb][E] (each 256-byte aligned).  The ticket, done counter,
-//   failure flag, flags and hist are zero between calls (the last block of every call clears
-//   them; the workspace starts zeroed).
+//   agg[nb][E] and inc[nb][E] (each 256-byte aligned).  The ticket, done counter, failure
+//   flag and flags are zero between calls (the last block of every call clears them; the
+//   workspace starts zeroed).
 constexpr int kScanMaxBlocks = 128;
 inline size_t round256(size_t n) { return (n + 255) / 256 * 256; }
 struct ScanWorkspace {
@@ -101,29 +99,35 @@ struct ScanWorkspace {
   int* done;
   int* fail;
   int* flags;   // [kScanMaxBlocks]
-  int* hist;    // [E] expert totals of the call
   int* agg;     // [nb][E] per-block counts
   int* inc;     // [nb][E] per-block inclusive prefixes over blocks
 };
 int scan_blocks(long long TK);                      // blocks (chunks) of one count/scan call
 size_t scan_ws_bytes(long long TK, int E);          // bytes of the state above
 ScanWorkspace scan_workspace(void* base, long long TK, int E);
-// hist[e] += #{a : ids[a] = e} (the caller's ids; the route kernel does this itself when given hist).
-cudaError_t launch_hist(const int32_t* ids, long long TK, int E, const ScanWorkspace& ws, cudaStream_t stream);
-// Needs ws.hist to hold the totals of ids (launch_hist or the route kernel, on the same stream before).
-cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, int32_t* counts, int32_t* offsets,
-                              int32_t* part_counts, int32_t* part_offsets, int32_t* row_of_assign,
-                              int32_t* assign_of_row, float* skew, const ScanWorkspace& ws, cudaStream_t stream);
+// One pass: ranks[a] = rank of assignment a among the assignments of its expert (stable), or -1
+// for an id outside [0, E); counts, offsets (offsets[E] = -1 after a device-side failure),
+// partition counts/offsets and the skew ratio (nullable).
+cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, int32_t* ranks, int32_t* counts,
+                              int32_t* offsets, int32_t* part_counts, int32_t* part_offsets, float* skew,
+                              const ScanWorkspace& ws, cudaStream_t stream);
+// row_of_assign (holding the ranks) becomes offsets[ids[a]] + rank in place; assign_of_row its inverse.
+cudaError_t launch_scan_finalize(const int32_t* ids, long long TK, int E, const int32_t* offsets,
+                                 int32_t* row_of_assign, int32_t* assign_of_row, cudaStream_t stream);
 cudaError_t launch_skew(const int32_t* counts, int E, float* ratio, cudaStream_t stream);
 
-cudaError_t launch_permute(const void* x, const int32_t* row_of_assign, const int32_t* ids, const float* w,
+// With rank_offsets != nullptr, row_of_assign holds count_scan's ranks: the row of assignment a
+// is rank_offsets[ids[a]] + rank, written back to row_of_assign[a] (and assign_of_row[row] = a).
+cudaError_t launch_permute(const void* x, int32_t* row_of_assign, const int32_t* ids, const float* w,
                            long long T, int H, int E, int K, int P, void* xp, int32_t* meta_token,
-                           int32_t* meta_slot, float* meta_w, int32_t* meta_local, cudaStream_t stream);
+                           int32_t* meta_slot, float* meta_w, int32_t* meta_local, const int32_t* rank_offsets,
+                           int32_t* assign_of_row, cudaStream_t stream);
 cudaError_t launch_quantize_fp8_rows(const void* x, long long rows, int cols, void* q, float* scales,
                                      cudaStream_t stream);
-cudaError_t launch_permute_fp8(const void* x, const int32_t* row_of_assign, const int32_t* ids, const float* w,
+cudaError_t launch_permute_fp8(const void* x, int32_t* row_of_assign, const int32_t* ids, const float* w,
                                long long T, int H, int E, int K, int P, void* xq, float* xs, int32_t* meta_token,
-                               int32_t* meta_slot, float* meta_w, int32_t* meta_local, cudaStream_t stream);
+                               int32_t* meta_slot, float* meta_w, int32_t* meta_local, const int32_t* rank_offsets,
+                               int32_t* assign_of_row, cudaStream_t stream);
 cudaError_t launch_combine(const void* y, const int32_t* row_of_assign, const float* w, const void* shared,
                            long long T, int H, int K, void* out, cudaStream_t stream);
 cudaError_t launch_pack_router(const float* w_g, int H, int E, void* w_split, cudaStream_t stream);

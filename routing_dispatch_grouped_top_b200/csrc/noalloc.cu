@@ -1,8 +1,8 @@
 // noalloc.cu - count/scan for callers that cannot allocate device memory.
 //
-// moe_count_scan needs scratch (a status word, the ticket and done counters of its
-// look-back scan, the expert totals and one row of per-expert counts per block) and takes
-// it from a caller-owned workspace.  Some callers cannot provide one: a plugin running
+// moe_count_scan needs scratch (a status word, the ticket and done counters and flags of its
+// look-back scan, and two rows of per-expert counts per block) and takes it from a
+// caller-owned workspace.  Some callers cannot provide one: a plugin running
 // inside a host framework that owns every device allocation, or a real-time loop that
 // must not allocate (cudaMalloc/cudaFree can also synchronize the device) once it is
 // running.  For them moe_count_scan_noalloc runs the same kernels on a fixed scratch array
@@ -55,14 +55,15 @@ extern "C" moe_status moe_count_scan_noalloc(const int32_t* topk_ids, const moe_
   uint8_t* base = static_cast<uint8_t*>(scratch_address());
   if (!base) return MOE_ERR_CUDA;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // The scratch keeps the previous call's contents.  The kernels leave the counters, the
-  // look-back flags and the expert totals at zero, but a previous call that failed between
-  // its two launches would not have: clear them (and the status word) on every call.
-  const size_t clear = ScanWorkspace::kFixedBytes + round256(static_cast<size_t>(d->E) * sizeof(int));
-  if (cudaMemsetAsync(base, 0, clear, s) != cudaSuccess) return MOE_ERR_CUDA;
+  // The scratch keeps the previous call's contents.  The kernel leaves its counters and
+  // look-back flags at zero, but a previous call whose kernel failed to launch or to finish
+  // would not have: clear them (and the status word) on every call.
+  if (cudaMemsetAsync(base, 0, ScanWorkspace::kFixedBytes, s) != cudaSuccess) return MOE_ERR_CUDA;
   const ScanWorkspace ws = scan_workspace(base, TK, d->E);
-  if (launch_hist(topk_ids, TK, d->E, ws, s) != cudaSuccess) return MOE_ERR_CUDA;
-  const cudaError_t e = launch_count_scan(topk_ids, TK, d->E, d->P, counts, offsets, part_counts, part_offsets,
-                                          row_of_assign, assign_of_row, nullptr, ws, s);
-  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  if (launch_count_scan(topk_ids, TK, d->E, d->P, row_of_assign, counts, offsets, part_counts, part_offsets, nullptr,
+                        ws, s) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  return launch_scan_finalize(topk_ids, TK, d->E, offsets, row_of_assign, assign_of_row, s) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }

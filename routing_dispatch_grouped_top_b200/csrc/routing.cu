@@ -45,7 +45,7 @@ constexpr int route_warps(int vpl) { return vpl <= 8 ? 8 : 4; }
 template <int VPL>
 __global__ void __launch_bounds__(32 * route_warps(VPL)) route_kernel(
     const float* __restrict__ logits, int nsplit, float* __restrict__ logits_out, long long T, int E, int K,
-    int renormalize, int P, int M, int32_t* __restrict__ ids, float* __restrict__ w, int* __restrict__ hist) {
+    int renormalize, int P, int M, int32_t* __restrict__ ids, float* __restrict__ w) {
   constexpr int W = route_warps(VPL);
   constexpr unsigned kFull = 0xffffffffu;
   __shared__ alignas(16) uint32_t s_key[W][32 * VPL];
@@ -202,18 +202,17 @@ __global__ void __launch_bounds__(32 * route_warps(VPL)) route_kernel(
     if (lane < K) {
       ids[t * K + lane] = my_id;
       w[t * K + lane] = num / den;
-      if (hist) atomicAdd(hist + my_id, 1);  // expert totals for the count/scan that follows
     }
   }
 }
 
 template <int VPL>
 cudaError_t launch_route_vpl(const float* logits, int nsplit, float* logits_out, long long T, int E, int K,
-                             int renorm, int P, int M, int32_t* ids, float* w, int* hist, cudaStream_t s) {
+                             int renorm, int P, int M, int32_t* ids, float* w, cudaStream_t s) {
   constexpr int W = route_warps(VPL);
   const long long blocks = std::min<long long>((T + W - 1) / W, 64LL * num_sms());
   return launch_pdl(route_kernel<VPL>, dim3(static_cast<unsigned>(std::max<long long>(blocks, 1))), dim3(32 * W), 0,
-                    s, logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, hist);
+                    s, logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w);
 }
 
 // out[i] = sum_{p < nsplit} partials[p * n + i], added in order p = 0, 1, ...
@@ -230,26 +229,28 @@ __global__ void sum_partials_kernel(const float* __restrict__ partials, int nspl
 }
 
 // ---------------------------------------------------------------------------
-// Count + scan + stable rank: a block-local histogram and a decoupled look-back scan.
+// Count + scan + stable rank in one pass: block-local histograms and a decoupled look-back
+// scan over the blocks.
 //
-// The expert totals come from a histogram taken before the scan: the route kernel adds
-// every id it writes to hist[E] (the layer path), or expert_hist_kernel counts a caller's
-// ids (moe_count_scan).  count_scan_kernel then makes one pass over the assignments in nb
-// chunks, one block per chunk, the chunk chosen by a ticket the block takes when it
-// starts (so a block only ever waits for blocks that are already running):
+// count_scan_kernel splits the assignments into nb chunks, one block per chunk, the chunk
+// chosen by a ticket the block takes when it starts (so a block only waits for blocks that
+// are already running):
 //   1. block histogram of its chunk, kept per warp (warp w owns a contiguous slice);
 //   2. the block publishes its per-expert counts (flag AGG) and looks back over its
-//      predecessors: one warp reads 32 flags at a time, and the counts of the blocks up
-//      to the nearest one that has published an inclusive prefix (flag INC) are added to
-//      that prefix; then it publishes its own inclusive prefix (flag INC);
-//   3. row of assignment a with expert e = offsets[e] (exclusive scan of hist) + the
-//      counts of e in earlier blocks + in earlier warps of this block + the number of
-//      earlier assignments of e in this warp (__match_any_sync): rows of one expert keep
-//      increasing a, a stable counting sort;
-//   4. the last block to finish clears hist and the flags and rewinds the ticket and
-//      the done counter for the next call.
-// Every wait is bounded: a block that gives up sets MOE_DEV_TIMEOUT and scatters nothing.
-// A call that met an invalid id or a wait that ran out leaves offsets[E] = -1.
+//      predecessors: one warp reads 32 flags at a time, and the counts of the blocks up to
+//      the nearest one that has published an inclusive prefix (flag INC) are added to that
+//      prefix; then it publishes its own inclusive prefix (flag INC);
+//   3. rank of assignment a (expert e) within its expert = the counts of e in earlier
+//      blocks + in earlier warps of this block + the number of earlier assignments of e in
+//      this warp (__match_any_sync): the stable order (increasing a) inside each expert.
+//      The rank is written to row_of_assign[a]; the row is offsets[e] + rank;
+//   4. the last block to finish takes the totals from the last chunk's inclusive prefix,
+//      scans them into offsets (and counts, partitions, skew), then clears the flags and
+//      rewinds the ticket and done counters for the next call.
+// The offsets exist only once every block is done, so the ranks become rows afterwards:
+// in the layer's permute (which reads them anyway), or in scan_finalize_kernel.  Every
+// wait is bounded: a block that gives up sets MOE_DEV_TIMEOUT and ranks nothing, and a call
+// that met an invalid id or a wait that ran out leaves offsets[E] = -1.
 // ---------------------------------------------------------------------------
 
 constexpr int kScanThreads = 256;
@@ -269,38 +270,63 @@ __device__ __forceinline__ void st_release(int* p, int v) {
   asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 
-// hist[e] += number of ids equal to e (ids outside [0, E) are skipped; count_scan reports them).
-__global__ void __launch_bounds__(kScanThreads) expert_hist_kernel(const int32_t* __restrict__ ids, long long TK,
-                                                                   int E, int* __restrict__ hist) {
-  extern __shared__ int s_h[];
-  for (int e = threadIdx.x; e < E; e += kScanThreads) s_h[e] = 0;
-  pdl_wait();
-  pdl_launch_dependents();
-  __syncthreads();
-  const long long stride = static_cast<long long>(gridDim.x) * kScanThreads;
-  for (long long a = static_cast<long long>(blockIdx.x) * kScanThreads + threadIdx.x; a < TK; a += stride) {
-    const int e = __ldg(ids + a);
-    if (e >= 0 && e < E) atomicAdd(&s_h[e], 1);
+// Exclusive scan of vals[0..n) (n <= 1024) in shared memory by the whole block; returns the
+// total and the maximum, out[n] = total.
+__device__ void block_exclusive_scan(const int* vals, int n, int* out, int* s_red, int* s_max, int& total,
+                                     int& mx) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int per = (n + kScanThreads - 1) / kScanThreads;
+  const int e0 = min(n, tid * per), e1 = min(n, e0 + per);
+  int local = 0, my_max = 0;
+  for (int e = e0; e < e1; ++e) {
+    const int c = vals[e];
+    local += c;
+    my_max = max(my_max, c);
   }
+  int incl = local;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += v;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, o));
+  __syncthreads();  // vals may alias out
+  if (lane == 31) s_red[warp] = incl;
+  if (lane == 0) s_max[warp] = my_max;
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += kScanThreads)
-    if (s_h[e]) atomicAdd(hist + e, s_h[e]);
+  int wbase = 0;
+  total = 0, mx = 0;
+  for (int w = 0; w < kScanWarps; ++w) {
+    if (w < warp) wbase += s_red[w];
+    total += s_red[w];
+    mx = max(mx, s_max[w]);
+  }
+  int run = wbase + incl - local;
+  int c_buf[kPerThreadE];
+  for (int e = e0; e < e1; ++e) c_buf[e - e0] = vals[e];
+  __syncthreads();
+  for (int e = e0; e < e1; ++e) {
+    out[e] = run;
+    run += c_buf[e - e0];
+  }
+  if (tid == 0) out[n] = total;
+  __syncthreads();
 }
 
 __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
-    const int32_t* __restrict__ ids, int TK, int E, int P, int chunk, int nb, int32_t* __restrict__ counts,
-    int32_t* __restrict__ offsets, int32_t* __restrict__ part_counts, int32_t* __restrict__ part_offsets,
-    int32_t* __restrict__ row_of_assign, int32_t* __restrict__ assign_of_row, float* __restrict__ skew,
-    const ScanWorkspace ws) {
+    const int32_t* __restrict__ ids, int TK, int E, int P, int chunk, int nb, int32_t* __restrict__ rank_out,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ part_counts,
+    int32_t* __restrict__ part_offsets, float* __restrict__ skew, const ScanWorkspace ws) {
   extern __shared__ int sm[];
-  int* s_run = sm;                        // [kScanWarps][E] warp counts, then each warp's next row
-  int* s_agg = s_run + kScanWarps * E;    // [E] this block's counts
-  int* s_off = s_agg + E;                 // [E + 1] exclusive scan of the totals
+  int* s_run = sm;                        // [kScanWarps][E] warp counts, then each warp's next rank
+  int* s_agg = s_run + kScanWarps * E;    // [E] this block's counts; the last block: totals
+  int* s_off = s_agg + E;                 // [E + 1] the last block: exclusive scan of the totals
   __shared__ int s_b, s_bad, s_ok, s_last, s_nwin, s_incpos, s_red[kScanWarps], s_max[kScanWarps];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   for (int i = tid; i < kScanWarps * E; i += kScanThreads) s_run[i] = 0;
-  pdl_wait();  // the ids and the histogram come from the previous kernel
+  pdl_wait();  // the ids come from the previous kernel
   pdl_launch_dependents();
   if (tid == 0) {
     s_b = atomicAdd(ws.ticket, 1);
@@ -308,58 +334,7 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
     s_ok = s_b < nb;  // a ticket beyond the grid: the previous call on this workspace did not finish
     if (!s_ok) report(ws.status, MOE_DEV_TIMEOUT);
   }
-
-  // global exclusive offsets from the totals (up to 4 experts per thread)
-  int my_max = 0;
-  {
-    const int per = (E + kScanThreads - 1) / kScanThreads;
-    const int e0 = min(E, tid * per), e1 = min(E, e0 + per);
-    int local = 0;
-    for (int e = e0; e < e1; ++e) {
-      const int c = __ldcg(ws.hist + e);
-      s_off[e] = c;
-      local += c;
-      my_max = max(my_max, c);
-    }
-    int incl = local;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, o);
-      if (lane >= o) incl += v;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) my_max = max(my_max, __shfl_xor_sync(0xffffffffu, my_max, o));
-    if (lane == 31) s_red[warp] = incl;
-    if (lane == 0) s_max[warp] = my_max;
-    __syncthreads();
-    int wbase = 0, total = 0, mx = 0;
-    for (int w = 0; w < kScanWarps; ++w) {
-      if (w < warp) wbase += s_red[w];
-      total += s_red[w];
-      mx = max(mx, s_max[w]);
-    }
-    int run = wbase + incl - local;
-    for (int e = e0; e < e1; ++e) {
-      const int c = s_off[e];
-      s_off[e] = run;
-      run += c;
-    }
-    if (tid == 0) s_off[E] = total;
-    __syncthreads();
-    if (s_b == 0) {  // the block holding ticket 0 writes the per-expert outputs
-      for (int e = tid; e <= E; e += kScanThreads) {
-        offsets[e] = s_off[e];
-        if (e < E) counts[e] = s_off[e + 1] - s_off[e];
-      }
-      const int epp = E / P;
-      for (int p = tid; p <= P; p += kScanThreads) {
-        part_offsets[p] = s_off[p * epp];
-        if (p < P) part_counts[p] = s_off[(p + 1) * epp] - s_off[p * epp];
-      }
-      if (tid == 0 && skew) skew[0] = total > 0 ? static_cast<float>(mx) * static_cast<float>(E) / total : 0.0f;
-    }
-  }
-
+  __syncthreads();
   const int b = s_b;
   const bool active = s_ok;  // block-uniform
   const int lo = min(TK, b * chunk), hi = min(TK, lo + chunk);
@@ -471,14 +446,13 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
         st_release(ws.flags + b, kFlagInc);
       }
     }
-    // 3. each warp's first row per expert, then the rows of its slice in order
+    // 3. each warp's first rank per expert, then the ranks of its slice in order
 #pragma unroll
     for (int j = 0; j < kPerThreadE; ++j) {
       const int e = tid + j * kScanThreads;
       if (e < E) {
-        const int base = s_off[e] + excl[j];
 #pragma unroll
-        for (int w = 0; w < kScanWarps; ++w) s_run[w * E + e] += base;
+        for (int w = 0; w < kScanWarps; ++w) s_run[w * E + e] += excl[j];
       }
     }
     __syncthreads();
@@ -490,22 +464,14 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
         if (e < 0 || e >= E) e = -1;
       }
       const unsigned same = __match_any_sync(0xffffffffu, e);
-      if (a < whi) {
-        if (e < 0) {
-          row_of_assign[a] = -1;  // an invalid id gets no row
-        } else {
-          const int r = s_run[warp * E + e] + __popc(same & lt_mask);
-          row_of_assign[a] = r;
-          assign_of_row[r] = a;
-        }
-      }
+      if (a < whi) rank_out[a] = e < 0 ? -1 : s_run[warp * E + e] + __popc(same & lt_mask);  // -1: no row
       __syncwarp();
       if (e >= 0 && lane == __ffs(same) - 1) s_run[warp * E + e] += __popc(same);
       __syncwarp();
     }
   }
 
-  // 4. the last block rewinds the workspace for the next call
+  // 4. the last block writes the per-expert outputs and rewinds the workspace for the next call
   __syncthreads();
   if (tid == 0) {
     if (s_bad) report(ws.status, MOE_DEV_BAD_INDEX);
@@ -516,13 +482,51 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
   __syncthreads();
   if (s_last) {
     __threadfence();
-    for (int e = tid; e < E; e += kScanThreads) ws.hist[e] = 0;
+    // totals: the inclusive prefix of the last chunk (every block published it before counting done)
+    const int* totals = ws.inc + static_cast<long long>(nb - 1) * E;
+    for (int e = tid; e < E; e += kScanThreads) s_agg[e] = TK > 0 ? __ldcg(totals + e) : 0;
+    __syncthreads();
+    int total = 0, mx = 0;
+    block_exclusive_scan(s_agg, E, s_off, s_red, s_max, total, mx);
+    const bool failed = *reinterpret_cast<volatile int*>(ws.fail) != 0;  // every block's flag is in
+    for (int e = tid; e <= E; e += kScanThreads) {
+      offsets[e] = (e == E && failed) ? -1 : s_off[e];
+      if (e < E) counts[e] = s_off[e + 1] - s_off[e];
+    }
+    const int epp = E / P;
+    for (int p = tid; p <= P; p += kScanThreads) {
+      part_offsets[p] = s_off[p * epp];
+      if (p < P) part_counts[p] = s_off[(p + 1) * epp] - s_off[p * epp];
+    }
+    if (tid == 0 && skew) skew[0] = total > 0 ? static_cast<float>(mx) * static_cast<float>(E) / total : 0.0f;
     for (int p = tid; p < kScanMaxBlocks; p += kScanThreads) ws.flags[p] = 0;
+    __syncthreads();
     if (tid == 0) {
-      if (atomicExch(ws.fail, 0)) offsets[E] = -1;  // after ticket 0's write: every block is done
+      *ws.fail = 0;
       *ws.ticket = 0;
       *ws.done = 0;
     }
+  }
+}
+
+// row_of_assign[a] = offsets[ids[a]] + rank (in place), assign_of_row[row] = a.
+__global__ void __launch_bounds__(kScanThreads) scan_finalize_kernel(const int32_t* __restrict__ ids, long long TK,
+                                                                     int E, const int32_t* __restrict__ offsets,
+                                                                     int32_t* __restrict__ row_of_assign,
+                                                                     int32_t* __restrict__ assign_of_row) {
+  pdl_wait();  // the ranks and offsets come from count_scan_kernel
+  pdl_launch_dependents();
+  for (long long a = static_cast<long long>(blockIdx.x) * kScanThreads + threadIdx.x; a < TK;
+       a += static_cast<long long>(gridDim.x) * kScanThreads) {
+    const int r = row_of_assign[a];
+    const int e = __ldg(ids + a);
+    int row = -1;
+    if (r >= 0 && e >= 0 && e < E) {
+      const long long v = static_cast<long long>(__ldg(offsets + e)) + r;
+      if (v >= 0 && v < TK) row = static_cast<int>(v);
+    }
+    row_of_assign[a] = row;
+    if (row >= 0) assign_of_row[row] = static_cast<int>(a);
   }
 }
 
@@ -560,10 +564,10 @@ cudaError_t launch_sum_partials(const float* partials, int nsplit, long long n, 
 }
 
 cudaError_t launch_route(const float* logits, int nsplit, float* logits_out, long long T, int E, int K, int renorm,
-                         int P, int M, int32_t* ids, float* w, int* hist, cudaStream_t s) {
+                         int P, int M, int32_t* ids, float* w, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int vpl = (E + 31) / 32;
-#define MOE_ROUTE(V) launch_route_vpl<V>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, hist, s)
+#define MOE_ROUTE(V) launch_route_vpl<V>(logits, nsplit, logits_out, T, E, K, renorm, P, M, ids, w, s)
   if (vpl <= 1) return MOE_ROUTE(1);
   if (vpl <= 2) return MOE_ROUTE(2);
   if (vpl <= 4) return MOE_ROUTE(4);
@@ -580,7 +584,7 @@ int scan_blocks(long long TK) {
 
 size_t scan_ws_bytes(long long TK, int E) {
   const size_t rows = static_cast<size_t>(scan_blocks(TK)) * E * sizeof(int);
-  return ScanWorkspace::kFixedBytes + round256(static_cast<size_t>(E) * sizeof(int)) + 2 * round256(rows);
+  return ScanWorkspace::kFixedBytes + 2 * round256(rows);
 }
 
 ScanWorkspace scan_workspace(void* base, long long TK, int E) {
@@ -591,25 +595,15 @@ ScanWorkspace scan_workspace(void* base, long long TK, int E) {
   w.done = reinterpret_cast<int*>(p + 96);
   w.fail = reinterpret_cast<int*>(p + 128);
   w.flags = reinterpret_cast<int*>(p + 256);
-  size_t off = ScanWorkspace::kFixedBytes;
-  w.hist = reinterpret_cast<int*>(p + off);
-  off += round256(static_cast<size_t>(E) * sizeof(int));
   const size_t rows = round256(static_cast<size_t>(scan_blocks(TK)) * E * sizeof(int));
-  w.agg = reinterpret_cast<int*>(p + off);
-  w.inc = reinterpret_cast<int*>(p + off + rows);
+  w.agg = reinterpret_cast<int*>(p + ScanWorkspace::kFixedBytes);
+  w.inc = reinterpret_cast<int*>(p + ScanWorkspace::kFixedBytes + rows);
   return w;
 }
 
-cudaError_t launch_hist(const int32_t* ids, long long TK, int E, const ScanWorkspace& ws, cudaStream_t s) {
-  if (TK == 0) return cudaSuccess;
-  const long long blocks = std::min<long long>((TK + 4 * kScanThreads - 1) / (4 * kScanThreads), num_sms());
-  return launch_pdl(expert_hist_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kScanThreads),
-                    static_cast<size_t>(E) * sizeof(int), s, ids, TK, E, ws.hist);
-}
-
-cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, int32_t* counts, int32_t* offsets,
-                              int32_t* part_counts, int32_t* part_offsets, int32_t* row_of_assign,
-                              int32_t* assign_of_row, float* skew, const ScanWorkspace& ws, cudaStream_t s) {
+cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, int32_t* ranks, int32_t* counts,
+                              int32_t* offsets, int32_t* part_counts, int32_t* part_offsets, float* skew,
+                              const ScanWorkspace& ws, cudaStream_t s) {
   static std::atomic<int> attr_done[kMaxDevices] = {};
   const cudaError_t attr = smem_attr_once(reinterpret_cast<const void*>(count_scan_kernel),
                                           static_cast<int>(scan_smem_bytes(MOE_MAX_E)), attr_done);
@@ -617,8 +611,16 @@ cudaError_t launch_count_scan(const int32_t* ids, long long TK, int E, int P, in
   const int nb = scan_blocks(TK);
   const long long chunk = (TK + nb - 1) / nb;
   return launch_pdl(count_scan_kernel, dim3(nb), dim3(kScanThreads), scan_smem_bytes(E), s, ids,
-                    static_cast<int>(TK), E, P, static_cast<int>(chunk), nb, counts, offsets, part_counts,
-                    part_offsets, row_of_assign, assign_of_row, skew, ws);
+                    static_cast<int>(TK), E, P, static_cast<int>(chunk), nb, ranks, counts, offsets, part_counts,
+                    part_offsets, skew, ws);
+}
+
+cudaError_t launch_scan_finalize(const int32_t* ids, long long TK, int E, const int32_t* offsets,
+                                 int32_t* row_of_assign, int32_t* assign_of_row, cudaStream_t s) {
+  if (TK == 0) return cudaSuccess;
+  const long long blocks = std::min<long long>((TK + kScanThreads - 1) / kScanThreads, 4LL * num_sms());
+  return launch_pdl(scan_finalize_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kScanThreads), 0, s, ids, TK, E,
+                    offsets, row_of_assign, assign_of_row);
 }
 
 cudaError_t launch_skew(const int32_t* counts, int E, float* ratio, cudaStream_t s) {
