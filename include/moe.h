@@ -166,7 +166,8 @@ moe_status moe_route(const float* logits, const moe_dims* d, int32_t* topk_ids,
  *   row_of_assign[TK]: row of assignment a in the expert-major buffer, a stable
  *     counting sort (rows of one expert keep increasing a),
  *   assign_of_row[TK]: its inverse.
- * Two launches: one pass over the assignments in up to 128 chunks, block-local histograms
+ * Two launches: one pass over the assignments in up to 128 chunks (1024 or more
+ * assignments each), block-local histograms
  * with a decoupled look-back scan across the chunks (each chunk's counts are published and
  * added up by its successors; no grid-wide barrier), which ranks every assignment within
  * its expert and leaves the offsets; then the ranks become rows.  Uses the workspace
@@ -189,9 +190,9 @@ moe_status moe_count_scan(const int32_t* topk_ids, const moe_dims* d, int32_t* c
  * call cudaMalloc/cudaFree, which can also synchronize the device, once it runs).
  * Same arguments, results and status codes as moe_count_scan minus the workspace.  The
  * scratch is a fixed device array inside the library holding the count/scan state: 768
- * bytes of counters and look-back flags and two int32 rows of E per chunk (ceil(T*K / 256)
+ * bytes of counters and look-back flags and two int32 rows of E per chunk (ceil(T*K / 1024)
  * chunks, at most 128), at most MOE_NOALLOC_SCRATCH_BYTES in all; larger shapes return
- * MOE_ERR_UNSUPPORTED_SHAPE (only E = 1024 with T*K > 32 512 exceeds it).  The call
+ * MOE_ERR_UNSUPPORTED_SHAPE (only E = 1024 with T*K > 130 048 exceeds it).  The call
  * allocates nothing: it clears the scratch's counters and flags with an async memset on
  * `stream`, then launches the count/scan kernel and the kernel that turns ranks into rows.
  * The first call on a device looks up the scratch's device address once (with that device

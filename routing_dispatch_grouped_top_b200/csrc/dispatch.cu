@@ -84,6 +84,11 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
   const int epp = E / P;
   const long long nwarps = static_cast<long long>(gridDim.x) * kWarps;
   for (long long t = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5); t < T; t += nwarps) {
+    const uint4* src = x + t * vpr;
+    uint4 v[kUnroll];  // the first vectors are on their way while the rows are looked up
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (lane + 32 * u < vpr) v[u] = ld_stream(src + lane + 32 * u);
     int row = -1;
     if (lane < K) {
       const long long a = t * K + lane;
@@ -95,12 +100,12 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
         if (meta_local) meta_local[row] = __ldg(ids + a) % epp;
       }
     }
-    const uint4* src = x + t * vpr;
     for (int v0 = lane; v0 < vpr; v0 += 32 * kUnroll) {
-      uint4 v[kUnroll];
+      if (v0 != lane) {
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        if (v0 + 32 * u < vpr) v[u] = ld_stream(src + v0 + 32 * u);
+        for (int u = 0; u < kUnroll; ++u)
+          if (v0 + 32 * u < vpr) v[u] = ld_stream(src + v0 + 32 * u);
+      }
       for (int k = 0; k < K; ++k) {
         const int rk = __shfl_sync(0xffffffffu, row, k);
         if (rk < 0) continue;

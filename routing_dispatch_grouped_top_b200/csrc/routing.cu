@@ -255,7 +255,7 @@ __global__ void sum_partials_kernel(const float* __restrict__ partials, int nspl
 
 constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
-constexpr int kScanMinChunk = 256;
+constexpr int kScanMinChunk = 1024;  // per block: 4 assignments per thread; short look-back chains
 constexpr int kLookWindow = 32;
 constexpr int kPerThreadE = MOE_MAX_E / kScanThreads;  // experts a thread scans and looks back for
 constexpr int kFlagAgg = 1, kFlagInc = 2;

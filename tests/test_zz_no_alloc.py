@@ -78,7 +78,7 @@ def test_noalloc_count_scan_marks_an_invalid_id_then_recovers():
 
 
 def test_noalloc_count_scan_rejects_shapes_beyond_its_scratch():
-    # E = 1024 with more than 127 chunks of 256 assignments needs more than the 1 MiB scratch
+    # E = 1024 with more than 127 chunks of 1024 assignments needs more than the 1 MiB scratch
     d = B.dims(T=32768, H=8, E=1024, K=8, F=8)
     st = B.lib().moe_count_scan_noalloc(None, C.byref(d), None, None, None, None, None, None, None)
     assert st == 1   # null outputs are refused first
@@ -86,7 +86,7 @@ def test_noalloc_count_scan_rejects_shapes_beyond_its_scratch():
     with pytest.raises(B.MoEError) as e:
         B.moe_count_scan_noalloc(torch.zeros((32768, 8), dtype=torch.int32, device=DEV), d, *bufs)
     assert e.value.status == 2   # MOE_ERR_UNSUPPORTED_SHAPE
-    T = 127 * 256 // 8           # 127 chunks: fits
+    T = 127 * 1024 // 8          # 127 chunks: fits
     ok = B.dims(T=T, H=8, E=1024, K=8, F=8)
     ids = inputs.random_topk_ids(T, 1024, 8, seed=3)
     bufs = outputs(1024, 1, T * 8, 0)
