@@ -455,7 +455,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     // With 8 epilogue warps, two share each lane quadrant and take alternate 32-token chunks.
     constexpr int kSplit = C::EW / 4;
     const int part = (warp - 2) >> 2;
-    uint32_t acc = 0, acc_phase = 0, rs = 0, rphase = 0;
+    uint32_t acc = 0, acc_phase = 0, chunk = 0, rs = 0, rphase = 0;
     for (;;) {
       if (!mbar_wait(&rfull[rs], rphase, abort_flag, args.status)) break;
       const int t = ring_tile[rs];
@@ -567,72 +567,57 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 // or 512 (bf16) output features x N <= 256 tokens.  Each CTA stages its own 128 rows of
 // each of the two weight operands and half of the token rows; the pair MMA (M = 256,
 // issued by the leader, rank 0) reads both token halves, so a token tile crosses L2 once
-// per pair and each SM fills 48 KB of shared memory per K-step for the MMA work that the
-// single-CTA tile needs 64 KB for.
+// per pair and each SM fills 48 KB of shared memory per K-step instead of the single-CTA
+// tile's 64 KB for the same MMA work per SM.
 //   SwiGLU: CTA r holds gate and up rows [n0 + 128 r, +128): gate and up accumulate in
 //           separate TMEM columns of the same lanes, so no exchange between warps; the two
 //           accumulators fill TMEM, so the epilogue of a tile runs between main loops.
 //   bf16:   CTA r holds rows [n0 + 128 r, +128) and [n0 + 256 + 128 r, +128) (NA = 2).
-// Weights and tokens travel in two rings of their own: WST weight stages (32 KB each) and BST
-// token stages (16 KB each), filled by two producer warps.  The weights stream from HBM and
-// the tokens mostly hit L2, so the shared memory goes to weight bytes in flight: measured on
-// B200, the kernel's weight stream was bound by the latency of its loads (the MMAs waited
-// with four 48 KB stages in flight while a pure TMA stream of the same boxes reached the
-// copy bandwidth), and with five weight stages more of that latency is covered.
-// Both CTAs' loads of a stage complete on the leader's "full" barriers; the leader's commits
-// release both CTAs' "empty" and "tmem full" barriers; both CTAs' epilogue warps release the
-// leader's "tmem empty" barrier.  The leader's weight producer claims tiles from the launch's
-// counter and publishes each id to both CTAs through a ring in shared memory (the peer's slot
-// written over the cluster), which every other role of both CTAs releases.
+// Both CTAs' TMA loads of a stage complete on the leader's "full" barrier; the leader's
+// commits release both CTAs' "empty" and "tmem full" barriers; both CTAs' epilogue warps
+// release the leader's "tmem empty" barrier.  The leader's producer claims tiles from the
+// launch's counter and publishes each id to both CTAs through a ring in shared memory (the
+// peer's slot written over the cluster), which both CTAs' consumers release.
 // ---------------------------------------------------------------------------
-constexpr int kPairThreads = 96 + 32 * 8;  // weight producer, MMA issuer, token producer, 8 epilogue warps
-
 template <int EPI>
 struct PairLayout {
   static constexpr int NT = 256;                                // tokens per pair tile (MMA N)
   static constexpr int NA = 2;                                  // weight operands (accumulators)
-  static constexpr int WST = 5;                                 // weight stages
-  static constexpr int BST = 2;                                 // token stages
+  static constexpr int STAGES = 4;
   static constexpr int EW = 8;                                  // epilogue warps per CTA
-  static constexpr int kEpiWarp0 = 3;                           // first epilogue warp
-  static constexpr int kThr = 32 * kEpiWarp0 + 32 * EW;
+  static constexpr int kThr = 64 + 32 * EW;
   static constexpr int FEAT = (EPI == kEpiBF16) ? 512 : 256;   // output features per pair tile
   static constexpr int kAPair = NA * kABytes;                   // this CTA's 128-row weight boxes (one atom)
   static constexpr int kBBytes = (NT / 2) * 128;                // this CTA's token rows (one atom)
-  static constexpr int kRingBytes = WST * kAPair + BST * kBBytes;
+  static constexpr int kStageBytes = kAPair + kBBytes;
   static constexpr uint32_t kAccCols = NA * NT;                 // one tile's accumulators
-  static constexpr uint32_t kTmemCols = kAccCols;               // single-buffered
+  static constexpr int kNumAcc = 1;                             // TMEM buffers
+  static constexpr uint32_t kTmemCols = kNumAcc * kAccCols;
   static constexpr int kStgBytes = EW * 32 * 32 * 2;
-  // wfull/wempty, bfull/bempty, tmem full/empty x2, drain, tile ring full/empty; then the TMEM
-  // address, the abort flag and the ring's tile ids
-  static constexpr int kBarBytes = (8 * (2 * WST + 2 * BST + 5 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
+  static constexpr int kBarBytes = (8 * (2 * STAGES + 5 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
   static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
-  static constexpr int kSmemBytes = 1024 + kRingBytes + kStgBytes + kBarBytes + kTableBytes;
+  static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kStgBytes + kBarBytes + kTableBytes;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kThr == kPairThreads, "block size");
-  static_assert(kAPair % 1024 == 0 && kBBytes % 1024 == 0, "stages stay 1024-byte aligned (128-byte swizzle)");
+  static_assert(kThr <= kMaxThreads, "block size");
 };
 
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                      const __grid_constant__ BoxMaps tmB, const GemmArgs args) {
   using L = PairLayout<EPI>;
-  constexpr int NT = L::NT, NA = L::NA, WST = L::WST, BST = L::BST, EW = L::EW;
+  constexpr int NT = L::NT, NA = L::NA, STAGES = L::STAGES, EW = L::EW;
   constexpr int KS = stage_k<EPI>();
   static_assert(EPI == kEpiSwiGLU || EPI == kEpiSwiGLUFp8 || EPI == kEpiBF16, "pair epilogues");
   static_assert(L::kTmemCols == 512, "TMEM allocation");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* wring = smem;                                   // WST x kAPair
-  uint8_t* bring = smem + WST * L::kAPair;                 // BST x kBBytes
-  __nv_bfloat16* stg_all = reinterpret_cast<__nv_bfloat16*>(smem + L::kRingBytes);
-  uint64_t* wfull = reinterpret_cast<uint64_t*>(smem + L::kRingBytes + L::kStgBytes);
-  uint64_t* wempty = wfull + WST;
-  uint64_t* bfull = wempty + WST;
-  uint64_t* bempty = bfull + BST;
-  uint64_t* tfull = bempty + BST;
+  uint8_t* ring = smem;
+  __nv_bfloat16* stg_all = reinterpret_cast<__nv_bfloat16*>(smem + STAGES * L::kStageBytes);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * L::kStageBytes + L::kStgBytes);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
   uint64_t* rfull = drain + 1;
@@ -640,9 +625,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(rempty + kRing);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   volatile int* ring_tile = reinterpret_cast<volatile int*>(tmem_slot + 2);
-  int* s_off = reinterpret_cast<int*>(smem + L::kRingBytes + L::kStgBytes + L::kBarBytes);
+  int* s_off = reinterpret_cast<int*>(smem + STAGES * L::kStageBytes + L::kStgBytes + L::kBarBytes);
   int* s_pre = s_off + (kMaxGroups + 1);
-  __shared__ int s_warp_sums[kPairThreads / 32];
+  __shared__ int s_warp_sums[kMaxThreads / 32];
   __shared__ int s_bad;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -654,24 +639,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   // Set-up that reads no global input runs before the wait on the previous kernel.
   if (threadIdx.x == 0) {
     s_bad = 0;
-    for (int s = 0; s < WST; ++s) {
-      mbar_init(&wfull[s], 1);
-      mbar_init(&wempty[s], 1);
-    }
-    for (int s = 0; s < BST; ++s) {
-      mbar_init(&bfull[s], 1);
-      mbar_init(&bempty[s], 1);
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tfull[a], 1);
       mbar_init(&tempty[a], 2 * EW);  // every epilogue warp of both CTAs
     }
     mbar_init(drain, 1);
-    // the leader's tile ring is released by its MMA thread, token producer and epilogue warps
-    // and by the peer's weight producer, token producer and epilogue warps
     for (int r = 0; r < kRing; ++r) {
       mbar_init(&rfull[r], 1);
-      mbar_init(&rempty[r], 4 + 2 * EW);
+      mbar_init(&rempty[r], 2 + 2 * EW);  // leader MMA + leader epilogue, peer producer + peer epilogue
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -679,9 +658,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmA0);
     tma_prefetch_map(&tmA1);
-  }
-  if (warp == 2 && lane == 0)
     for (int i = 1; i < kNumBoxes; ++i) tma_prefetch_map(&tmB.box[i]);
+  }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, L::kTmemCols);
     tmem_relinquish_pair();
@@ -708,49 +686,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   const int total = s_pre[G];
-  const uint32_t wfull_leader = mapa_shared(smem_u32(wfull), 0);
-  const uint32_t bfull_leader = mapa_shared(smem_u32(bfull), 0);
+  const uint32_t full_leader = mapa_shared(smem_u32(full), 0);
   const uint32_t rempty_leader = mapa_shared(smem_u32(rempty), 0);
   const uint32_t tempty_leader = mapa_shared(smem_u32(tempty), 0);
 
-  // Next tile id for every role but the leader's weight producer (which claims and publishes):
-  // wait for the ring slot, read it, release it to the leader.  -2 when a wait gave up.
-  auto next_tile = [&](uint32_t& rs, uint32_t& rphase) -> int {
-    if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) return -2;
-    const int t = ring_tile[rs];
-    return t;
-  };
-  auto release_slot = [&](uint32_t& rs, uint32_t& rphase) {
-    if (rank == 0) mbar_arrive(&rempty[rs]);
-    else mbar_arrive_cluster(rempty_leader + 8 * rs);
-    if (++rs == kRing) {
-      rs = 0;
-      rphase ^= 1u;
-    }
-  };
-  // After an abort: let this CTA's own copies land before it exits (the peer's complete on the
-  // leader's barriers, so the peer just gives them time).
-  auto drain_copies = [&](uint64_t* full_bars, const bool* pend, const uint32_t* pend_phase, int n) {
-    if (rank == 0) {
-      for (int s = 0; s < n; ++s)
-        if (pend[s]) mbar_drain(&full_bars[s], pend_phase[s], 200000000ull);
-    } else {
-      const uint64_t t0 = global_timer_ns();
-      while (global_timer_ns() - t0 < 2000000ull) {
-      }
-    }
-  };
-
   if (warp == 0) {
-    // ------------------------------------------------------------ weight producer (both CTAs)
+    // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
       const uint32_t rfull_peer = mapa_shared(smem_u32(rfull), 1);
       const uint32_t ring_peer = mapa_shared(smem_u32(const_cast<int*>(ring_tile)), 1);
       uint32_t stage = 0, phase = 0, rs = 0, rphase = 0;
-      uint32_t pend_phase[WST];
-      bool pend[WST];
+      uint32_t pend_phase[STAGES];
+      bool pend[STAGES];
 #pragma unroll
-      for (int s = 0; s < WST; ++s) pend[s] = false, pend_phase[s] = 0;
+      for (int s = 0; s < STAGES; ++s) pend[s] = false, pend_phase[s] = 0;
       bool ok = true;
       for (;;) {
         int t;
@@ -765,28 +714,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           st_shared_cluster(ring_peer + 4 * rs, t);
           mbar_arrive(&rfull[rs]);
           mbar_arrive_cluster(rfull_peer + 8 * rs);
-          if (++rs == kRing) {
-            rs = 0;
-            rphase ^= 1u;
-          }
         } else {
-          t = next_tile(rs, rphase);
-          if (t == -2) {
+          if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) {
             ok = false;
             break;
           }
-          release_slot(rs, rphase);
+          t = ring_tile[rs];
+          mbar_arrive_cluster(rempty_leader + 8 * rs);
+        }
+        if (++rs == kRing) {
+          rs = 0;
+          rphase ^= 1u;
         }
         if (t < 0) break;
         const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
+        const int half = tl.nround >> 1;  // token rows staged by each CTA (a multiple of 16)
+        const int rbase = tl.row0 + static_cast<int>(rank) * half;
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&wempty[stage], phase ^ 1u, abort_flag, args.status)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
           }
-          const uint32_t bar = wfull_leader + stage * 8;
-          if (rank == 0) mbar_arrive_expect_tx(&wfull[stage], 2u * L::kAPair);
-          uint8_t* st = wring + stage * L::kAPair;
+          const uint32_t bar = full_leader + stage * 8;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kAPair + half * 128));
+          uint8_t* st = ring + stage * L::kStageBytes;
           const int kx = kb * KS;
           if constexpr (EPI == kEpiBF16) {
             tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
@@ -796,81 +747,54 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
             tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
           }
-          pend[stage] = true;
-          pend_phase[stage] = phase;
-          if (++stage == WST) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-        if (!ok) break;
-      }
-      if (!ok) drain_copies(wfull, pend, pend_phase, WST);
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ token producer (both CTAs)
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0, rs = 0, rphase = 0;
-      uint32_t pend_phase[BST];
-      bool pend[BST];
-#pragma unroll
-      for (int s = 0; s < BST; ++s) pend[s] = false, pend_phase[s] = 0;
-      bool ok = true;
-      for (;;) {
-        const int t = next_tile(rs, rphase);
-        if (t == -2) {
-          ok = false;
-          break;
-        }
-        release_slot(rs, rphase);
-        if (t < 0) break;
-        const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
-        const int half = tl.nround >> 1;  // token rows staged by each CTA (a multiple of 16)
-        const int rbase = tl.row0 + static_cast<int>(rank) * half;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&bempty[stage], phase ^ 1u, abort_flag, args.status)) {
-            ok = false;
-            break;
-          }
-          const uint32_t bar = bfull_leader + stage * 8;
-          if (rank == 0) mbar_arrive_expect_tx(&bfull[stage], 2u * half * 128);
-          uint8_t* st = bring + stage * L::kBBytes;
-          const int kx = kb * KS;
           int r = 0;
 #pragma unroll
           for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
             const int rows = 256 >> i;
             if (half & rows) {
-              tma_load_2d_pair(st + r * 128, &tmB.box[i], bar, kx, rbase + r);
+              tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
               r += rows;
             }
           }
           pend[stage] = true;
           pend_phase[stage] = phase;
-          if (++stage == BST) {
+          if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
           }
         }
         if (!ok) break;
       }
-      if (!ok) drain_copies(bfull, pend, pend_phase, BST);
+      if (!ok) {
+        if (rank == 0) {
+#pragma unroll
+          for (int s = 0; s < STAGES; ++s)
+            if (pend[s]) mbar_drain(&full[s], pend_phase[s], 200000000ull);
+        } else {  // the peer's copies complete on the leader's barrier: give them time to land
+          const uint64_t t0 = global_timer_ns();
+          while (global_timer_ns() - t0 < 2000000ull) {
+          }
+        }
+      }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader only)
     if (lane == 0 && rank == 0) {
-      const uint32_t wempty_peer = mapa_shared(smem_u32(wempty), 1);
-      const uint32_t bempty_peer = mapa_shared(smem_u32(bempty), 1);
+      const uint32_t empty_peer = mapa_shared(smem_u32(empty), 1);
       const uint32_t tfull_peer = mapa_shared(smem_u32(tfull), 1);
-      uint32_t ws = 0, wph = 0, bs = 0, bph = 0, acc = 0, acc_phase = 0, rs = 0, rphase = 0;
+      uint32_t stage = 0, phase = 0, acc = 0, acc_phase = 0, rs = 0, rphase = 0;
       bool ok = true;
       for (;;) {
-        const int t = next_tile(rs, rphase);
-        if (t == -2) {
+        if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) {
           ok = false;
           break;
         }
-        release_slot(rs, rphase);
+        const int t = ring_tile[rs];
+        mbar_arrive(&rempty[rs]);
+        if (++rs == kRing) {
+          rs = 0;
+          rphase ^= 1u;
+        }
         if (t < 0) break;
         const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) {
@@ -882,14 +806,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         const uint32_t idesc =
             (EPI == kEpiSwiGLUFp8) ? idesc_e4m3_f32(256, tl.nround) : idesc_bf16_f32(256, tl.nround);
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&wfull[ws], wph, abort_flag, args.status) ||
-              !mbar_wait(&bfull[bs], bph, abort_flag, args.status)) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sa = smem_u32(wring + ws * L::kAPair);
-          const uint32_t sb = smem_u32(bring + bs * L::kBBytes);
+          const uint32_t sa = smem_u32(ring + stage * L::kStageBytes);
+          const uint32_t sb = sa + L::kAPair;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t bdesc = sw128_kmajor_desc(sb + kk * 32);
@@ -901,24 +824,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
               else umma_bf16_pair(d0 + i * NT, adesc, bdesc, idesc, accum);
             }
           }
-          // both CTAs' stage buffers are free again once these MMAs have read them
-          umma_commit_pair(smem_u32(&wempty[ws]));
-          umma_commit_pair(wempty_peer + ws * 8);
-          umma_commit_pair(smem_u32(&bempty[bs]));
-          umma_commit_pair(bempty_peer + bs * 8);
-          if (++ws == WST) {
-            ws = 0;
-            wph ^= 1u;
-          }
-          if (++bs == BST) {
-            bs = 0;
-            bph ^= 1u;
+          umma_commit_pair(smem_u32(&empty[stage]));  // both CTAs' stage buffers are free again
+          umma_commit_pair(empty_peer + stage * 8);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
           }
         }
         if (!ok) break;
         umma_commit_pair(smem_u32(&tfull[acc]));
         umma_commit_pair(tfull_peer + acc * 8);
-        if (++acc == 1) {
+        if (++acc == L::kNumAcc) {
           acc = 0;
           acc_phase ^= 1u;
         }
@@ -930,17 +846,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;                           // TMEM lanes [32q, 32q + 32)
-    const int part = (warp - L::kEpiWarp0) >> 2;      // two warps per lane quadrant take alternate chunks
-    __nv_bfloat16* stg = stg_all + (warp - L::kEpiWarp0) * 32 * 32;
+    const int q = warp & 3;               // TMEM lanes [32q, 32q + 32)
+    const int part = (warp - 2) >> 2;     // two warps per lane quadrant take alternate chunks
+    __nv_bfloat16* stg = stg_all + (warp - 2) * 32 * 32;
     __nv_bfloat16* outb = reinterpret_cast<__nv_bfloat16*>(args.out);
     uint32_t acc = 0, acc_phase = 0, rs = 0, rphase = 0;
     for (;;) {
-      const int t = next_tile(rs, rphase);
-      if (t == -2) break;
+      if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) break;
+      const int t = ring_tile[rs];
       __syncwarp();
-      if (lane == 0) release_slot(rs, rphase);
-      else if (++rs == kRing) rs = 0, rphase ^= 1u;
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(&rempty[rs]);
+        else mbar_arrive_cluster(rempty_leader + 8 * rs);
+      }
+      if (++rs == kRing) {
+        rs = 0;
+        rphase ^= 1u;
+      }
       if (t < 0) break;
       const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
@@ -992,7 +914,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (rank == 0) mbar_arrive(&tempty[acc]);
         else mbar_arrive_cluster(tempty_leader + acc * 8);
       }
-      if (++acc == 1) {
+      if (++acc == L::kNumAcc) {
         acc = 0;
         acc_phase ^= 1u;
       }
