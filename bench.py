@@ -52,6 +52,9 @@ def parse():
                    help="add a shared expert of this width, run on a second stream beside the routed path")
     p.add_argument("--fp8-dispatch", action="store_true",
                    help="dispatch E4M3 rows with per-token scales and run gate/up on E4M3 weights")
+    p.add_argument("--gather", action="store_true",
+                   help="bf16 dispatch without the permuted copy: the gate/up GEMM gathers each row's token "
+                        "in place (saves the xp buffer; slower on B200, its 4-row TMA gathers bound the loads)")
     p.add_argument("--shape", action="append", default=[], metavar="FIELD=INT",
                    help="override one integer field of the workload (T, E, H, F, K, P); for reduced-size "
                         "profiling captures of a workload's kernels, e.g. --shape T=1024 --shape E=32")
@@ -348,10 +351,18 @@ def fp8_accuracy(cfg, inp, bufs, dev) -> dict:
             "format": "E4M3 codes, one fp32 scale per token (amax/448); gate/up weights E4M3 per output feature"}
 
 
-def config_dict(cfg, world: int) -> dict:
+def gathers(cfg, args) -> bool:
+    """bf16 dispatch without the permuted copy: the gate/up GEMM gathers the token rows."""
+    return not cfg.fp8_dispatch and getattr(args, "gather", False)
+
+
+def config_dict(cfg, world: int, gather: bool = False) -> dict:
     return {"workload": cfg.name, "T": cfg.T, "H": cfg.H, "E": cfg.E, "K": cfg.K, "F": cfg.F, "P": cfg.P,
             "d_model": cfg.d_model, "group_limit": cfg.group_limit, "F_shared": cfg.F_shared,
             "fp8_dispatch": cfg.fp8_dispatch,
+            "dispatch": ("e4m3 rows permuted with per-row scales" if cfg.fp8_dispatch else
+                         "token rows gathered by the gate/up GEMM (no permuted copy)" if gather else
+                         "bf16 rows permuted into an expert-major copy"),
             "parallelism": f"replicas{world}",
             "l2": "flushed (256 MiB write) before every timed step, outside its events"}
 
@@ -372,7 +383,7 @@ def run_reference(args, cfg):
             "warmup": args.warmup, "ms_per_step": 1000.0 * oracle_sample_tokens(cfg) / val,
             "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "impl": "reference", "config": config_dict(cfg, ws),
+            "impl": "reference", "config": config_dict(cfg, ws, gathers(cfg, args)),
             "cpu_baseline": cb, "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
                                         "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -415,7 +426,8 @@ def main():
     inp = inputs.make_layer(cfg, dev)
     w = B.pack_layer_weights(d, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"], inp["w_dp"],
                              inp["w_upp"], shared=inp["shared"])
-    bufs = B.alloc_layer_buffers(d, dev)
+    gather = gathers(cfg, args)
+    bufs = B.alloc_layer_buffers(d, dev, gather=gather)
     if cfg.F_shared:
         B.attach_aux_stream(bufs, torch.cuda.Stream(dev))
     ws = B.make_workspace(d, dev)
@@ -480,7 +492,7 @@ def main():
     d_in = cfg.d_model or cfg.H
     lanes = []
     for i in range(E2E_LANES):
-        lb = bufs if i == 0 else B.alloc_layer_buffers(d, dev)
+        lb = bufs if i == 0 else B.alloc_layer_buffers(d, dev, gather=gather)
         if cfg.F_shared and i > 0:
             B.attach_aux_stream(lb, torch.cuda.Stream(dev))
         lanes.append(dict(stream=torch.cuda.Stream(dev), bufs=lb,
@@ -533,11 +545,13 @@ def main():
         # algorithmic work per launch: (flops, HBM bytes)
         fp8 = cfg.fp8_dispatch
         xb = 1 if fp8 else 2            # bytes per dispatched activation element and gate/up weight
+        # gathered rows: each token's row need cross HBM once (T H 2), the permute step only
+        # reads the ranks and ids and writes rows and metadata
         work = {
-            "gate_up": (4 * H * F * TK, 2 * H * F * xb * n_touched + TK * H * xb + TK * F * 2
-                        + (2 * F * 4 * n_touched + TK * 4 if fp8 else 0)),
+            "gate_up": (4 * H * F * TK, 2 * H * F * xb * n_touched + (T * H * 2 if gather else TK * H * xb)
+                        + TK * F * 2 + (2 * F * 4 * n_touched + TK * 4 if fp8 else 0)),
             "down": (2 * H * F * TK, H * F * 2 * n_touched + TK * F * 2 + TK * H * 2),
-            "permute": (0, T * H * 2 + TK * H * xb + TK * (4 + 8 + 16) + (TK * 4 if fp8 else 0)),
+            "permute": (0, (0 if gather else T * H * 2 + TK * H * xb) + TK * (4 + 8 + 16) + (TK * 4 if fp8 else 0)),
             "combine": (0, TK * H * 2 + T * H * 2 + TK * 8),
             "gating": (2 * T * H * cfg.E * 3, T * H * 2 + 3 * cfg.E * H * 2 + T * cfg.E * 4),
             "route": (0, T * cfg.E * 4 + TK * 8),
@@ -586,7 +600,7 @@ def main():
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "e4m3 gate/up, bf16 elsewhere" if fp8 else "bf16", "data": "synthetic",
-            "config": config_dict(cfg, world),
+            "config": config_dict(cfg, world, gather),
             "roofline": roof,
             "stages_ms": stage_mean,
             **({"shared_expert": shared_diag} if shared_diag else {}),

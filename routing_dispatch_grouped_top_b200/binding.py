@@ -78,6 +78,7 @@ _SIGS = {
     "moe_permute": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "moe_grouped_ffn": (C.c_int, [_VP, _VP, _VP, _VP, _VP, _DP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_gate_up": (C.c_int, [_VP, _VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
+    "moe_grouped_gate_up_gather": (C.c_int, [_VP, _VP, _VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
     "moe_grouped_down": (C.c_int, [_VP, _VP, _VP, _DP, _VP, _VP, _SZ, _VP]),
     "moe_set_pair_min_rows": (None, [_I32]),
     "moe_quantize_fp8_rows": (C.c_int, [_VP, _I64, _I32, _VP, _VP, _VP]),
@@ -312,6 +313,16 @@ def moe_grouped_gate_up(xp, offsets, w_gate, w_up, d: moe_dims, h, ws, stream=No
         _stream(stream)))
 
 
+def moe_grouped_gate_up_gather(x, assign_of_row, offsets, w_gate, w_up, d: moe_dims, h, ws, stream=None):
+    """moe_grouped_gate_up on the unpermuted x [T][H]: row r is token assign_of_row[r] // K."""
+    TK = d.T * d.K
+    _check("moe_grouped_gate_up_gather", lib().moe_grouped_gate_up_gather(
+        _ptr(x, torch.bfloat16, "x", d.T * d.H), _ptr(assign_of_row, torch.int32, "assign_of_row", TK),
+        _ptr(offsets, torch.int32, "offsets", d.E + 1), _ptr(w_gate, torch.bfloat16, "w_gate", d.E * d.F * d.H),
+        _ptr(w_up, torch.bfloat16, "w_up", d.E * d.F * d.H), C.byref(d), _ptr(h, torch.bfloat16, "h", TK * d.F),
+        _ptr(ws, torch.uint8, "ws"), ws.numel(), _stream(stream)))
+
+
 def moe_grouped_down(h, offsets, w_down, d: moe_dims, y, ws, stream=None):
     TK = d.T * d.K
     _check("moe_grouped_down", lib().moe_grouped_down(
@@ -352,15 +363,16 @@ def moe_dense(a, w, out, ws, stream=None):
 # Whole layer
 # ---------------------------------------------------------------------------
 
-def alloc_layer_buffers(d: moe_dims, device="cuda", meta=True) -> dict:
-    """Device buffers for every output of moe_layer_forward (torch allocations)."""
+def alloc_layer_buffers(d: moe_dims, device="cuda", meta=True, gather=False) -> dict:
+    """Device buffers for every output of moe_layer_forward (torch allocations).  gather=True
+    leaves out xp: the layer's gate/up GEMM then reads the token rows in place."""
     T, TK = d.T, d.T * d.K
     i32, f32, bf = torch.int32, torch.float32, torch.bfloat16
     e = lambda shape, dt: torch.empty(shape, dtype=dt, device=device)  # noqa: E731
     b = dict(z=e((T, d.H), bf) if d.d_model else None, logits=e((T, d.E), f32), topk_ids=e((T, d.K), i32),
              topk_w=e((T, d.K), f32), counts=e((d.E,), i32), offsets=e((d.E + 1,), i32), part_counts=e((d.P,), i32),
              part_offsets=e((d.P + 1,), i32), row_of_assign=e((TK,), i32), assign_of_row=e((TK,), i32),
-             xp=None if d.fp8_dispatch else e((TK, d.H), bf), meta_token=e((TK,), i32) if meta else None,
+             xp=None if d.fp8_dispatch or gather else e((TK, d.H), bf), meta_token=e((TK,), i32) if meta else None,
              meta_slot=e((TK,), i32) if meta else None, meta_w=e((TK,), f32) if meta else None,
              meta_local_expert=e((TK,), i32) if meta else None, h=e((TK, d.F), bf), y=e((TK, d.H), bf),
              out=e((T, d.H), bf), final_out=e((T, d.d_model), bf) if d.d_model else None, skew=e((1,), f32),

@@ -289,6 +289,19 @@ moe_status moe_grouped_gate_up(const void* xp, const int32_t* offsets, const voi
                                   d->F, h, ws_status(ws), ws_sched(ws, kSchedGateUp), as_stream(stream)));
 }
 
+moe_status moe_grouped_gate_up_gather(const void* x, const int32_t* assign_of_row, const int32_t* offsets,
+                                      const void* w_gate, const void* w_up, const moe_dims* d, void* h, void* ws,
+                                      size_t ws_bytes, void* stream) {
+  MOE_TRY(common_checks(d));
+  MOE_TRY(check_ws_header(ws, ws_bytes));
+  if (d->T == 0) return MOE_OK;
+  if (!x || !assign_of_row || !offsets || !w_gate || !w_up || !h) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(w_gate) || !aligned16(w_up) || !aligned16(h)) return MOE_ERR_INVALID_ARG;
+  return cuda_status(gemm_gate_up(x, offsets, w_gate, w_up, d->E, d->T * static_cast<long long>(d->K), d->H, d->F, h,
+                                  ws_status(ws), ws_sched(ws, kSchedGateUp), as_stream(stream), assign_of_row, d->K,
+                                  d->T));
+}
+
 moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w_down, const moe_dims* d, void* y,
                             void* ws, size_t ws_bytes, void* stream) {
   MOE_TRY(common_checks(d));
@@ -368,8 +381,10 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
     return MOE_ERR_INVALID_ARG;
   if (shared && b->aux_stream && (!b->fork_event || !b->join_event)) return MOE_ERR_INVALID_ARG;
   if (!b->logits || !b->topk_ids || !b->topk_w || !b->counts || !b->offsets || !b->part_counts ||
-      !b->part_offsets || !b->row_of_assign || !b->assign_of_row || (!fp8 && !b->xp) || !b->h || !b->y || !b->out)
+      !b->part_offsets || !b->row_of_assign || !b->assign_of_row || !b->h || !b->y || !b->out)
     return MOE_ERR_INVALID_ARG;
+  // bf16 dispatch without an xp buffer: the gate/up GEMM reads each row's token in place
+  const bool gather = !fp8 && !b->xp;
   // every bf16 row buffer is read or written in 16-byte pieces
   for (const void* p : {x, static_cast<const void*>(b->xp), static_cast<const void*>(b->h), static_cast<const void*>(b->y),
                         static_cast<const void*>(b->out), static_cast<const void*>(b->z),
@@ -417,7 +432,8 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
                         b->topk_w, s));
   MOE_TRY(mark(3));
   // count/scan leaves each assignment's rank within its expert in row_of_assign; the permute
-  // turns it into the row (offsets[e] + rank) and writes assign_of_row
+  // turns it into the row (offsets[e] + rank) and writes assign_of_row (and, without a
+  // gather, copies the rows)
   MOE_CUDA(launch_count_scan(b->topk_ids, TK, d->E, d->P, b->row_of_assign, b->counts, b->offsets, b->part_counts,
                              b->part_offsets, b->skew, scan_ws(ws, d), s));
   MOE_TRY(mark(4));
@@ -435,8 +451,8 @@ moe_status moe_layer_forward(const void* x, const moe_layer_weights* w, const mo
       MOE_CUDA(gemm_gate_up_fp8(b->xq, b->xs, b->offsets, w->w_gate_q, w->w_up_q, w->s_gate, w->s_up, d->E, TK, d->H,
                                 d->F, b->h, status, ws_sched(ws, kSchedGateUp), s));
     else
-      MOE_CUDA(gemm_gate_up(b->xp, b->offsets, w->w_gate, w->w_up, d->E, TK, d->H, d->F, b->h, status,
-                            ws_sched(ws, kSchedGateUp), s));
+      MOE_CUDA(gemm_gate_up(gather ? routed : b->xp, b->offsets, w->w_gate, w->w_up, d->E, TK, d->H, d->F, b->h,
+                            status, ws_sched(ws, kSchedGateUp), s, gather ? b->assign_of_row : nullptr, d->K, T));
   }
   MOE_TRY(mark(6));
   if (T > 0)

@@ -71,6 +71,7 @@ __device__ __forceinline__ int assignment_row(int32_t* roa, const int32_t* __res
 // One warp per token: lanes k < K find the rows of the token's K assignments (and write their
 // metadata), then the warp copies the token's row of 16-byte vectors to those K rows, kUnroll
 // loads in flight per lane; consecutive lanes touch consecutive vectors (coalesced both ways).
+// Without xp (the gate/up GEMM gathers the rows itself) only the rows and metadata are made.
 __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
     const uint4* __restrict__ x, int32_t* roa, const int32_t* __restrict__ ids, const float* __restrict__ w,
     long long T, int vpr, int E, int K, int P, uint4* __restrict__ xp, int32_t* __restrict__ meta_token,
@@ -88,7 +89,7 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
     uint4 v[kUnroll];  // the first vectors are on their way while the rows are looked up
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u)
-      if (lane + 32 * u < vpr) v[u] = ld_stream(src + lane + 32 * u);
+      if (xp && lane + 32 * u < vpr) v[u] = ld_stream(src + lane + 32 * u);
     int row = -1;
     if (lane < K) {
       const long long a = t * K + lane;
@@ -100,6 +101,7 @@ __global__ void __launch_bounds__(kCopyThreads) permute_kernel(
         if (meta_local) meta_local[row] = __ldg(ids + a) % epp;
       }
     }
+    if (!xp) continue;
     for (int v0 = lane; v0 < vpr; v0 += 32 * kUnroll) {
       if (v0 != lane) {
 #pragma unroll

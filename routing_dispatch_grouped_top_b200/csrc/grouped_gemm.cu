@@ -223,6 +223,18 @@ __device__ void build_tile_table(int* s_pre, const int* s_off, int G, int NT, in
   __syncthreads();
 }
 
+// Source row of token operand row r when the operand is gathered in place (GemmArgs::gather).
+// An entry that names no source row is reported (bad index) and row 0 is read instead.
+__device__ __forceinline__ int gather_source(const GemmArgs& args, int r) {
+  const int a = __ldg(args.gather + r);
+  const int src = a >= 0 ? a / args.gather_div : -1;
+  if (static_cast<unsigned>(src) >= static_cast<unsigned>(args.gather_rows)) {
+    report(args.status, MOE_DEV_BAD_INDEX);
+    return 0;
+  }
+  return src;
+}
+
 template <int EPI>
 __global__ void __launch_bounds__(kMaxThreads, 1)
     grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
@@ -314,7 +326,11 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
+    // Lane 0 claims tiles, waits on the stages and issues the weight loads; a gathered token
+    // operand (SwiGLU only) is fetched by the whole warp, four rows per lane and gather.
+    const bool gather = EPI == kEpiSwiGLU && args.gather != nullptr;
+    if (lane == 0 || gather) {
+      const unsigned lmask = gather ? 0xffffffffu : 1u;
       uint32_t stage = 0, phase = 0;
       uint32_t pend_phase[STAGES];
       bool pend[STAGES];
@@ -325,13 +341,20 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       for (;;) {
         // Dynamic schedule: the next unclaimed tile of the launch (tiles differ in their token
         // count, so a fixed round-robin leaves some SMs with much more work than others).
-        if (!mbar_wait(&rempty[rs], rphase ^ 1u, abort_flag, args.status)) {
+        int t = 0, got = 1;
+        if (lane == 0) {
+          got = mbar_wait(&rempty[rs], rphase ^ 1u, abort_flag, args.status);
+          if (got) {
+            t = atomicAdd(&args.sched[0], 1);
+            ring_tile[rs] = t < total ? t : -1;
+            mbar_arrive(&rfull[rs]);
+          }
+        }
+        if (!__shfl_sync(lmask, got, 0)) {
           ok = false;
           break;
         }
-        const int t = atomicAdd(&args.sched[0], 1);
-        ring_tile[rs] = t < total ? t : -1;
-        mbar_arrive(&rfull[rs]);
+        t = __shfl_sync(lmask, t, 0);
         if (++rs == kRing) {
           rs = 0;
           rphase ^= 1u;
@@ -340,33 +363,57 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const int tb = t / S, ks = t - tb * S;
         const Tile tl = decode_tile<NT, 16, C::FEAT>(tb, s_pre, s_off, G);
         const uint32_t bytes = NA * kABytes + tl.nround * 128;
+        // gathered rows: lane l fetches tile rows 4 l .. 4 l + 3 and 128 + 4 l .. 128 + 4 l + 3;
+        // rows past the tile's valid ones repeat its first row (computed, never stored)
+        int src[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+        const bool g0 = gather && 4 * lane < tl.nround, g1 = gather && 128 + 4 * lane < tl.nround;
+        if (g0) {
+          const int first = gather_source(args, tl.row0);
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int j = (i < 4 ? 0 : 128) + 4 * lane + (i & 3);
+            src[i] = j < tl.nvalid ? gather_source(args, tl.row0 + j) : first;
+          }
+        }
         for (int kb = ks * KB / S; kb < (ks + 1) * KB / S; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
+          got = 1;
+          if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status);
+          if (!__shfl_sync(lmask, got, 0)) {
             ok = false;
             break;
           }
           uint8_t* st = ring + stage * L::kStageBytes;
-          mbar_arrive_expect_tx(&full[stage], bytes);
           const int kx = kb * KS;
-          if constexpr (EPI == kEpiBF16) {
-            // both 128-row weight tiles in one 256-row box
-            tma_load_3d(st, &tmA0, &full[stage], kx, tl.n0, tl.g);
-          } else {
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            if constexpr (EPI == kEpiBF16) {
+              // both 128-row weight tiles in one 256-row box
+              tma_load_3d(st, &tmA0, &full[stage], kx, tl.n0, tl.g);
+            } else {
 #pragma unroll
-            for (int i = 0; i < NA; ++i) {
-              const CUtensorMap* m = (i == 0) ? &tmA0 : ((i == 1) ? &tmA1 : &tmA2);
-              tma_load_3d(st + i * kABytes, m, &full[stage], kx, tl.n0, (EPI == kEpiF32) ? i : tl.g);
+              for (int i = 0; i < NA; ++i) {
+                const CUtensorMap* m = (i == 0) ? &tmA0 : ((i == 1) ? &tmA1 : &tmA2);
+                tma_load_3d(st + i * kABytes, m, &full[stage], kx, tl.n0, (EPI == kEpiF32) ? i : tl.g);
+              }
+            }
+            if (!gather) {
+              int r = 0;
+#pragma unroll
+              for (int i = 0; i < kNumBoxes; ++i) {
+                const int rows = 256 >> i;
+                if (tl.nround & rows) {
+                  tma_load_2d(st + NA * kABytes + r * 128, &tmB.box[i], &full[stage], kx, tl.row0 + r);
+                  r += rows;
+                }
+              }
             }
           }
-          int r = 0;
-#pragma unroll
-          for (int i = 0; i < kNumBoxes; ++i) {
-            const int rows = 256 >> i;
-            if (tl.nround & rows) {
-              tma_load_2d(st + NA * kABytes + r * 128, &tmB.box[i], &full[stage], kx, tl.row0 + r);
-              r += rows;
-            }
-          }
+          if (g0)
+            tma_gather4(st + NA * kABytes + 4 * lane * 128, &tmB.box[0], &full[stage], kx, src[0], src[1], src[2],
+                        src[3]);
+          if (g1)
+            tma_gather4(st + NA * kABytes + (128 + 4 * lane) * 128, &tmB.box[0], &full[stage], kx, src[4], src[5],
+                        src[6], src[7]);
           pend[stage] = true;
           pend_phase[stage] = phase;
           if (++stage == STAGES) {
@@ -376,7 +423,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         }
         if (!ok) break;
       }
-      if (!ok) {  // let the copies already issued land before the CTA exits
+      if (!ok && lane == 0) {  // let the copies already issued land before the CTA exits
 #pragma unroll
         for (int s = 0; s < STAGES; ++s)
           if (pend[s]) mbar_drain(&full[s], pend_phase[s], 200000000ull);
@@ -658,7 +705,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_map(&tmA0);
     tma_prefetch_map(&tmA1);
-    for (int i = 1; i < kNumBoxes; ++i) tma_prefetch_map(&tmB.box[i]);
+    for (int i = 0; i < kNumBoxes; ++i) tma_prefetch_map(&tmB.box[i]);
   }
   if (warp == 1) {
     tmem_alloc_pair(tmem_slot, L::kTmemCols);
@@ -692,7 +739,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
+    // Lane 0 takes the tile ids, waits on the stages and issues the weight loads; a gathered
+    // token operand (SwiGLU only) is fetched by the whole warp, four of this CTA's rows per lane.
+    const bool gather = EPI == kEpiSwiGLU && args.gather != nullptr;
+    if (lane == 0 || gather) {
+      const unsigned lmask = gather ? 0xffffffffu : 1u;
       const uint32_t rfull_peer = mapa_shared(smem_u32(rfull), 1);
       const uint32_t ring_peer = mapa_shared(smem_u32(const_cast<int*>(ring_tile)), 1);
       uint32_t stage = 0, phase = 0, rs = 0, rphase = 0;
@@ -702,26 +753,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
       for (int s = 0; s < STAGES; ++s) pend[s] = false, pend_phase[s] = 0;
       bool ok = true;
       for (;;) {
-        int t;
-        if (rank == 0) {
-          if (!mbar_wait_cluster(&rempty[rs], rphase ^ 1u, abort_flag, args.status)) {
-            ok = false;
-            break;
+        int t = -1, got = 1;
+        if (lane == 0) {
+          if (rank == 0) {
+            got = mbar_wait_cluster(&rempty[rs], rphase ^ 1u, abort_flag, args.status);
+            if (got) {
+              const int claimed = atomicAdd(&args.sched[0], 1);
+              t = claimed < total ? claimed : -1;
+              ring_tile[rs] = t;
+              st_shared_cluster(ring_peer + 4 * rs, t);
+              mbar_arrive(&rfull[rs]);
+              mbar_arrive_cluster(rfull_peer + 8 * rs);
+            }
+          } else {
+            got = mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status);
+            if (got) {
+              t = ring_tile[rs];
+              mbar_arrive_cluster(rempty_leader + 8 * rs);
+            }
           }
-          const int claimed = atomicAdd(&args.sched[0], 1);
-          t = claimed < total ? claimed : -1;
-          ring_tile[rs] = t;
-          st_shared_cluster(ring_peer + 4 * rs, t);
-          mbar_arrive(&rfull[rs]);
-          mbar_arrive_cluster(rfull_peer + 8 * rs);
-        } else {
-          if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) {
-            ok = false;
-            break;
-          }
-          t = ring_tile[rs];
-          mbar_arrive_cluster(rempty_leader + 8 * rs);
         }
+        if (!__shfl_sync(lmask, got, 0)) {
+          ok = false;
+          break;
+        }
+        t = __shfl_sync(lmask, t, 0);
         if (++rs == kRing) {
           rs = 0;
           rphase ^= 1u;
@@ -730,32 +786,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
         const int half = tl.nround >> 1;  // token rows staged by each CTA (a multiple of 16)
         const int rbase = tl.row0 + static_cast<int>(rank) * half;
+        // gathered rows: lane l fetches this CTA's rows 4 l .. 4 l + 3; rows past the tile's
+        // valid ones repeat its first row (computed, never stored)
+        int src[4] = {0, 0, 0, 0};
+        const bool gl = gather && 4 * lane < half;
+        if (gl) {
+          const int first = gather_source(args, tl.row0);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const int j = static_cast<int>(rank) * half + 4 * lane + i;
+            src[i] = j < tl.nvalid ? gather_source(args, tl.row0 + j) : first;
+          }
+        }
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
+          got = 1;
+          if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status);
+          if (!__shfl_sync(lmask, got, 0)) {
             ok = false;
             break;
           }
           const uint32_t bar = full_leader + stage * 8;
-          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kAPair + half * 128));
           uint8_t* st = ring + stage * L::kStageBytes;
           const int kx = kb * KS;
-          if constexpr (EPI == kEpiBF16) {
-            tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
-            tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
-          } else {
-            const int fr = tl.n0 + 128 * static_cast<int>(rank);
-            tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
-            tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
-          }
-          int r = 0;
+          if (lane == 0) {
+            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kAPair + half * 128));
+            if constexpr (EPI == kEpiBF16) {
+              tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
+              tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
+            } else {
+              const int fr = tl.n0 + 128 * static_cast<int>(rank);
+              tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
+              tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
+            }
+            if (!gather) {
+              int r = 0;
 #pragma unroll
-          for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
-            const int rows = 256 >> i;
-            if (half & rows) {
-              tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
-              r += rows;
+              for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
+                const int rows = 256 >> i;
+                if (half & rows) {
+                  tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
+                  r += rows;
+                }
+              }
             }
           }
+          if (gl)
+            tma_gather4_pair(st + L::kAPair + 4 * lane * 128, &tmB.box[0], bar, kx, src[0], src[1], src[2], src[3]);
           pend[stage] = true;
           pend_phase[stage] = phase;
           if (++stage == STAGES) {
@@ -765,7 +841,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         }
         if (!ok) break;
       }
-      if (!ok) {
+      if (!ok && lane == 0) {
         if (rank == 0) {
 #pragma unroll
           for (int s = 0; s < STAGES; ++s)
@@ -1054,13 +1130,24 @@ static bool use_pair(long long rows, int groups) {
 
 void set_pair_min_rows(int rows) { g_pair_min_rows.store(rows, std::memory_order_relaxed); }
 
-// h = silu(xp Wg^T) * (xp Wu^T) per expert group.
-cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
-                         long long rows, int H, int F, void* h, int* status, int* sched, cudaStream_t stream) {
+// h = silu(xp Wg^T) * (xp Wu^T) per expert group; xp is x itself, or x's rows gathered
+// through `gather` (row r of xp = row gather[r] / K of x) by the GEMM's own loads.
+cudaError_t gemm_gate_up(const void* x, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
+                         long long rows, int H, int F, void* h, int* status, int* sched, cudaStream_t stream,
+                         const int32_t* gather, int K, long long x_rows) {
   GemmArgs args{offsets, E, static_cast<int>(rows), F, H, h, F, nullptr, status, nullptr, nullptr, nullptr, sched};
   CUtensorMap a0, a1;
   BoxMaps b;
-  if (!map_token_boxes(&b, xp, H, rows)) return cudaErrorInvalidValue;
+  if (gather) {
+    if (K < 1 || x_rows < 1 || x_rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+    args.gather = gather;
+    args.gather_div = K;
+    args.gather_rows = static_cast<int>(x_rows);
+    // box 0 fetches one row per coordinate (four per gather); the others stay valid maps
+    if (!map_token_boxes(&b, x, H, x_rows) || !map_bf16_2d(&b.box[0], x, H, x_rows, 1)) return cudaErrorInvalidValue;
+  } else if (!map_token_boxes(&b, x, H, rows)) {
+    return cudaErrorInvalidValue;
+  }
   if (!map_bf16_3d(&a0, w_gate, H, F, E, kBM) || !map_bf16_3d(&a1, w_up, H, F, E, kBM)) return cudaErrorInvalidValue;
   if (use_pair(rows, E))
     return launch_pair<kEpiSwiGLU>(a0, a1, b, args,

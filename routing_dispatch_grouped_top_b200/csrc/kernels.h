@@ -28,6 +28,12 @@ struct GemmArgs {
   int* sched;              // two device ints {next tile, finished CTAs}, zero between launches
   int ksplit;              // kEpiF32: reduction split into this many partial outputs (0 or 1: none)
   long long split_stride;  // elements between the partial outputs of consecutive splits
+  // kEpiSwiGLU only: token operand gathered in place.  Row r of the operand is row
+  // gather[r] / gather_div of the source (gather_rows rows, token box map 0 one row high)
+  // instead of row r of a permuted copy; nullptr: rows are read as they lie.
+  const int32_t* gather;
+  int gather_div;
+  int gather_rows;
 };
 
 int num_sms();             // SM count of the current device (cached per device)
@@ -62,8 +68,11 @@ int gemm_smem_bytes(int epi);
 // Average rows per group from which the grouped GEMMs use the CTA-pair kernel (< 0: never).
 void set_pair_min_rows(int rows);
 
-cudaError_t gemm_gate_up(const void* xp, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
-                         long long rows, int H, int F, void* h, int* status, int* sched, cudaStream_t stream);
+// With `gather` (assign_of_row of the layer's count/scan), the token operand's row r is row
+// gather[r] / K of x ([x_rows][H]), read in place; otherwise x holds the permuted rows.
+cudaError_t gemm_gate_up(const void* x, const int32_t* offsets, const void* w_gate, const void* w_up, int E,
+                         long long rows, int H, int F, void* h, int* status, int* sched, cudaStream_t stream,
+                         const int32_t* gather = nullptr, int K = 1, long long x_rows = 0);
 // h = silu(s_x s_g (xq Wg_q^T)) * (s_x s_u (xq Wu_q^T)) on E4M3 operands.
 cudaError_t gemm_gate_up_fp8(const void* xq, const float* xs, const int32_t* offsets, const void* wq_gate,
                              const void* wq_up, const float* s_gate, const float* s_up, int E, long long rows, int H,

@@ -51,11 +51,11 @@ def cpu(t):
     return t.detach().cpu().numpy()
 
 
-def run_gpu_layer(cfg, inp, aux=False):
+def run_gpu_layer(cfg, inp, aux=False, gather=False):
     d = B.dims_of(cfg)
     w = B.pack_layer_weights(d, inp["w_g"], inp["bias"], inp["w_gate"], inp["w_up"], inp["w_down"], inp["w_dp"],
                              inp["w_upp"], shared=inp["shared"])
-    bufs = B.alloc_layer_buffers(d)
+    bufs = B.alloc_layer_buffers(d, gather=gather)
     if aux:
         B.attach_aux_stream(bufs, torch.cuda.Stream())
     ws = B.make_workspace(d)
@@ -267,6 +267,30 @@ def test_layer_stage_events_are_recorded():
 # Full workloads: sampled tokens + size-independent properties
 # ---------------------------------------------------------------------------
 
+LAYER_KEYS = ("logits", "topk_ids", "topk_w", "counts", "offsets", "part_counts", "part_offsets", "row_of_assign",
+              "assign_of_row", "meta_token", "meta_slot", "meta_w", "meta_local_expert", "h", "y", "out", "z",
+              "final_out", "h_shared", "y_shared", "skew")
+
+
+def assert_same_layer_outputs(a, b):
+    for k in LAYER_KEYS:
+        if a.get(k) is not None:
+            assert torch.equal(a[k].view(torch.uint8), b[k].view(torch.uint8)), k
+
+
+@pytest.mark.parametrize("cfg", [c for c in SMALL if not c.fp8_dispatch], ids=lambda c: c.name)
+def test_layer_gathering_rows_in_place_equals_the_permuted_copy(cfg, gemm_kernel):
+    # without an xp buffer the gate/up GEMM gathers each row's token itself: every output of the
+    # layer must be bit for bit the one of the run with the permuted copy (checked above
+    # against the oracle)
+    inp = inputs.make_layer(cfg, DEV)
+    copy = run_gpu_layer(cfg, inp)
+    gath = run_gpu_layer(cfg, inp, gather=True)
+    torch.cuda.synchronize()
+    assert gath["xp"] is None
+    assert_same_layer_outputs(copy, gath)
+
+
 FULL = [QWEN3_30B_A3B_PREFILL, DEEPSEEK_R1_PREFILL, DEEPSEEK_R1_DECODE, LATENT_896E,
         DEEPSEEK_R1_PREFILL.with_(name=DEEPSEEK_R1_PREFILL.name + "_fp8_dispatch", fp8_dispatch=True)]
 HOST_EXPERT_BUDGET = 2.5e9   # bytes of expert weights copied to the host for the oracle
@@ -278,6 +302,12 @@ def test_full_size_sampled(cfg):
     torch.cuda.empty_cache()
     inp = inputs.make_layer(cfg, DEV)
     g = run_gpu_layer(cfg, inp)
+    if not cfg.fp8_dispatch:
+        # the same layer without the permuted copy (bench.py --gather) must give these outputs
+        gath = run_gpu_layer(cfg, inp, gather=True)
+        torch.cuda.synchronize()
+        assert_same_layer_outputs(g, gath)
+        del gath
     T, K, E, H, F = cfg.T, cfg.K, cfg.E, cfg.H, cfg.F
     latent = bool(cfg.d_model)
     # properties at full size

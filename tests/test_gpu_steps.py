@@ -303,6 +303,66 @@ def test_grouped_ffn_matches_oracle(E, H, F, rows, zipf, zf, gemm_kernel):
     check_bf16("y", bits(y), ry)
 
 
+GATHER_CASES = [  # T, H, E, K, F, zipf
+    (300, 256, 8, 2, 512, None), (130, 200, 4, 2, 200, None), (2000, 2048, 16, 8, 768, 1.1),
+    (1, 64, 3, 1, 136, None), (64, 128, 64, 1, 128, None), (700, 512, 32, 4, 256, 2.0),
+]
+
+
+def gather_inputs(T, H, E, K, F, zipf, seed=0):
+    ids = inputs.random_topk_ids(T, E, K, seed=seed + T, zipf_s=zipf)
+    cs = oracle.count_scan(ids.numpy(), E, 1)
+    x = inputs.random_bf16((T, H), seed=seed + 1)
+    wg = inputs.random_bf16((E, F, H), seed=seed + 2, std=H ** -0.5)
+    wu = inputs.random_bf16((E, F, H), seed=seed + 3, std=H ** -0.5)
+    return cs, x, wg, wu
+
+
+@pytest.mark.parametrize("T,H,E,K,F,zipf", GATHER_CASES)
+def test_grouped_gate_up_gather_equals_the_permuted_copy_bit_for_bit(T, H, E, K, F, zipf, gemm_kernel):
+    # row r of the gathered operand is token assign_of_row[r] // K: the same bytes reach the same
+    # MMAs in the same order as with the permuted copy, so h is identical, not just close
+    cs, x, wg, wu = gather_inputs(T, H, E, K, F, zipf)
+    TK = T * K
+    d = B.dims(T=T, H=H, E=E, K=K, F=F)
+    ws = B.make_workspace(d)
+    aor = torch.from_numpy(cs["assign_of_row"]).to(DEV)
+    off = torch.from_numpy(cs["offsets"]).to(DEV)
+    xp = x[torch.from_numpy(cs["assign_of_row"] // K)]
+    h_copy = torch.full((TK, F), -1.0, dtype=torch.bfloat16, device=DEV)
+    h_gather = torch.full((TK, F), -2.0, dtype=torch.bfloat16, device=DEV)
+    B.moe_grouped_gate_up(xp.to(DEV), off, wg.to(DEV), wu.to(DEV), d, h_copy, ws)
+    B.moe_grouped_gate_up_gather(x.to(DEV), aor, off, wg.to(DEV), wu.to(DEV), d, h_gather, ws)
+    torch.cuda.synchronize()
+    assert B.read_device_status(ws) == 0
+    assert torch.equal(h_gather.view(torch.int16), h_copy.view(torch.int16))
+    rh, _ = oracle.grouped_ffn(bits(xp), cs["offsets"], bits(wg), bits(wu), np.zeros((E, 8, F), np.uint16))
+    check_bf16("h", bits(h_gather), rh)
+
+
+def test_grouped_gate_up_gather_reports_a_row_outside_the_tokens_then_recovers():
+    T, H, E, K, F = 200, 256, 4, 2, 128
+    cs, x, wg, wu = gather_inputs(T, H, E, K, F, None, seed=5)
+    d = B.dims(T=T, H=H, E=E, K=K, F=F)
+    off = torch.from_numpy(cs["offsets"]).to(DEV)
+    xd, wgd, wud = x.to(DEV), wg.to(DEV), wu.to(DEV)
+    h = torch.zeros((T * K, F), dtype=torch.bfloat16, device=DEV)
+    for bad in (T * K + 7, -3):
+        ws = B.make_workspace(d)
+        aor = cs["assign_of_row"].copy()
+        aor[17] = bad                      # names no token: reported, row 0 read instead
+        B.moe_grouped_gate_up_gather(xd, torch.from_numpy(aor).to(DEV), off, wgd, wud, d, h, ws)
+        torch.cuda.synchronize()
+        assert B.read_device_status(ws) & B.DEV_BAD_INDEX
+    ws = B.make_workspace(d)
+    B.moe_grouped_gate_up_gather(xd, torch.from_numpy(cs["assign_of_row"]).to(DEV), off, wgd, wud, d, h, ws)
+    torch.cuda.synchronize()
+    assert B.read_device_status(ws) == 0
+    xp = x[torch.from_numpy(cs["assign_of_row"] // K)]
+    rh, _ = oracle.grouped_ffn(bits(xp), cs["offsets"], bits(wg), bits(wu), np.zeros((E, 8, F), np.uint16))
+    check_bf16("h", bits(h), rh)
+
+
 # ---------------------------------------------------------------------------
 # FP8 dispatch: E4M3 codes with per-row scales, gate/up on E4M3
 # ---------------------------------------------------------------------------
