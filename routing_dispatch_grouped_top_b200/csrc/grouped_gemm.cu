@@ -502,7 +502,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
     // With 8 epilogue warps, two share each lane quadrant and take alternate 32-token chunks.
     constexpr int kSplit = C::EW / 4;
     const int part = (warp - 2) >> 2;
-    uint32_t acc = 0, acc_phase = 0, chunk = 0, rs = 0, rphase = 0;
+    uint32_t acc = 0, acc_phase = 0, rs = 0, rphase = 0;
     for (;;) {
       if (!mbar_wait(&rfull[rs], rphase, abort_flag, args.status)) break;
       const int t = ring_tile[rs];

@@ -257,6 +257,8 @@ constexpr int kScanThreads = 256;
 constexpr int kScanWarps = kScanThreads / 32;
 constexpr int kScanMinChunk = 1024;  // per block: 4 assignments per thread; short look-back chains
 constexpr int kLookWindow = 32;
+constexpr int kLookBatch = 8;  // look-back rows loaded together
+constexpr int kIdBatch = 4;    // ids per lane loaded together
 constexpr int kPerThreadE = MOE_MAX_E / kScanThreads;  // experts a thread scans and looks back for
 constexpr int kFlagAgg = 1, kFlagInc = 2;
 
@@ -346,20 +348,23 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
   for (int j = 0; j < kPerThreadE; ++j) excl[j] = 0;
 
   if (active) {
-    // 1. counts of this warp's slice
-    for (int base = wlo; base < whi; base += 32) {
-      const int a = base + lane;
-      int e = -1;
-      if (a < whi) {
-        e = __ldg(ids + a);
-        if (e < 0 || e >= E) {
-          e = -1;
-          s_bad = 1;
-        }
+    // 1. counts of this warp's slice (kIdBatch ids per lane in flight at once)
+    for (int base = wlo; base < whi; base += 32 * kIdBatch) {
+      int ev[kIdBatch];
+#pragma unroll
+      for (int u = 0; u < kIdBatch; ++u) {
+        const int a = base + 32 * u + lane;
+        ev[u] = a < whi ? __ldg(ids + a) : -1;
       }
-      const unsigned same = __match_any_sync(0xffffffffu, e);
-      if (e >= 0 && lane == __ffs(same) - 1) s_run[warp * E + e] += __popc(same);
-      __syncwarp();
+#pragma unroll
+      for (int u = 0; u < kIdBatch; ++u) {
+        int e = ev[u];
+        if (base + 32 * u + lane < whi && (e < 0 || e >= E)) s_bad = 1;
+        if (e < 0 || e >= E) e = -1;
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        if (e >= 0 && lane == __ffs(same) - 1) s_run[warp * E + e] += __popc(same);
+        __syncwarp();
+      }
     }
     __syncthreads();
     // per expert: counts of the earlier warps of the block, and the block's count, published
@@ -420,10 +425,17 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
       for (int j = 0; j < kPerThreadE; ++j) {
         const int e = tid + j * kScanThreads;
         if (e < E) {
+          // the window's rows in batches of independent loads (one round trip per batch)
           int acc = 0;
-          for (int i = 0; i < n; ++i) {
-            const int* src = (i == ip) ? ws.inc : ws.agg;
-            acc += __ldcg(src + static_cast<long long>(top - i) * E + e);
+          for (int i0 = 0; i0 < n; i0 += kLookBatch) {
+            int v[kLookBatch];
+#pragma unroll
+            for (int u = 0; u < kLookBatch; ++u) {
+              const int i = i0 + u;
+              v[u] = i < n ? __ldcg(((i == ip) ? ws.inc : ws.agg) + static_cast<long long>(top - i) * E + e) : 0;
+            }
+#pragma unroll
+            for (int u = 0; u < kLookBatch; ++u) acc += v[u];
           }
           excl[j] += acc;
         }
@@ -456,18 +468,23 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
       }
     }
     __syncthreads();
-    for (int base = wlo; base < whi; base += 32) {
-      const int a = base + lane;
-      int e = -1;
-      if (a < whi) {
-        e = __ldg(ids + a);
-        if (e < 0 || e >= E) e = -1;
+    for (int base = wlo; base < whi; base += 32 * kIdBatch) {
+      int ev[kIdBatch];
+#pragma unroll
+      for (int u = 0; u < kIdBatch; ++u) {
+        const int a = base + 32 * u + lane;
+        ev[u] = a < whi ? __ldg(ids + a) : -1;
       }
-      const unsigned same = __match_any_sync(0xffffffffu, e);
-      if (a < whi) rank_out[a] = e < 0 ? -1 : s_run[warp * E + e] + __popc(same & lt_mask);  // -1: no row
-      __syncwarp();
-      if (e >= 0 && lane == __ffs(same) - 1) s_run[warp * E + e] += __popc(same);
-      __syncwarp();
+#pragma unroll
+      for (int u = 0; u < kIdBatch; ++u) {
+        const int a = base + 32 * u + lane;
+        const int e = (ev[u] < 0 || ev[u] >= E) ? -1 : ev[u];
+        const unsigned same = __match_any_sync(0xffffffffu, e);
+        if (a < whi) rank_out[a] = e < 0 ? -1 : s_run[warp * E + e] + __popc(same & lt_mask);  // -1: no row
+        __syncwarp();
+        if (e >= 0 && lane == __ffs(same) - 1) s_run[warp * E + e] += __popc(same);
+        __syncwarp();
+      }
     }
   }
 
