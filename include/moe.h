@@ -264,10 +264,13 @@ moe_status moe_grouped_down(const void* h, const int32_t* offsets, const void* w
                             const moe_dims* d, void* y, void* ws, size_t ws_bytes, void* stream);
 
 /* moe_grouped_gate_up without the permuted copy: row r of the operand is row
- * assign_of_row[r] / K of x ([T][H] bf16, the unpermuted activations), fetched by the
- * GEMM's own TMA row gathers, so h equals moe_grouped_gate_up(xp, ...) bit for bit for
+ * assign_of_row[r] / K of x ([T][H] bf16, the unpermuted activations), copied into the
+ * GEMM's shared-memory stages by its own gather warps (16-byte cp.async, CTA-pair kernel
+ * at every row count), so h equals moe_grouped_gate_up(xp, ...) bit for bit for
  * xp = moe_permute(x).  assign_of_row [TK] from moe_count_scan.  An entry outside
- * [0, T*K) is reported as MOE_ERR_DEVICE_BAD_INDEX (row 0 of x is read in its place). */
+ * [0, T*K) is reported as MOE_ERR_DEVICE_BAD_INDEX (row 0 of x is read in its place).
+ * Saves the T*K*H*2-byte xp buffer and its write and read; on B200 the row-by-row
+ * operand fetch makes the GEMM slower than reading xp (about 1.5x at prefill sizes). */
 moe_status moe_grouped_gate_up_gather(const void* x, const int32_t* assign_of_row, const int32_t* offsets,
                                       const void* w_gate, const void* w_up, const moe_dims* d, void* h,
                                       void* ws, size_t ws_bytes, void* stream);
@@ -418,9 +421,9 @@ typedef struct moe_layer_buffers {
  * moe_permute_fp8 (into b->xq, b->xs; b->xp may be NULL) and gate/up runs on
  * w->w_gate_q / w->w_up_q with their scales.  With bf16 dispatch and b->xp NULL no
  * permuted copy is made: the permute step only writes the rows (row_of_assign,
- * assign_of_row) and the metadata, and the gate/up GEMM loads each row's token
- * straight from the routed activations (row r is token assign_of_row[r] / K, four
- * rows per TMA gather); h, y and out are bit-identical to the run with xp.  With d->F_shared > 0 the shared
+ * assign_of_row) and the metadata, and the gate/up GEMM copies each row's token
+ * straight from the routed activations (row r is token assign_of_row[r] / K, as in
+ * moe_grouped_gate_up_gather); h, y and out are bit-identical to the run with xp.  With d->F_shared > 0 the shared
  * expert (gate/up+SwiGLU and down over all T tokens of the routed activations) runs
  * on b->aux_stream, forked after the routed activations are ready and joined before
  * the combine, or on `stream` when aux_stream is NULL.  x: [T][d_in] bf16 with

@@ -26,7 +26,10 @@
 //   warps 2..   epilogue: tcgen05.ld of the fp32 accumulator (warp w reads the TMEM
 //               lane quadrant w % 4; with eight warps two share a quadrant and take
 //               alternate 32-token chunks), activation, and bf16 rows written through a
-//               per-warp shared-memory transpose as 16-byte pieces.
+//               per-warp shared-memory transpose as 16-byte pieces;
+//   (pair, SwiGLU) four gather warps, one per stage, that copy the token rows with 16-byte
+//               cp.async through the rows' source indices when the operand is gathered in
+//               place instead of read from a permuted copy.
 // Tiles are numbered group-major, then weight tile, then token chunk, and claimed in
 // that order: CTAs working at the same time share weight and token tiles through L2,
 // so each expert's weights cross HBM about once, and SMs that draw short tiles take
@@ -52,6 +55,7 @@ struct BoxMaps {
   CUtensorMap box[kNumBoxes];  // box[i] is (256 >> i) rows x 64 columns
 };
 constexpr int kMaxThreads = 320;         // single-CTA kernel with 8 epilogue warps
+constexpr int kMaxPairThreads = 448;     // CTA-pair kernel with 8 epilogue and 4 gather warps
 constexpr int kMaxGroups = MOE_MAX_E;
 constexpr int kRing = 8;                 // tile ids in flight from the producer to the MMA and epilogue warps
 
@@ -326,11 +330,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    // Lane 0 claims tiles, waits on the stages and issues the weight loads; a gathered token
-    // operand (SwiGLU only) is fetched by the whole warp, four rows per lane and gather.
-    const bool gather = EPI == kEpiSwiGLU && args.gather != nullptr;
-    if (lane == 0 || gather) {
-      const unsigned lmask = gather ? 0xffffffffu : 1u;
+    if (lane == 0) {
       uint32_t stage = 0, phase = 0;
       uint32_t pend_phase[STAGES];
       bool pend[STAGES];
@@ -341,20 +341,13 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
       for (;;) {
         // Dynamic schedule: the next unclaimed tile of the launch (tiles differ in their token
         // count, so a fixed round-robin leaves some SMs with much more work than others).
-        int t = 0, got = 1;
-        if (lane == 0) {
-          got = mbar_wait(&rempty[rs], rphase ^ 1u, abort_flag, args.status);
-          if (got) {
-            t = atomicAdd(&args.sched[0], 1);
-            ring_tile[rs] = t < total ? t : -1;
-            mbar_arrive(&rfull[rs]);
-          }
-        }
-        if (!__shfl_sync(lmask, got, 0)) {
+        if (!mbar_wait(&rempty[rs], rphase ^ 1u, abort_flag, args.status)) {
           ok = false;
           break;
         }
-        t = __shfl_sync(lmask, t, 0);
+        const int t = atomicAdd(&args.sched[0], 1);
+        ring_tile[rs] = t < total ? t : -1;
+        mbar_arrive(&rfull[rs]);
         if (++rs == kRing) {
           rs = 0;
           rphase ^= 1u;
@@ -363,57 +356,33 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         const int tb = t / S, ks = t - tb * S;
         const Tile tl = decode_tile<NT, 16, C::FEAT>(tb, s_pre, s_off, G);
         const uint32_t bytes = NA * kABytes + tl.nround * 128;
-        // gathered rows: lane l fetches tile rows 4 l .. 4 l + 3 and 128 + 4 l .. 128 + 4 l + 3;
-        // rows past the tile's valid ones repeat its first row (computed, never stored)
-        int src[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-        const bool g0 = gather && 4 * lane < tl.nround, g1 = gather && 128 + 4 * lane < tl.nround;
-        if (g0) {
-          const int first = gather_source(args, tl.row0);
-#pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            const int j = (i < 4 ? 0 : 128) + 4 * lane + (i & 3);
-            src[i] = j < tl.nvalid ? gather_source(args, tl.row0 + j) : first;
-          }
-        }
         for (int kb = ks * KB / S; kb < (ks + 1) * KB / S; ++kb) {
-          got = 1;
-          if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status);
-          if (!__shfl_sync(lmask, got, 0)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
           }
           uint8_t* st = ring + stage * L::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], bytes);
           const int kx = kb * KS;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(&full[stage], bytes);
-            if constexpr (EPI == kEpiBF16) {
-              // both 128-row weight tiles in one 256-row box
-              tma_load_3d(st, &tmA0, &full[stage], kx, tl.n0, tl.g);
-            } else {
+          if constexpr (EPI == kEpiBF16) {
+            // both 128-row weight tiles in one 256-row box
+            tma_load_3d(st, &tmA0, &full[stage], kx, tl.n0, tl.g);
+          } else {
 #pragma unroll
-              for (int i = 0; i < NA; ++i) {
-                const CUtensorMap* m = (i == 0) ? &tmA0 : ((i == 1) ? &tmA1 : &tmA2);
-                tma_load_3d(st + i * kABytes, m, &full[stage], kx, tl.n0, (EPI == kEpiF32) ? i : tl.g);
-              }
-            }
-            if (!gather) {
-              int r = 0;
-#pragma unroll
-              for (int i = 0; i < kNumBoxes; ++i) {
-                const int rows = 256 >> i;
-                if (tl.nround & rows) {
-                  tma_load_2d(st + NA * kABytes + r * 128, &tmB.box[i], &full[stage], kx, tl.row0 + r);
-                  r += rows;
-                }
-              }
+            for (int i = 0; i < NA; ++i) {
+              const CUtensorMap* m = (i == 0) ? &tmA0 : ((i == 1) ? &tmA1 : &tmA2);
+              tma_load_3d(st + i * kABytes, m, &full[stage], kx, tl.n0, (EPI == kEpiF32) ? i : tl.g);
             }
           }
-          if (g0)
-            tma_gather4(st + NA * kABytes + 4 * lane * 128, &tmB.box[0], &full[stage], kx, src[0], src[1], src[2],
-                        src[3]);
-          if (g1)
-            tma_gather4(st + NA * kABytes + (128 + 4 * lane) * 128, &tmB.box[0], &full[stage], kx, src[4], src[5],
-                        src[6], src[7]);
+          int r = 0;
+#pragma unroll
+          for (int i = 0; i < kNumBoxes; ++i) {
+            const int rows = 256 >> i;
+            if (tl.nround & rows) {
+              tma_load_2d(st + NA * kABytes + r * 128, &tmB.box[i], &full[stage], kx, tl.row0 + r);
+              r += rows;
+            }
+          }
           pend[stage] = true;
           pend_phase[stage] = phase;
           if (++stage == STAGES) {
@@ -423,7 +392,7 @@ __global__ void __launch_bounds__(kMaxThreads, 1)
         }
         if (!ok) break;
       }
-      if (!ok && lane == 0) {  // let the copies already issued land before the CTA exits
+      if (!ok) {  // let the copies already issued land before the CTA exits
 #pragma unroll
         for (int s = 0; s < STAGES; ++s)
           if (pend[s]) mbar_drain(&full[s], pend_phase[s], 200000000ull);
@@ -632,7 +601,9 @@ struct PairLayout {
   static constexpr int NA = 2;                                  // weight operands (accumulators)
   static constexpr int STAGES = 4;
   static constexpr int EW = 8;                                  // epilogue warps per CTA
-  static constexpr int kThr = 64 + 32 * EW;
+  // bf16 SwiGLU: one warp per stage that fills the stage's token rows when they are gathered
+  static constexpr int GW = EPI == kEpiSwiGLU ? STAGES : 0;
+  static constexpr int kThr = 64 + 32 * (EW + GW);
   static constexpr int FEAT = (EPI == kEpiBF16) ? 512 : 256;   // output features per pair tile
   static constexpr int kAPair = NA * kABytes;                   // this CTA's 128-row weight boxes (one atom)
   static constexpr int kBBytes = (NT / 2) * 128;                // this CTA's token rows (one atom)
@@ -643,13 +614,15 @@ struct PairLayout {
   static constexpr int kStgBytes = EW * 32 * 32 * 2;
   static constexpr int kBarBytes = (8 * (2 * STAGES + 5 + 2 * kRing) + 8 + 4 * kRing + 15) / 16 * 16;
   static constexpr int kTableBytes = 2 * (kMaxGroups + 1) * 4;
-  static constexpr int kSmemBytes = 1024 + STAGES * kStageBytes + kStgBytes + kBarBytes + kTableBytes;
+  static constexpr int kSrcBytes = GW * (NT / 2) * 4;          // each gather warp's source rows of a tile
+  static constexpr int kSmemBytes =
+      1024 + STAGES * kStageBytes + kStgBytes + kBarBytes + kTableBytes + kSrcBytes;
   static_assert(kSmemBytes <= 232448, "shared memory budget");
-  static_assert(kThr <= kMaxThreads, "block size");
+  static_assert(kThr <= kMaxPairThreads, "block size");
 };
 
 template <int EPI>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<EPI>::kThr, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
                      const __grid_constant__ BoxMaps tmB, const GemmArgs args) {
   using L = PairLayout<EPI>;
@@ -674,11 +647,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
   volatile int* ring_tile = reinterpret_cast<volatile int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(smem + STAGES * L::kStageBytes + L::kStgBytes + L::kBarBytes);
   int* s_pre = s_off + (kMaxGroups + 1);
-  __shared__ int s_warp_sums[kMaxThreads / 32];
+  int* s_src = s_pre + (kMaxGroups + 1);
+  __shared__ int s_warp_sums[kMaxPairThreads / 32];
   __shared__ int s_bad;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
+  // Gathered token rows (bf16 SwiGLU): the gather warps copy each stage's token rows with
+  // 16-byte cp.async through assign_of_row instead of the producer's token boxes; a stage is
+  // then full after the producer's weight bytes and one gather warp of each CTA.
+  const bool gather = L::GW > 0 && args.gather != nullptr;
   const int G = args.offsets ? args.G : 1;
   const int NFT = (args.N + L::FEAT - 1) / L::FEAT;
   const int KB = (args.Kd + KS - 1) / KS;  // K-steps (a K atom beyond Kd reads the zero fill)
@@ -687,7 +665,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
   if (threadIdx.x == 0) {
     s_bad = 0;
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&full[s], 1);
+      mbar_init(&full[s], gather ? 3 : 1);
       mbar_init(&empty[s], 1);
     }
     for (int a = 0; a < 2; ++a) {
@@ -697,7 +675,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
     mbar_init(drain, 1);
     for (int r = 0; r < kRing; ++r) {
       mbar_init(&rfull[r], 1);
-      mbar_init(&rempty[r], 2 + 2 * EW);  // leader MMA + leader epilogue, peer producer + peer epilogue
+      // leader MMA + leader epilogue, peer producer + peer epilogue (+ both CTAs' gather warps)
+      mbar_init(&rempty[r], 2 + 2 * EW + (gather ? 2 * L::GW : 0));
     }
     *abort_flag = 0;
     mbar_init_fence();
@@ -739,11 +718,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
-    // Lane 0 takes the tile ids, waits on the stages and issues the weight loads; a gathered
-    // token operand (SwiGLU only) is fetched by the whole warp, four of this CTA's rows per lane.
-    const bool gather = EPI == kEpiSwiGLU && args.gather != nullptr;
-    if (lane == 0 || gather) {
-      const unsigned lmask = gather ? 0xffffffffu : 1u;
+    if (lane == 0) {
       const uint32_t rfull_peer = mapa_shared(smem_u32(rfull), 1);
       const uint32_t ring_peer = mapa_shared(smem_u32(const_cast<int*>(ring_tile)), 1);
       uint32_t stage = 0, phase = 0, rs = 0, rphase = 0;
@@ -753,31 +728,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
       for (int s = 0; s < STAGES; ++s) pend[s] = false, pend_phase[s] = 0;
       bool ok = true;
       for (;;) {
-        int t = -1, got = 1;
-        if (lane == 0) {
-          if (rank == 0) {
-            got = mbar_wait_cluster(&rempty[rs], rphase ^ 1u, abort_flag, args.status);
-            if (got) {
-              const int claimed = atomicAdd(&args.sched[0], 1);
-              t = claimed < total ? claimed : -1;
-              ring_tile[rs] = t;
-              st_shared_cluster(ring_peer + 4 * rs, t);
-              mbar_arrive(&rfull[rs]);
-              mbar_arrive_cluster(rfull_peer + 8 * rs);
-            }
-          } else {
-            got = mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status);
-            if (got) {
-              t = ring_tile[rs];
-              mbar_arrive_cluster(rempty_leader + 8 * rs);
-            }
+        int t;
+        if (rank == 0) {
+          if (!mbar_wait_cluster(&rempty[rs], rphase ^ 1u, abort_flag, args.status)) {
+            ok = false;
+            break;
           }
+          const int claimed = atomicAdd(&args.sched[0], 1);
+          t = claimed < total ? claimed : -1;
+          ring_tile[rs] = t;
+          st_shared_cluster(ring_peer + 4 * rs, t);
+          mbar_arrive(&rfull[rs]);
+          mbar_arrive_cluster(rfull_peer + 8 * rs);
+        } else {
+          if (!mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status)) {
+            ok = false;
+            break;
+          }
+          t = ring_tile[rs];
+          mbar_arrive_cluster(rempty_leader + 8 * rs);
         }
-        if (!__shfl_sync(lmask, got, 0)) {
-          ok = false;
-          break;
-        }
-        t = __shfl_sync(lmask, t, 0);
         if (++rs == kRing) {
           rs = 0;
           rphase ^= 1u;
@@ -786,52 +756,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
         const int half = tl.nround >> 1;  // token rows staged by each CTA (a multiple of 16)
         const int rbase = tl.row0 + static_cast<int>(rank) * half;
-        // gathered rows: lane l fetches this CTA's rows 4 l .. 4 l + 3; rows past the tile's
-        // valid ones repeat its first row (computed, never stored)
-        int src[4] = {0, 0, 0, 0};
-        const bool gl = gather && 4 * lane < half;
-        if (gl) {
-          const int first = gather_source(args, tl.row0);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const int j = static_cast<int>(rank) * half + 4 * lane + i;
-            src[i] = j < tl.nvalid ? gather_source(args, tl.row0 + j) : first;
-          }
-        }
         for (int kb = 0; kb < KB; ++kb) {
-          got = 1;
-          if (lane == 0) got = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status);
-          if (!__shfl_sync(lmask, got, 0)) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
             ok = false;
             break;
           }
           const uint32_t bar = full_leader + stage * 8;
+          if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kAPair + (gather ? 0 : half * 128)));
           uint8_t* st = ring + stage * L::kStageBytes;
           const int kx = kb * KS;
-          if (lane == 0) {
-            if (rank == 0) mbar_arrive_expect_tx(&full[stage], 2u * (L::kAPair + half * 128));
-            if constexpr (EPI == kEpiBF16) {
-              tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
-              tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
-            } else {
-              const int fr = tl.n0 + 128 * static_cast<int>(rank);
-              tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
-              tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
-            }
-            if (!gather) {
-              int r = 0;
+          if constexpr (EPI == kEpiBF16) {
+            tma_load_3d_pair(st, &tmA0, bar, kx, tl.n0 + 128 * static_cast<int>(rank), tl.g);
+            tma_load_3d_pair(st + kABytes, &tmA0, bar, kx, tl.n0 + 256 + 128 * static_cast<int>(rank), tl.g);
+          } else {
+            const int fr = tl.n0 + 128 * static_cast<int>(rank);
+            tma_load_3d_pair(st, &tmA0, bar, kx, fr, tl.g);            // gate rows
+            tma_load_3d_pair(st + kABytes, &tmA1, bar, kx, fr, tl.g);  // up rows
+          }
+          if (!gather) {
+            int r = 0;
 #pragma unroll
-              for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
-                const int rows = 256 >> i;
-                if (half & rows) {
-                  tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
-                  r += rows;
-                }
+            for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
+              const int rows = 256 >> i;
+              if (half & rows) {
+                tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
+                r += rows;
               }
             }
           }
-          if (gl)
-            tma_gather4_pair(st + L::kAPair + 4 * lane * 128, &tmB.box[0], bar, kx, src[0], src[1], src[2], src[3]);
           pend[stage] = true;
           pend_phase[stage] = phase;
           if (++stage == STAGES) {
@@ -841,7 +793,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         }
         if (!ok) break;
       }
-      if (!ok && lane == 0) {
+      if (!ok) {
         if (rank == 0) {
 #pragma unroll
           for (int s = 0; s < STAGES; ++s)
@@ -882,7 +834,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         const uint32_t idesc =
             (EPI == kEpiSwiGLUFp8) ? idesc_e4m3_f32(256, tl.nround) : idesc_bf16_f32(256, tl.nround);
         for (int kb = 0; kb < KB; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, args.status)) {
+          // gathered rows: the peer's gather warp wrote its rows with plain stores and arrived
+          // with cluster-scope release, so this wait acquires at cluster scope
+          if (!(gather ? mbar_wait_cluster(&full[stage], phase, abort_flag, args.status)
+                       : mbar_wait(&full[stage], phase, abort_flag, args.status))) {
             ok = false;
             break;
           }
@@ -920,7 +875,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         mbar_drain(drain, 0, 200000000ull);
       }
     }
-  } else {
+  } else if (warp < 2 + EW) {
     // ------------------------------------------------------------ epilogue (both CTAs)
     const int q = warp & 3;               // TMEM lanes [32q, 32q + 32)
     const int part = (warp - 2) >> 2;     // two warps per lane quadrant take alternate chunks
@@ -994,6 +949,85 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kMaxThreads, 1)
         acc = 0;
         acc_phase ^= 1u;
       }
+    }
+  } else if (gather) {
+    // ------------------------------------------------------------ token-row gather (both CTAs)
+    // Warp gw fills the token rows of stage gw, i.e. K-steps gw, gw + STAGES, ... of the CTA's
+    // sequence (the producer's stage counter).  Per tile it looks up the source row of each of
+    // this CTA's rows once; per K-step each lane copies one 16-byte piece of four rows' 128-byte
+    // K slices into the 128-byte-swizzled layout the producer's token boxes would have written
+    // (piece c of row r at r * 128 + (c ^ (r % 8)) * 16), waits for its copies, fences them
+    // against the tensor core's async-proxy reads and the warp arrives on the leader's barrier.
+    const int gw = warp - 2 - EW;
+    int* srow = s_src + gw * (NT / 2);
+    const __nv_bfloat16* xsrc = reinterpret_cast<const __nv_bfloat16*>(args.gather_x);
+    const uint32_t full_arrive = rank == 0 ? smem_u32(&full[gw]) : full_leader + gw * 8;
+    const int c = lane & 7;  // this lane's 16-byte piece of a row's K slice
+    constexpr int kGatherRows = NT / 2 / 4;  // rows per lane: four rows per warp-wide copy
+    constexpr int kGatherBatch = 8;
+    uint32_t rs = 0, rphase = 0, kstep = 0;
+    for (;;) {
+      int t = 0, got = 1;
+      if (lane == 0) {
+        got = mbar_wait_cluster(&rfull[rs], rphase, abort_flag, args.status);
+        if (got) {
+          t = ring_tile[rs];
+          if (rank == 0) mbar_arrive(&rempty[rs]);
+          else mbar_arrive_cluster(rempty_leader + 8 * rs);
+        }
+      }
+      if (!__shfl_sync(0xffffffffu, got, 0)) break;
+      t = __shfl_sync(0xffffffffu, t, 0);
+      if (++rs == kRing) {
+        rs = 0;
+        rphase ^= 1u;
+      }
+      if (t < 0) break;
+      const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
+      const int half = tl.nround >> 1;
+      // this CTA's rows are tile rows rank * half + i; rows past the valid ones repeat row 0
+      // (computed, never stored)
+      for (int i = lane; i < half; i += 32) {
+        const int j = static_cast<int>(rank) * half + i;
+        srow[i] = gather_source(args, tl.row0 + (j < tl.nvalid ? j : 0));
+      }
+      __syncwarp();
+      bool ok = true;
+      for (int kb = 0; kb < KB; ++kb, ++kstep) {
+        if (static_cast<int>(kstep % STAGES) != gw) continue;
+        got = 1;
+        if (lane == 0) got = mbar_wait(&empty[gw], ((kstep / STAGES) & 1u) ^ 1u, abort_flag, args.status);
+        if (!__shfl_sync(0xffffffffu, got, 0)) {
+          ok = false;
+          break;
+        }
+        const uint32_t dst = smem_u32(ring + gw * L::kStageBytes + L::kAPair);
+        const int k0 = kb * KS + 8 * c;  // first K element of this lane's piece
+        const uint32_t nbytes = k0 < args.Kd ? 16u : 0u;  // past the reduction: zero fill
+        const __nv_bfloat16* xk = xsrc + (nbytes ? k0 : 0);
+        // this lane's rows lane / 8 + 4 i: their source rows read in batches, then the copies
+#pragma unroll
+        for (int i0 = 0; i0 < kGatherRows; i0 += kGatherBatch) {
+          int sr[kGatherBatch];
+#pragma unroll
+          for (int u = 0; u < kGatherBatch; ++u) sr[u] = srow[min((lane >> 3) + 4 * (i0 + u), half - 1)];
+#pragma unroll
+          for (int u = 0; u < kGatherBatch; ++u) {
+            const int r = (lane >> 3) + 4 * (i0 + u);
+            if (r < half)
+              cp_async_16(dst + r * 128 + ((c ^ (r & 7)) << 4), xk + static_cast<long long>(sr[u]) * args.Kd, nbytes);
+          }
+        }
+        cp_async_wait_all();
+        fence_proxy_async_shared();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(&full[gw]);
+          else mbar_arrive_cluster(full_arrive);
+        }
+      }
+      if (!ok) break;
+      __syncwarp();  // srow is rewritten for the next tile
     }
   }
 
@@ -1139,17 +1173,18 @@ cudaError_t gemm_gate_up(const void* x, const int32_t* offsets, const void* w_ga
   CUtensorMap a0, a1;
   BoxMaps b;
   if (gather) {
+    // gathered rows: the CTA-pair kernel's gather warps copy them, whatever the row count
     if (K < 1 || x_rows < 1 || x_rows > 0x7fffffffLL) return cudaErrorInvalidValue;
+    if (!MOE_GEMM_PAIR || num_sms() < 2) return cudaErrorNotSupported;
     args.gather = gather;
     args.gather_div = K;
     args.gather_rows = static_cast<int>(x_rows);
-    // box 0 fetches one row per coordinate (four per gather); the others stay valid maps
-    if (!map_token_boxes(&b, x, H, x_rows) || !map_bf16_2d(&b.box[0], x, H, x_rows, 1)) return cudaErrorInvalidValue;
-  } else if (!map_token_boxes(&b, x, H, rows)) {
-    return cudaErrorInvalidValue;
+    args.gather_x = x;
   }
+  // the token maps are not read when the rows are gathered, but stay valid maps
+  if (!map_token_boxes(&b, x, H, gather ? x_rows : rows)) return cudaErrorInvalidValue;
   if (!map_bf16_3d(&a0, w_gate, H, F, E, kBM) || !map_bf16_3d(&a1, w_up, H, F, E, kBM)) return cudaErrorInvalidValue;
-  if (use_pair(rows, E))
+  if (gather || use_pair(rows, E))
     return launch_pair<kEpiSwiGLU>(a0, a1, b, args,
                                    tile_bound(rows, E, PairLayout<kEpiSwiGLU>::NT, F, PairLayout<kEpiSwiGLU>::FEAT),
                                    stream);

@@ -28,12 +28,13 @@ struct GemmArgs {
   int* sched;              // two device ints {next tile, finished CTAs}, zero between launches
   int ksplit;              // kEpiF32: reduction split into this many partial outputs (0 or 1: none)
   long long split_stride;  // elements between the partial outputs of consecutive splits
-  // kEpiSwiGLU only: token operand gathered in place.  Row r of the operand is row
-  // gather[r] / gather_div of the source (gather_rows rows, token box map 0 one row high)
-  // instead of row r of a permuted copy; nullptr: rows are read as they lie.
+  // CTA-pair kEpiSwiGLU only: token operand gathered in place.  Row r of the operand is row
+  // gather[r] / gather_div of gather_x ([gather_rows][Kd] bf16) instead of row r of a permuted
+  // copy; nullptr: rows are read as they lie.
   const int32_t* gather;
   int gather_div;
   int gather_rows;
+  const void* gather_x;
 };
 
 int num_sms();             // SM count of the current device (cached per device)
