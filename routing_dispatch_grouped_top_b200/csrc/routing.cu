@@ -347,6 +347,11 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
 #pragma unroll
   for (int j = 0; j < kPerThreadE; ++j) excl[j] = 0;
 
+  // a warp slice of at most 32 * kIdBatch ids is loaded once and kept for the ranking pass
+  const bool keep = whi - wlo <= 32 * kIdBatch;
+  int kept[kIdBatch];
+#pragma unroll
+  for (int u = 0; u < kIdBatch; ++u) kept[u] = -1;
   if (active) {
     // 1. counts of this warp's slice (kIdBatch ids per lane in flight at once)
     for (int base = wlo; base < whi; base += 32 * kIdBatch) {
@@ -355,6 +360,7 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
       for (int u = 0; u < kIdBatch; ++u) {
         const int a = base + 32 * u + lane;
         ev[u] = a < whi ? __ldg(ids + a) : -1;
+        kept[u] = ev[u];
       }
 #pragma unroll
       for (int u = 0; u < kIdBatch; ++u) {
@@ -473,7 +479,7 @@ __global__ void __launch_bounds__(kScanThreads) count_scan_kernel(
 #pragma unroll
       for (int u = 0; u < kIdBatch; ++u) {
         const int a = base + 32 * u + lane;
-        ev[u] = a < whi ? __ldg(ids + a) : -1;
+        ev[u] = keep ? kept[u] : (a < whi ? __ldg(ids + a) : -1);
       }
 #pragma unroll
       for (int u = 0; u < kIdBatch; ++u) {
