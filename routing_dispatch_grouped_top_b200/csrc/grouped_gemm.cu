@@ -167,6 +167,32 @@ __device__ __forceinline__ void store_rows32(__nv_bfloat16* stg, int lane, const
   __syncwarp();
 }
 
+// store_rows32 through a TMA tile store: the 32 x 32 chunk (tokens x features) is staged as 32
+// rows of 64 bytes and one lane stores it as one box of `map` (the output, box 32 x 32, no
+// swizzle), which completes in the background: the warp goes on (and hands TMEM back) while the
+// rows drain.  A chunk with fewer than 32 valid rows takes store_rows32's 16-byte stores, since
+// the box would also write the first rows of the next group.  The staging tile is reused only
+// after the previous chunk's store has read it.
+__device__ __forceinline__ void store_rows32_tma(__nv_bfloat16* stg, int lane, const float (&v)[32],
+                                                 const CUtensorMap* map, __nv_bfloat16* out, long long ldo, int N,
+                                                 int fbase, long long row0, int jn) {
+  if (lane == 0) bulk_wait_read_all();
+  __syncwarp();
+  if (jn < 32) {
+    store_rows32(stg, lane, v, out, ldo, N, fbase, row0, jn);
+    return;
+  }
+  if (fbase >= N) return;
+#pragma unroll
+  for (int j = 0; j < 32; ++j) stg[j * 32 + lane] = __float2bfloat16_rn(v[j]);
+  fence_proxy_async_shared();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(map, stg, fbase, static_cast<int>(row0));
+    bulk_commit_group();
+  }
+}
+
 // Tile t -> (group, weight tile, token chunk).  s_pre[g] = first tile of group g.  A group of
 // cnt rows is cut into ceil(cnt / NT) balanced chunks of a multiple of ROUND rows; a weight
 // tile covers FEAT output features.
@@ -624,7 +650,8 @@ struct PairLayout {
 template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<EPI>::kThr, 1)
     pair_gemm_kernel(const __grid_constant__ CUtensorMap tmA0, const __grid_constant__ CUtensorMap tmA1,
-                     const __grid_constant__ BoxMaps tmB, const GemmArgs args) {
+                     const __grid_constant__ BoxMaps tmB, const __grid_constant__ CUtensorMap tmO,
+                     const GemmArgs args) {
   using L = PairLayout<EPI>;
   constexpr int NT = L::NT, NA = L::NA, STAGES = L::STAGES, EW = L::EW;
   constexpr int KS = stage_k<EPI>();
@@ -921,10 +948,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<EPI>::kTh
         if constexpr (EPI == kEpiBF16) {
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r0[j]);
-          store_rows32(stg, lane, v, outb, args.ldo, args.N, fa, row0, jn);
+          store_rows32_tma(stg, lane, v, &tmO, outb, args.ldo, args.N, fa, row0, jn);
 #pragma unroll
           for (int j = 0; j < 32; ++j) v[j] = __uint_as_float(r1[j]);
-          store_rows32(stg, lane, v, outb, args.ldo, args.N, fa + 256, row0, jn);
+          store_rows32_tma(stg, lane, v, &tmO, outb, args.ldo, args.N, fa + 256, row0, jn);
         } else {
 #pragma unroll
           for (int j = 0; j < 32; ++j) {
@@ -949,6 +976,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<EPI>::kTh
         acc = 0;
         acc_phase ^= 1u;
       }
+    }
+    if constexpr (EPI == kEpiBF16) {
+      if (lane == 0) bulk_wait_all();  // the tile stores are complete before the CTA exits
     }
   } else if (gather) {
     // ------------------------------------------------------------ token-row gather (both CTAs)
@@ -1116,6 +1146,19 @@ cudaError_t launch(const CUtensorMap& a0, const CUtensorMap& a1, const CUtensorM
   return launch_pdl(grouped_gemm_kernel<EPI>, dim3(grid), dim3(L::kThr), L::kSmemBytes, stream, a0, a1, a2, b, args);
 }
 
+// Output map of the pair kernel's tile stores: out [M][N] bf16 (row stride ldo), box 32 x 32.
+bool map_out_tiles(CUtensorMap* m, const GemmArgs& args) {
+  EncodeTiledFn enc = encoder();
+  if (!enc || args.N <= 0 || args.M <= 0) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(args.N), static_cast<cuuint64_t>(args.M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(args.ldo) * 2};
+  const cuuint32_t box[2] = {32, 32};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, args.out, dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int EPI>
 cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const BoxMaps& b, const GemmArgs& args,
                         long long tile_bound, cudaStream_t stream) {
@@ -1126,7 +1169,10 @@ cudaError_t launch_pair(const CUtensorMap& a0, const CUtensorMap& a1, const BoxM
   if (attr_err != cudaSuccess) return attr_err;
   if (tile_bound <= 0) return cudaSuccess;
   const int pairs = static_cast<int>(std::min<long long>(num_sms() / 2, tile_bound));
-  return launch_pdl(pair_gemm_kernel<EPI>, dim3(2 * pairs), dim3(L::kThr), L::kSmemBytes, stream, a0, a1, b, args);
+  CUtensorMap o;
+  if (!map_out_tiles(&o, args)) return cudaErrorInvalidValue;
+  return launch_pdl(pair_gemm_kernel<EPI>, dim3(2 * pairs), dim3(L::kThr), L::kSmemBytes, stream, a0, a1, b, o,
+                    args);
 }
 
 long long tile_bound(long long rows, int groups, int NT, int N, int feat) {
