@@ -159,6 +159,43 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(self.samples), "source": "nvml"}
 
 
+class GpuLocalCpus:
+    """Runs the enclosed host work on the CPUs of the GPU's own NUMA node (from sysfs), so that
+    pinned buffers first touched there sit next to the GPU's PCIe root; the previous affinity is
+    restored on exit.  A no-op where the node or the call is unavailable."""
+
+    def __init__(self, device: int):
+        self.device = device
+        self.saved = None
+
+    def _local(self):
+        p = torch.cuda.get_device_properties(self.device)
+        bus = f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        cpus = set()
+        with open(f"/sys/bus/pci/devices/{bus}/local_cpulist") as f:
+            for part in f.read().strip().split(","):
+                lo, _, hi = part.partition("-")
+                cpus.update(range(int(lo), int(hi or lo) + 1))
+        return cpus & os.sched_getaffinity(0)
+
+    def __enter__(self):
+        try:
+            local = self._local()
+            if local:
+                self.saved = os.sched_getaffinity(0)
+                os.sched_setaffinity(0, local)
+        except Exception:
+            self.saved = None
+        return self
+
+    def __exit__(self, *a):
+        if self.saved:
+            try:
+                os.sched_setaffinity(0, self.saved)
+            except Exception:
+                pass
+
+
 def code_fingerprint(path: str) -> str:
     """sha256[:12] of a CUDA source with its // comments and blank lines removed: a comment
     edit keeps the fingerprint, any change to the code changes it."""
@@ -491,14 +528,15 @@ def main():
     # for its copy-out and the copies are only half hidden; three lanes keep the SMs busy.
     d_in = cfg.d_model or cfg.H
     lanes = []
-    for i in range(E2E_LANES):
-        lb = bufs if i == 0 else B.alloc_layer_buffers(d, dev, gather=gather)
-        if cfg.F_shared and i > 0:
-            B.attach_aux_stream(lb, torch.cuda.Stream(dev))
-        lanes.append(dict(stream=torch.cuda.Stream(dev), bufs=lb,
-                          ws=ws if i == 0 else B.make_workspace(d, dev), xd=torch.empty_like(inp["x"]),
-                          oh=torch.empty((cfg.T, d_in), dtype=torch.bfloat16).pin_memory()))
-    xh = inp["x"].cpu().pin_memory()
+    with GpuLocalCpus(local) as numa:  # the pinned host buffers on the GPU's NUMA node
+        for i in range(E2E_LANES):
+            lb = bufs if i == 0 else B.alloc_layer_buffers(d, dev, gather=gather)
+            if cfg.F_shared and i > 0:
+                B.attach_aux_stream(lb, torch.cuda.Stream(dev))
+            lanes.append(dict(stream=torch.cuda.Stream(dev), bufs=lb,
+                              ws=ws if i == 0 else B.make_workspace(d, dev), xd=torch.empty_like(inp["x"]),
+                              oh=torch.empty((cfg.T, d_in), dtype=torch.bfloat16).pin_memory()))
+        xh = inp["x"].cpu().pin_memory()
 
     def e2e_step(j):
         ln = lanes[j % E2E_LANES]
@@ -607,7 +645,7 @@ def main():
             **({"fp8_dispatch": fp8_diag} if fp8_diag else {}),
             "fractions": frac,
             "e2e": {"value": e2e_value, "unit": UNIT, "streams": E2E_LANES, "h2d_bytes_per_step": cfg.T * d_in * 2,
-                    "d2h_bytes_per_step": cfg.T * d_in * 2},
+                    "d2h_bytes_per_step": cfg.T * d_in * 2, "pinned_on_gpu_numa_node": numa.saved is not None},
             "gpu_launches": (7 + (2 if cfg.d_model else 0) + (2 if cfg.F_shared else 0)) * args.steps,
             "clocks": clocks,
             "skew_max_over_mean": float(bufs["skew"].item()),
