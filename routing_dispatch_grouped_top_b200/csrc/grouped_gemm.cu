@@ -49,8 +49,9 @@ constexpr int kBM = 128;                  // output features per tile (MMA M)
 constexpr int kBK = 64;                   // K per stage: one 128-byte swizzle atom of bf16
 constexpr int kABytes = kBM * kBK * 2;    // 16 KB per weight tile
 // The token operand of a tile (nround rows, a multiple of 16) is fetched with one TMA box
-// per set bit of nround / 16: boxes of 256, 128, 64, 32 and 16 rows, at most 4 per stage.
-constexpr int kNumBoxes = 5;
+// per set bit of nround: boxes of 256, 128, 64, 32 and 16 rows (single CTA), or of 128 down to 8
+// rows for each CTA's half of a CTA-pair tile.
+constexpr int kNumBoxes = 6;
 struct BoxMaps {
   CUtensorMap box[kNumBoxes];  // box[i] is (256 >> i) rows x 64 columns
 };
@@ -631,6 +632,9 @@ struct PairLayout {
   static constexpr int GW = EPI == kEpiSwiGLU ? STAGES : 0;
   static constexpr int kThr = 64 + 32 * (EW + GW);
   static constexpr int FEAT = (EPI == kEpiBF16) ? 512 : 256;   // output features per pair tile
+  // token rows per tile rounded to ROUND (MMA N): 16 for bf16 operands (N = 16..256 in steps of
+  // 16 for a CTA pair), 32 for E4M3 operands
+  static constexpr int ROUND = EPI == kEpiSwiGLUFp8 ? 32 : 16;
   static constexpr int kAPair = NA * kABytes;                   // this CTA's 128-row weight boxes (one atom)
   static constexpr int kBBytes = (NT / 2) * 128;                // this CTA's token rows (one atom)
   static constexpr int kStageBytes = kAPair + kBBytes;
@@ -780,8 +784,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<EPI>::kTh
           rphase ^= 1u;
         }
         if (t < 0) break;
-        const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
-        const int half = tl.nround >> 1;  // token rows staged by each CTA (a multiple of 16)
+        const Tile tl = decode_tile<NT, L::ROUND, L::FEAT>(t, s_pre, s_off, G);
+        const int half = tl.nround >> 1;  // token rows staged by each CTA (a multiple of ROUND / 2)
         const int rbase = tl.row0 + static_cast<int>(rank) * half;
         for (int kb = 0; kb < KB; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status)) {
@@ -803,7 +807,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<EPI>::kTh
           if (!gather) {
             int r = 0;
 #pragma unroll
-            for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16 rows
+            for (int i = 1; i < kNumBoxes; ++i) {  // boxes of 128, 64, 32, 16, 8 rows
               const int rows = 256 >> i;
               if (half & rows) {
                 tma_load_2d_pair(st + L::kAPair + r * 128, &tmB.box[i], bar, kx, rbase + r);
@@ -851,7 +855,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<EPI>::kTh
           rphase ^= 1u;
         }
         if (t < 0) break;
-        const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
+        const Tile tl = decode_tile<NT, L::ROUND, L::FEAT>(t, s_pre, s_off, G);
         if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, args.status)) {
           ok = false;
           break;
@@ -922,7 +926,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<EPI>::kTh
         rphase ^= 1u;
       }
       if (t < 0) break;
-      const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
+      const Tile tl = decode_tile<NT, L::ROUND, L::FEAT>(t, s_pre, s_off, G);
       if (!mbar_wait(&tfull[acc], acc_phase, abort_flag, args.status)) break;
       tc_fence_after();
       const uint32_t tbase = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * L::kAccCols;
@@ -1013,7 +1017,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairLayout<EPI>::kTh
         rphase ^= 1u;
       }
       if (t < 0) break;
-      const Tile tl = decode_tile<NT, 32, L::FEAT>(t, s_pre, s_off, G);
+      const Tile tl = decode_tile<NT, L::ROUND, L::FEAT>(t, s_pre, s_off, G);
       const int half = tl.nround >> 1;
       // this CTA's rows are tile rows rank * half + i; rows past the valid ones repeat row 0
       // (computed, never stored)
@@ -1192,7 +1196,7 @@ int gemm_smem_bytes(int epi) {
 }
 
 // The CTA-pair kernel serves groups of at least MOE_PAIR_MIN_ROWS rows on average (its
-// token tiles are cut in multiples of 32 rows and split between the two SMs); smaller
+// token tiles are cut in multiples of 16 (E4M3: 32) rows and split between the two SMs); smaller
 // groups (decode) and the fp32 gating use the single-CTA kernel.  MOE_GEMM_PAIR=0 builds
 // the single-CTA kernel only.
 #ifndef MOE_GEMM_PAIR
