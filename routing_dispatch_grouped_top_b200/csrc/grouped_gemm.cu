@@ -20,13 +20,14 @@
 //   warp 0      TMA producer: claims the next tile of the launch from a counter in
 //               the workspace (the last CTA rewinds it), publishes its id through a
 //               ring of tile ids in shared memory, and streams weight boxes of 128 or
-//               256 rows and token boxes of 16..256 rows (128-byte swizzle) into a
+//               256 rows and token boxes of 8..256 rows (128-byte swizzle) into a
 //               STAGES-deep ring of shared memory;
 //   warp 1      TMEM owner and single-thread tcgen05.mma issuer;
 //   warps 2..   epilogue: tcgen05.ld of the fp32 accumulator (warp w reads the TMEM
 //               lane quadrant w % 4; with eight warps two share a quadrant and take
 //               alternate 32-token chunks), activation, and bf16 rows written through a
-//               per-warp shared-memory transpose as 16-byte pieces;
+//               per-warp shared-memory transpose as 16-byte pieces (the pair kernel's bf16
+//               epilogue stores each full 32 x 32 chunk with one TMA tile store instead);
 //   (pair, SwiGLU) four gather warps, one per stage, that copy the token rows with 16-byte
 //               cp.async through the rows' source indices when the operand is gathered in
 //               place instead of read from a permuted copy.
